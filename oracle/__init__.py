@@ -1,0 +1,159 @@
+"""CPU oracle for the PATCH hybrid tile-sparse linear layer (test infrastructure).
+
+Only the test suite, the package smoke check and the benchmark's CPU-baseline
+leg may import this package.  The arithmetic lives in ``patch_oracle.c``
+(plain C, fp64, OpenMP over output elements); this module only compiles it
+with gcc and marshals numpy arrays.  It shares no code with the CUDA library.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "patch_oracle.c"
+_LIB = _HERE / "liboracle.so"
+
+TILE = 128
+_lib = None
+
+
+def build(force: bool = False) -> Path:
+    """Compile patch_oracle.c into liboracle.so (gcc -O2 -fopenmp)."""
+    if force or not _LIB.exists() or _LIB.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB.with_suffix(f".so.{os.getpid()}.tmp")
+        subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall",
+                        "-o", str(tmp), str(_SRC)], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(str(build()))
+        P, I64 = ctypes.c_void_p, ctypes.c_int64
+        for name, args in {
+            "oracle_apply_mask": [P, I64, I64, P, P, P],
+            "oracle_hard_mask": [P, I64, I64, P, P, P, P, P],
+            "oracle_pack": [P, I64, I64, P, P, I64, P, P, P],
+            "oracle_unpack": [P, P, P, I64, I64, P],
+            "oracle_gemm_rows": [P, I64, P, I64, P, I64, I64, P],
+            "oracle_hybrid_gemm": [P, I64, P, I64, P, I64, I64, P, P, P],
+        }.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        lib.oracle_pack_sizes.argtypes = [I64, I64, I64, P, P, P]
+        lib.oracle_pack_sizes.restype = None
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise OracleError(f"{what}: oracle error {rc}")
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def apply_mask(w: np.ndarray, bitmap: np.ndarray, pat_id: np.ndarray) -> np.ndarray:
+    w = np.ascontiguousarray(w, np.uint16)
+    N, K = w.shape
+    out = np.empty_like(w)
+    _check(_load().oracle_apply_mask(_ptr(w), N, K, _ptr(np.ascontiguousarray(bitmap, np.uint8)),
+                                     _ptr(np.ascontiguousarray(pat_id, np.uint8)), _ptr(out)),
+           "apply_mask")
+    return out
+
+
+def hard_mask(w: np.ndarray, tile_logits: np.ndarray, pattern_logits: np.ndarray):
+    """Returns (W_masked, bitmap [Tn][Tk] u8, pat_id [N][K/4] u8)."""
+    w = np.ascontiguousarray(w, np.uint16)
+    N, K = w.shape
+    wm = np.empty_like(w)
+    bitmap = np.empty((N // TILE, K // TILE), np.uint8)
+    pid = np.empty((N, K // 4), np.uint8)
+    _check(_load().oracle_hard_mask(_ptr(w), N, K, _ptr(np.ascontiguousarray(tile_logits, np.float32)),
+                                    _ptr(np.ascontiguousarray(pattern_logits, np.float32)),
+                                    _ptr(wm), _ptr(bitmap), _ptr(pid)), "hard_mask")
+    return wm, bitmap, pid
+
+
+def pack_sizes(N: int, K: int, n_sparse: int):
+    v, m, d = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    _load().oracle_pack_sizes(N, K, n_sparse, ctypes.byref(v), ctypes.byref(m), ctypes.byref(d))
+    return v.value, m.value, d.value
+
+
+def pack(w: np.ndarray, bitmap: np.ndarray, pat_id: np.ndarray):
+    """Returns (values u8, meta u8, desc u8) blobs of the packed format."""
+    w = np.ascontiguousarray(w, np.uint16)
+    N, K = w.shape
+    bitmap = np.ascontiguousarray(bitmap, np.uint8)
+    ns = int(np.count_nonzero(bitmap))
+    vb, mb, db = pack_sizes(N, K, ns)
+    values = np.zeros(vb, np.uint8)
+    meta = np.zeros(max(mb, 1), np.uint8)
+    desc = np.zeros(db, np.uint8)
+    _check(_load().oracle_pack(_ptr(w), N, K, _ptr(bitmap), _ptr(np.ascontiguousarray(pat_id, np.uint8)),
+                               ns, _ptr(values), _ptr(meta), _ptr(desc)), "pack")
+    return values, meta[:mb], desc
+
+
+def unpack(values: np.ndarray, meta: np.ndarray, desc: np.ndarray, N: int, K: int) -> np.ndarray:
+    out = np.empty((N, K), np.uint16)
+    meta = np.ascontiguousarray(meta, np.uint8) if meta.size else np.zeros(1, np.uint8)
+    _check(_load().oracle_unpack(_ptr(np.ascontiguousarray(values, np.uint8)), _ptr(meta),
+                                 _ptr(np.ascontiguousarray(desc, np.uint8)), N, K, _ptr(out)), "unpack")
+    return out
+
+
+def gemm(x: np.ndarray, w_eff: np.ndarray, rows: np.ndarray | None = None) -> np.ndarray:
+    """fp64 Y = X * W_eff^T over bf16 bit inputs (optionally only the given rows of X)."""
+    x = np.ascontiguousarray(x, np.uint16)
+    w_eff = np.ascontiguousarray(w_eff, np.uint16)
+    M, K = x.shape
+    N = w_eff.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    R = M if r is None else r.size
+    y = np.empty((R, N), np.float64)
+    _check(_load().oracle_gemm_rows(_ptr(x), M, _ptr(r), 0 if r is None else r.size,
+                                    _ptr(w_eff), N, K, _ptr(y)), "gemm")
+    return y
+
+
+def hybrid_gemm(x: np.ndarray, w: np.ndarray, bitmap: np.ndarray, pat_id: np.ndarray,
+                rows: np.ndarray | None = None) -> np.ndarray:
+    """The layer: hybrid mask applied to W, then fp64 Y = X * W_eff^T."""
+    x = np.ascontiguousarray(x, np.uint16)
+    w = np.ascontiguousarray(w, np.uint16)
+    M, K = x.shape
+    N = w.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    R = M if r is None else r.size
+    y = np.empty((R, N), np.float64)
+    _check(_load().oracle_hybrid_gemm(_ptr(x), M, _ptr(r), 0 if r is None else r.size, _ptr(w), N, K,
+                                      _ptr(np.ascontiguousarray(bitmap, np.uint8)),
+                                      _ptr(np.ascontiguousarray(pat_id, np.uint8)), _ptr(y)),
+           "hybrid_gemm")
+    return y

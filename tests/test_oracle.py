@@ -1,0 +1,315 @@
+"""Pins of the CPU oracle against facts fixed outside it (no GPU needed).
+
+Each test checks the oracle against something it does not compute itself:
+the method's invariants (PATCH: Learnable Tile-level Hybrid Sparsity for LLMs,
+section 2 "Methodology: PATCH"), brute force over the 6 patterns, numpy's
+library matmul / argmax, closed-form sizes, and the pattern table under
+tests/golden/.
+"""
+import itertools
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth_inputs as si
+
+TILE = 128
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pattern_codes.txt")
+PAIRS = list(itertools.combinations(range(4), 2))  # lexicographic, library-generated
+ONE = np.uint16(0x3F80)  # bf16 1.0
+
+
+def golden_codes():
+    rows = []
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                i, a, b, c = line.split()
+                rows.append((int(i), int(a), int(b), int(c, 16)))
+    return rows
+
+
+def mask_from_pairs(bitmap, pat_id, N, K):
+    """Keep-mask built from the itertools pair list (independent of the oracle's table)."""
+    keep = np.ones((N, K), bool)
+    pos = np.arange(K) % 4
+    for n in range(N):
+        for tk in range(K // TILE):
+            if bitmap[n // TILE, tk]:
+                sl = slice(tk * TILE, (tk + 1) * TILE)
+                ids = np.repeat(pat_id[n, tk * 32:(tk + 1) * 32], 4)
+                a = np.array([PAIRS[i][0] for i in ids])
+                b = np.array([PAIRS[i][1] for i in ids])
+                keep[n, sl] = (pos[sl] == a) | (pos[sl] == b)
+    return keep
+
+
+def f64(bits):
+    return si.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+# ---------------------------------------------------------------- hard mask
+
+
+@pytest.mark.parametrize("pid", range(6))
+def test_hard_mask_one_hot_pattern(pid):
+    N = K = TILE
+    w = np.full((N, K), ONE, np.uint16)
+    tl = np.zeros((1, 1, 2), np.float32)
+    tl[..., 1] = 1.0  # sparse
+    pl = np.zeros((N, K // 4, 6), np.float32)
+    pl[..., pid] = 1.0
+    wm, bm, ids = oracle.hard_mask(w, tl, pl)
+    assert bm.tolist() == [[1]]
+    assert np.all(ids == pid)
+    keep = np.zeros(4, bool)
+    keep[list(PAIRS[pid])] = True
+    expect = np.where(np.tile(keep, K // 4)[None, :], ONE, np.uint16(0))
+    assert np.array_equal(wm, np.broadcast_to(expect, (N, K)))
+
+
+def test_hard_mask_tile_choice_and_ties():
+    N, K = 2 * TILE, 2 * TILE
+    w = np.full((N, K), ONE, np.uint16)
+    tl = np.array([[[1.0, 0.0], [0.0, 1.0]], [[0.5, 0.5], [-1.0, -0.5]]], np.float32)
+    pl = np.zeros((N, K // 4, 6), np.float32)  # all tied -> pattern 0
+    wm, bm, ids = oracle.hard_mask(w, tl, pl)
+    assert bm.tolist() == [[0, 1], [0, 1]]  # tie -> dense (index 0)
+    assert np.all(ids == 0)
+    # sparse tiles keep positions 0,1 of each group; dense tiles keep all
+    assert np.all(wm[:TILE, :TILE] == ONE)
+    assert np.all(wm[:TILE, TILE:].reshape(TILE, -1, 4)[:, :, 2:] == 0)
+    assert np.all(wm[:TILE, TILE:].reshape(TILE, -1, 4)[:, :, :2] == ONE)
+
+
+def test_hard_mask_pattern_ties_and_nan_reading():
+    N = K = TILE
+    w = np.full((N, K), ONE, np.uint16)
+    tl = np.array([[[0.0, 1.0]]], np.float32)
+    pl = np.zeros((N, K // 4, 6), np.float32)
+    pl[0, 0] = [0, 1, 1, 0, 0, 0]          # tie between 1 and 2 -> 1
+    pl[0, 1] = [np.nan, 5, 6, 7, 8, 9]     # NaN first: no later value beats it -> 0
+    pl[0, 2] = [0, np.nan, 1, 0, 0, 0]     # NaN later never wins -> 2
+    pl[0, 3] = [-3, -2, -1, -1, -5, -1]    # first maximum -> 2
+    _, _, ids = oracle.hard_mask(w, tl, pl)
+    assert ids[0, :4].tolist() == [1, 0, 2, 2]
+
+
+def test_hard_mask_matches_numpy_argmax_random():
+    N, K = 256, 384
+    w = si.gen_w(N, K, 1, 0)
+    tl = si.gen_tile_logits(N, K, 1, 0)
+    pl = si.gen_pattern_logits(N, K, 1, 0)
+    wm, bm, ids = oracle.hard_mask(w, tl, pl)
+    assert np.array_equal(bm, np.argmax(tl, axis=-1).astype(np.uint8))
+    assert np.array_equal(ids, np.argmax(pl, axis=-1).astype(np.uint8))
+    keep = mask_from_pairs(bm, ids, N, K)
+    assert np.array_equal(wm, np.where(keep, w, np.uint16(0)))
+
+
+def test_pruned_weights_are_positive_zero():
+    N = K = TILE
+    w = np.full((N, K), np.uint16(0xBF80), np.uint16)  # -1.0
+    bm = np.ones((1, 1), np.uint8)
+    ids = np.full((N, K // 4), 5, np.uint8)
+    wm = oracle.apply_mask(w, bm, ids)
+    g = wm.reshape(N, -1, 4)
+    assert np.all(g[:, :, :2] == 0x0000) and np.all(g[:, :, 2:] == 0xBF80)
+
+
+# --------------------------------------------------------------- invariants
+
+
+@pytest.mark.parametrize("frac", [0.0, 0.25, 0.5, 0.75, 1.0])
+def test_two_of_four_and_global_sparsity(frac):
+    N, K = 3 * TILE, 4 * TILE
+    w = np.full((N, K), ONE, np.uint16)
+    bm = si.tiles_exact(N, K, frac, 3, 7)
+    ids = np.random.default_rng(5).integers(0, 6, (N, K // 4)).astype(np.uint8)
+    wm = oracle.apply_mask(w, bm, ids)
+    nz = (wm != 0).reshape(N // TILE, TILE, K // TILE, TILE // 4, 4).sum(-1)
+    for tn in range(N // TILE):
+        for tk in range(K // TILE):
+            expect = 2 if bm[tn, tk] else 4
+            assert np.all(nz[tn, :, tk, :] == expect)
+    T = bm.size
+    ns = int(bm.sum())
+    pruned = int(np.count_nonzero(wm == 0))
+    assert pruned * 2 * T == N * K * ns  # sparsity == 0.5 * ns / T exactly
+    assert 0.0 <= pruned / (N * K) <= 0.5
+
+
+# ---------------------------------------------------------------- packing
+
+
+def test_pack_sizes_closed_form():
+    for N, K, ns in [(128, 128, 0), (128, 128, 1), (4096, 4096, 512), (11008, 4096, 1376)]:
+        T = (N // TILE) * (K // TILE)
+        assert oracle.pack_sizes(N, K, ns) == ((T - ns) * 32768 + ns * 16384, ns * 2048, 16 * T)
+
+
+@pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
+def test_pack_unpack_round_trip(frac):
+    N, K = 3 * TILE, 5 * TILE
+    w = si.gen_w(N, K, 2, 1)
+    bm = si.tiles_exact(N, K, frac, 2, 1)
+    ids = si.patterns_top2(w)
+    values, meta, desc = oracle.pack(w, bm, ids)
+    vb, mb, db = oracle.pack_sizes(N, K, int(bm.sum()))
+    assert (values.size, meta.size, desc.size) == (vb, mb, db)
+    w_eff = oracle.unpack(values, meta, desc, N, K)
+    assert np.array_equal(w_eff, oracle.apply_mask(w, bm, ids))
+    # masked and unmasked W pack to the same bytes
+    v2, m2, d2 = oracle.pack(oracle.apply_mask(w, bm, ids), bm, ids)
+    assert np.array_equal(values, v2) and np.array_equal(meta, m2) and np.array_equal(desc, d2)
+
+
+def test_descriptor_table():
+    N, K = 2 * TILE, 3 * TILE
+    w = si.gen_w(N, K)
+    bm = np.array([[1, 0, 1], [0, 0, 1]], np.uint8)
+    _, _, desc = oracle.pack(w, bm, si.patterns_top2(w))
+    d = desc.reshape(-1, 16)
+    kinds = d[:, 0:4].copy().view("<u4").ravel()
+    ords = d[:, 4:8].copy().view("<u4").ravel()
+    offs = d[:, 8:16].copy().view("<u8").ravel()
+    assert kinds.tolist() == [1, 0, 1, 0, 0, 1]
+    assert ords.tolist() == [0, 0xFFFFFFFF, 1, 0xFFFFFFFF, 0xFFFFFFFF, 2]
+    sizes = [16384 if k else 32768 for k in kinds]
+    assert offs.tolist() == list(np.concatenate([[0], np.cumsum(sizes)[:-1]]))
+
+
+def test_pattern_codes_against_golden():
+    codes = golden_codes()
+    assert [(a, b) for _, a, b, _ in codes] == PAIRS
+    N = K = TILE
+    w = np.full((N, K), ONE, np.uint16)
+    bm = np.ones((1, 1), np.uint8)
+    for pid, a, b, code in codes:
+        assert code == a | (b << 2)
+        _, meta, _ = oracle.pack(w, bm, np.full((N, K // 4), pid, np.uint8))
+        assert np.all(meta == (code | (code << 4)))
+
+
+def hw_meta_position(r, g):
+    """Byte and nibble of group g of tile row r, restated from the tensor-memory
+    placement the 16-bit sparse MMA (M = 128) reads: lane = r%8 + 8*((k//16)%2)
+    + 16*(r//16), 32-bit column = k//32, byte in column = (k%16)//8 + 2*((r//8)%2),
+    nibble = (k//4)%2, with k = 4g; a tcgen05.cp 128x128b copy puts 16 bytes per lane."""
+    k = 4 * g
+    lane = r % 8 + 8 * ((k // 16) % 2) + 16 * (r // 16)
+    col = k // 32
+    byte = (k % 16) // 8 + 2 * ((r // 8) % 2)
+    return lane * 16 + col * 4 + byte, (k // 4) % 2
+
+
+def test_metadata_layout_positions():
+    N = K = TILE
+    w = np.full((N, K), ONE, np.uint16)
+    bm = np.ones((1, 1), np.uint8)
+    seen = set()
+    rng = np.random.default_rng(11)
+    cells = [(r, g) for r in range(TILE) for g in range(32)]
+    for idx in rng.permutation(len(cells))[:512]:
+        r, g = cells[idx]
+        ids = np.zeros((N, K // 4), np.uint8)  # code 0x4 everywhere
+        ids[r, g] = 5                          # code 0xE at one group
+        _, meta, _ = oracle.pack(w, bm, ids)
+        byte, nib = hw_meta_position(r, g)
+        assert (meta[byte] >> (4 * nib)) & 0xF == 0xE
+        others = meta.copy()
+        others[byte] &= ~np.uint8(0xF << (4 * nib))
+        others[byte] |= np.uint8(0x4 << (4 * nib))
+        assert np.all(others == 0x44)
+        seen.add((byte, nib))
+    assert len(seen) == 512
+    # the restated placement is a bijection onto the 2048 bytes x 2 nibbles
+    allpos = {hw_meta_position(r, g) for r, g in cells}
+    assert len(allpos) == TILE * 32
+
+
+# ------------------------------------------------------------------- GEMM
+
+
+def test_gemm_all_dense_is_dense_matmul():
+    M, N, K = 5, 2 * TILE, 3 * TILE
+    x, w = si.gen_x(M, K, 4, 0), si.gen_w(N, K, 4, 0)
+    bm = np.zeros((N // TILE, K // TILE), np.uint8)
+    y = oracle.hybrid_gemm(x, w, bm, si.patterns_top2(w))
+    ref = f64(x) @ f64(w).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_gemm_all_sparse_is_24_matmul():
+    M, N, K = 4, 2 * TILE, 2 * TILE
+    x, w = si.gen_x(M, K, 4, 1), si.gen_w(N, K, 4, 1)
+    bm = np.ones((N // TILE, K // TILE), np.uint8)
+    ids = np.random.default_rng(3).integers(0, 6, (N, K // 4)).astype(np.uint8)
+    y = oracle.hybrid_gemm(x, w, bm, ids)
+    keep = mask_from_pairs(bm, ids, N, K)
+    ref = f64(x) @ np.where(keep, f64(w), 0.0).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_gemm_one_hot_columns_brute_force():
+    N = K = TILE
+    w = si.gen_w(N, K, 4, 2)
+    bm = np.ones((1, 1), np.uint8)
+    ids = (np.arange(N * (K // 4)) % 6).astype(np.uint8).reshape(N, K // 4)  # all 6 patterns
+    x = np.zeros((K, K), np.uint16)
+    x[np.arange(K), np.arange(K)] = ONE       # row m is the unit vector e_m
+    y = oracle.hybrid_gemm(x, w, bm, ids)     # y[m][n] = W_eff[n][m]
+    for n in range(N):
+        for g in range(K // 4):
+            a, b = PAIRS[ids[n, g]]
+            for i in range(4):
+                expect = f64(w[n, 4 * g + i]) if i in (a, b) else 0.0
+                assert y[4 * g + i, n] == expect
+
+
+def test_gemm_linear_over_tiles():
+    M, N, K = 3, 3 * TILE, 3 * TILE
+    x, w = si.gen_x(M, K, 4, 3), si.gen_w(N, K, 4, 3)
+    bm = si.tiles_exact(N, K, 0.5, 4, 3)
+    ids = si.patterns_top2(w)
+    y = oracle.hybrid_gemm(x, w, bm, ids)
+    tile_is_sparse = np.kron(bm, np.ones((TILE, TILE), np.uint8)).astype(bool)
+    keep = mask_from_pairs(bm, ids, N, K)
+    w_dense_part = np.where(~tile_is_sparse, f64(w), 0.0)
+    w_sparse_part = np.where(tile_is_sparse & keep, f64(w), 0.0)
+    ref = f64(x) @ w_dense_part.T + f64(x) @ w_sparse_part.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_gemm_row_sample_equals_full():
+    M, N, K = 9, TILE, 2 * TILE
+    x, w = si.gen_x(M, K, 4, 4), si.gen_w(N, K, 4, 4)
+    bm = si.tiles_bernoulli(N, K, 0.5, 4, 4)
+    ids = si.patterns_top2(w)
+    full = oracle.hybrid_gemm(x, w, bm, ids)
+    rows = np.array([8, 0, 3])
+    assert np.array_equal(oracle.hybrid_gemm(x, w, bm, ids, rows=rows), full[rows])
+
+
+# ---------------------------------------------------------- input recipe
+
+
+def test_top2_patterns_are_magnitude_argmax():
+    """Generator's top-2 ids == argmax over the 6 pairs of |wi|+|wj| (fp64, ties low)."""
+    w = si.gen_w(TILE, TILE, 6, 0)
+    w[0, :4] = [0x3F80, 0xBF80, 0x3F80, 0x0000]  # |1|,|-1|,|1|,0 -> tie resolved to (0,1)
+    ids = si.patterns_top2(w)
+    mag = np.abs(f64(w)).reshape(TILE, -1, 4)
+    score = np.stack([mag[:, :, a] + mag[:, :, b] for a, b in PAIRS], axis=-1)
+    assert np.array_equal(ids, np.argmax(score, axis=-1).astype(np.uint8))
+    assert ids[0, 0] == 0
+
+
+def test_bf16_rounding_is_rne():
+    f = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 3.0e-3], np.float32)
+    b = si.f32_to_bf16_bits(f)
+    assert b.tolist()[:4] == [0x3F80, 0x3F80, 0x3F82, 0xC020]  # ties go to even
+    assert abs(si.bf16_bits_to_f32(b)[4] - 3.0e-3) < 3.0e-3 * 2 ** -8
