@@ -1,0 +1,399 @@
+"""Benchmark of the PATCH hybrid tile-sparse linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill]
+                    [--impl ours|reference]
+
+Default workload ("decode"): the 7 LLaMA-2-7B linear layers (q/k/v/o 4096x4096,
+gate/up 11008x4096, down 4096x11008), 50% of the 128x128 tiles 2:4 sparse
+(exact count, seeded uniform positions), magnitude-top-2 patterns, at
+M = 1, 4 and 16 tokens.  One step = the 21 patch_gemm calls (7 layers x 3 M)
+over packed weights resident in HBM; the metric is HBM GB/s counting only the
+bytes the layer must move: stored weight bytes (dense tiles 32 KiB, sparse
+tiles 16 KiB values + 2 KiB metadata, 16 B descriptor per tile) + X + Y.
+
+"prefill": the same 7 shapes at M = 2048, sparse-tile fraction swept over
+{0, 0.25, 0.5, 0.75, 1}; metric dense-equivalent TFLOP/s (2*M*N*K / time).
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle (plain
+C, fp64) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth_inputs as si  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+DECODE_MS = (1, 4, 16)
+PREFILL_M = 2048
+FRACS = (0.0, 0.25, 0.5, 0.75, 1.0)
+DECODE_CONFIG = 2   # seeds of the decode workload
+PREFILL_CONFIG = 3  # seeds of the prefill workload
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def stored_bytes(N, K, n_sparse):
+    T = (N // 128) * (K // 128)
+    return (T - n_sparse) * 32768 + n_sparse * (16384 + 2048) + 16 * T
+
+
+# ------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) of the SM clock and throttle reasons."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ workloads
+
+
+def build_layers(workload):
+    """Host inputs of every layer in the step: list of dicts."""
+    layers = []
+    if workload == "decode":
+        for i, (name, N, K) in enumerate(si.LLAMA2_7B):
+            w = si.gen_w(N, K, DECODE_CONFIG, i)
+            bm = si.tiles_exact(N, K, 0.5, DECODE_CONFIG, i)
+            layers.append(dict(name=name, N=N, K=K, w=w, bm=bm, ids=si.patterns_top2(w), frac=0.5,
+                               xs={M: si.gen_x(M, K, DECODE_CONFIG, i) for M in DECODE_MS}))
+    else:
+        for i, (name, N, K) in enumerate(si.LLAMA2_7B):
+            w = si.gen_w(N, K, PREFILL_CONFIG, i)
+            ids = si.patterns_top2(w)
+            x = si.gen_x(PREFILL_M, K, PREFILL_CONFIG, i)
+            for f in FRACS:
+                bm = si.tiles_exact(N, K, f, PREFILL_CONFIG, i)
+                layers.append(dict(name=name, N=N, K=K, w=w, bm=bm, ids=ids, frac=f, xs={PREFILL_M: x}))
+    return layers
+
+
+def calls_of(layers):
+    """(layer index, M) for every GEMM of one step, in order."""
+    return [(li, M) for M in sorted({m for L in layers for m in L["xs"]}) for li, L in enumerate(layers)
+            if M in L["xs"]]
+
+
+def call_bytes(L, M):
+    return stored_bytes(L["N"], L["K"], int(L["bm"].sum())) + 2 * M * L["K"] + 2 * M * L["N"]
+
+
+def call_flops(L, M):
+    return 2.0 * M * L["N"] * L["K"]
+
+
+# ------------------------------------------------------------ CPU oracle
+
+
+def cpu_baseline(workload, budget_s=15.0):
+    """Time the CPU oracle on a bounded sample of the workload (same metric)."""
+    import oracle
+    layers = build_layers(workload)
+    done_units, spent, what = 0.0, 0.0, []
+    for li, M in calls_of(layers):
+        L = layers[li]
+        x = L["xs"][M]
+        rows = None
+        if workload == "prefill":
+            rows = np.arange(0, M, M // 16)[:16]  # 16 of the 2048 rows
+        t0 = time.perf_counter()
+        oracle.hybrid_gemm(x, L["w"], L["bm"], L["ids"], rows=rows)
+        dt = time.perf_counter() - t0
+        spent += dt
+        if workload == "decode":
+            done_units += call_bytes(L, M) / 1e9
+            what.append(f"{L['name']}@M={M}")
+        else:
+            done_units += call_flops(L, 16) / 1e12
+            what.append(f"{L['name']}/f={L['frac']}@16rows")
+        if spent >= budget_s:
+            break
+    return {"value": done_units / spent, "unit": "GB/s" if workload == "decode" else "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle", "seconds": round(spent, 3),
+            "sample": ("decode GEMMs " if workload == "decode" else "prefill GEMMs, 16 of 2048 token rows each: ")
+            + ", ".join(what[:8]) + (" ..." if len(what) > 8 else "") + f" ({len(what)} calls)"}
+
+
+# ------------------------------------------------------------ GPU arm
+
+
+def run_ours(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    import tile_sparse_gemm_b200 as tsg
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    layers = build_layers(args.workload)
+    calls = calls_of(layers)
+    status = tsg.new_status(dev)
+    packed = []
+    for L in layers:
+        pw = tsg.patch_pack(torch.from_numpy(L["w"].view(np.int16)).view(torch.bfloat16).to(dev),
+                            torch.from_numpy(L["bm"]).to(dev), torch.from_numpy(L["ids"]).to(dev),
+                            int(L["bm"].sum()), status=status)
+        packed.append(pw)
+    xs = {(li, M): torch.from_numpy(layers[li]["xs"][M].view(np.int16)).view(torch.bfloat16).to(dev)
+          for li, M in calls}
+    ys = {(li, M): torch.empty((M, layers[li]["N"]), dtype=torch.bfloat16, device=dev) for li, M in calls}
+    ws_bytes = max(tsg.patch_gemm_workspace_size(M, packed[li]) for li, M in calls)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    launches_per_call = {c: (2 if tsg.patch_gemm_workspace_size(c[1], packed[c[0]]) > 0 else 1) for c in calls}
+    stream = torch.cuda.current_stream()
+    resident = sum(p.stored_bytes for p in packed)
+
+    def step(per_call_events=None):
+        for j, (li, M) in enumerate(calls):
+            if per_call_events is not None:
+                per_call_events[j][0].record(stream)
+            tsg.patch_gemm(xs[(li, M)], packed[li], Y=ys[(li, M)], workspace=ws, status=status)
+            if per_call_events is not None:
+                per_call_events[j][1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    code, bits = tsg.patch_read_status(status)
+    if code != 0:
+        raise RuntimeError(f"device status {code} bits {bits} after warm-up")
+
+    # timed region: whole-step events plus per-call events for the roofline
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        t_start.record(stream)
+        for s in range(args.steps):
+            step(ev[s])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t_start.elapsed_time(t_end)
+    call_ms = np.array([[a.elapsed_time(b) for a, b in ev[s]] for s in range(args.steps)])  # [steps][calls]
+    code, bits = tsg.patch_read_status(status)
+    if code != 0:
+        raise RuntimeError(f"device status {code} bits {bits} after timing")
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    xh = {c: xs[c].cpu().pin_memory() for c in calls}
+    yh = {c: torch.empty(ys[c].shape, dtype=torch.bfloat16).pin_memory() for c in calls}
+    h2d = sum(xh[c].numel() * 2 for c in calls)
+    d2h = sum(yh[c].numel() * 2 for c in calls)
+
+    def e2e_step():
+        for li, M in calls:
+            xs[(li, M)].copy_(xh[(li, M)], non_blocking=True)
+            tsg.patch_gemm(xs[(li, M)], packed[li], Y=ys[(li, M)], workspace=ws, status=status)
+            yh[(li, M)].copy_(ys[(li, M)], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    if args.workload == "decode":
+        unit, per_step = "GB/s", sum(call_bytes(layers[li], M) for li, M in calls) / 1e9
+        metric = "hybrid GEMM HBM GB/s over stored bytes (decode)"
+    else:
+        unit, per_step = "TFLOP/s", sum(call_flops(layers[li], M) for li, M in calls) / 1e12
+        metric = "hybrid GEMM TFLOP/s, dense-equivalent (prefill)"
+    value = per_step * args.steps * world / (ms / 1e3)
+    e2e_value = per_step * args.steps * world / (e2e_ms / 1e3)
+
+    # roofline of the dominant kernel: algorithmic bytes (or FLOPs) per launch / mean launch time
+    mean_call_ms = call_ms.mean(axis=0)
+    if args.workload == "decode":
+        alg = np.array([call_bytes(layers[li], M) for li, M in calls]) / 1e9
+        achieved = float(alg.sum() / (mean_call_ms.sum() / 1e3))
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                "kernel": "decode_gemm_kernel (+ split-K reduce)", "peak_source": pk["source"]}
+        detail = {f"{layers[li]['name']}@M={M}": {"us": round(1e3 * mean_call_ms[j], 2),
+                                                  "GB/s": round(alg[j] / (mean_call_ms[j] / 1e3), 1)}
+                  for j, (li, M) in enumerate(calls)}
+    else:
+        # mixed roofline: dense tiles at the dense peak, sparse tiles at 2x (the datasheet ratio)
+        P = pk["bf16_tflops"]
+        t_roof = np.array([2.0 * M * 128 * 128 * ((layers[li]["N"] * layers[li]["K"] // 16384 - int(layers[li]["bm"].sum()))
+                                                  / P + int(layers[li]["bm"].sum()) / (2 * P)) / 1e12
+                           for li, M in calls])
+        alg = np.array([call_flops(layers[li], M) for li, M in calls]) / 1e12
+        achieved = float(alg.sum() / (mean_call_ms.sum() / 1e3))
+        frac_roof = float(t_roof.sum() / (mean_call_ms.sum() / 1e3))
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": P, "unit": "TFLOP/s",
+                "frac": round(frac_roof, 4), "traffic": None, "kernel": "prefill_kernel (tcgen05)",
+                "peak_source": pk["source"], "note": "frac = mixed roofline time (dense tiles at peak, sparse at 2x peak) / measured"}
+        detail = {}
+        for j, (li, M) in enumerate(calls):
+            L = layers[li]
+            detail[f"{L['name']}/f={L['frac']}"] = {"us": round(1e3 * mean_call_ms[j], 1),
+                                                   "TFLOP/s": round(alg[j] / (mean_call_ms[j] / 1e3), 1),
+                                                   "roofline_frac": round(t_roof[j] / (mean_call_ms[j] / 1e3), 3)}
+
+    out = {
+        "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"LLaMA-2-7B linear layers ({args.workload})",
+                   "shapes": [f"{n}:{N}x{K}" for n, N, K in si.LLAMA2_7B],
+                   "tokens": sorted({M for _, M in calls}),
+                   "sparse_tile_fraction": sorted({L["frac"] for L in layers}),
+                   "resident_weight_bytes": resident,
+                   "l2": f"inputs larger than L2: {resident / 2**20:.0f} MiB of packed weights read in rotation",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(sum(launches_per_call[c] for c in calls) * args.steps),
+        "clocks": clocks.summary(),
+        "per_call": detail,
+    }
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        # the CPU oracle, timed as it stands on the host cores; rank 0 only
+        if rank != 0:
+            return
+        steps = []
+        cb = None
+        for _ in range(args.warmup):
+            cpu_baseline(args.workload, budget_s=1.0)
+        for _ in range(args.steps):
+            cb = cpu_baseline(args.workload, budget_s=5.0)
+            steps.append(cb["value"])
+        value = statistics.median(steps)
+        cb = dict(cb, value=round(value, 4))
+        print(json.dumps({"impl": "reference", "metric": "hybrid GEMM HBM GB/s over stored bytes (decode)"
+                          if args.workload == "decode" else "hybrid GEMM TFLOP/s, dense-equivalent (prefill)",
+                          "value": round(value, 4), "unit": cb["unit"], "n_gpus": args.gpus, "steps": args.steps,
+                          "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": f"LLaMA-2-7B linear layers ({args.workload})"},
+                          "cpu_baseline": cb,
+                          "e2e": {"value": round(value, 4), "unit": cb["unit"], "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    out = run_ours(args, rank, world)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(args.workload)
+        print(json.dumps(out))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+/*
+ * patch.h - C ABI of libpatch.so, the B200 (sm_100a) implementation of the
+ * inference hot path of PATCH, the hybrid tile-sparse linear layer
+ *
+ *     Y[m][n] = sum_k X[m][k] * W_eff[n][k]        (Y = X * W_eff^T)
+ *
+ * Source: "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs"
+ * (arXiv 2509.23410), as summarised on gist.science/paper/2509.23410:
+ *   - section 2 "Methodology: PATCH", "Core Mechanism": W is cut into tiles,
+ *     each tile is dense (0% sparsity) or 2:4 sparse (50% sparsity); the
+ *     final mask is a combination of a dense and a 2:4 option;
+ *   - "Learnable Distributions": a 2-way tile logit distribution chooses
+ *     dense vs sparse; inside sparse tiles a separate distribution chooses one
+ *     of the 6 possible 2:4 patterns;
+ *   - "Inference & Deployment": 128 x 128 execution tiles; dense tiles run on
+ *     dense tensor-core MMA, sparse tiles on the 2:4 sparse tensor cores.
+ *
+ * Conventions shared by every entry point
+ *   - bf16 values travel as uint16_t bit patterns.
+ *   - W is N x K row-major (K contiguous), X is M x K row-major, Y is M x N
+ *     row-major.  N and K must be positive multiples of 128.
+ *   - Tiles are numbered row-major: t = tn*Tk + tk, Tn = N/128, Tk = K/128.
+ *   - Groups of 4 run along K: group g of row n covers k = 4g .. 4g+3.
+ *   - Pattern ids number the kept pair (i0, i1), i0 < i1, lexicographically:
+ *       0:(0,1) 1:(0,2) 2:(0,3) 3:(1,2) 4:(1,3) 5:(2,3).
+ *   - Every pointer argument except the patch_weight struct itself and the
+ *     size outputs of *_sizes / *_workspace_size is a DEVICE pointer.  The
+ *     caller allocates and owns every buffer; the library allocates no device
+ *     memory, keeps no state between calls and never synchronises the stream
+ *     (except patch_read_status).  All calls are asynchronous on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream).
+ *   - Host-detectable errors (shape, alignment, null pointer, workspace too
+ *     small, not an sm_100 device) return immediately without launching.
+ *   - Errors found on the device are OR-ed into the int32 word *dev_status
+ *     (PATCH_DEV_* bits); read it with patch_read_status.  dev_status must be
+ *     a valid device pointer; the library never clears it.
+ *
+ * Packed weight format (this library's specification; the paper fixes none)
+ *   - Descriptor table: one patch_tile_desc (16 bytes) per tile, row-major.
+ *   - Values blob: a sequence of panels; a panel is 128 rows x 64 bf16, row
+ *     major with 128-byte rows (16384 bytes).  A dense tile occupies 2 panels
+ *     (the tile's k 0..63, then k 64..127).  A sparse tile occupies 1 panel in
+ *     which row r holds, for each group g = 0..31, its two kept values in
+ *     ascending k at positions 2g and 2g+1.
+ *   - Metadata blob: 2048 bytes per sparse tile, at sparse_ordinal*2048.
+ *     Group g of tile row r has the 4-bit code i0 | (i1 << 2), stored in the
+ *     low nibble of its byte when g is even and the high nibble when g is
+ *     odd; the byte is
+ *         ((g>>1)&1) | ((r>>3)&1)<<1 | (g>>3)<<2 | (r&7)<<4
+ *         | ((g>>2)&1)<<7 | (r>>4)<<8.
+ *     This is the order in which the 16-bit sparse tensor-core MMA (M = 128)
+ *     reads its metadata from tensor memory after a 128x128b copy (16 bytes
+ *     per tensor-memory lane, 4 bytes per 32-K column), so the GEMM moves it
+ *     without reshuffling.
+ *   - All blobs must be 16-byte aligned.
+ */
+#ifndef PATCH_H
+#define PATCH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define PATCH_API __attribute__((visibility("default")))
+#else
+#define PATCH_API
+#endif
+
+#define PATCH_TILE 128
+#define PATCH_PANEL_BYTES 16384
+#define PATCH_DENSE_TILE_BYTES 32768
+#define PATCH_SPARSE_TILE_BYTES 16384
+#define PATCH_META_TILE_BYTES 2048
+#define PATCH_DECODE_MAX_M 16
+
+typedef enum {
+    PATCH_OK = 0,
+    PATCH_ERR_INVALID_ARG = 1, /* null pointer, M < 0, bad path selector */
+    PATCH_ERR_SHAPE = 2,       /* N or K not a positive multiple of 128 */
+    PATCH_ERR_ALIGN = 3,       /* a pointer not 16-byte aligned */
+    PATCH_ERR_DEVICE = 4,      /* current device is not compute capability 10.x */
+    PATCH_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed */
+    PATCH_ERR_BAD_PATTERN = 6, /* device: pattern id > 5 inside a sparse tile */
+    PATCH_ERR_TIMEOUT = 7,     /* device: a bounded wait in a kernel ran out */
+    PATCH_ERR_WORKSPACE = 8,   /* workspace pointer null or too small */
+    PATCH_ERR_COUNT = 9        /* device: bitmap's sparse-tile count != n_sparse */
+} patch_status_t;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define PATCH_DEV_BAD_PATTERN 0x1
+#define PATCH_DEV_TIMEOUT 0x2
+#define PATCH_DEV_COUNT 0x4
+
+/* Path selector of patch_gemm_ex. */
+#define PATCH_PATH_AUTO 0    /* M <= PATCH_DECODE_MAX_M: decode, else prefill */
+#define PATCH_PATH_DECODE 1  /* CUDA-core split-K GEMV, any M in 1..16 */
+#define PATCH_PATH_PREFILL 2 /* TMA + tcgen05 (dense and 2:4 sparse MMA), any M >= 1 */
+/* Test hook, OR-ed into PATCH_PATH_PREFILL: the prefill producer stops after
+ * its first K-tile, so the consumers' bounded waits run out and the kernel
+ * reports PATCH_DEV_TIMEOUT and exits cleanly (needs K >= 256 or several
+ * output tiles).  Used only to test the timeout path. */
+#define PATCH_PATH_TEST_STALL 0x100
+
+/* One descriptor per 128 x 128 tile (16 bytes). */
+typedef struct {
+    uint32_t kind;           /* 0 = dense, 1 = 2:4 sparse */
+    uint32_t sparse_ordinal; /* index of this tile among sparse tiles; 0xFFFFFFFF if dense */
+    uint64_t val_offset;     /* byte offset of the tile's first panel in the values blob */
+} patch_tile_desc;
+
+/* A packed weight: host struct of device pointers, all owned by the caller. */
+typedef struct {
+    int64_t N, K;                /* logical shape of W */
+    int64_t n_sparse;            /* number of sparse tiles */
+    const void *values;          /* values blob, patch_pack_sizes bytes */
+    const void *meta;            /* metadata blob (may be NULL when n_sparse == 0) */
+    const patch_tile_desc *desc; /* Tn*Tk descriptors */
+} patch_weight;
+
+/*
+ * patch_pack_sizes: byte sizes of the three blobs of a packed N x K weight
+ * with n_sparse sparse tiles (host only, no device work):
+ *   values = (T - n_sparse)*32768 + n_sparse*16384, meta = n_sparse*2048,
+ *   desc = 16*T.
+ * Errors: PATCH_ERR_SHAPE; PATCH_ERR_INVALID_ARG for n_sparse outside [0, T]
+ * or a NULL output pointer.
+ */
+PATCH_API patch_status_t patch_pack_sizes(int64_t N, int64_t K, int64_t n_sparse, size_t *values_bytes,
+                                size_t *meta_bytes, size_t *desc_bytes);
+
+/*
+ * patch_hard_mask: the inference-time hard form of the hybrid mask
+ * ("Learnable Distributions": tile selection and pattern selection).
+ *   bitmap[t]          = argmax(tile_logits[t][0..1])   (0 dense, 1 sparse)
+ *   pat_id[n][g]       = argmax(pattern_logits[n][g][0..5])
+ *   W_masked[n][k]     = W[n][k] if the tile is dense, or the tile is sparse
+ *                        and k%4 is kept by pat_id[n][k/4]; else +0.0 (0x0000)
+ * argmax takes the first maximum: a later entry wins only when strictly
+ * greater, so ties go to the lowest index and a NaN never displaces an
+ * earlier entry.  pat_id is written for every group, dense tiles included.
+ *   W              bf16 [N][K]
+ *   tile_logits    fp32 [Tn][Tk][2]
+ *   pattern_logits fp32 [N][K/4][6]
+ *   W_masked       bf16 [N][K], or NULL to skip
+ *   bitmap         u8 [Tn][Tk];  pat_id  u8 [N][K/4]
+ * Alignment: W, W_masked, pattern_logits 16 bytes.
+ */
+PATCH_API patch_status_t patch_hard_mask(const uint16_t *W, int64_t N, int64_t K, const float *tile_logits,
+                               const float *pattern_logits, uint16_t *W_masked, uint8_t *bitmap,
+                               uint8_t *pat_id, int32_t *dev_status, void *stream);
+
+/*
+ * patch_pack: build the packed format ("Core Mechanism": dense tiles kept
+ * whole, sparse tiles stored as their 2 kept values per group of 4 plus the
+ * 2-bit positions).  W may be masked or not: only kept positions of sparse
+ * tiles are read, so both give identical blobs.  Two launches: a scan of the
+ * bitmap that writes the descriptors, then one CTA per tile.
+ *   W        bf16 [N][K]; bitmap u8 [Tn][Tk] (nonzero = sparse);
+ *   pat_id   u8 [N][K/4] (read only inside sparse tiles);
+ *   n_sparse must equal the number of nonzero bitmap entries: the kernel
+ *   sets PATCH_DEV_COUNT and writes nothing past the blob sizes otherwise;
+ *   values/meta/desc sized by patch_pack_sizes (meta may be NULL if n_sparse == 0).
+ * An id > 5 in a sparse tile sets PATCH_DEV_BAD_PATTERN and is packed as id 0.
+ */
+PATCH_API patch_status_t patch_pack(const uint16_t *W, int64_t N, int64_t K, const uint8_t *bitmap,
+                          const uint8_t *pat_id, int64_t n_sparse, void *values, void *meta,
+                          patch_tile_desc *desc, int32_t *dev_status, void *stream);
+
+/*
+ * patch_gemm_workspace_size: device scratch bytes patch_gemm needs for M rows
+ * of X and this weight (0 when none is needed).  Host only.
+ */
+PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight *W, size_t *bytes);
+
+/*
+ * patch_gemm: Y = X * W_eff^T with fp32 accumulation and one round to
+ * bf16 (nearest-even) at the end ("Inference & Deployment": dense tiles on
+ * the dense tensor-core MMA, sparse tiles on the 2:4 sparse tensor-core MMA).
+ *   X  bf16 [M][K] (16-byte aligned, M >= 0; M == 0 is a no-op)
+ *   W  packed weight (host struct)
+ *   Y  bf16 [M][N] (16-byte aligned)
+ *   workspace: patch_gemm_workspace_size bytes (may be NULL when that is 0)
+ * M <= 16 runs the decode path (split-K GEMV on CUDA cores over the stored
+ * bytes, fp32 partials reduced in a fixed order), larger M the prefill path
+ * (TMA-fed tcgen05 kernel, dense and sparse MMAs into one TMEM fp32 tile).
+ * A bounded wait that runs out sets PATCH_DEV_TIMEOUT (Y is then undefined).
+ */
+PATCH_API patch_status_t patch_gemm(const uint16_t *X, int64_t M, const patch_weight *W, uint16_t *Y,
+                          void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                          void *stream);
+
+/*
+ * patch_gemm_ex: patch_gemm with an explicit path (PATCH_PATH_*) and the
+ * bounded-wait limit of the prefill kernel in microseconds (0 = default,
+ * 2 s).  PATCH_PATH_DECODE requires M <= 16.  PATCH_PATH_TEST_STALL is only
+ * accepted together with PATCH_PATH_PREFILL.
+ */
+PATCH_API patch_status_t patch_gemm_ex(const uint16_t *X, int64_t M, const patch_weight *W, uint16_t *Y,
+                             void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                             void *stream, int path, uint64_t wait_limit_us);
+
+/*
+ * patch_read_status: synchronise `stream`, copy *dev_status to *host_bits and
+ * return the first error it encodes (PATCH_ERR_TIMEOUT, then BAD_PATTERN,
+ * then COUNT) or PATCH_OK.  host_bits may be NULL.
+ */
+PATCH_API patch_status_t patch_read_status(const int32_t *dev_status, void *stream, int32_t *host_bits);
+
+/* Static message for a status code. */
+PATCH_API const char *patch_strerror(patch_status_t status);
+
+/* Library version string. */
+PATCH_API const char *patch_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PATCH_H */

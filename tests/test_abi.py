@@ -1,0 +1,79 @@
+"""The C-ABI library loads and exports every entry point include/patch.h declares
+(no GPU needed: only host-side calls that launch nothing)."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import tile_sparse_gemm_b200 as tsg
+from tile_sparse_gemm_b200 import build as tsg_build
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tsg_build.build()
+    return tsg.lib()
+
+
+def declared_symbols():
+    text = (ROOT / "include" / "patch.h").read_text()
+    return sorted(set(re.findall(r"PATCH_API\s+[\w\s\*]+?\b(patch_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 9, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in patch.h but not exported"
+
+
+def test_version_and_strerror(lib):
+    assert b"sm_100a" in lib.patch_version()
+    for code in range(10):
+        assert lib.patch_strerror(code)
+    assert lib.patch_strerror(99) == b"unknown status"
+
+
+def test_pack_sizes_host_only(lib):
+    assert tsg.patch_pack_sizes(512, 512, 8) == (8 * 32768 + 8 * 16384, 8 * 2048, 16 * 16)
+    with pytest.raises(tsg.PatchError) as e:
+        tsg.patch_pack_sizes(500, 512, 0)
+    assert e.value.code == 2  # PATCH_ERR_SHAPE
+    with pytest.raises(tsg.PatchError) as e:
+        tsg.patch_pack_sizes(128, 128, 2)
+    assert e.value.code == 1  # n_sparse > T
+
+
+def test_host_checks_reject_before_any_launch(lib):
+    P = ctypes.c_void_p
+    fake = P(0x10000)  # never dereferenced: every call below fails its host checks first
+    # bad shape
+    assert lib.patch_hard_mask(fake, 100, 128, fake, fake, None, fake, fake, fake, None) == 2
+    # null required pointer
+    assert lib.patch_hard_mask(fake, 128, 128, None, fake, None, fake, fake, fake, None) == 1
+    # misaligned pointer
+    assert lib.patch_pack(P(0x10001), 128, 128, fake, fake, 0, fake, None, fake, fake, None) == 3
+    # n_sparse out of range
+    assert lib.patch_pack(fake, 128, 128, fake, fake, 5, fake, fake, fake, fake, None) == 1
+    # gemm: bad path selector, decode path with M > 16, negative M
+    w = tsg._Weight(128, 128, 0, 0x10000, None, 0x10000)
+    assert lib.patch_gemm_ex(fake, 4, ctypes.byref(w), fake, None, 0, fake, None, 7, 0) == 1
+    assert lib.patch_gemm_ex(fake, 17, ctypes.byref(w), fake, None, 0, fake, None, 1, 0) == 1
+    assert lib.patch_gemm_ex(fake, -1, ctypes.byref(w), fake, None, 0, fake, None, 0, 0) == 1
+    # the stall test hook is refused outside the prefill path
+    assert lib.patch_gemm_ex(fake, 4, ctypes.byref(w), fake, None, 0, fake, None, 0x101, 0) == 1
+    # M == 0 is a no-op that needs no device
+    assert lib.patch_gemm_ex(None, 0, ctypes.byref(w), None, None, 0, fake, None, 0, 0) == 0
+    # weight with a bad shape
+    wbad = tsg._Weight(128, 130, 0, 0x10000, None, 0x10000)
+    assert lib.patch_gemm(fake, 4, ctypes.byref(wbad), fake, None, 0, fake, None) == 2
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(tsg, "_lib", None)
+    monkeypatch.setattr(tsg, "_LIB_PATH", tmp_path / "libpatch.so")
+    with pytest.raises(ImportError):
+        tsg.lib()

@@ -1,0 +1,267 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+hard mask and pack are compared byte for byte; the GEMM against the fp64
+oracle with the layer's tolerance (relative Frobenius error <= 5e-3 and
+|err| <= 1e-2 * (1 + |ref|) elementwise).  Sizes here run in seconds on the
+oracle and still span several tiles, ragged token counts and the degenerate
+all-dense / all-sparse bitmaps; the full-size workloads are in
+test_gpu_full_size.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+import tile_sparse_gemm_b200 as tsg
+from _util import bits_of, check_gemm, to_dev, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+TILE = 128
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    assert torch.cuda.get_device_capability()[0] == 10, "GPU tests need an sm_100 device"
+    tsg.lib()  # fails loudly when libpatch.so is missing
+
+
+def pack_on_gpu(w, bm, ids):
+    status = tsg.new_status()
+    pw = tsg.patch_pack(to_dev_bf16(w), to_dev(bm), to_dev(ids), int(bm.sum()), status=status)
+    code, bits = tsg.patch_read_status(status)
+    assert code == 0, (code, bits)
+    return pw
+
+
+def gemm_on_gpu(x, pw, path=tsg.PATH_AUTO):
+    status = tsg.new_status()
+    y = tsg.patch_gemm_ex(to_dev_bf16(x), pw, status=status, path=path)
+    code, bits = tsg.patch_read_status(status)
+    assert code == 0, (code, bits)
+    return bits_of(y)
+
+
+# ------------------------------------------------------------- hard mask
+
+
+@pytest.mark.parametrize("N,K,cfg", [(512, 512, 1), (128, 128, 0), (384, 640, 7), (1024, 256, 8)])
+def test_hard_mask_bit_exact(N, K, cfg):
+    w = si.gen_w(N, K, cfg, 0)
+    tl = si.gen_tile_logits(N, K, cfg, 0)
+    pl = si.gen_pattern_logits(N, K, cfg, 0)
+    wm_ref, bm_ref, id_ref = oracle.hard_mask(w, tl, pl)
+    status = tsg.new_status()
+    wm, bm, ids = tsg.patch_hard_mask(to_dev_bf16(w), to_dev(tl), to_dev(pl), status=status)
+    assert tsg.patch_read_status(status)[0] == 0
+    assert np.array_equal(bm.cpu().numpy(), bm_ref)
+    assert np.array_equal(ids.cpu().numpy(), id_ref)
+    assert np.array_equal(bits_of(wm), wm_ref)
+
+
+def test_hard_mask_ties_nan_and_negative_weights():
+    N = K = 256
+    w = np.full((N, K), np.uint16(0xBF80), np.uint16)  # -1.0 everywhere
+    tl = np.array([[[0.0, 0.0], [0.0, 1.0]], [[np.nan, 1.0], [1.0, np.nan]]], np.float32)
+    rng = np.random.default_rng(0)
+    pl = rng.integers(-2, 3, (N, K // 4, 6)).astype(np.float32)  # many ties
+    pl[::7, ::5, 3] = np.nan
+    pl[::11, ::3, 0] = np.nan
+    wm_ref, bm_ref, id_ref = oracle.hard_mask(w, tl, pl)
+    wm, bm, ids = tsg.patch_hard_mask(to_dev_bf16(w), to_dev(tl), to_dev(pl))
+    assert np.array_equal(bm.cpu().numpy(), bm_ref)
+    assert np.array_equal(ids.cpu().numpy(), id_ref)
+    assert np.array_equal(bits_of(wm), wm_ref)
+    assert bm_ref.tolist() == [[0, 1], [0, 0]]
+
+
+def test_hard_mask_without_masked_output():
+    N, K = 256, 384
+    tl = si.gen_tile_logits(N, K, 2, 0)
+    pl = si.gen_pattern_logits(N, K, 2, 0)
+    _, bm_ref, id_ref = oracle.hard_mask(si.gen_w(N, K, 2, 0), tl, pl)
+    wm, bm, ids = tsg.patch_hard_mask(None, to_dev(tl), to_dev(pl), want_masked=False)
+    assert wm is None
+    assert np.array_equal(bm.cpu().numpy(), bm_ref) and np.array_equal(ids.cpu().numpy(), id_ref)
+
+
+# ------------------------------------------------------------------ pack
+
+
+@pytest.mark.parametrize("N,K,kind,frac", [
+    (512, 512, "bernoulli", 0.5), (128, 128, "exact", 1.0), (128, 128, "exact", 0.0),
+    (384, 640, "exact", 0.5), (640, 384, "clustered", 0.5), (256, 1024, "exact", 0.25)])
+def test_pack_bit_exact(N, K, kind, frac):
+    w = si.gen_w(N, K, 1, 3)
+    bm = {"bernoulli": si.tiles_bernoulli, "exact": si.tiles_exact, "clustered": si.tiles_clustered}[kind](
+        N, K, frac, 1, 3)
+    ids = si.patterns_top2(w)
+    v_ref, m_ref, d_ref = oracle.pack(w, bm, ids)
+    pw = pack_on_gpu(w, bm, ids)
+    assert np.array_equal(pw.desc.cpu().numpy(), d_ref)
+    assert np.array_equal(pw.values.cpu().numpy(), v_ref)
+    assert np.array_equal(pw.meta.cpu().numpy(), m_ref)
+
+
+def test_pack_of_masked_and_random_patterns():
+    N, K = 384, 384
+    w = si.gen_w(N, K, 5, 0)
+    bm = si.tiles_exact(N, K, 0.5, 5, 0)
+    ids = np.random.default_rng(9).integers(0, 6, (N, K // 4)).astype(np.uint8)
+    v_ref, m_ref, d_ref = oracle.pack(w, bm, ids)
+    pw = pack_on_gpu(oracle.apply_mask(w, bm, ids), bm, ids)
+    assert np.array_equal(pw.values.cpu().numpy(), v_ref)
+    assert np.array_equal(pw.meta.cpu().numpy(), m_ref)
+    assert np.array_equal(pw.desc.cpu().numpy(), d_ref)
+
+
+def test_pack_flags_bad_pattern_id():
+    N = K = 256
+    w = si.gen_w(N, K, 6, 0)
+    bm = np.array([[1, 0], [0, 1]], np.uint8)
+    ids = si.patterns_top2(w)
+    ids[3, 5] = 9   # inside sparse tile (0, 0)
+    ids[3, 40] = 7  # inside dense tile (0, 1): never read
+    status = tsg.new_status()
+    tsg.patch_pack(to_dev_bf16(w), to_dev(bm), to_dev(ids), 2, status=status)
+    code, bits = tsg.patch_read_status(status)
+    assert code == 6 and bits == tsg.DEV_BAD_PATTERN
+
+
+def test_pack_flags_count_mismatch_without_overrun():
+    N = K = 256
+    w = si.gen_w(N, K, 6, 1)
+    bm = np.array([[1, 1], [0, 1]], np.uint8)  # 3 sparse tiles
+    ids = si.patterns_top2(w)
+    vb, mb, db = tsg.patch_pack_sizes(N, K, 1)
+    guard = 4096
+    values = torch.full((vb + guard,), 0xAB, dtype=torch.uint8, device="cuda")
+    meta = torch.full((mb + guard,), 0xCD, dtype=torch.uint8, device="cuda")
+    desc = torch.zeros(db, dtype=torch.uint8, device="cuda")
+    status = tsg.new_status()
+    import ctypes
+    rc = tsg.lib().patch_pack(ctypes.c_void_p(to_dev_bf16(w).data_ptr()), N, K,
+                              ctypes.c_void_p(to_dev(bm).data_ptr()), ctypes.c_void_p(to_dev(ids).data_ptr()),
+                              1, ctypes.c_void_p(values.data_ptr()), ctypes.c_void_p(meta.data_ptr()),
+                              ctypes.c_void_p(desc.data_ptr()), ctypes.c_void_p(status.data_ptr()),
+                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    code, bits = tsg.patch_read_status(status)
+    assert code == 9 and bits & tsg.DEV_COUNT
+    assert torch.all(values[vb:] == 0xAB) and torch.all(meta[mb:] == 0xCD)
+
+
+def test_gpu_pack_then_hard_mask_chain():
+    """hard mask -> pack on the GPU equals the oracle's chain."""
+    N, K = 512, 512
+    w = si.gen_w(N, K, 1, 0)
+    tl, pl = si.gen_tile_logits(N, K, 1, 0), si.gen_pattern_logits(N, K, 1, 0)
+    wm_ref, bm_ref, id_ref = oracle.hard_mask(w, tl, pl)
+    v_ref, m_ref, d_ref = oracle.pack(w, bm_ref, id_ref)
+    wm, bm, ids = tsg.patch_hard_mask(to_dev_bf16(w), to_dev(tl), to_dev(pl))
+    pw = tsg.patch_pack(wm, bm, ids)
+    assert np.array_equal(pw.values.cpu().numpy(), v_ref)
+    assert np.array_equal(pw.meta.cpu().numpy(), m_ref)
+    assert np.array_equal(pw.desc.cpu().numpy(), d_ref)
+
+
+# ------------------------------------------------------------------ GEMM
+
+
+def _layer(N, K, M, kind, frac, cfg=3, shape_idx=0):
+    x = si.gen_x(M, K, cfg, shape_idx)
+    w = si.gen_w(N, K, cfg, shape_idx)
+    if kind == "bernoulli":
+        bm = si.tiles_bernoulli(N, K, frac, cfg, shape_idx)
+    elif kind == "clustered":
+        bm = si.tiles_clustered(N, K, frac, cfg, shape_idx)
+    else:
+        bm = si.tiles_exact(N, K, frac, cfg, shape_idx)
+    return x, w, bm, si.patterns_top2(w)
+
+
+def test_gemm_config1_decode():
+    """512 x 512 weight, Bernoulli(0.5) tiles, M = 16 tokens."""
+    x, w, bm, ids = _layer(512, 512, 16, "bernoulli", 0.5, cfg=1)
+    ref = oracle.hybrid_gemm(x, w, bm, ids)
+    y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids))
+    check_gemm(y, ref, "config 1")
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 7, 8, 13, 16])
+@pytest.mark.parametrize("N,K,frac", [(384, 640, 0.5), (256, 1280, 0.0), (640, 256, 1.0)])
+def test_gemm_decode_parity(M, N, K, frac):
+    x, w, bm, ids = _layer(N, K, M, "exact", frac, shape_idx=M)
+    ref = oracle.hybrid_gemm(x, w, bm, ids)
+    y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids), tsg.PATH_DECODE)
+    check_gemm(y, ref, f"decode M={M} {N}x{K} f={frac}")
+
+
+@pytest.mark.parametrize("frac", [0.0, 1.0, 0.5])
+@pytest.mark.parametrize("M", [17, 129, 256, 300])
+def test_gemm_prefill_parity(M, frac):
+    N, K = 384, 640
+    x, w, bm, ids = _layer(N, K, M, "exact", frac, shape_idx=int(10 * frac))
+    ref = oracle.hybrid_gemm(x, w, bm, ids)
+    y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids), tsg.PATH_PREFILL)
+    check_gemm(y, ref, f"prefill M={M} f={frac}")
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_prefill_path_small_m_matches_decode(M):
+    x, w, bm, ids = _layer(256, 512, M, "bernoulli", 0.5, cfg=4)
+    pw = pack_on_gpu(w, bm, ids)
+    ref = oracle.hybrid_gemm(x, w, bm, ids)
+    yp = gemm_on_gpu(x, pw, tsg.PATH_PREFILL)
+    yd = gemm_on_gpu(x, pw, tsg.PATH_DECODE)
+    check_gemm(yp, ref, "prefill small M")
+    check_gemm(yd, ref, "decode")
+
+
+def test_prefill_many_output_tiles():
+    """More output tiles than SMs: the persistent schedule wraps around."""
+    N, K, M = 128 * 40, 256, 1100
+    x, w, bm, ids = _layer(N, K, M, "exact", 0.5, cfg=5)
+    rows = np.array([0, 1, 255, 256, 511, 700, 1023, 1099])
+    ref = oracle.hybrid_gemm(x, w, bm, ids, rows=rows)
+    y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids), tsg.PATH_PREFILL)
+    check_gemm(y[rows], ref, "prefill wrap")
+
+
+def test_gemm_all_sparse_equals_24_and_all_dense_equals_dense():
+    N, K, M = 256, 256, 64
+    x = si.gen_x(M, K, 9, 0)
+    w = si.gen_w(N, K, 9, 0)
+    ids = si.patterns_top2(w)
+    for frac in (0.0, 1.0):
+        bm = np.full((N // TILE, K // TILE), int(frac), np.uint8)
+        pw = pack_on_gpu(w, bm, ids)
+        xd = to_dev_bf16(x).float()
+        w_eff = torch.from_numpy(oracle.apply_mask(w, bm, ids).view(np.int16)).view(torch.bfloat16).cuda().float()
+        torch_ref = (xd @ w_eff.T).double().cpu().numpy()   # plain fp32 reference of the same op
+        for path in (tsg.PATH_PREFILL, tsg.PATH_DECODE):
+            if path == tsg.PATH_DECODE:
+                y = gemm_on_gpu(x[:16], pw, path)
+                check_gemm(y, torch_ref[:16], f"decode f={frac}")
+            else:
+                y = gemm_on_gpu(x, pw, path)
+                check_gemm(y, torch_ref, f"prefill f={frac}")
+
+
+def test_gemm_zero_tokens_is_noop():
+    x, w, bm, ids = _layer(256, 256, 4, "exact", 0.5)
+    pw = pack_on_gpu(w, bm, ids)
+    y = torch.full((0, 256), 1.0, dtype=torch.bfloat16, device="cuda")
+    out = tsg.patch_gemm(torch.empty((0, 256), dtype=torch.bfloat16, device="cuda"), pw, Y=y)
+    assert out.shape == (0, 256)
+
+
+def test_decode_workspace_too_small_is_rejected():
+    x, w, bm, ids = _layer(4096, 4096, 4, "exact", 0.5)
+    pw = pack_on_gpu(w, bm, ids)
+    need = tsg.patch_gemm_workspace_size(4, pw)
+    assert need > 0
+    with pytest.raises(tsg.PatchError) as e:
+        tsg.patch_gemm(to_dev_bf16(x), pw, workspace=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
+    assert e.value.code == 8

@@ -1,0 +1,220 @@
+"""B200-native PATCH hybrid tile-sparse linear layer (Y = X * W_eff^T).
+
+Thin Python binding over the C ABI of ``libpatch.so`` (declared in
+include/patch.h).  It only marshals arguments: torch supplies device memory
+and the current CUDA stream, every step of the hot path runs in the
+library's sm_100a kernels.  There is no CPU fallback: importing the binding
+works anywhere, but every call fails loudly unless the in-tree library has
+been built (``python -m tile_sparse_gemm_b200.build``) and a B200 is present.
+
+Entry points (same names as the C ABI):
+    patch_pack_sizes(N, K, n_sparse)          -> (values_bytes, meta_bytes, desc_bytes)
+    patch_hard_mask(W, tile_logits, pattern_logits) -> (W_masked, bitmap, pat_id)
+    patch_pack(W, bitmap, pat_id, n_sparse)   -> PackedWeight
+    patch_gemm_workspace_size(M, weight)      -> bytes
+    patch_gemm(X, weight)                     -> Y
+    patch_gemm_ex(X, weight, path=..., wait_limit_us=...) -> Y
+    patch_read_status(status)                 -> (status code, device bits)
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from pathlib import Path
+
+import torch
+
+_LIB_PATH = Path(__file__).resolve().parent / "libpatch.so"
+
+TILE = 128
+PANEL_BYTES = 16384
+DECODE_MAX_M = 16
+
+PATCH_OK = 0
+STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_INVALID_ARG", 2: "PATCH_ERR_SHAPE", 3: "PATCH_ERR_ALIGN",
+                4: "PATCH_ERR_DEVICE", 5: "PATCH_ERR_CUDA", 6: "PATCH_ERR_BAD_PATTERN",
+                7: "PATCH_ERR_TIMEOUT", 8: "PATCH_ERR_WORKSPACE", 9: "PATCH_ERR_COUNT"}
+DEV_BAD_PATTERN, DEV_TIMEOUT, DEV_COUNT = 0x1, 0x2, 0x4
+PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_TEST_STALL = 0, 1, 2, 0x100
+
+
+class PatchError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)} ({_strerror(code)})")
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64), ("n_sparse", ctypes.c_int64),
+                ("values", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("desc", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libpatch.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not _LIB_PATH.exists():
+            raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m tile_sparse_gemm_b200.build`")
+        L = ctypes.CDLL(str(_LIB_PATH))
+        P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        WP = ctypes.POINTER(_Weight)
+        sigs = {
+            "patch_pack_sizes": [I64, I64, I64, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)],
+            "patch_hard_mask": [P, I64, I64, P, P, P, P, P, P, P],
+            "patch_pack": [P, I64, I64, P, P, I64, P, P, P, P, P],
+            "patch_gemm_workspace_size": [I64, WP, ctypes.POINTER(SZ)],
+            "patch_gemm": [P, I64, WP, P, P, SZ, P, P],
+            "patch_gemm_ex": [P, I64, WP, P, P, SZ, P, P, I32, ctypes.c_uint64],
+            "patch_read_status": [P, P, ctypes.POINTER(ctypes.c_int32)],
+        }
+        for name, args in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = I32
+        L.patch_strerror.argtypes = [I32]
+        L.patch_strerror.restype = ctypes.c_char_p
+        L.patch_version.argtypes = []
+        L.patch_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _strerror(code: int) -> str:
+    try:
+        return lib().patch_strerror(code).decode()
+    except Exception:  # the library itself may be what is missing
+        return "?"
+
+
+def _check(code: int, what: str):
+    if code != PATCH_OK:
+        raise PatchError(code, what)
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor | None, name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def new_status(device=None) -> torch.Tensor:
+    """A zeroed device status word for the kernels to OR error bits into."""
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+@dataclass
+class PackedWeight:
+    """A packed hybrid weight: three device blobs plus its shape."""
+    N: int
+    K: int
+    n_sparse: int
+    values: torch.Tensor  # uint8, patch_pack_sizes bytes
+    meta: torch.Tensor    # uint8 (may be empty)
+    desc: torch.Tensor    # uint8, 16 bytes per tile
+
+    def struct(self) -> _Weight:
+        return _Weight(self.N, self.K, self.n_sparse, self.values.data_ptr(),
+                       self.meta.data_ptr() if self.meta.numel() else None, self.desc.data_ptr())
+
+    @property
+    def stored_bytes(self) -> int:
+        return self.values.numel() + self.meta.numel() + self.desc.numel()
+
+
+def patch_pack_sizes(N: int, K: int, n_sparse: int) -> tuple[int, int, int]:
+    v, m, d = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().patch_pack_sizes(N, K, n_sparse, ctypes.byref(v), ctypes.byref(m), ctypes.byref(d)),
+           "patch_pack_sizes")
+    return v.value, m.value, d.value
+
+
+def patch_hard_mask(W: torch.Tensor | None, tile_logits: torch.Tensor, pattern_logits: torch.Tensor,
+                    status: torch.Tensor | None = None, want_masked: bool = True, stream=None):
+    """Argmax hard mask.  Returns (W_masked or None, bitmap u8 [Tn][Tk], pat_id u8 [N][K/4])."""
+    N, K4, _ = pattern_logits.shape
+    K = 4 * K4
+    dev = pattern_logits.device
+    status = new_status(dev) if status is None else status
+    wm = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if want_masked else None
+    bitmap = torch.empty((N // TILE, K // TILE), dtype=torch.uint8, device=dev)
+    pid = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+    _check(lib().patch_hard_mask(_dev(W, "W"), N, K, _dev(tile_logits, "tile_logits"),
+                                 _dev(pattern_logits, "pattern_logits"), _dev(wm, "W_masked"),
+                                 _dev(bitmap, "bitmap"), _dev(pid, "pat_id"), _dev(status, "status"),
+                                 _stream(stream)), "patch_hard_mask")
+    return wm, bitmap, pid
+
+
+def patch_pack(W: torch.Tensor, bitmap: torch.Tensor, pat_id: torch.Tensor, n_sparse: int | None = None,
+               status: torch.Tensor | None = None, stream=None) -> PackedWeight:
+    """Pack W (bf16 [N][K]) under a tile bitmap and pattern ids into the mixed layout."""
+    N, K = W.shape
+    if n_sparse is None:
+        n_sparse = int(torch.count_nonzero(bitmap).item())
+    vb, mb, db = patch_pack_sizes(N, K, n_sparse)
+    dev = W.device
+    status = new_status(dev) if status is None else status
+    values = torch.empty(vb, dtype=torch.uint8, device=dev)
+    meta = torch.empty(mb, dtype=torch.uint8, device=dev)
+    desc = torch.empty(db, dtype=torch.uint8, device=dev)
+    _check(lib().patch_pack(_dev(W, "W"), N, K, _dev(bitmap, "bitmap"), _dev(pat_id, "pat_id"), n_sparse,
+                            _dev(values, "values"), _dev(meta, "meta") if mb else None, _dev(desc, "desc"),
+                            _dev(status, "status"), _stream(stream)), "patch_pack")
+    return PackedWeight(N, K, n_sparse, values, meta, desc)
+
+
+def patch_gemm_workspace_size(M: int, weight: PackedWeight) -> int:
+    b = ctypes.c_size_t()
+    st = weight.struct()
+    _check(lib().patch_gemm_workspace_size(M, ctypes.byref(st), ctypes.byref(b)), "patch_gemm_workspace_size")
+    return b.value
+
+
+def patch_gemm_ex(X: torch.Tensor, weight: PackedWeight, Y: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                  path: int = PATH_AUTO, wait_limit_us: int = 0, stream=None) -> torch.Tensor:
+    M, K = X.shape
+    if K != weight.K:
+        raise ValueError(f"X has K={K}, weight has K={weight.K}")
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, weight.N), dtype=torch.bfloat16, device=dev)
+    status = new_status(dev) if status is None else status
+    st = weight.struct()
+    if workspace is None:
+        need = patch_gemm_workspace_size(M, weight) if (path & 0xFF) != PATH_PREFILL else 0
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().patch_gemm_ex(_dev(X, "X"), M, ctypes.byref(st), _dev(Y, "Y"), _dev(workspace, "workspace"),
+                               workspace.numel(), _dev(status, "status"), _stream(stream), path, wait_limit_us),
+           "patch_gemm")
+    return Y
+
+
+def patch_gemm(X: torch.Tensor, weight: PackedWeight, Y: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Y = X * W_eff^T (bf16 out, fp32 accumulate); M <= 16 decode path, else prefill."""
+    return patch_gemm_ex(X, weight, Y, workspace, status, PATH_AUTO, 0, stream)
+
+
+def patch_read_status(status: torch.Tensor, stream=None) -> tuple[int, int]:
+    """Synchronise the stream and decode the status word: (status code, raw bits)."""
+    bits = ctypes.c_int32()
+    code = lib().patch_read_status(_dev(status, "status"), _stream(stream), ctypes.byref(bits))
+    return code, bits.value
+
+
+def version() -> str:
+    return lib().patch_version().decode()

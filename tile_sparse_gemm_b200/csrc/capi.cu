@@ -1,0 +1,174 @@
+// C ABI of libpatch: argument checks, path dispatch, status handling.
+// Every entry point is declared and documented in include/patch.h.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace patch {
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool shape_ok(int64_t N, int64_t K) {
+  return N > 0 && K > 0 && N % kTile == 0 && K % kTile == 0 && N <= (int64_t(1) << 31) &&
+         K <= (int64_t(1) << 31);
+}
+
+// SM count of the current device; PATCH_ERR_DEVICE unless it is compute capability 10.x
+static patch_status_t device_sms(int* sms) {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PATCH_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return PATCH_ERR_CUDA;
+  if (major != 10) return PATCH_ERR_DEVICE;
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
+static patch_status_t check_weight(const patch_weight* W) {
+  if (!W || !W->values || !W->desc) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(W->N, W->K)) return PATCH_ERR_SHAPE;
+  const int64_t T = (W->N / kTile) * (W->K / kTile);
+  if (W->n_sparse < 0 || W->n_sparse > T) return PATCH_ERR_INVALID_ARG;
+  if (W->n_sparse > 0 && !W->meta) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(W->values) || !aligned16(W->desc) || (W->meta && !aligned16(W->meta)))
+    return PATCH_ERR_ALIGN;
+  return PATCH_OK;
+}
+
+}  // namespace patch
+
+using namespace patch;
+
+extern "C" {
+
+const char* patch_version(void) { return "patch-b200 0.1 (sm_100a)"; }
+
+const char* patch_strerror(patch_status_t s) {
+  switch (s) {
+    case PATCH_OK: return "ok";
+    case PATCH_ERR_INVALID_ARG: return "invalid argument";
+    case PATCH_ERR_SHAPE: return "N and K must be positive multiples of 128";
+    case PATCH_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case PATCH_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+    case PATCH_ERR_CUDA: return "CUDA call failed";
+    case PATCH_ERR_BAD_PATTERN: return "pattern id > 5 inside a sparse tile";
+    case PATCH_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case PATCH_ERR_WORKSPACE: return "workspace missing or too small";
+    case PATCH_ERR_COUNT: return "bitmap's sparse-tile count differs from n_sparse";
+  }
+  return "unknown status";
+}
+
+patch_status_t patch_pack_sizes(int64_t N, int64_t K, int64_t n_sparse, size_t* values_bytes,
+                                size_t* meta_bytes, size_t* desc_bytes) {
+  if (!values_bytes || !meta_bytes || !desc_bytes) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return PATCH_ERR_SHAPE;
+  const int64_t T = (N / kTile) * (K / kTile);
+  if (n_sparse < 0 || n_sparse > T) return PATCH_ERR_INVALID_ARG;
+  *values_bytes = size_t(T - n_sparse) * PATCH_DENSE_TILE_BYTES + size_t(n_sparse) * PATCH_SPARSE_TILE_BYTES;
+  *meta_bytes = size_t(n_sparse) * PATCH_META_TILE_BYTES;
+  *desc_bytes = size_t(T) * sizeof(patch_tile_desc);
+  return PATCH_OK;
+}
+
+patch_status_t patch_hard_mask(const uint16_t* W, int64_t N, int64_t K, const float* tile_logits,
+                               const float* pattern_logits, uint16_t* W_masked, uint8_t* bitmap,
+                               uint8_t* pat_id, int32_t* dev_status, void* stream) {
+  if (!tile_logits || !pattern_logits || !bitmap || !pat_id || !dev_status) return PATCH_ERR_INVALID_ARG;
+  if (W_masked && !W) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return PATCH_ERR_SHAPE;
+  if ((W && !aligned16(W)) || (W_masked && !aligned16(W_masked)) || !aligned16(pattern_logits) ||
+      !aligned16(pat_id))
+    return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_hard_mask(W, N, K, tile_logits, pattern_logits, W_masked, bitmap, pat_id, sms,
+                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
+patch_status_t patch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap,
+                          const uint8_t* pat_id, int64_t n_sparse, void* values, void* meta,
+                          patch_tile_desc* desc, int32_t* dev_status, void* stream) {
+  if (!W || !bitmap || !pat_id || !values || !desc || !dev_status) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return PATCH_ERR_SHAPE;
+  const int64_t T = (N / kTile) * (K / kTile);
+  if (n_sparse < 0 || n_sparse > T) return PATCH_ERR_INVALID_ARG;
+  if (n_sparse > 0 && !meta) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(desc) || (meta && !aligned16(meta)))
+    return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_pack(W, N, K, bitmap, pat_id, n_sparse, values, meta, desc, dev_status, sms,
+                  static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
+patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight* W, size_t* bytes) {
+  if (!bytes || !W || M < 0) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(W->N, W->K)) return PATCH_ERR_SHAPE;
+  *bytes = 0;
+  if (M == 0 || M > PATCH_DECODE_MAX_M) return PATCH_OK;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  *bytes = decode_plan(M, W->N, W->K, sms).ws_bytes;
+  return PATCH_OK;
+}
+
+patch_status_t patch_gemm_ex(const uint16_t* X, int64_t M, const patch_weight* W, uint16_t* Y,
+                             void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                             void* stream, int path, uint64_t wait_limit_us) {
+  if (M < 0 || !dev_status) return PATCH_ERR_INVALID_ARG;
+  const int inject = (path & PATCH_PATH_TEST_STALL) ? 1 : 0;
+  path &= ~PATCH_PATH_TEST_STALL;
+  if (inject && path != PATCH_PATH_PREFILL) return PATCH_ERR_INVALID_ARG;
+  patch_status_t st = check_weight(W);
+  if (st != PATCH_OK) return st;
+  if (path == PATCH_PATH_AUTO) path = M <= PATCH_DECODE_MAX_M ? PATCH_PATH_DECODE : PATCH_PATH_PREFILL;
+  if (path != PATCH_PATH_DECODE && path != PATCH_PATH_PREFILL) return PATCH_ERR_INVALID_ARG;
+  if (path == PATCH_PATH_DECODE && M > PATCH_DECODE_MAX_M) return PATCH_ERR_INVALID_ARG;
+  if (M == 0) return PATCH_OK;
+  if (!X || !Y) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y)) return PATCH_ERR_ALIGN;
+  if (M > (int64_t(1) << 30)) return PATCH_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (path == PATCH_PATH_DECODE) {
+    const DecodePlan p = decode_plan(M, W->N, W->K, sms);
+    if (p.ws_bytes > 0 && (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace)))
+      return PATCH_ERR_WORKSPACE;
+    e = launch_decode(X, M, *W, Y, workspace, sms, s);
+  } else {
+    const uint64_t limit_ns = (wait_limit_us ? wait_limit_us : 2000000ull) * 1000ull;
+    e = launch_prefill(X, M, *W, Y, dev_status, sms, limit_ns, inject, s);
+  }
+  return e == cudaSuccess ? PATCH_OK : PATCH_ERR_CUDA;
+}
+
+patch_status_t patch_gemm(const uint16_t* X, int64_t M, const patch_weight* W, uint16_t* Y,
+                          void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  return patch_gemm_ex(X, M, W, Y, workspace, workspace_bytes, dev_status, stream, PATCH_PATH_AUTO, 0);
+}
+
+patch_status_t patch_read_status(const int32_t* dev_status, void* stream, int32_t* host_bits) {
+  if (!dev_status) return PATCH_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PATCH_ERR_CUDA;
+  int32_t bits = 0;
+  if (cudaMemcpy(&bits, dev_status, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess) return PATCH_ERR_CUDA;
+  if (host_bits) *host_bits = bits;
+  if (bits & PATCH_DEV_TIMEOUT) return PATCH_ERR_TIMEOUT;
+  if (bits & PATCH_DEV_BAD_PATTERN) return PATCH_ERR_BAD_PATTERN;
+  if (bits & PATCH_DEV_COUNT) return PATCH_ERR_COUNT;
+  return PATCH_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,481 @@
+// Prefill path of patch_gemm (M > 16): a persistent, warp-specialised
+// TMA + tcgen05 kernel for sm_100a in which dense tiles run on the dense
+// tensor-core MMA and 2:4 sparse tiles on the structured-sparse MMA, both
+// accumulating into one fp32 tile in tensor memory.
+//
+// "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs", section 2
+// "Methodology: PATCH", "Inference & Deployment": hybrid execution over
+// 128 x 128 tiles; dense tiles use dense tensor-core kernels, sparse tiles the
+// 2:4 sparse tensor cores.
+//
+// The sparse operand of the tensor-core MMA is A (the M side), so the kernel
+// computes Y^T = W_eff * X^T: the MMA's M = 128 rows of W (one tile row), its
+// N = BT tokens, K streams over the tiles of the row.
+//
+// CTA = 6 warps, one CTA per SM, static round-robin over output tiles
+// (tile row tn, token block tb):
+//   warp 0  producer: per K-tile reads the descriptor; TMA-loads a dense tile's
+//           2 panels (or a sparse tile's 1 value panel + its 2 KB of metadata
+//           by bulk copy) into the A ring and the 2 matching 64-k panels of X
+//           into the B ring.
+//   warp 1  MMA issuer (one thread) and TMEM owner: dense panel -> 4 x
+//           tcgen05.mma kind::f16 (K = 16); sparse tile -> tcgen05.cp of the
+//           metadata into TMEM, then 4 x tcgen05.mma.sp kind::f16 (K = 32
+//           logical); tcgen05.commit releases ring slots and, per output tile,
+//           signals the epilogue.
+//   warps 2-5 epilogue: tcgen05.ld of the 128 x BT fp32 accumulator, one
+//           round to bf16 (nearest even), stores to Y[m][n].
+// Every mbarrier wait is bounded in time; when one runs out the kernel sets
+// PATCH_DEV_TIMEOUT, the other roles stop at their next wait, the producer
+// waits for its copies in flight, the MMA thread for its MMAs, and TMEM is
+// freed before the CTA exits.  No cluster multicast is used anywhere.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace patch {
+namespace prefill {
+
+constexpr int BM = 128;                  // W rows per output tile (MMA M)
+constexpr int BT = 256;                  // tokens per output tile (MMA N)
+constexpr int NA = 4;                    // A ring: W panels of 128 x 64 bf16
+constexpr int NB = 4;                    // B ring: X panels of BT x 64 bf16
+constexpr int NE = 4;                    // metadata ring
+constexpr int A_BYTES = PATCH_PANEL_BYTES;
+constexpr int B_BYTES = BT * 64 * 2;
+constexpr int E_BYTES = PATCH_META_TILE_BYTES;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;      // accumulator [0, BT) + metadata slots
+constexpr uint32_t META_COL0 = BT;
+
+// instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
+// (bits 7-9 = 1, bits 10-12 = 1), both K-major, N >> 3 at bits 17-22,
+// M >> 4 at bits 24-28; bit 2 marks the sparse form, bits 0-1 select the
+// metadata column pair half.
+constexpr uint32_t IDESC_DENSE =
+    (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BT >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+constexpr uint32_t IDESC_SPARSE = IDESC_DENSE | (1u << 2);
+
+struct Shared {
+  alignas(1024) uint8_t a[NA][A_BYTES];
+  alignas(1024) uint8_t b[NB][B_BYTES];
+  alignas(128) uint8_t e[NE][E_BYTES];
+  uint64_t a_full[NA], a_empty[NA], b_full[NB], b_empty[NB], e_full[NE], e_empty[NE];
+  uint64_t acc_full, acc_empty, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr size_t SMEM_BYTES = sizeof(Shared) + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+// ---------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar`.  Returns false when the wait outlived
+// limit_ns (the CTA is then marked aborted and PATCH_DEV_TIMEOUT raised) or,
+// unless `drain` is set, when another role of the CTA aborted first.
+__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Shared& s,
+                                          uint64_t limit_ns, int32_t* status, bool drain) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  volatile int* abort_flag = &s.abort_flag;
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((spin & 31u) == 0) {
+      if (!drain && *abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        set_status(status, PATCH_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mma_dense(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_sparse(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
+        "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
+        "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: start address,
+// leading offset unused (1), 8-row groups 1024 B apart, sm_100 version bit 46,
+// layout type 2 (SWIZZLE_128B) in bits 61-63.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+// Descriptor of a 128-row x 16-byte metadata block for tcgen05.cp 128x128b:
+// no swizzle, rows 16 B apart, 8-row core matrices 128 B apart.
+__device__ __forceinline__ uint64_t meta_desc(uint32_t saddr) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(128 >> 4) << 16) | (uint64_t(128 >> 4) << 32) |
+         (uint64_t(1) << 46);
+}
+
+// ---------------------------------------------------------------- roles
+
+struct Args {
+  const uint8_t* meta;
+  const patch_tile_desc* desc;
+  uint16_t* Y;
+  int M, N, Tk, n_items;
+  uint64_t limit_ns;
+  int32_t* status;
+  int inject;  // 1: producer stops after the first K-tile (exercises the timeout path)
+};
+
+__device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap* tmap_w, const Args& p) {
+  const int Tn = p.N / BM;
+  uint32_t a_i = 0, b_i = 0, e_i = 0;  // loads issued per ring
+  bool ok = true;
+  for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+    const int tn = item % Tn, tb = item / Tn;
+    for (int kt = 0; ok && kt < p.Tk; ++kt) {
+      if (p.inject && (item != int(blockIdx.x) || kt > 0)) {
+        ok = false;
+        break;
+      }
+      const patch_tile_desc d = p.desc[int64_t(tn) * p.Tk + kt];
+      const int panel = int(d.val_offset / A_BYTES);
+      if (d.kind) {
+        const uint32_t es = e_i % NE;
+        if (!(ok = wait_bounded(&s.e_empty[es], ((e_i / NE) & 1) ^ 1, s, p.limit_ns, p.status, false))) break;
+        mbar_expect_tx(&s.e_full[es], E_BYTES);
+        bulk_load(s.e[es], p.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.e_full[es]);
+        ++e_i;
+      }
+      const int n_a = d.kind ? 1 : 2;
+      for (int h = 0; h < 2; ++h) {
+        if (h < n_a) {
+          const uint32_t as = a_i % NA;
+          if (!(ok = wait_bounded(&s.a_empty[as], ((a_i / NA) & 1) ^ 1, s, p.limit_ns, p.status, false)))
+            break;
+          mbar_expect_tx(&s.a_full[as], A_BYTES);
+          tma_load_2d(s.a[as], tmap_w, &s.a_full[as], 0, (panel + h) * 128);
+          ++a_i;
+        }
+        const uint32_t bs = b_i % NB;
+        if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, s, p.limit_ns, p.status, false)))
+          break;
+        mbar_expect_tx(&s.b_full[bs], B_BYTES);
+        tma_load_2d(s.b[bs], tmap_x, &s.b_full[bs], kt * kTile + 64 * h, tb * BT);
+        ++b_i;
+      }
+    }
+  }
+  // every copy issued must have landed before the CTA may exit
+  for (uint32_t i = (a_i > NA ? a_i - NA : 0); i < a_i; ++i)
+    wait_bounded(&s.a_full[i % NA], (i / NA) & 1, s, p.limit_ns, p.status, true);
+  for (uint32_t i = (b_i > NB ? b_i - NB : 0); i < b_i; ++i)
+    wait_bounded(&s.b_full[i % NB], (i / NB) & 1, s, p.limit_ns, p.status, true);
+  for (uint32_t i = (e_i > NE ? e_i - NE : 0); i < e_i; ++i)
+    wait_bounded(&s.e_full[i % NE], (i / NE) & 1, s, p.limit_ns, p.status, true);
+}
+
+__device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
+  const int Tn = p.N / BM;
+  uint32_t a_i = 0, b_i = 0, e_i = 0;
+  bool ok = true;
+  int it = 0;
+  for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
+    const int tn = item % Tn;
+    if (!(ok = wait_bounded(&s.acc_empty, (it & 1) ^ 1, s, p.limit_ns, p.status, false))) break;
+    tc_fence_after();
+    uint32_t accumulate = 0;
+    for (int kt = 0; ok && kt < p.Tk; ++kt) {
+      const patch_tile_desc d = p.desc[int64_t(tn) * p.Tk + kt];
+      if (d.kind) {
+        const uint32_t es = e_i % NE, as = a_i % NA;
+        if (!(ok = wait_bounded(&s.e_full[es], (e_i / NE) & 1, s, p.limit_ns, p.status, false))) break;
+        if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, s, p.limit_ns, p.status, false))) break;
+        tc_fence_after();
+        const uint32_t e_tmem = tmem + META_COL0 + 4 * es;
+        tmem_cp_128x128b(e_tmem, meta_desc(smem_u32(s.e[es])));
+        const uint64_t a0 = sw128_desc(smem_u32(s.a[as]));
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t bs = b_i % NB;
+          if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, s, p.limit_ns, p.status, false))) break;
+          tc_fence_after();
+          const uint64_t b0 = sw128_desc(smem_u32(s.b[bs]));
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t kb = 2 * h + j;  // 32-k block of the tile: 16 kept values = 32 B of A
+            mma_sparse(tmem, a0 + (kb * 32 >> 4), b0 + (j * 64 >> 4), e_tmem + (kb & 2u),
+                       IDESC_SPARSE | (kb & 1u), accumulate);
+            accumulate = 1;
+          }
+          tc_commit(&s.b_empty[bs]);
+          ++b_i;
+        }
+        if (!ok) break;
+        tc_commit(&s.a_empty[as]);
+        ++a_i;
+        tc_commit(&s.e_empty[es]);
+        ++e_i;
+      } else {
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t as = a_i % NA, bs = b_i % NB;
+          if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, s, p.limit_ns, p.status, false))) break;
+          if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, s, p.limit_ns, p.status, false))) break;
+          tc_fence_after();
+          const uint64_t a0 = sw128_desc(smem_u32(s.a[as]));
+          const uint64_t b0 = sw128_desc(smem_u32(s.b[bs]));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {  // K = 16 per MMA = 32 B along the swizzled row
+            mma_dense(tmem, a0 + (j * 32 >> 4), b0 + (j * 32 >> 4), IDESC_DENSE, accumulate);
+            accumulate = 1;
+          }
+          tc_commit(&s.a_empty[as]);
+          ++a_i;
+          tc_commit(&s.b_empty[bs]);
+          ++b_i;
+        }
+      }
+    }
+    if (ok) tc_commit(&s.acc_full);
+  }
+  // all MMAs and copies issued must be complete before TMEM is freed
+  tc_commit(&s.drain);
+  wait_bounded(&s.drain, 0, s, p.limit_ns, p.status, true);
+}
+
+__device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
+  const int Tn = p.N / BM;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3;  // the TMEM lane quarter this warp may access
+  int it = 0;
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
+    const int tn = item % Tn, tb = item / Tn;
+    if (!wait_bounded(&s.acc_full, it & 1, s, p.limit_ns, p.status, false)) break;
+    tc_fence_after();
+    const int64_t n = int64_t(tn) * BM + 32 * q + lane;
+    const int m0 = tb * BT;
+    for (int c = 0; c < BT / 32; ++c) {
+      if (m0 + 32 * c >= p.M) break;  // warp-uniform
+      uint32_t v[32];
+      tmem_ld_32cols(tmem + (uint32_t(32 * q) << 16) + uint32_t(32 * c), v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int m = m0 + 32 * c + j;
+        if (m < p.M) p.Y[int64_t(m) * p.N + n] = f32_to_bf16_rne(__uint_as_float(v[j]));
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.acc_empty);
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                   const Args p) {
+  extern __shared__ uint8_t smem_raw[];
+  Shared& s = *reinterpret_cast<Shared*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(&s.a_full[i], 1);
+      mbar_init(&s.a_empty[i], 1);
+    }
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(&s.b_full[i], 1);
+      mbar_init(&s.b_empty[i], 1);
+    }
+    for (int i = 0; i < NE; ++i) {
+      mbar_init(&s.e_full[i], 1);
+      mbar_init(&s.e_empty[i], 1);
+    }
+    mbar_init(&s.acc_full, 1);
+    mbar_init(&s.acc_empty, 4);
+    mbar_init(&s.drain, 1);
+    s.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s.tmem_base)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) producer(s, &tmap_x, &tmap_w, p);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) mma_issuer(s, tmem, p);
+    __syncwarp();
+  } else {
+    epilogue(s, tmem, p);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace prefill
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor map, 128-byte swizzle, out-of-bounds reads fill zeros.
+static bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
+                           int32_t* status, int num_sms, uint64_t limit_ns, int inject,
+                           cudaStream_t stream) {
+  using namespace prefill;
+  const int64_t Tn = W.N / BM, Tk = W.K / kTile, T = Tn * Tk;
+  const uint64_t n_panels = uint64_t(2 * (T - W.n_sparse) + W.n_sparse);
+  CUtensorMap tmap_x, tmap_w;
+  if (!make_map_2d(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, BT)) return cudaErrorUnknown;
+  if (!make_map_2d(&tmap_w, W.values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
+  Args p;
+  p.meta = static_cast<const uint8_t*>(W.meta);
+  p.desc = W.desc;
+  p.Y = Y;
+  p.M = int(M);
+  p.N = int(W.N);
+  p.Tk = int(Tk);
+  p.n_items = int(Tn * ((M + BT - 1) / BT));
+  p.limit_ns = limit_ns;
+  p.status = status;
+  p.inject = inject;
+  const int grid = p.n_items < num_sms ? p.n_items : num_sms;
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES));
+  if (e != cudaSuccess) return e;
+  prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmap_x, tmap_w, p);
+  return cudaGetLastError();
+}
+
+}  // namespace patch

@@ -1,0 +1,101 @@
+// patch_hard_mask kernel: the inference-time (argmax) form of PATCH's hybrid
+// mask.  "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs", section 2
+// "Methodology: PATCH", "Learnable Distributions": a 2-way tile logit chooses
+// dense vs 2:4 sparse, a 6-way pattern logit per group of 4 chooses the kept
+// pair inside sparse tiles.
+//
+// HBM-bound elementwise pass: per weight it reads 2 B of W and 6 B of pattern
+// logits and writes 2 B of masked W plus 1/4 B of pattern id.  One thread
+// handles 8 consecutive groups (32 weights) of one row: 4 x 16 B loads of W,
+// 12 x 16 B loads of logits, 4 x 16 B stores, one 8 B store of ids.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace patch {
+
+// Index of the first maximum (a later value wins only when strictly greater).
+__device__ __forceinline__ uint32_t argmax6(const float* v) {
+  uint32_t best = 0;
+  float bv = v[0];
+#pragma unroll
+  for (uint32_t j = 1; j < 6; ++j) {
+    if (v[j] > bv) {
+      bv = v[j];
+      best = j;
+    }
+  }
+  return best;
+}
+
+__global__ void __launch_bounds__(256) hard_mask_kernel(
+    const uint4* __restrict__ W, int64_t N, int64_t K, const float* __restrict__ tile_logits,
+    const float4* __restrict__ pattern_logits, uint4* __restrict__ W_masked,
+    uint8_t* __restrict__ bitmap, uint2* __restrict__ pat_id) {
+  const int64_t items_per_row = K / 32;  // 8 groups per item
+  const int64_t n_items = N * items_per_row;
+  const int64_t Tk = K / kTile;
+  for (int64_t it = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; it < n_items;
+       it += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t n = it / items_per_row;
+    const int64_t j = it - n * items_per_row;  // item within row: k = 32j .. 32j+31
+    const int64_t tn = n / kTile, tk = (32 * j) / kTile;
+    const float l0 = __ldg(tile_logits + 2 * (tn * Tk + tk));
+    const float l1 = __ldg(tile_logits + 2 * (tn * Tk + tk) + 1);
+    const bool sparse = l1 > l0;  // argmax of (dense, sparse), ties -> dense
+    if (bitmap && n % kTile == 0 && (32 * j) % kTile == 0) bitmap[tn * Tk + tk] = sparse ? 1 : 0;
+
+    // 8 groups x 6 logits = 48 floats = 12 float4, contiguous
+    float lg[48];
+    const float4* lp = pattern_logits + it * 12;
+#pragma unroll
+    for (int q = 0; q < 12; ++q) {
+      float4 v = __ldcs(lp + q);
+      lg[4 * q] = v.x;
+      lg[4 * q + 1] = v.y;
+      lg[4 * q + 2] = v.z;
+      lg[4 * q + 3] = v.w;
+    }
+    uint32_t ids[8];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) ids[g] = argmax6(lg + 6 * g);
+    uint2 packed;
+    packed.x = ids[0] | ids[1] << 8 | ids[2] << 16 | ids[3] << 24;
+    packed.y = ids[4] | ids[5] << 8 | ids[6] << 16 | ids[7] << 24;
+    __stcs(pat_id + it, packed);
+
+    if (W_masked) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {  // 16 B = 8 weights = groups 2q, 2q+1
+        uint4 w = __ldcs(W + it * 4 + q);
+        if (sparse) {
+          const uint32_t c0 = pattern_code(ids[2 * q]), c1 = pattern_code(ids[2 * q + 1]);
+          // keep-masks of the 4 bf16 lanes of each group (bit i set = keep position i)
+          const uint32_t k0 = (1u << (c0 & 3)) | (1u << (c0 >> 2));
+          const uint32_t k1 = (1u << (c1 & 3)) | (1u << (c1 >> 2));
+          w.x &= ((k0 & 1) ? 0x0000FFFFu : 0u) | ((k0 & 2) ? 0xFFFF0000u : 0u);
+          w.y &= ((k0 & 4) ? 0x0000FFFFu : 0u) | ((k0 & 8) ? 0xFFFF0000u : 0u);
+          w.z &= ((k1 & 1) ? 0x0000FFFFu : 0u) | ((k1 & 2) ? 0xFFFF0000u : 0u);
+          w.w &= ((k1 & 4) ? 0x0000FFFFu : 0u) | ((k1 & 8) ? 0xFFFF0000u : 0u);
+        }
+        __stcs(W_masked + it * 4 + q, w);
+      }
+    }
+  }
+}
+
+cudaError_t launch_hard_mask(const uint16_t* W, int64_t N, int64_t K, const float* tile_logits,
+                             const float* pattern_logits, uint16_t* W_masked, uint8_t* bitmap,
+                             uint8_t* pat_id, int num_sms, cudaStream_t stream) {
+  const int64_t n_items = N * (K / 32);
+  const int threads = 256;
+  int64_t blocks = (n_items + threads - 1) / threads;
+  const int64_t cap = int64_t(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  hard_mask_kernel<<<int(blocks), threads, 0, stream>>>(
+      reinterpret_cast<const uint4*>(W), N, K, tile_logits,
+      reinterpret_cast<const float4*>(pattern_logits), reinterpret_cast<uint4*>(W_masked), bitmap,
+      reinterpret_cast<uint2*>(pat_id));
+  return cudaGetLastError();
+}
+
+}  // namespace patch

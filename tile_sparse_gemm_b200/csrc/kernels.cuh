@@ -1,0 +1,34 @@
+// Host-side launchers of libpatch's kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "patch.h"
+
+namespace patch {
+
+cudaError_t launch_hard_mask(const uint16_t* W, int64_t N, int64_t K, const float* tile_logits,
+                             const float* pattern_logits, uint16_t* W_masked, uint8_t* bitmap,
+                             uint8_t* pat_id, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap,
+                        const uint8_t* pat_id, int64_t n_sparse, void* values, void* meta,
+                        patch_tile_desc* desc, int32_t* status, int num_sms, cudaStream_t stream);
+
+// Decode split: L K-tiles per unit, S K-splits, units CTAs, smem bytes, fp32 workspace bytes.
+struct DecodePlan {
+  int L, S, units;
+  size_t smem, ws_bytes;
+};
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int num_sms);
+
+cudaError_t launch_decode(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
+                          void* workspace, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
+                           int32_t* status, int num_sms, uint64_t limit_ns, int inject,
+                           cudaStream_t stream);
+
+}  // namespace patch

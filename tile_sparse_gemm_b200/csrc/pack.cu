@@ -1,0 +1,137 @@
+// patch_pack kernels: build the mixed layout of dense tiles, compressed 2:4
+// tiles (2 kept values per group of 4 plus a 4-bit position code) and the tile
+// descriptor table.  "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs",
+// section 2 "Methodology: PATCH", "Core Mechanism" (each 128 x 128 tile dense
+// or 2:4 sparse) and "Inference & Deployment" (sparse tiles must feed the 2:4
+// sparse tensor cores, dense tiles the dense ones).
+//
+// Launch 1 (one CTA): exclusive scan of the tile kinds in row-major tile
+// order -> descriptors {kind, sparse ordinal, byte offset}.
+// Launch 2 (one CTA per tile): dense tile -> 2 panels of 128 x 64 bf16;
+// sparse tile -> 1 panel of kept values + 2048 B of metadata in the order the
+// tensor-core sparse MMA reads it.  Integer/bit work only; HBM-bound.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace patch {
+
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) pack_scan_kernel(
+    const uint8_t* __restrict__ bitmap, int64_t T, int64_t n_sparse,
+    patch_tile_desc* __restrict__ desc, int32_t* status) {
+  __shared__ uint32_t warp_sums[kScanThreads / 32];
+  __shared__ uint64_t carry_s;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry_s = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < T; base += kScanThreads) {
+    const int64_t t = base + threadIdx.x;
+    const uint32_t kind = (t < T && bitmap[t] != 0) ? 1u : 0u;
+    // inclusive warp scan
+    uint32_t v = kind;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      uint32_t y = __shfl_up_sync(0xFFFFFFFFu, v, d);
+      if (lane >= d) v += y;
+    }
+    if (lane == 31) warp_sums[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t s = warp_sums[lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        uint32_t y = __shfl_up_sync(0xFFFFFFFFu, s, d);
+        if (lane >= d) s += y;
+      }
+      warp_sums[lane] = s;  // inclusive prefix over warps
+    }
+    __syncthreads();
+    const uint64_t carry = carry_s;
+    const uint64_t before = carry + (warp > 0 ? warp_sums[warp - 1] : 0u) + v - kind;
+    if (t < T) {
+      patch_tile_desc d;
+      d.kind = kind;
+      d.sparse_ordinal = kind ? uint32_t(before) : 0xFFFFFFFFu;
+      // dense tiles before t take 2 panels each, sparse ones 1
+      d.val_offset = uint64_t(PATCH_PANEL_BYTES) * (2ull * uint64_t(t) - before);
+      desc[t] = d;
+    }
+    __syncthreads();
+    if (threadIdx.x == kScanThreads - 1) carry_s = carry + warp_sums[31];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && carry_s != uint64_t(n_sparse)) set_status(status, PATCH_DEV_COUNT);
+}
+
+__global__ void __launch_bounds__(256) pack_tiles_kernel(
+    const uint16_t* __restrict__ W, int64_t K, const uint8_t* __restrict__ pat_id,
+    const patch_tile_desc* __restrict__ desc, int64_t T, int64_t n_sparse, uint64_t values_bytes,
+    uint8_t* __restrict__ values, uint8_t* __restrict__ meta, int32_t* status) {
+  __shared__ __align__(16) uint8_t meta_s[PATCH_META_TILE_BYTES];
+  const int64_t Tk = K / kTile;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const patch_tile_desc d = desc[t];
+    const int64_t tn = t / Tk, tk = t - tn * Tk;
+    const uint64_t size = d.kind ? PATCH_SPARSE_TILE_BYTES : PATCH_DENSE_TILE_BYTES;
+    // a bitmap whose count disagrees with n_sparse must not write past the blobs
+    if (d.val_offset + size > values_bytes || (d.kind && int64_t(d.sparse_ordinal) >= n_sparse))
+      continue;  // PATCH_DEV_COUNT is raised by the scan
+    uint8_t* panel = values + d.val_offset;
+    const uint16_t* wt = W + (tn * kTile) * K + tk * kTile;
+    if (d.kind == 0) {
+      // 2 panels x 128 rows x 8 chunks of 16 B
+      for (int c = threadIdx.x; c < 2048; c += blockDim.x) {
+        const int h = c >> 10, r = (c >> 3) & 127, q = c & 7;
+        const uint4 v = __ldcs(reinterpret_cast<const uint4*>(wt + int64_t(r) * K + h * 64 + q * 8));
+        *reinterpret_cast<uint4*>(panel + h * PATCH_PANEL_BYTES + r * 128 + q * 16) = v;
+      }
+    } else {
+      // 128 rows x 16 pairs of groups; each item reads 8 weights, writes 4 values + 1 byte
+      for (int c = threadIdx.x; c < 2048; c += blockDim.x) {
+        const int r = c >> 4, p = c & 15;
+        const uint4 w = __ldcs(reinterpret_cast<const uint4*>(wt + int64_t(r) * K + p * 8));
+        const uint16_t ids2 = *reinterpret_cast<const uint16_t*>(
+            pat_id + (tn * kTile + r) * (K / 4) + tk * 32 + 2 * p);
+        uint32_t id0 = ids2 & 0xFF, id1 = ids2 >> 8;
+        if (id0 > 5 || id1 > 5) {
+          set_status(status, PATCH_DEV_BAD_PATTERN);
+          if (id0 > 5) id0 = 0;
+          if (id1 > 5) id1 = 0;
+        }
+        const uint32_t c0 = pattern_code(id0), c1 = pattern_code(id1);
+        // the 4 bf16 of each group as one 64-bit word; position i is bits 16i..16i+15
+        const uint64_t g0 = uint64_t(w.y) << 32 | w.x, g1 = uint64_t(w.w) << 32 | w.z;
+        uint2 out;
+        out.x = uint32_t((g0 >> (16 * (c0 & 3))) & 0xFFFFu) | uint32_t((g0 >> (16 * (c0 >> 2))) & 0xFFFFu) << 16;
+        out.y = uint32_t((g1 >> (16 * (c1 & 3))) & 0xFFFFu) | uint32_t((g1 >> (16 * (c1 >> 2))) & 0xFFFFu) << 16;
+        *reinterpret_cast<uint2*>(panel + r * 128 + p * 8) = out;
+        meta_s[meta_byte_index(r, 2 * p)] = uint8_t(c0 | (c1 << 4));
+      }
+      __syncthreads();
+      uint8_t* mt = meta + uint64_t(d.sparse_ordinal) * PATCH_META_TILE_BYTES;
+      for (int c = threadIdx.x; c < PATCH_META_TILE_BYTES / 16; c += blockDim.x)
+        reinterpret_cast<uint4*>(mt)[c] = reinterpret_cast<const uint4*>(meta_s)[c];
+      __syncthreads();
+    }
+  }
+}
+
+cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap,
+                        const uint8_t* pat_id, int64_t n_sparse, void* values, void* meta,
+                        patch_tile_desc* desc, int32_t* status, int num_sms,
+                        cudaStream_t stream) {
+  const int64_t T = (N / kTile) * (K / kTile);
+  const uint64_t values_bytes =
+      uint64_t(T - n_sparse) * PATCH_DENSE_TILE_BYTES + uint64_t(n_sparse) * PATCH_SPARSE_TILE_BYTES;
+  pack_scan_kernel<<<1, kScanThreads, 0, stream>>>(bitmap, T, n_sparse, desc, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int64_t blocks = T < int64_t(num_sms) * 16 ? T : int64_t(num_sms) * 16;
+  pack_tiles_kernel<<<int(blocks), 256, 0, stream>>>(W, K, pat_id, desc, T, n_sparse, values_bytes,
+                                                     static_cast<uint8_t*>(values),
+                                                     static_cast<uint8_t*>(meta), status);
+  return cudaGetLastError();
+}
+
+}  // namespace patch
