@@ -204,6 +204,37 @@ PATCH_API patch_status_t patch_gemm_ex(const uint16_t *X, int64_t M, const patch
                              void *stream, int path, uint64_t wait_limit_us);
 
 /*
+ * patch_gemm_decode_noalloc: the decode GEMM (M <= 16) for callers that
+ * cannot allocate device memory.  The paper has no counterpart; this is a
+ * deployment convenience of this library.
+ *
+ * Some callers have no way to get scratch memory: a plugin inside a host
+ * framework that owns the device memory pool and passes the plugin only its
+ * input and output buffers, or a latency-critical loop where a cudaMalloc
+ * (which may synchronise the whole device) is not acceptable.  This entry
+ * point computes exactly what patch_gemm computes on its decode path, with
+ * the same kernels, but keeps the split-K partial sums in a buffer compiled
+ * into the library instead of a caller-provided workspace:
+ *   - the buffer is PATCH_NOALLOC_SCRATCH_BYTES of device memory that every
+ *     GPU which loads the library holds until the process exits;
+ *   - the first call on each device looks the buffer's device address up
+ *     (cudaGetSymbolAddress, with that device current), so make that first
+ *     call before any stream capture;
+ *   - a problem whose partial sums need more than the buffer holds is
+ *     rejected with PATCH_ERR_WORKSPACE (no launch);
+ *   - every call shares the one buffer: calls whose kernels may overlap on
+ *     the GPU (different streams, or different host threads) race and give
+ *     wrong results; serialise them, e.g. on one stream.  Nothing in the
+ *     buffer needs to start at zero: each call overwrites what it reads.
+ * Arguments are as for patch_gemm (X, Y, the packed weight and dev_status
+ * are caller-owned device memory); M must be in 0..16.  The call allocates
+ * nothing and never synchronises the stream.
+ */
+#define PATCH_NOALLOC_SCRATCH_BYTES (4u << 20) /* 4 MiB */
+PATCH_API patch_status_t patch_gemm_decode_noalloc(const uint16_t *X, int64_t M, const patch_weight *W,
+                                                   uint16_t *Y, int32_t *dev_status, void *stream);
+
+/*
  * patch_read_status: synchronise `stream`, copy *dev_status to *host_bits and
  * return the first error it encodes (PATCH_ERR_TIMEOUT, then BAD_PATTERN,
  * then COUNT) or PATCH_OK.  host_bits may be NULL.
