@@ -62,22 +62,27 @@ def stored_bytes(N, K, n_sparse):
 
 
 class ClockSampler:
-    """nvidia-smi samples (every 100 ms) of the SM clock and throttle reasons."""
+    """nvidia-smi samples (every 20 ms) of the SM clock and throttle reasons.
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+    The timed region may be shorter than the sampling period, so the summary
+    uses the samples from 0.25 s before the region starts (the warm-up, at the
+    same load) until it ends."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.samples = []  # (host time, line)
+        self.marks = {}
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except OSError:
@@ -86,9 +91,18 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.samples.append((time.monotonic(), line.strip()))
+
+    def wait_first_sample(self, timeout=3.0):
+        t0 = time.monotonic()
+        while self.proc and not self.samples and time.monotonic() - t0 < timeout:
+            time.sleep(0.01)
+
+    def mark(self, name):
+        self.marks[name] = time.monotonic()
 
     def __exit__(self, *exc):
+        time.sleep(0.05)
         if self.proc:
             self.proc.terminate()
             try:
@@ -97,46 +111,56 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        t0 = self.marks.get("start", 0.0) - 0.25
+        t1 = self.marks.get("end", float("inf")) + 0.03
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.samples:
+            if not (t0 <= ts <= t1):
+                continue
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 7:
+            if len(parts) < 6:
                 continue
             try:
                 sm.append(float(parts[0]))
                 smax.append(float(parts[1]))
             except ValueError:
                 continue
-            for name, v in zip(names, parts[3:7]):
+            for name, v in zip(names, parts[2:6]):
                 if v.lower() == "active":
                     reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "window": "0.25 s before the timed region to its end"}
 
 
 # ------------------------------------------------------------ workloads
 
 
-def build_layers(workload):
-    """Host inputs of every layer in the step: list of dicts."""
+def build_layers(workload, only=None, fracs=None, tokens=None):
+    """Host inputs of every layer in the step: list of dicts.  `only`, `fracs` and
+    `tokens` select a subset (profiling runs); the default is the whole workload."""
     layers = []
+    ms = tuple(tokens) if tokens else (DECODE_MS if workload == "decode" else (PREFILL_M,))
     if workload == "decode":
         for i, (name, N, K) in enumerate(si.LLAMA2_7B):
+            if only and name not in only:
+                continue
             w = si.gen_w(N, K, DECODE_CONFIG, i)
             bm = si.tiles_exact(N, K, 0.5, DECODE_CONFIG, i)
             layers.append(dict(name=name, N=N, K=K, w=w, bm=bm, ids=si.patterns_top2(w), frac=0.5,
-                               xs={M: si.gen_x(M, K, DECODE_CONFIG, i) for M in DECODE_MS}))
+                               xs={M: si.gen_x(M, K, DECODE_CONFIG, i) for M in ms}))
     else:
         for i, (name, N, K) in enumerate(si.LLAMA2_7B):
+            if only and name not in only:
+                continue
             w = si.gen_w(N, K, PREFILL_CONFIG, i)
             ids = si.patterns_top2(w)
-            x = si.gen_x(PREFILL_M, K, PREFILL_CONFIG, i)
-            for f in FRACS:
+            xs = {M: si.gen_x(M, K, PREFILL_CONFIG, i) for M in ms}
+            for f in (fracs or FRACS):
                 bm = si.tiles_exact(N, K, f, PREFILL_CONFIG, i)
-                layers.append(dict(name=name, N=N, K=K, w=w, bm=bm, ids=ids, frac=f, xs={PREFILL_M: x}))
+                layers.append(dict(name=name, N=N, K=K, w=w, bm=bm, ids=ids, frac=f, xs=xs))
     return layers
 
 
@@ -198,7 +222,7 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     pk = peaks()
-    layers = build_layers(args.workload)
+    layers = build_layers(args.workload, args.layers, args.fracs, args.tokens)
     calls = calls_of(layers)
     status = tsg.new_status(dev)
     packed = []
@@ -212,7 +236,7 @@ def run_ours(args, rank, world):
     ys = {(li, M): torch.empty((M, layers[li]["N"]), dtype=torch.bfloat16, device=dev) for li, M in calls}
     ws_bytes = max(tsg.patch_gemm_workspace_size(M, packed[li]) for li, M in calls)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    launches_per_call = {c: (2 if tsg.patch_gemm_workspace_size(c[1], packed[c[0]]) > 0 else 1) for c in calls}
+    launches_per_call = {c: (2 if c[1] <= tsg.DECODE_MAX_M else 1) for c in calls}  # decode: main + fixup
     stream = torch.cuda.current_stream()
     resident = sum(p.stored_bytes for p in packed)
 
@@ -235,24 +259,48 @@ def run_ours(args, rank, world):
     if code != 0:
         raise RuntimeError(f"device status {code} bits {bits} after warm-up")
 
-    # timed region: whole-step events plus per-call events for the roofline
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
-          for _ in range(args.steps)]
+    # The K timed steps are captured once as one CUDA graph (launch-bound small
+    # kernels), with an event pair around every call; one replay is the timed region.
+    # external events become event-record nodes when captured, so they keep their timestamps
+    ev = [[(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in calls] for _ in range(args.steps)]
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream()
+            for st in range(args.steps):
+                for j, (li, M) in enumerate(calls):
+                    ev[st][j][0].record(cap)
+                    tsg.patch_gemm(xs[(li, M)], packed[li], Y=ys[(li, M)], workspace=ws, status=status)
+                    ev[st][j][1].record(cap)
+        graph.replay()  # untimed: first replay uploads the graph
+        torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
     with ClockSampler(dev.index) as clocks:
+        clocks.wait_first_sample()
+        barrier()
+        torch.cuda.synchronize()
+        clocks.mark("start")
         t_start.record(stream)
-        for s in range(args.steps):
-            step(ev[s])
+        if graph is not None:
+            graph.replay()
+        else:
+            for st in range(args.steps):
+                step(ev[st])
         t_end.record(stream)
         torch.cuda.synchronize()
-    barrier()
+        clocks.mark("end")
+        barrier()
     ms = t_start.elapsed_time(t_end)
-    call_ms = np.array([[a.elapsed_time(b) for a, b in ev[s]] for s in range(args.steps)])  # [steps][calls]
+    try:
+        call_ms = np.array([[a.elapsed_time(b) for a, b in ev[st]] for st in range(args.steps)])  # [steps][calls]
+    except RuntimeError:  # no per-call timestamps: attribute the step time to the calls by bytes/FLOPs
+        call_ms = None
     code, bits = tsg.patch_read_status(status)
     if code != 0:
         raise RuntimeError(f"device status {code} bits {bits} after timing")
+    del graph
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     xh = {c: xs[c].cpu().pin_memory() for c in calls}
@@ -294,13 +342,18 @@ def run_ours(args, rank, world):
     e2e_value = per_step * args.steps * world / (e2e_ms / 1e3)
 
     # roofline of the dominant kernel: algorithmic bytes (or FLOPs) per launch / mean launch time
-    mean_call_ms = call_ms.mean(axis=0)
+    if call_ms is None:
+        w_ = np.array([call_bytes(layers[li], M) if args.workload == "decode" else call_flops(layers[li], M)
+                       for li, M in calls], dtype=np.float64)
+        mean_call_ms = (ms / args.steps) * w_ / w_.sum()
+    else:
+        mean_call_ms = call_ms.mean(axis=0)
     if args.workload == "decode":
         alg = np.array([call_bytes(layers[li], M) for li, M in calls]) / 1e9
         achieved = float(alg.sum() / (mean_call_ms.sum() / 1e3))
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
-                "kernel": "decode_gemm_kernel (+ split-K reduce)", "peak_source": pk["source"]}
+                "kernel": "decode_tc_kernel (+ decode_fixup_kernel)", "peak_source": pk["source"]}
         detail = {f"{layers[li]['name']}@M={M}": {"us": round(1e3 * mean_call_ms[j], 2),
                                                   "GB/s": round(alg[j] / (mean_call_ms[j] / 1e3), 1)}
                   for j, (li, M) in enumerate(calls)}
@@ -346,11 +399,15 @@ def run_ours(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", choices=["decode", "prefill"], default="decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the timed calls eagerly instead of one CUDA graph")
+    ap.add_argument("--layers", nargs="*", help="profiling: only these projections (q k v o gate up down)")
+    ap.add_argument("--fracs", nargs="*", type=float, help="profiling (prefill): only these sparse-tile fractions")
+    ap.add_argument("--tokens", nargs="*", type=int, help="profiling: only these token counts M")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

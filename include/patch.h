@@ -97,8 +97,9 @@ typedef enum {
 
 /* Path selector of patch_gemm_ex. */
 #define PATCH_PATH_AUTO 0    /* M <= PATCH_DECODE_MAX_M: decode, else prefill */
-#define PATCH_PATH_DECODE 1  /* CUDA-core split-K GEMV, any M in 1..16 */
+#define PATCH_PATH_DECODE 1  /* stream-K weight streaming kernel (TMA + tcgen05, N = 16), M in 1..16 */
 #define PATCH_PATH_PREFILL 2 /* TMA + tcgen05 (dense and 2:4 sparse MMA), any M >= 1 */
+#define PATCH_PATH_DECODE_SIMT 3 /* split-K GEMV on CUDA cores (16-byte loads, fp32 FMA), M in 1..16 */
 /* Test hook, OR-ed into PATCH_PATH_PREFILL: the prefill producer stops after
  * its first K-tile, so the consumers' bounded waits run out and the kernel
  * reports PATCH_DEV_TIMEOUT and exits cleanly (needs K >= 256 or several
@@ -172,7 +173,8 @@ PATCH_API patch_status_t patch_pack(const uint16_t *W, int64_t N, int64_t K, con
 
 /*
  * patch_gemm_workspace_size: device scratch bytes patch_gemm needs for M rows
- * of X and this weight (0 when none is needed).  Host only.
+ * of X and this weight (0 when none is needed; for M <= 16 enough for either
+ * decode kernel).  Host only, but queries the current device's SM count.
  */
 PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight *W, size_t *bytes);
 
@@ -184,9 +186,12 @@ PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight
  *   W  packed weight (host struct)
  *   Y  bf16 [M][N] (16-byte aligned)
  *   workspace: patch_gemm_workspace_size bytes (may be NULL when that is 0)
- * M <= 16 runs the decode path (split-K GEMV on CUDA cores over the stored
- * bytes, fp32 partials reduced in a fixed order), larger M the prefill path
- * (TMA-fed tcgen05 kernel, dense and sparse MMAs into one TMEM fp32 tile).
+ * M <= 16 runs the decode path: one CTA per SM streams an equal share of
+ * the stored panels through a TMA ring (stream-K), the tensor cores reduce
+ * them (N = 16 tokens, zero-padded), tile rows cut between CTAs are summed
+ * by a second kernel in a fixed order from fp32 partials in the workspace.
+ * Larger M runs the prefill path (TMA-fed tcgen05 kernel, dense and sparse
+ * MMAs into one TMEM fp32 tile per 128 x 256 output tile).
  * A bounded wait that runs out sets PATCH_DEV_TIMEOUT (Y is then undefined).
  */
 PATCH_API patch_status_t patch_gemm(const uint16_t *X, int64_t M, const patch_weight *W, uint16_t *Y,
@@ -195,9 +200,10 @@ PATCH_API patch_status_t patch_gemm(const uint16_t *X, int64_t M, const patch_we
 
 /*
  * patch_gemm_ex: patch_gemm with an explicit path (PATCH_PATH_*) and the
- * bounded-wait limit of the prefill kernel in microseconds (0 = default,
- * 2 s).  PATCH_PATH_DECODE requires M <= 16.  PATCH_PATH_TEST_STALL is only
- * accepted together with PATCH_PATH_PREFILL.
+ * bounded-wait limit of the tensor-core kernels in microseconds (0 =
+ * default, 2 s).  PATCH_PATH_DECODE and PATCH_PATH_DECODE_SIMT require
+ * M <= 16.  PATCH_PATH_TEST_STALL is only accepted together with
+ * PATCH_PATH_PREFILL.  patch_gemm_workspace_size covers every path.
  */
 PATCH_API patch_status_t patch_gemm_ex(const uint16_t *X, int64_t M, const patch_weight *W, uint16_t *Y,
                              void *workspace, size_t workspace_bytes, int32_t *dev_status,

@@ -96,11 +96,11 @@ def tiles_clustered(N: int, K: int, frac: float, config: int = 0, shape_idx: int
 def patterns_top2(w_bits: np.ndarray) -> np.ndarray:
     """Pattern ids [N][K/4] uint8: keep the two largest |w| of each group of 4 (ties -> lower index)."""
     N, K = w_bits.shape
-    mag = (w_bits.astype(np.uint16) & np.uint16(0x7FFF)).reshape(N, K // 4, 4)  # |w| order == bit order
-    # stable sort on -mag keeps the lower index first among equal magnitudes
-    order = np.argsort(-mag.astype(np.int32), axis=2, kind="stable")[:, :, :2]
-    lo = np.minimum(order[:, :, 0], order[:, :, 1])
-    hi = np.maximum(order[:, :, 0], order[:, :, 1])
+    mag = (w_bits.astype(np.uint16) & np.uint16(0x7FFF)).reshape(N, K // 4, 4).astype(np.int32)  # |w| order
+    first = np.argmax(mag, axis=2)                      # largest, lowest index among equals
+    np.put_along_axis(mag, first[:, :, None], -1, axis=2)
+    second = np.argmax(mag, axis=2)                     # next largest, lowest index among equals
+    lo, hi = np.minimum(first, second), np.maximum(first, second)
     table = np.full((4, 4), 255, dtype=np.uint8)
     for (a, b), pid in _PAIR_ID.items():
         table[a, b] = pid

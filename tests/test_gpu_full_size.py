@@ -34,7 +34,7 @@ def _cuda():
     tsg.lib()
 
 
-@functools.lru_cache(maxsize=4)
+@functools.lru_cache(maxsize=16)
 def weight(N, K, cfg, idx):
     w = si.gen_w(N, K, cfg, idx)
     return w, si.patterns_top2(w)

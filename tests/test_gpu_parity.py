@@ -189,13 +189,30 @@ def test_gemm_config1_decode():
     check_gemm(y, ref, "config 1")
 
 
+@pytest.mark.parametrize("path", [tsg.PATH_DECODE, tsg.PATH_DECODE_SIMT])
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 7, 8, 13, 16])
 @pytest.mark.parametrize("N,K,frac", [(384, 640, 0.5), (256, 1280, 0.0), (640, 256, 1.0)])
-def test_gemm_decode_parity(M, N, K, frac):
+def test_gemm_decode_parity(M, N, K, frac, path):
     x, w, bm, ids = _layer(N, K, M, "exact", frac, shape_idx=M)
     ref = oracle.hybrid_gemm(x, w, bm, ids)
+    y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids), path)
+    check_gemm(y, ref, f"decode path {path} M={M} {N}x{K} f={frac}")
+
+
+@pytest.mark.parametrize("N,K,frac,kind", [
+    (128, 128, 1.0, "exact"),        # 1 panel: most CTAs idle
+    (128, 896, 0.5, "clustered"),    # fewer panels than SMs
+    (4864, 896, 0.5, "clustered"),   # many tile rows cut between CTAs
+    (2048, 4096, 0.3, "bernoulli"),  # mixed kinds, rows longer than a CTA share
+    (128, 16384, 0.5, "exact"),      # one tile row shared by every CTA
+])
+@pytest.mark.parametrize("M", [1, 16])
+def test_stream_k_decode_cuts(N, K, frac, kind, M):
+    """The stream-K split cuts tile rows anywhere; every cut must be summed exactly once."""
+    x, w, bm, ids = _layer(N, K, M, kind, frac, cfg=12, shape_idx=N % 97)
+    ref = oracle.hybrid_gemm(x, w, bm, ids)
     y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids), tsg.PATH_DECODE)
-    check_gemm(y, ref, f"decode M={M} {N}x{K} f={frac}")
+    check_gemm(y, ref, f"stream-K {N}x{K} f={frac} M={M}")
 
 
 @pytest.mark.parametrize("frac", [0.0, 1.0, 0.5])
@@ -215,8 +232,10 @@ def test_prefill_path_small_m_matches_decode(M):
     ref = oracle.hybrid_gemm(x, w, bm, ids)
     yp = gemm_on_gpu(x, pw, tsg.PATH_PREFILL)
     yd = gemm_on_gpu(x, pw, tsg.PATH_DECODE)
+    ys = gemm_on_gpu(x, pw, tsg.PATH_DECODE_SIMT)
     check_gemm(yp, ref, "prefill small M")
     check_gemm(yd, ref, "decode")
+    check_gemm(ys, ref, "decode simt")
 
 
 def test_prefill_many_output_tiles():
@@ -240,8 +259,8 @@ def test_gemm_all_sparse_equals_24_and_all_dense_equals_dense():
         xd = to_dev_bf16(x).float()
         w_eff = torch.from_numpy(oracle.apply_mask(w, bm, ids).view(np.int16)).view(torch.bfloat16).cuda().float()
         torch_ref = (xd @ w_eff.T).double().cpu().numpy()   # plain fp32 reference of the same op
-        for path in (tsg.PATH_PREFILL, tsg.PATH_DECODE):
-            if path == tsg.PATH_DECODE:
+        for path in (tsg.PATH_PREFILL, tsg.PATH_DECODE, tsg.PATH_DECODE_SIMT):
+            if path != tsg.PATH_PREFILL:
                 y = gemm_on_gpu(x[:16], pw, path)
                 check_gemm(y, torch_ref[:16], f"decode f={frac}")
             else:

@@ -35,7 +35,7 @@ STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_INVALID_ARG", 2: "PATCH_ERR_SHAPE",
                 4: "PATCH_ERR_DEVICE", 5: "PATCH_ERR_CUDA", 6: "PATCH_ERR_BAD_PATTERN",
                 7: "PATCH_ERR_TIMEOUT", 8: "PATCH_ERR_WORKSPACE", 9: "PATCH_ERR_COUNT"}
 DEV_BAD_PATTERN, DEV_TIMEOUT, DEV_COUNT = 0x1, 0x2, 0x4
-PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_TEST_STALL = 0, 1, 2, 0x100
+PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_DECODE_SIMT, PATH_TEST_STALL = 0, 1, 2, 3, 0x100
 
 
 class PatchError(RuntimeError):
@@ -205,7 +205,10 @@ def patch_gemm_ex(X: torch.Tensor, weight: PackedWeight, Y: torch.Tensor | None 
 def patch_gemm(X: torch.Tensor, weight: PackedWeight, Y: torch.Tensor | None = None,
                workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
-    """Y = X * W_eff^T (bf16 out, fp32 accumulate); M <= 16 decode path, else prefill."""
+    """Y = X * W_eff^T (bf16 out, fp32 accumulate); M <= 16 decode path, else prefill.
+
+    Every call runs on the current stream and launches only libpatch kernels, so a
+    sequence of calls can be captured in a CUDA graph (after one eager call)."""
     return patch_gemm_ex(X, weight, Y, workspace, status, PATH_AUTO, 0, stream)
 
 

@@ -111,12 +111,16 @@ patch_status_t patch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t
 patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight* W, size_t* bytes) {
   if (!bytes || !W || M < 0) return PATCH_ERR_INVALID_ARG;
   if (!shape_ok(W->N, W->K)) return PATCH_ERR_SHAPE;
+  const int64_t T = (W->N / kTile) * (W->K / kTile);
+  if (W->n_sparse < 0 || W->n_sparse > T) return PATCH_ERR_INVALID_ARG;
   *bytes = 0;
   if (M == 0 || M > PATCH_DECODE_MAX_M) return PATCH_OK;
   int sms = 0;
   patch_status_t st = device_sms(&sms);
   if (st != PATCH_OK) return st;
-  *bytes = decode_plan(M, W->N, W->K, sms).ws_bytes;
+  // enough for either decode kernel
+  const size_t tc = decode_tc_workspace_bytes(M, *W, sms), simt = decode_plan(M, W->N, W->K, sms).ws_bytes;
+  *bytes = tc > simt ? tc : simt;
   return PATCH_OK;
 }
 
@@ -130,8 +134,9 @@ patch_status_t patch_gemm_ex(const uint16_t* X, int64_t M, const patch_weight* W
   patch_status_t st = check_weight(W);
   if (st != PATCH_OK) return st;
   if (path == PATCH_PATH_AUTO) path = M <= PATCH_DECODE_MAX_M ? PATCH_PATH_DECODE : PATCH_PATH_PREFILL;
-  if (path != PATCH_PATH_DECODE && path != PATCH_PATH_PREFILL) return PATCH_ERR_INVALID_ARG;
-  if (path == PATCH_PATH_DECODE && M > PATCH_DECODE_MAX_M) return PATCH_ERR_INVALID_ARG;
+  if (path != PATCH_PATH_DECODE && path != PATCH_PATH_PREFILL && path != PATCH_PATH_DECODE_SIMT)
+    return PATCH_ERR_INVALID_ARG;
+  if (path != PATCH_PATH_PREFILL && M > PATCH_DECODE_MAX_M) return PATCH_ERR_INVALID_ARG;
   if (M == 0) return PATCH_OK;
   if (!X || !Y) return PATCH_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Y)) return PATCH_ERR_ALIGN;
@@ -140,14 +145,18 @@ patch_status_t patch_gemm_ex(const uint16_t* X, int64_t M, const patch_weight* W
   st = device_sms(&sms);
   if (st != PATCH_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint64_t limit_ns = (wait_limit_us ? wait_limit_us : 2000000ull) * 1000ull;
   cudaError_t e;
   if (path == PATCH_PATH_DECODE) {
+    const size_t need = decode_tc_workspace_bytes(M, *W, sms);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PATCH_ERR_WORKSPACE;
+    e = launch_decode_tc(X, M, *W, Y, workspace, dev_status, sms, limit_ns, s);
+  } else if (path == PATCH_PATH_DECODE_SIMT) {
     const DecodePlan p = decode_plan(M, W->N, W->K, sms);
     if (p.ws_bytes > 0 && (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace)))
       return PATCH_ERR_WORKSPACE;
     e = launch_decode(X, M, *W, Y, workspace, sms, s);
   } else {
-    const uint64_t limit_ns = (wait_limit_us ? wait_limit_us : 2000000ull) * 1000ull;
     e = launch_prefill(X, M, *W, Y, dev_status, sms, limit_ns, inject, s);
   }
   return e == cudaSuccess ? PATCH_OK : PATCH_ERR_CUDA;

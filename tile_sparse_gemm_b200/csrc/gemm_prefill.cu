@@ -33,9 +33,12 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tc_ptx.cuh"
 
 namespace patch {
 namespace prefill {
+
+using namespace tc;
 
 constexpr int BM = 128;                  // W rows per output tile (MMA M)
 constexpr int BT = 256;                  // tokens per output tile (MMA N)
@@ -49,13 +52,8 @@ constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;      // accumulator [0, BT) + metadata slots
 constexpr uint32_t META_COL0 = BT;
 
-// instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A and B bf16
-// (bits 7-9 = 1, bits 10-12 = 1), both K-major, N >> 3 at bits 17-22,
-// M >> 4 at bits 24-28; bit 2 marks the sparse form, bits 0-1 select the
-// metadata column pair half.
-constexpr uint32_t IDESC_DENSE =
-    (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BT >> 3) << 17) | (uint32_t(BM >> 4) << 24);
-constexpr uint32_t IDESC_SPARSE = IDESC_DENSE | (1u << 2);
+constexpr uint32_t IDESC_DENSE = tc::idesc_bf16(BM, BT, false);
+constexpr uint32_t IDESC_SPARSE = tc::idesc_bf16(BM, BT, true);
 
 struct Shared {
   alignas(1024) uint8_t a[NA][A_BYTES];
@@ -68,140 +66,6 @@ struct Shared {
 };
 constexpr size_t SMEM_BYTES = sizeof(Shared) + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-
-// ---------------------------------------------------------------- PTX helpers
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for phase `parity` of `bar`.  Returns false when the wait outlived
-// limit_ns (the CTA is then marked aborted and PATCH_DEV_TIMEOUT raised) or,
-// unless `drain` is set, when another role of the CTA aborted first.
-__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Shared& s,
-                                          uint64_t limit_ns, int32_t* status, bool drain) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  volatile int* abort_flag = &s.abort_flag;
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((spin & 31u) == 0) {
-      if (!drain && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        set_status(status, PATCH_DEV_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                            int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void mma_dense(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-__device__ __forceinline__ void mma_sparse(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                           uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate));
-}
-
-__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
-        "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
-        "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor, K-major, 128-byte swizzle: start address,
-// leading offset unused (1), 8-row groups 1024 B apart, sm_100 version bit 46,
-// layout type 2 (SWIZZLE_128B) in bits 61-63.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
-         (uint64_t(1) << 46) | (uint64_t(2) << 61);
-}
-
-// Descriptor of a 128-row x 16-byte metadata block for tcgen05.cp 128x128b:
-// no swizzle, rows 16 B apart, 8-row core matrices 128 B apart.
-__device__ __forceinline__ uint64_t meta_desc(uint32_t saddr) {
-  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(128 >> 4) << 16) | (uint64_t(128 >> 4) << 32) |
-         (uint64_t(1) << 46);
-}
 
 // ---------------------------------------------------------------- roles
 
@@ -230,7 +94,7 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
       const int panel = int(d.val_offset / A_BYTES);
       if (d.kind) {
         const uint32_t es = e_i % NE;
-        if (!(ok = wait_bounded(&s.e_empty[es], ((e_i / NE) & 1) ^ 1, s, p.limit_ns, p.status, false))) break;
+        if (!(ok = wait_bounded(&s.e_empty[es], ((e_i / NE) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
         mbar_expect_tx(&s.e_full[es], E_BYTES);
         bulk_load(s.e[es], p.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.e_full[es]);
         ++e_i;
@@ -239,14 +103,14 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
       for (int h = 0; h < 2; ++h) {
         if (h < n_a) {
           const uint32_t as = a_i % NA;
-          if (!(ok = wait_bounded(&s.a_empty[as], ((a_i / NA) & 1) ^ 1, s, p.limit_ns, p.status, false)))
+          if (!(ok = wait_bounded(&s.a_empty[as], ((a_i / NA) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
             break;
           mbar_expect_tx(&s.a_full[as], A_BYTES);
           tma_load_2d(s.a[as], tmap_w, &s.a_full[as], 0, (panel + h) * 128);
           ++a_i;
         }
         const uint32_t bs = b_i % NB;
-        if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, s, p.limit_ns, p.status, false)))
+        if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
           break;
         mbar_expect_tx(&s.b_full[bs], B_BYTES);
         tma_load_2d(s.b[bs], tmap_x, &s.b_full[bs], kt * kTile + 64 * h, tb * BT);
@@ -256,11 +120,11 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
   }
   // every copy issued must have landed before the CTA may exit
   for (uint32_t i = (a_i > NA ? a_i - NA : 0); i < a_i; ++i)
-    wait_bounded(&s.a_full[i % NA], (i / NA) & 1, s, p.limit_ns, p.status, true);
+    wait_bounded(&s.a_full[i % NA], (i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, true);
   for (uint32_t i = (b_i > NB ? b_i - NB : 0); i < b_i; ++i)
-    wait_bounded(&s.b_full[i % NB], (i / NB) & 1, s, p.limit_ns, p.status, true);
+    wait_bounded(&s.b_full[i % NB], (i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, true);
   for (uint32_t i = (e_i > NE ? e_i - NE : 0); i < e_i; ++i)
-    wait_bounded(&s.e_full[i % NE], (i / NE) & 1, s, p.limit_ns, p.status, true);
+    wait_bounded(&s.e_full[i % NE], (i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, true);
 }
 
 __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
@@ -270,22 +134,22 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
     const int tn = item % Tn;
-    if (!(ok = wait_bounded(&s.acc_empty, (it & 1) ^ 1, s, p.limit_ns, p.status, false))) break;
+    if (!(ok = wait_bounded(&s.acc_empty, (it & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
     tc_fence_after();
     uint32_t accumulate = 0;
     for (int kt = 0; ok && kt < p.Tk; ++kt) {
       const patch_tile_desc d = p.desc[int64_t(tn) * p.Tk + kt];
       if (d.kind) {
         const uint32_t es = e_i % NE, as = a_i % NA;
-        if (!(ok = wait_bounded(&s.e_full[es], (e_i / NE) & 1, s, p.limit_ns, p.status, false))) break;
-        if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, s, p.limit_ns, p.status, false))) break;
+        if (!(ok = wait_bounded(&s.e_full[es], (e_i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+        if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
         tc_fence_after();
         const uint32_t e_tmem = tmem + META_COL0 + 4 * es;
         tmem_cp_128x128b(e_tmem, meta_desc(smem_u32(s.e[es])));
         const uint64_t a0 = sw128_desc(smem_u32(s.a[as]));
         for (int h = 0; h < 2; ++h) {
           const uint32_t bs = b_i % NB;
-          if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, s, p.limit_ns, p.status, false))) break;
+          if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
           tc_fence_after();
           const uint64_t b0 = sw128_desc(smem_u32(s.b[bs]));
 #pragma unroll
@@ -306,8 +170,8 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
       } else {
         for (int h = 0; h < 2; ++h) {
           const uint32_t as = a_i % NA, bs = b_i % NB;
-          if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, s, p.limit_ns, p.status, false))) break;
-          if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, s, p.limit_ns, p.status, false))) break;
+          if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+          if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
           tc_fence_after();
           const uint64_t a0 = sw128_desc(smem_u32(s.a[as]));
           const uint64_t b0 = sw128_desc(smem_u32(s.b[bs]));
@@ -327,7 +191,7 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
   }
   // all MMAs and copies issued must be complete before TMEM is freed
   tc_commit(&s.drain);
-  wait_bounded(&s.drain, 0, s, p.limit_ns, p.status, true);
+  wait_bounded(&s.drain, 0, &s.abort_flag, p.limit_ns, p.status, true);
 }
 
 __device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
@@ -337,7 +201,7 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
     const int tn = item % Tn, tb = item / Tn;
-    if (!wait_bounded(&s.acc_full, it & 1, s, p.limit_ns, p.status, false)) break;
+    if (!wait_bounded(&s.acc_full, it & 1, &s.abort_flag, p.limit_ns, p.status, false)) break;
     tc_fence_after();
     const int64_t n = int64_t(tn) * BM + 32 * q + lane;
     const int m0 = tb * BT;
@@ -438,7 +302,7 @@ static EncodeTiledFn get_encode_fn() {
 }
 
 // 2D bf16 tensor map, 128-byte swizzle, out-of-bounds reads fill zeros.
-static bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+bool make_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                         uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
@@ -458,8 +322,8 @@ cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, 
   const int64_t Tn = W.N / BM, Tk = W.K / kTile, T = Tn * Tk;
   const uint64_t n_panels = uint64_t(2 * (T - W.n_sparse) + W.n_sparse);
   CUtensorMap tmap_x, tmap_w;
-  if (!make_map_2d(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, BT)) return cudaErrorUnknown;
-  if (!make_map_2d(&tmap_w, W.values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
+  if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, BT)) return cudaErrorUnknown;
+  if (!make_map_2d_bf16(&tmap_w, W.values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
   Args p;
   p.meta = static_cast<const uint8_t*>(W.meta);
   p.desc = W.desc;

@@ -1,6 +1,7 @@
 // Host-side launchers of libpatch's kernels (internal to the library).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -30,5 +31,14 @@ cudaError_t launch_decode(const uint16_t* X, int64_t M, const patch_weight& W, u
 cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
                            int32_t* status, int num_sms, uint64_t limit_ns, int inject,
                            cudaStream_t stream);
+
+// Tensor-core decode (stream-K over panels, M <= 16): main kernel + fixup.
+size_t decode_tc_workspace_bytes(int64_t M, const patch_weight& W, int num_sms);
+cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
+                             int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream);
+
+// 2D bf16 tensor map with 128-byte swizzle (out-of-bounds reads fill zeros).
+bool make_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                      uint32_t box_inner, uint32_t box_outer);
 
 }  // namespace patch
