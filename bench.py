@@ -210,6 +210,57 @@ def cpu_baseline(workload, budget_s=15.0):
             + ", ".join(what[:8]) + (" ..." if len(what) > 8 else "") + f" ({len(what)} calls)"}
 
 
+# ------------------------------------------------------------ offline steps
+
+
+def offline_steps(layers, dev, pk, reps=5):
+    """HBM throughput of the once-per-model steps on the step's layers: the hard
+    mask (argmax of tile and pattern logits, masked W) and the packer."""
+    import torch
+
+    import tile_sparse_gemm_b200 as tsg
+
+    out = {}
+    status = tsg.new_status(dev)
+    mask_bytes = pack_bytes = 0
+    mask_ms = pack_ms = 0.0
+    for i, L in enumerate(layers):
+        N, K = L["N"], L["K"]
+        w = torch.from_numpy(L["w"].view(np.int16)).view(torch.bfloat16).to(dev)
+        tl = torch.from_numpy(si.gen_tile_logits(N, K, DECODE_CONFIG, i)).to(dev)
+        pl = torch.from_numpy(si.gen_pattern_logits(N, K, DECODE_CONFIG, i)).to(dev)
+        bm = torch.from_numpy(L["bm"]).to(dev)
+        ids = torch.from_numpy(L["ids"]).to(dev)
+        ns = int(L["bm"].sum())
+        for _ in range(2):
+            tsg.patch_hard_mask(w, tl, pl, status=status)
+            tsg.patch_pack(w, bm, ids, ns, status=status)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        torch.cuda.synchronize()
+        e[0].record()
+        for _ in range(reps):
+            tsg.patch_hard_mask(w, tl, pl, status=status)
+        e[1].record()
+        for _ in range(reps):
+            tsg.patch_pack(w, bm, ids, ns, status=status)
+        e[2].record()
+        torch.cuda.synchronize()
+        mask_ms += e[0].elapsed_time(e[1]) / reps
+        pack_ms += e[1].elapsed_time(e[2]) / reps
+        mask_bytes += N * K * (2 + 6 + 2) + N * K // 4 + (N // 128) * (K // 128) * 9
+        # reads W (dense tiles whole, sparse tiles whole 16 B rows) + ids of sparse tiles + bitmap; writes the blobs
+        pack_bytes += 2 * N * K + ns * 128 * 32 + (N // 128) * (K // 128) + stored_bytes(N, K, ns)
+        del w, tl, pl, bm, ids
+    code, bits = tsg.patch_read_status(status)
+    if code != 0:
+        raise RuntimeError(f"offline steps: device status {code} bits {bits}")
+    for name, b, ms in (("hard_mask", mask_bytes, mask_ms), ("pack", pack_bytes, pack_ms)):
+        gbs = b / 1e9 / (ms / 1e3)
+        out[name] = {"GB/s": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4), "ms_total": round(ms, 3),
+                     "bytes": int(b), "note": "7 LLaMA-2-7B layers, mean of %d calls each (eager launches)" % reps}
+    return out
+
+
 # ------------------------------------------------------------ GPU arm
 
 
@@ -392,6 +443,7 @@ def run_ours(args, rank, world):
         "gpu_launches": int(sum(launches_per_call[c] for c in calls) * args.steps),
         "clocks": clocks.summary(),
         "per_call": detail,
+        "offline": offline_steps(layers, dev, pk) if args.workload == "decode" and not args.layers else None,
     }
     return out
 

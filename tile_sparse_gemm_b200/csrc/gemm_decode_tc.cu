@@ -49,6 +49,7 @@ constexpr uint32_t META_COL0 = NACC * BT;
 constexpr uint32_t IDESC_DENSE = idesc_bf16(BM, BT, false);
 constexpr uint32_t IDESC_SPARSE = idesc_bf16(BM, BT, true);
 constexpr int WS_FLOATS_PER_CTA = 2 * BT * BM;  // [2 slots][16 tokens][128 rows]
+constexpr int DCAP = 1024;               // descriptors of the CTA's tiles staged in shared memory
 
 struct Shared {
   alignas(1024) uint8_t a[NA][A_BYTES];
@@ -56,9 +57,11 @@ struct Shared {
   alignas(128) uint8_t e[NE][E_BYTES];
   uint64_t a_full[NA], a_empty[NA], b_full[NB], b_empty[NB], e_full[NE], e_empty[NE];
   uint64_t acc_full[NACC], acc_empty[NACC], drain;
+  alignas(16) patch_tile_desc dcache[DCAP];  // tiles t_first .. t_last (when they fit)
   uint32_t tmem_base;
   int abort_flag;
   int t_first, t_last;  // tiles holding the CTA's first and last panel
+  int cached;           // dcache holds the CTA's tiles
 };
 constexpr size_t SMEM_BYTES = sizeof(Shared) + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -84,22 +87,30 @@ __device__ __forceinline__ int64_t panel_of(const patch_tile_desc& d) {
   return int64_t(d.val_offset / PATCH_PANEL_BYTES);
 }
 
-// Tile holding panel p: the last t with panel_of(desc[t]) <= p.
-__device__ int find_tile(const patch_tile_desc* desc, int T, int64_t p) {
-  int lo = 0, hi = T - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (panel_of(desc[mid]) <= p)
-      lo = mid;
-    else
-      hi = mid - 1;
+// Tiles holding panels pa and pb: the last t with panel_of(desc[t]) <= p.
+// Called by every thread of the block: each round probes blockDim.x tiles at
+// once and narrows the span by that factor, so a search costs a few global
+// latencies instead of log2(T) dependent ones.
+__device__ void find_tiles(const patch_tile_desc* desc, int T, int64_t pa, int64_t pb, int& ta, int& tb) {
+  const int n = blockDim.x, i = threadIdx.x;
+  int lo_a = 0, lo_b = 0, span = T;
+  while (span > 1) {
+    const int step = (span + n - 1) / n;
+    const int ia = lo_a + i * step, ib = lo_b + i * step;
+    const bool in = i * step < span;
+    const int ca = __syncthreads_count(in && ia < T && panel_of(desc[ia]) <= pa);
+    const int cb = __syncthreads_count(in && ib < T && panel_of(desc[ib]) <= pb);
+    lo_a += (ca - 1) * step;
+    lo_b += (cb - 1) * step;
+    span = step;
   }
-  return lo;
+  ta = lo_a;
+  tb = lo_b;
 }
 
-// First panel of tile row tn (P for tn == Tn).
-__device__ __forceinline__ int64_t row_begin(const Args& a, int tn) {
-  return tn < a.Tn ? panel_of(a.desc[int64_t(tn) * a.Tk]) : a.P;
+// Descriptor of tile t (staged in shared memory when the CTA's tiles fit).
+__device__ __forceinline__ patch_tile_desc tile_desc(const Shared& s, const Args& a, int t) {
+  return s.cached ? s.dcache[t - s.t_first] : a.desc[t];
 }
 
 __device__ __forceinline__ void advance(const patch_tile_desc& d, int& t, int& h) {
@@ -115,10 +126,10 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
                          int64_t p0, int64_t p1) {
   uint32_t a_i = 0, b_i = 0, e_i = 0;
   int t = s.t_first;
-  int h = p0 < p1 ? int(p0 - panel_of(a.desc[t])) : 0;
+  int h = p0 < p1 ? int(p0 - panel_of(tile_desc(s, a, t))) : 0;
   bool ok = true;
   for (int64_t p = p0; ok && p < p1; ++p) {
-    const patch_tile_desc d = a.desc[t];
+    const patch_tile_desc d = tile_desc(s, a, t);
     const int kt = t % a.Tk;
     if (d.kind) {
       const uint32_t es = e_i % NE;
@@ -156,12 +167,12 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
 __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& a, int64_t p0, int64_t p1) {
   uint32_t a_i = 0, b_i = 0, e_i = 0;
   int t = s.t_first;
-  int h = p0 < p1 ? int(p0 - panel_of(a.desc[t])) : 0;
+  int h = p0 < p1 ? int(p0 - panel_of(tile_desc(s, a, t))) : 0;
   int seg = -1, cur_tn = -1;
   uint32_t acc = tmem, accumulate = 0;
   bool ok = true;
   for (int64_t p = p0; ok && p < p1; ++p) {
-    const patch_tile_desc d = a.desc[t];
+    const patch_tile_desc d = tile_desc(s, a, t);
     const int tn = t / a.Tk;
     if (tn != cur_tn) {  // a new tile row starts a new accumulation segment
       ++seg;
@@ -244,8 +255,11 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, in
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.acc_empty[buf]);
     const int r = 32 * q + lane;
-    const int64_t rb = row_begin(a, tn), re = row_begin(a, tn + 1);
-    if (p0 <= rb && p1 >= re) {  // the whole row is ours
+    // does this CTA hold the row's first and last panel?
+    const patch_tile_desc df = tile_desc(s, a, s.t_first), dl = tile_desc(s, a, s.t_last);
+    const bool starts = tn > tn_first || (s.t_first % a.Tk == 0 && p0 == panel_of(df));
+    const bool ends = tn < tn_last || (s.t_last % a.Tk == a.Tk - 1 && p1 == panel_of(dl) + (dl.kind ? 1 : 2));
+    if (starts && ends) {  // the whole row is ours
       const int64_t n = int64_t(tn) * BM + r;
 #pragma unroll
       for (int m = 0; m < BT; ++m)
@@ -287,12 +301,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
-    const int T = a.Tn * a.Tk;
-    s.t_first = p0 < p1 ? find_tile(a.desc, T, p0) : 0;
-    s.t_last = p0 < p1 ? find_tile(a.desc, T, p1 - 1) : 0;
     fence_barrier_init();
     prefetch_tensormap(&tmap_x);
     prefetch_tensormap(&tmap_w);
+  }
+  // locate the CTA's first and last tile, then stage their descriptors
+  if (p0 < p1) {
+    int ta, tb;
+    find_tiles(a.desc, a.Tn * a.Tk, p0, p1 - 1, ta, tb);
+    const int count = tb - ta + 1;
+    if (threadIdx.x == 0) {
+      s.t_first = ta;
+      s.t_last = tb;
+      s.cached = count <= DCAP;
+    }
+    if (count <= DCAP)
+      for (int i = threadIdx.x; i < count; i += blockDim.x) s.dcache[i] = a.desc[ta + i];
+  } else if (threadIdx.x == 0) {
+    s.t_first = s.t_last = 0;
+    s.cached = 0;
   }
   if (warp == 1) tmem_alloc(&s.tmem_base, TMEM_COLS);
   tc_fence_before();

@@ -24,7 +24,9 @@
 //           logical); tcgen05.commit releases ring slots and, per output tile,
 //           signals the epilogue.
 //   warps 2-5 epilogue: tcgen05.ld of the 128 x BT fp32 accumulator, one
-//           round to bf16 (nearest even), stores to Y[m][n].
+//           round to bf16 (nearest even), stores to Y[m][n]; two TMEM
+//           accumulators let it drain one output tile while the MMAs of the
+//           next one run.
 // Every mbarrier wait is bounded in time; when one runs out the kernel sets
 // PATCH_DEV_TIMEOUT, the other roles stop at their next wait, the producer
 // waits for its copies in flight, the MMA thread for its MMAs, and TMEM is
@@ -41,16 +43,20 @@ namespace prefill {
 using namespace tc;
 
 constexpr int BM = 128;                  // W rows per output tile (MMA M)
-constexpr int BT = 256;                  // tokens per output tile (MMA N)
-constexpr int NA = 4;                    // A ring: W panels of 128 x 64 bf16
+constexpr int BT = 240;                  // tokens per output tile (MMA N; 2 x 240 + metadata fit TMEM)
+constexpr int NA = 5;                    // A ring: W panels of 128 x 64 bf16
 constexpr int NB = 4;                    // B ring: X panels of BT x 64 bf16
 constexpr int NE = 4;                    // metadata ring
 constexpr int A_BYTES = PATCH_PANEL_BYTES;
 constexpr int B_BYTES = BT * 64 * 2;
 constexpr int E_BYTES = PATCH_META_TILE_BYTES;
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 512;      // accumulator [0, BT) + metadata slots
+constexpr int MAXTK = 256;               // descriptors of one tile row staged in shared memory
+constexpr int NACC = 2;                  // accumulators: the epilogue of one tile overlaps the next
+constexpr uint32_t TMEM_COLS = 512;      // accumulators at columns 0 and 256, metadata slots at BT..
+constexpr uint32_t ACC_STRIDE = 256;
 constexpr uint32_t META_COL0 = BT;
+static_assert(META_COL0 + 4 * 4 <= ACC_STRIDE && ACC_STRIDE + BT <= TMEM_COLS, "TMEM layout");
 
 constexpr uint32_t IDESC_DENSE = tc::idesc_bf16(BM, BT, false);
 constexpr uint32_t IDESC_SPARSE = tc::idesc_bf16(BM, BT, true);
@@ -60,7 +66,10 @@ struct Shared {
   alignas(1024) uint8_t b[NB][B_BYTES];
   alignas(128) uint8_t e[NE][E_BYTES];
   uint64_t a_full[NA], a_empty[NA], b_full[NB], b_empty[NB], e_full[NE], e_empty[NE];
-  uint64_t acc_full, acc_empty, drain;
+  uint64_t acc_full[NACC], acc_empty[NACC], drain;
+  uint64_t pdesc_full[2];             // descriptor rows, bulk-copied by the producer
+  alignas(16) patch_tile_desc pdesc[2][MAXTK];
+  uint32_t a_kind[NA];                // tile kind of the panel in each A slot (producer -> MMA)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -79,18 +88,46 @@ struct Args {
   int inject;  // 1: producer stops after the first K-tile (exercises the timeout path)
 };
 
+// Descriptor of tile (tn, kt): from the staged row when it fits, else from global memory.
+__device__ __forceinline__ patch_tile_desc row_desc(const Shared& s, const Args& p, bool staged, int buf, int tn,
+                                                    int kt) {
+  return staged ? s.pdesc[buf][kt] : p.desc[int64_t(tn) * p.Tk + kt];
+}
+
 __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap* tmap_w, const Args& p) {
   const int Tn = p.N / BM;
-  uint32_t a_i = 0, b_i = 0, e_i = 0;  // loads issued per ring
+  const bool staged = p.Tk <= MAXTK;
+  uint32_t a_i = 0, b_i = 0, e_i = 0, d_i = 0;  // loads issued per ring / descriptor rows staged
   bool ok = true;
-  for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+  // stage the first item's descriptor row
+  if (staged && int(blockIdx.x) < p.n_items) {
+    const int tn0 = int(blockIdx.x) % Tn;
+    mbar_expect_tx(&s.pdesc_full[0], uint32_t(p.Tk * sizeof(patch_tile_desc)));
+    bulk_load(s.pdesc[0], p.desc + int64_t(tn0) * p.Tk, uint32_t(p.Tk * sizeof(patch_tile_desc)), &s.pdesc_full[0]);
+    ++d_i;
+  }
+  int it = 0;
+  for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
     const int tn = item % Tn, tb = item / Tn;
+    const int buf = it & 1;
+    if (staged) {
+      if (!(ok = wait_bounded(&s.pdesc_full[buf], (it >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
+        break;
+      // prefetch the next item's row into the other buffer (its previous row is done)
+      const int next = item + gridDim.x;
+      if (next < p.n_items) {
+        mbar_expect_tx(&s.pdesc_full[buf ^ 1], uint32_t(p.Tk * sizeof(patch_tile_desc)));
+        bulk_load(s.pdesc[buf ^ 1], p.desc + int64_t(next % Tn) * p.Tk, uint32_t(p.Tk * sizeof(patch_tile_desc)),
+                  &s.pdesc_full[buf ^ 1]);
+        ++d_i;
+      }
+    }
     for (int kt = 0; ok && kt < p.Tk; ++kt) {
       if (p.inject && (item != int(blockIdx.x) || kt > 0)) {
         ok = false;
         break;
       }
-      const patch_tile_desc d = p.desc[int64_t(tn) * p.Tk + kt];
+      const patch_tile_desc d = row_desc(s, p, staged, buf, tn, kt);
       const int panel = int(d.val_offset / A_BYTES);
       if (d.kind) {
         const uint32_t es = e_i % NE;
@@ -105,6 +142,7 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
           const uint32_t as = a_i % NA;
           if (!(ok = wait_bounded(&s.a_empty[as], ((a_i / NA) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
             break;
+          s.a_kind[as] = d.kind;  // published to the MMA thread by the barrier's release
           mbar_expect_tx(&s.a_full[as], A_BYTES);
           tma_load_2d(s.a[as], tmap_w, &s.a_full[as], 0, (panel + h) * 128);
           ++a_i;
@@ -125,24 +163,29 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
     wait_bounded(&s.b_full[i % NB], (i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, true);
   for (uint32_t i = (e_i > NE ? e_i - NE : 0); i < e_i; ++i)
     wait_bounded(&s.e_full[i % NE], (i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+  for (uint32_t i = (d_i > 2 ? d_i - 2 : 0); i < d_i; ++i)
+    wait_bounded(&s.pdesc_full[i & 1], (i >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, true);
 }
 
 __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
-  const int Tn = p.N / BM;
   uint32_t a_i = 0, b_i = 0, e_i = 0;
   bool ok = true;
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const int tn = item % Tn;
-    if (!(ok = wait_bounded(&s.acc_empty, (it & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+    const int buf = it % NACC;
+    if (!(ok = wait_bounded(&s.acc_empty[buf], ((it / NACC) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
+      break;
     tc_fence_after();
+    const uint32_t acc = tmem + ACC_STRIDE * buf;
     uint32_t accumulate = 0;
     for (int kt = 0; ok && kt < p.Tk; ++kt) {
-      const patch_tile_desc d = p.desc[int64_t(tn) * p.Tk + kt];
-      if (d.kind) {
-        const uint32_t es = e_i % NE, as = a_i % NA;
+      // the tile's kind arrives with its first A panel
+      uint32_t as = a_i % NA;
+      if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+      const uint32_t kind = *reinterpret_cast<volatile uint32_t*>(&s.a_kind[as]);
+      if (kind) {
+        const uint32_t es = e_i % NE;
         if (!(ok = wait_bounded(&s.e_full[es], (e_i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
-        if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
         tc_fence_after();
         const uint32_t e_tmem = tmem + META_COL0 + 4 * es;
         tmem_cp_128x128b(e_tmem, meta_desc(smem_u32(s.e[es])));
@@ -155,7 +198,7 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const uint32_t kb = 2 * h + j;  // 32-k block of the tile: 16 kept values = 32 B of A
-            mma_sparse(tmem, a0 + (kb * 32 >> 4), b0 + (j * 64 >> 4), e_tmem + (kb & 2u),
+            mma_sparse(acc, a0 + (kb * 32 >> 4), b0 + (j * 64 >> 4), e_tmem + (kb & 2u),
                        IDESC_SPARSE | (kb & 1u), accumulate);
             accumulate = 1;
           }
@@ -169,15 +212,18 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
         ++e_i;
       } else {
         for (int h = 0; h < 2; ++h) {
-          const uint32_t as = a_i % NA, bs = b_i % NB;
-          if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+          as = a_i % NA;
+          const uint32_t bs = b_i % NB;
+          if (h == 1 &&
+              !(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
+            break;
           if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
           tc_fence_after();
           const uint64_t a0 = sw128_desc(smem_u32(s.a[as]));
           const uint64_t b0 = sw128_desc(smem_u32(s.b[bs]));
 #pragma unroll
           for (int j = 0; j < 4; ++j) {  // K = 16 per MMA = 32 B along the swizzled row
-            mma_dense(tmem, a0 + (j * 32 >> 4), b0 + (j * 32 >> 4), IDESC_DENSE, accumulate);
+            mma_dense(acc, a0 + (j * 32 >> 4), b0 + (j * 32 >> 4), IDESC_DENSE, accumulate);
             accumulate = 1;
           }
           tc_commit(&s.a_empty[as]);
@@ -187,7 +233,7 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
         }
       }
     }
-    if (ok) tc_commit(&s.acc_full);
+    if (ok) tc_commit(&s.acc_full[buf]);
   }
   // all MMAs and copies issued must be complete before TMEM is freed
   tc_commit(&s.drain);
@@ -201,23 +247,25 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
     const int tn = item % Tn, tb = item / Tn;
-    if (!wait_bounded(&s.acc_full, it & 1, &s.abort_flag, p.limit_ns, p.status, false)) break;
+    const int buf = it % NACC;
+    if (!wait_bounded(&s.acc_full[buf], (it / NACC) & 1, &s.abort_flag, p.limit_ns, p.status, false)) break;
     tc_fence_after();
     const int64_t n = int64_t(tn) * BM + 32 * q + lane;
     const int m0 = tb * BT;
-    for (int c = 0; c < BT / 32; ++c) {
-      if (m0 + 32 * c >= p.M) break;  // warp-uniform
-      uint32_t v[32];
-      tmem_ld_32cols(tmem + (uint32_t(32 * q) << 16) + uint32_t(32 * c), v);
+    const uint32_t acc = tmem + (uint32_t(32 * q) << 16) + ACC_STRIDE * buf;
+    for (int c = 0; c < BT / 16; ++c) {
+      if (m0 + 16 * c >= p.M) break;  // warp-uniform
+      uint32_t v[16];
+      tmem_ld_16cols(acc + uint32_t(16 * c), v);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int m = m0 + 32 * c + j;
+      for (int j = 0; j < 16; ++j) {
+        const int m = m0 + 16 * c + j;
         if (m < p.M) p.Y[int64_t(m) * p.N + n] = f32_to_bf16_rne(__uint_as_float(v[j]));
       }
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.acc_empty);
+    if (lane == 0) mbar_arrive(&s.acc_empty[buf]);
   }
 }
 
@@ -241,9 +289,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&s.e_full[i], 1);
       mbar_init(&s.e_empty[i], 1);
     }
-    mbar_init(&s.acc_full, 1);
-    mbar_init(&s.acc_empty, 4);
+    for (int i = 0; i < NACC; ++i) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 4);
+    }
     mbar_init(&s.drain, 1);
+    mbar_init(&s.pdesc_full[0], 1);
+    mbar_init(&s.pdesc_full[1], 1);
     s.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
