@@ -185,11 +185,16 @@ PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight
  *   X  bf16 [M][K] (16-byte aligned, M >= 0; M == 0 is a no-op)
  *   W  packed weight (host struct)
  *   Y  bf16 [M][N] (16-byte aligned)
- *   workspace: patch_gemm_workspace_size bytes (may be NULL when that is 0)
+ *   workspace: patch_gemm_workspace_size bytes (may be NULL when that is 0).
+ *     It must be zero-filled before its first use; every successful call
+ *     leaves it zero-filled again (the decode path keeps per-row arrival
+ *     counters there), so one zero-fill at allocation suffices.  After a call
+ *     that reported an error, zero it again.
  * M <= 16 runs the decode path: one CTA per SM streams an equal share of
  * the stored panels through a TMA ring (stream-K), the tensor cores reduce
- * them (N = 16 tokens, zero-padded), tile rows cut between CTAs are summed
- * by a second kernel in a fixed order from fp32 partials in the workspace.
+ * them (N = 16 tokens, zero-padded); a tile row cut between CTAs is finished
+ * by the last CTA to reach it, which adds the fp32 partials in the
+ * workspace in CTA order (deterministic).
  * Larger M runs the prefill path (TMA-fed tcgen05 kernel, dense and sparse
  * MMAs into one TMEM fp32 tile per 128 x 256 output tile).
  * A bounded wait that runs out sets PATCH_DEV_TIMEOUT (Y is then undefined).

@@ -268,6 +268,21 @@ def test_gemm_all_sparse_equals_24_and_all_dense_equals_dense():
                 check_gemm(y, torch_ref, f"prefill f={frac}")
 
 
+def test_decode_workspace_reused_across_calls():
+    """The decode path leaves its workspace zero-filled, so back-to-back calls on
+    one workspace keep finishing the rows cut between CTAs."""
+    x, w, bm, ids = _layer(4864, 896, 16, "clustered", 0.5, cfg=12, shape_idx=5)
+    pw = pack_on_gpu(w, bm, ids)
+    ws = torch.zeros(tsg.patch_gemm_workspace_size(16, pw), dtype=torch.uint8, device="cuda")
+    ref = oracle.hybrid_gemm(x, w, bm, ids)
+    xd = to_dev_bf16(x)
+    for it in range(4):
+        status = tsg.new_status()
+        y = tsg.patch_gemm(xd[: 16 - it], pw, workspace=ws, status=status)
+        assert tsg.patch_read_status(status)[0] == 0
+        check_gemm(bits_of(y), ref[: 16 - it], f"call {it}")
+
+
 def test_gemm_zero_tokens_is_noop():
     x, w, bm, ids = _layer(256, 256, 4, "exact", 0.5)
     pw = pack_on_gpu(w, bm, ids)

@@ -195,7 +195,7 @@ def patch_gemm_ex(X: torch.Tensor, weight: PackedWeight, Y: torch.Tensor | None 
     st = weight.struct()
     if workspace is None:
         need = patch_gemm_workspace_size(M, weight) if (path & 0xFF) != PATH_PREFILL else 0
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)  # must start zero-filled
     _check(lib().patch_gemm_ex(_dev(X, "X"), M, ctypes.byref(st), _dev(Y, "Y"), _dev(workspace, "workspace"),
                                workspace.numel(), _dev(status, "status"), _stream(stream), path, wait_limit_us),
            "patch_gemm")

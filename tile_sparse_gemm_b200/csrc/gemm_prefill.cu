@@ -122,8 +122,13 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
         ++d_i;
       }
     }
-    for (int kt = 0; ok && kt < p.Tk; ++kt) {
-      if (p.inject && (item != int(blockIdx.x) || kt > 0)) {
+    // CTAs that share an X block (same tb) or a W tile row (same tn) start
+    // their K loop at different tiles, so they do not all hit the same L2 lines
+    // at the same moment; the sum order is the only thing that changes
+    const int rot = (tn + 7 * tb) % p.Tk;
+    for (int j = 0; ok && j < p.Tk; ++j) {
+      const int kt = (j + rot) % p.Tk;
+      if (p.inject && (item != int(blockIdx.x) || j > 0)) {
         ok = false;
         break;
       }

@@ -42,8 +42,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // limit_ns (the CTA's shared abort flag is then set and PATCH_DEV_TIMEOUT
 // raised) or, unless `drain` is set, when another role of the CTA aborted
 // first.  Spins are bounded by time, never unbounded.
-static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, int* abort_flag_smem,
-                                          uint64_t limit_ns, int32_t* status, bool drain) {
+static __device__ __noinline__ bool wait_bounded_slow(uint64_t* bar, uint32_t parity, int* abort_flag_smem,
+                                               uint64_t limit_ns, int32_t* status, bool drain) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -59,6 +59,13 @@ static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
       }
     }
   }
+}
+
+// Inline fast path: one try_wait, then the bounded slow loop if needed.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, int* abort_flag_smem, uint64_t limit_ns,
+                                             int32_t* status, bool drain) {
+  if (mbar_try_wait(smem_u32(bar), parity)) return true;
+  return wait_bounded_slow(bar, parity, abort_flag_smem, limit_ns, status, drain);
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
