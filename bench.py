@@ -312,22 +312,28 @@ def run_ours(args, rank, world):
         raise RuntimeError(f"device status {code} bits {bits} after warm-up")
 
     # The K timed steps are captured once as one CUDA graph (launch-bound small
-    # kernels), with an event pair around every call; one replay is the timed region.
-    # external events become event-record nodes when captured, so they keep their timestamps
-    ev = [[(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-           for _ in calls] for _ in range(args.steps)]
-    graph = None
-    if not args.no_graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+    # kernels); one replay is the timed region.  A second graph of the same steps
+    # with an (external) event pair around every call gives the per-call split;
+    # event nodes add a few microseconds each, so it is not used for the totals.
+    def capture(with_events):
+        g = torch.cuda.CUDAGraph()
+        evs = [[(torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True)) for _ in calls]
+               for _ in range(args.steps)] if with_events else None
+        with torch.cuda.graph(g):
             cap = torch.cuda.current_stream()
             for st in range(args.steps):
                 for j, (li, M) in enumerate(calls):
-                    ev[st][j][0].record(cap)
+                    if evs:
+                        evs[st][j][0].record(cap)
                     tsg.patch_gemm(xs[(li, M)], packed[li], Y=ys[(li, M)], workspace=ws, status=status)
-                    ev[st][j][1].record(cap)
-        graph.replay()  # untimed: first replay uploads the graph
+                    if evs:
+                        evs[st][j][1].record(cap)
+        g.replay()  # untimed: the first replay uploads the graph
         torch.cuda.synchronize()
+        return g, evs
+
+    graph = None if args.no_graph else capture(False)[0]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clocks:
         clocks.wait_first_sample()
@@ -339,20 +345,26 @@ def run_ours(args, rank, world):
             graph.replay()
         else:
             for st in range(args.steps):
-                step(ev[st])
+                step()
         t_end.record(stream)
         torch.cuda.synchronize()
         clocks.mark("end")
         barrier()
     ms = t_start.elapsed_time(t_end)
-    try:
-        call_ms = np.array([[a.elapsed_time(b) for a, b in ev[st]] for st in range(args.steps)])  # [steps][calls]
-    except RuntimeError:  # no per-call timestamps: attribute the step time to the calls by bytes/FLOPs
-        call_ms = None
+    del graph
+    call_ms = None
+    if not args.no_graph:
+        g_ev, ev = capture(True)
+        g_ev.replay()
+        torch.cuda.synchronize()
+        try:
+            call_ms = np.array([[a.elapsed_time(b) for a, b in ev[st]] for st in range(args.steps)])
+        except RuntimeError:
+            call_ms = None
+        del g_ev
     code, bits = tsg.patch_read_status(status)
     if code != 0:
         raise RuntimeError(f"device status {code} bits {bits} after timing")
-    del graph
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     xh = {c: xs[c].cpu().pin_memory() for c in calls}
@@ -393,13 +405,18 @@ def run_ours(args, rank, world):
     value = per_step * args.steps * world / (ms / 1e3)
     e2e_value = per_step * args.steps * world / (e2e_ms / 1e3)
 
-    # roofline of the dominant kernel: algorithmic bytes (or FLOPs) per launch / mean launch time
+    # roofline of the dominant kernel: algorithmic bytes (or FLOPs) per launch / mean launch time.
+    # Every call of the step is one launch of that kernel, so the mean over the
+    # timed region is the step's bytes (FLOPs) over the step's time; the per-call
+    # split below comes from the event-instrumented graph.
+    w_ = np.array([call_bytes(layers[li], M) if args.workload == "decode" else call_flops(layers[li], M)
+                   for li, M in calls], dtype=np.float64)
+    step_ms = ms / args.steps
     if call_ms is None:
-        w_ = np.array([call_bytes(layers[li], M) if args.workload == "decode" else call_flops(layers[li], M)
-                       for li, M in calls], dtype=np.float64)
-        mean_call_ms = (ms / args.steps) * w_ / w_.sum()
+        split_ms = step_ms * w_ / w_.sum()
     else:
-        mean_call_ms = call_ms.mean(axis=0)
+        split_ms = call_ms.mean(axis=0)
+    mean_call_ms = split_ms * (step_ms / split_ms.sum())  # scaled to the event-free step time
     if args.workload == "decode":
         alg = np.array([call_bytes(layers[li], M) for li, M in calls]) / 1e9
         achieved = float(alg.sum() / (mean_call_ms.sum() / 1e3))
@@ -444,6 +461,7 @@ def run_ours(args, rank, world):
         "gpu_launches": int(sum(launches_per_call[c] for c in calls) * args.steps),
         "clocks": clocks.summary(),
         "per_call": detail,
+        "per_call_note": "split of the event-free step time in proportion to an event-instrumented replay",
         "offline": offline_steps(layers, dev, pk) if args.workload == "decode" and not (args.layers or args.fracs) else None,
     }
     return out

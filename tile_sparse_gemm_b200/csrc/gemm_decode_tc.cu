@@ -14,11 +14,11 @@
 // Inside its range a CTA accumulates each tile row's panels into a TMEM
 // accumulator (M = 128 rows of W, N = 16 tokens, zero-padded by TMA).  A
 // tile row entirely inside one CTA's range is rounded to bf16 and stored
-// directly.  A row cut by range boundaries is finished by whichever
-// epilogue warp of the covering CTAs arrives last: every warp stores its fp32
-// partial sums in the workspace and bumps the row's arrival counter; the
-// last one adds all partials in CTA order (deterministic), stores Y and
-// resets the counter to zero for the next call.
+// directly.  A row cut by range boundaries is finished, per 32-row quarter,
+// by whichever covering CTA's epilogue warp arrives last: every warp stores
+// its fp32 partial sums in the workspace and bumps the quarter's arrival
+// counter; the last one adds all partials in CTA order (deterministic),
+// stores Y and resets the counter to zero for the next call.
 //
 // One pipeline stage per panel holds the 16 KiB weight panel, the 64-k
 // slices of X it multiplies (1 for a dense panel, 2 for a sparse one) and,
@@ -73,6 +73,8 @@ struct Shared {
   int abort_flag;
   int t_first, t_last;  // tiles holding the CTA's first and last panel
   int cached;           // dcache holds the CTA's tiles
+  int64_t row_lo[2];    // first panel of the CTA's first row, and of the row after it
+  int64_t row_hi[2];    // first panel of the CTA's last row, and of the row after it
 };
 constexpr size_t SMEM_BYTES = sizeof(Shared) + 1024;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -82,7 +84,7 @@ struct Args {
   const uint8_t* meta;
   uint16_t* Y;
   float* ws;           // [G][2][16][128] fp32 partials
-  uint32_t* counters;  // [Tn] arrivals per tile row (zero between calls)
+  uint32_t* counters;  // [Tn][4] arrivals per tile row and TMEM lane quarter (zero between calls)
   int M, N, Tk, Tn;
   int64_t P;  // panels in the values blob
   uint64_t limit_ns;
@@ -125,6 +127,21 @@ __device__ __forceinline__ patch_tile_desc tile_desc(const Shared& s, const Args
   return s.cached ? s.dcache[t - s.t_first] : a.desc[t];
 }
 
+// X slice loads of one stage (after the previous kernel in the stream is done)
+__device__ __forceinline__ void load_x(Stage& g, uint64_t* full, const CUtensorMap* tmap_x, uint32_t xinfo) {
+  const int kt = int(xinfo >> 2), h = int((xinfo >> 1) & 1);
+  if (xinfo & 1) {
+    tma_load_2d(g.x[0], tmap_x, full, kt * kTile, 0);
+    tma_load_2d(g.x[1], tmap_x, full, kt * kTile + 64, 0);
+  } else {
+    tma_load_2d(g.x[0], tmap_x, full, kt * kTile + 64 * h, 0);
+  }
+}
+
+// The weight panels (and metadata) of the first NS stages are requested
+// before this kernel waits for the previous kernel in the stream (they do
+// not depend on it); the X slices of those stages, which may be that
+// kernel's output, are requested once it has completed.
 __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap* tmap_w, const Args& a,
                          int64_t p0, int64_t p1) {
   int t = s.t_first;
@@ -132,8 +149,19 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
   int h = int(p0 - panel_of(d));
   int kt = t % a.Tk;
   uint32_t i = 0;
+  bool waited = false;
+  uint32_t deferred[NS];
+  auto release_deferred = [&]() {
+    pdl_wait_previous();
+    waited = true;
+    const uint32_t n = i < NS ? i : NS;
+#pragma unroll
+    for (uint32_t j = 0; j < NS; ++j)
+      if (j < n) load_x(s.st[j], &s.full[j], tmap_x, deferred[j]);
+  };
   for (int64_t p = p0; p < p1; ++p, ++i) {
     const uint32_t st = i % NS;
+    if (i == NS && !waited) release_deferred();  // stage 0 must be consumable before it is reused
     if (!wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false)) break;
     const bool sparse = d.kind != 0;
     const bool last_panel_of_tile = sparse || h == 1;
@@ -144,13 +172,12 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
     Stage& g = s.st[st];
     mbar_expect_tx(&s.full[st], A_BYTES + (sparse ? 2 * X_BYTES + E_BYTES : X_BYTES));
     tma_load_2d(g.a, tmap_w, &s.full[st], 0, int(p * 128));
-    if (sparse) {
-      tma_load_2d(g.x[0], tmap_x, &s.full[st], kt * kTile, 0);
-      tma_load_2d(g.x[1], tmap_x, &s.full[st], kt * kTile + 64, 0);
-      bulk_load(g.e, a.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.full[st]);
-    } else {
-      tma_load_2d(g.x[0], tmap_x, &s.full[st], kt * kTile + 64 * h, 0);
-    }
+    if (sparse) bulk_load(g.e, a.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.full[st]);
+    const uint32_t xinfo = uint32_t(kt) << 2 | uint32_t(h) << 1 | (sparse ? 1u : 0u);
+#pragma unroll
+    for (uint32_t j = 0; j < NS; ++j)
+      if (!waited && j == i) deferred[j] = xinfo;
+    if (waited) load_x(g, &s.full[st], tmap_x, xinfo);
     // next panel: second half of a dense tile, or the next tile
     if (last_panel_of_tile) {
       h = 0;
@@ -161,6 +188,7 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
       h = 1;
     }
   }
+  if (!waited) release_deferred();
   // every copy issued must have landed before the CTA may exit
   for (uint32_t j = (i > NS ? i - NS : 0); j < i; ++j)
     wait_bounded(&s.full[j % NS], (j / NS) & 1, &s.abort_flag, a.limit_ns, a.status, true);
@@ -235,41 +263,38 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, in
         if (m < a.M) a.Y[int64_t(m) * a.N + n] = f32_to_bf16_rne(__uint_as_float(v[m]));
       continue;
     }
-    // A cut row: publish this warp's 32 rows of partial sums, then count the
-    // arrival of the warp; the last of the row's 4 x (covering CTAs) warps to
-    // arrive adds up every partial (in CTA order) and finishes the row.
+    // A cut row: publish this warp's 32 rows (its TMEM lane quarter q) of
+    // partial sums and count the arrival; the last covering CTA to arrive for
+    // quarter q adds up that quarter's partials (in CTA order) and stores them.
     float* mine = a.ws + int64_t(blockIdx.x) * WS_FLOATS_PER_CTA + (tn == tn_first ? 0 : BT * BM);
 #pragma unroll
     for (int m = 0; m < BT; ++m)
       if (m < a.M) mine[m * BM + r] = __uint_as_float(v[m]);
-    const int64_t rb = panel_of(a.desc[int64_t(tn) * a.Tk]);
-    const int64_t re = tn + 1 < a.Tn ? panel_of(a.desc[int64_t(tn + 1) * a.Tk]) : a.P;
+    const int64_t rb = tn == tn_first ? s.row_lo[0] : s.row_hi[0];
+    const int64_t re = tn == tn_first ? s.row_lo[1] : s.row_hi[1];
     const int64_t c_lo = cta_of_panel(rb, a.P, G), c_hi = cta_of_panel(re - 1, a.P, G);
     __threadfence();
     __syncwarp();
     uint32_t old = 0;
-    if (lane == 0) old = atomicAdd(&a.counters[tn], 1u);
+    if (lane == 0) old = atomicAdd(&a.counters[4 * tn + q], 1u);
     old = __shfl_sync(0xFFFFFFFFu, old, 0);
-    if (old != uint32_t(4 * (c_hi - c_lo + 1) - 1)) continue;
+    if (old != uint32_t(c_hi - c_lo)) continue;
     __threadfence();
-    for (int rr = lane; rr < BM; rr += 32) {
-      float sum[BT];
+    float sum[BT];
 #pragma unroll
-      for (int m = 0; m < BT; ++m) sum[m] = 0.0f;
-      for (int64_t c = c_lo; c <= c_hi; ++c) {
-        // only the first covering CTA can have started before the row (its "last row" slot)
-        const int slot = (c == c_lo && range_begin(c, a.P, G) < rb) ? 1 : 0;
-        const float* src = a.ws + c * WS_FLOATS_PER_CTA + slot * BT * BM;
-#pragma unroll
-        for (int m = 0; m < BT; ++m)
-          if (m < a.M) sum[m] += __ldcg(src + m * BM + rr);
-      }
-      const int64_t nn = int64_t(tn) * BM + rr;
+    for (int m = 0; m < BT; ++m) sum[m] = 0.0f;
+    for (int64_t c = c_lo; c <= c_hi; ++c) {
+      // only the first covering CTA can have started before the row (its "last row" slot)
+      const int slot = (c == c_lo && range_begin(c, a.P, G) < rb) ? 1 : 0;
+      const float* src = a.ws + c * WS_FLOATS_PER_CTA + slot * BT * BM + r;
 #pragma unroll
       for (int m = 0; m < BT; ++m)
-        if (m < a.M) a.Y[int64_t(m) * a.N + nn] = f32_to_bf16_rne(sum[m]);
+        if (m < a.M) sum[m] += __ldcg(src + m * BM);
     }
-    if (lane == 0) a.counters[tn] = 0;  // ready for the next call
+#pragma unroll
+    for (int m = 0; m < BT; ++m)
+      if (m < a.M) a.Y[int64_t(m) * a.N + n] = f32_to_bf16_rne(sum[m]);
+    if (lane == 0) a.counters[4 * tn + q] = 0;  // ready for the next call
   }
 }
 
@@ -281,6 +306,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t G = gridDim.x;
   const int64_t p0 = range_begin(blockIdx.x, a.P, G), p1 = range_begin(blockIdx.x + 1, a.P, G);
+  pdl_launch_dependents();  // the next kernel may run its prologue as our CTAs finish
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -309,6 +335,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (count <= DCAP)
     for (int i = threadIdx.x; i < count; i += blockDim.x) s.dcache[i] = a.desc[ta + i];
+  // tile-row boundaries the epilogue needs for rows cut by this CTA's range
+  if (threadIdx.x < 4) {
+    const int tn = (threadIdx.x < 2 ? ta : tb) / a.Tk + (threadIdx.x & 1);
+    const int64_t v = tn < a.Tn ? panel_of(a.desc[int64_t(tn) * a.Tk]) : a.P;
+    if (threadIdx.x < 2)
+      s.row_lo[threadIdx.x] = v;
+    else
+      s.row_hi[threadIdx.x - 2] = v;
+  }
   if (warp == 1) tmem_alloc(&s.tmem_base, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -345,7 +380,7 @@ static Plan plan(const patch_weight& W, int num_sms) {
   p.P = 2 * (T - W.n_sparse) + W.n_sparse;
   p.G = p.P < num_sms ? p.P : num_sms;
   p.ws_floats_bytes = size_t(p.G) * WS_FLOATS_PER_CTA * sizeof(float);
-  p.counter_bytes = (size_t(p.Tn) * sizeof(uint32_t) + 255) & ~size_t(255);
+  p.counter_bytes = (size_t(p.Tn) * 4 * sizeof(uint32_t) + 255) & ~size_t(255);
   return p;
 }
 
@@ -379,8 +414,7 @@ cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W
   a.status = status;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES));
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<<<int(pl.G), THREADS, SMEM_BYTES, stream>>>(tmap_x, tmap_w, a);
-  return cudaGetLastError();
+  return launch_pdl(decode_tc_kernel, dim3(unsigned(pl.G)), dim3(THREADS), SMEM_BYTES, stream, tmap_x, tmap_w, a);
 }
 
 }  // namespace patch

@@ -98,7 +98,7 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
   const int Tn = p.N / BM;
   const bool staged = p.Tk <= MAXTK;
   uint32_t a_i = 0, b_i = 0, e_i = 0, d_i = 0;  // loads issued per ring / descriptor rows staged
-  bool ok = true;
+  bool ok = true, waited = false;
   // stage the first item's descriptor row
   if (staged && int(blockIdx.x) < p.n_items) {
     const int tn0 = int(blockIdx.x) % Tn;
@@ -142,16 +142,22 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
         ++e_i;
       }
       const int n_a = d.kind ? 1 : 2;
+      for (int h = 0; h < n_a; ++h) {
+        const uint32_t as = a_i % NA;
+        if (!(ok = wait_bounded(&s.a_empty[as], ((a_i / NA) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
+          break;
+        s.a_kind[as] = d.kind;  // published to the MMA thread by the barrier's release
+        mbar_expect_tx(&s.a_full[as], A_BYTES);
+        tma_load_2d(s.a[as], tmap_w, &s.a_full[as], 0, (panel + h) * 128);
+        ++a_i;
+      }
+      if (!ok) break;
+      // X may be the previous kernel's output: wait for it before the first X load
+      if (!waited) {
+        pdl_wait_previous();
+        waited = true;
+      }
       for (int h = 0; h < 2; ++h) {
-        if (h < n_a) {
-          const uint32_t as = a_i % NA;
-          if (!(ok = wait_bounded(&s.a_empty[as], ((a_i / NA) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
-            break;
-          s.a_kind[as] = d.kind;  // published to the MMA thread by the barrier's release
-          mbar_expect_tx(&s.a_full[as], A_BYTES);
-          tma_load_2d(s.a[as], tmap_w, &s.a_full[as], 0, (panel + h) * 128);
-          ++a_i;
-        }
         const uint32_t bs = b_i % NB;
         if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
           break;
@@ -280,6 +286,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   Shared& s = *reinterpret_cast<Shared*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();  // the next kernel may run its prologue as our CTAs finish
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NA; ++i) {
@@ -395,8 +402,7 @@ cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, 
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES));
   if (e != cudaSuccess) return e;
-  prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmap_x, tmap_w, p);
-  return cudaGetLastError();
+  return launch_pdl(prefill_kernel, dim3(unsigned(grid)), dim3(THREADS), SMEM_BYTES, stream, tmap_x, tmap_w, p);
 }
 
 }  // namespace patch
