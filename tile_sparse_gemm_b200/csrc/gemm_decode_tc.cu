@@ -40,7 +40,7 @@ using namespace tc;
 
 constexpr int BM = 128;
 constexpr int BT = 16;                   // MMA N (tokens)
-constexpr int NS = 9;                    // pipeline stages (panels in flight per SM)
+constexpr int NS = 4;                    // pipeline stages per CTA (2 CTAs per SM: ~8 panels in flight)
 constexpr int NACC = 2;                  // accumulator buffers (epilogue overlaps the next row)
 constexpr int A_BYTES = PATCH_PANEL_BYTES;
 constexpr int X_BYTES = BT * 64 * 2;     // one 64-k slice of X (16 token rows)
@@ -52,7 +52,7 @@ static_assert(META_COL0 + 4 * NS <= TMEM_COLS, "TMEM layout");
 constexpr uint32_t IDESC_DENSE = idesc_bf16(BM, BT, false);
 constexpr uint32_t IDESC_SPARSE = idesc_bf16(BM, BT, true);
 constexpr int WS_FLOATS_PER_CTA = 2 * BT * BM;  // [2 slots][16 tokens][128 rows]
-constexpr int DCAP = 1024;                      // descriptors of the CTA's tiles staged in shared memory
+constexpr int DCAP = 256;                       // descriptors of the CTA's tiles staged in shared memory
 
 // stage info word written by the producer, read by the MMA thread
 constexpr uint32_t INFO_SPARSE = 1u, INFO_SEG_START = 2u, INFO_SEG_END = 4u;
@@ -77,7 +77,9 @@ struct Shared {
   int64_t row_hi[2];    // first panel of the CTA's last row, and of the row after it
 };
 constexpr size_t SMEM_BYTES = sizeof(Shared) + 1024;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+// two CTAs fit on an SM, so the next layer's CTAs can start (and stream their
+// weight) while this kernel's last CTAs finish
+static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "shared memory budget: 2 CTAs per SM");
 
 struct Args {
   const patch_tile_desc* desc;
@@ -97,25 +99,48 @@ __host__ __device__ __forceinline__ int64_t cta_of_panel(int64_t p, int64_t P, i
   return ((p + 1) * G - 1) / P;
 }
 
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ int64_t panel_of(const patch_tile_desc& d) {
   return int64_t(d.val_offset / PATCH_PANEL_BYTES);
 }
 
 // Tiles holding panels pa and pb: the last t with panel_of(desc[t]) <= p.
-// Called by every thread of the block: each round probes blockDim.x tiles at
-// once and narrows the span by that factor, so a search costs a few global
-// latencies instead of log2(T) dependent ones.
-__device__ void find_tiles(const patch_tile_desc* desc, int T, int64_t pa, int64_t pb, int& ta, int& tb) {
+// Called by every thread of the block.  The first round probes blockDim.x
+// consecutive tiles around the proportional estimate p*T/P, which holds the
+// answer unless the sparse tiles are very unevenly spread; otherwise each
+// further round probes blockDim.x tiles at once and narrows the span by that
+// factor, so a search costs a few global latencies, not log2(T) dependent ones.
+__device__ void find_tiles(const patch_tile_desc* desc, int T, int64_t P, int64_t pa, int64_t pb, int& ta,
+                           int& tb) {
   const int n = blockDim.x, i = threadIdx.x;
+  auto window = [&](int64_t p) {
+    int64_t w = p * T / P - n / 2;
+    if (w > T - n) w = T - n;
+    return int(w < 0 ? 0 : w);
+  };
+  const int wa = window(pa), wb = window(pb);
+  const int ca = __syncthreads_count(wa + i < T && panel_of(desc[wa + i]) <= pa);
+  const int cb = __syncthreads_count(wb + i < T && panel_of(desc[wb + i]) <= pb);
+  const int na = T - wa < n ? T - wa : n, nb = T - wb < n ? T - wb : n;
+  if (ca >= 1 && (ca < na || wa + na == T) && cb >= 1 && (cb < nb || wb + nb == T)) {
+    ta = wa + ca - 1;
+    tb = wb + cb - 1;
+    return;
+  }
   int lo_a = 0, lo_b = 0, span = T;
   while (span > 1) {
     const int step = (span + n - 1) / n;
     const int ia = lo_a + i * step, ib = lo_b + i * step;
     const bool in = i * step < span;
-    const int ca = __syncthreads_count(in && ia < T && panel_of(desc[ia]) <= pa);
-    const int cb = __syncthreads_count(in && ib < T && panel_of(desc[ib]) <= pb);
-    lo_a += (ca - 1) * step;
-    lo_b += (cb - 1) * step;
+    const int ka = __syncthreads_count(in && ia < T && panel_of(desc[ia]) <= pa);
+    const int kb = __syncthreads_count(in && ib < T && panel_of(desc[ib]) <= pb);
+    lo_a += (ka - 1) * step;
+    lo_b += (kb - 1) * step;
     span = step;
   }
   ta = lo_a;
@@ -138,10 +163,10 @@ __device__ __forceinline__ void load_x(Stage& g, uint64_t* full, const CUtensorM
   }
 }
 
-// The weight panels (and metadata) of the first NS stages are requested
-// before this kernel waits for the previous kernel in the stream (they do
-// not depend on it); the X slices of those stages, which may be that
-// kernel's output, are requested once it has completed.
+// The weight panels of the first NS stages are requested at kernel entry and
+// their metadata before this kernel waits for the previous kernel in the
+// stream (neither depends on it); the X slices of those stages, which may be
+// that kernel's output, are requested once it has completed.
 __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap* tmap_w, const Args& a,
                          int64_t p0, int64_t p1) {
   int t = s.t_first;
@@ -162,7 +187,9 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
   for (int64_t p = p0; p < p1; ++p, ++i) {
     const uint32_t st = i % NS;
     if (i == NS && !waited) release_deferred();  // stage 0 must be consumable before it is reused
-    if (!wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false)) break;
+    const bool early = i < NS;  // weight panel already requested at kernel entry
+    if (!early && !wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false))
+      break;
     const bool sparse = d.kind != 0;
     const bool last_panel_of_tile = sparse || h == 1;
     uint32_t info = sparse ? INFO_SPARSE : 0u;
@@ -170,8 +197,9 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
     if (p + 1 == p1 || (kt == a.Tk - 1 && last_panel_of_tile)) info |= INFO_SEG_END;
     s.info[st] = info;  // published to the MMA thread by the barrier's release
     Stage& g = s.st[st];
-    mbar_expect_tx(&s.full[st], A_BYTES + (sparse ? 2 * X_BYTES + E_BYTES : X_BYTES));
-    tma_load_2d(g.a, tmap_w, &s.full[st], 0, int(p * 128));
+    const uint32_t rest = sparse ? 2 * X_BYTES + E_BYTES : X_BYTES;
+    mbar_expect_tx(&s.full[st], early ? rest : A_BYTES + rest);
+    if (!early) tma_load_2d(g.a, tmap_w, &s.full[st], 0, int(p * 128));
     if (sparse) bulk_load(g.e, a.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.full[st]);
     const uint32_t xinfo = uint32_t(kt) << 2 | uint32_t(h) << 1 | (sparse ? 1u : 0u);
 #pragma unroll
@@ -273,13 +301,15 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, in
     const int64_t rb = tn == tn_first ? s.row_lo[0] : s.row_hi[0];
     const int64_t re = tn == tn_first ? s.row_lo[1] : s.row_hi[1];
     const int64_t c_lo = cta_of_panel(rb, a.P, G), c_hi = cta_of_panel(re - 1, a.P, G);
-    __threadfence();
+    // the warp's partial stores are ordered before lane 0's release-acquire
+    // increment; the last arriver's acquire makes every covering CTA's
+    // partials visible to its later (L2) loads
     __syncwarp();
     uint32_t old = 0;
-    if (lane == 0) old = atomicAdd(&a.counters[4 * tn + q], 1u);
+    if (lane == 0) old = atom_add_acq_rel_gpu(&a.counters[4 * tn + q], 1u);
     old = __shfl_sync(0xFFFFFFFFu, old, 0);
     if (old != uint32_t(c_hi - c_lo)) continue;
-    __threadfence();
+    __syncwarp();  // orders lane 0's acquire before every lane's loads
     float sum[BT];
 #pragma unroll
     for (int m = 0; m < BT; ++m) sum[m] = 0.0f;
@@ -298,7 +328,7 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, in
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const Args a) {
   extern __shared__ uint8_t smem_raw[];
@@ -320,13 +350,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
     fence_barrier_init();
-    prefetch_tensormap(&tmap_x);
     prefetch_tensormap(&tmap_w);
+    // The first weight panels need nothing but their index: request them now,
+    // before the tile search, so HBM is busy from the CTA's first microsecond.
+    // Their stages expect the rest of their bytes when the producer arms them.
+    const int64_t n0 = p1 - p0 < NS ? p1 - p0 : NS;
+    for (int j = 0; j < n0; ++j) {
+      mbar_add_tx(&s.full[j], A_BYTES);
+      tma_load_2d(s.st[j].a, &tmap_w, &s.full[j], 0, int((p0 + j) * 128));
+    }
+    prefetch_tensormap(&tmap_x);
   }
   // locate the CTA's first and last tile, then stage their descriptors
   // (G <= P, so every CTA has at least one panel)
   int ta, tb;
-  find_tiles(a.desc, a.Tn * a.Tk, p0, p1 - 1, ta, tb);
+  find_tiles(a.desc, a.Tn * a.Tk, a.P, p0, p1 - 1, ta, tb);
   const int count = tb - ta + 1;
   if (threadIdx.x == 0) {
     s.t_first = ta;
