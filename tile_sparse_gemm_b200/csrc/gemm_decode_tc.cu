@@ -43,7 +43,7 @@ constexpr int BT = 16;                   // MMA N (tokens)
 constexpr int NS = 4;                    // pipeline stages per CTA (2 CTAs per SM: ~8 panels in flight)
 constexpr int NACC = 2;                  // accumulator buffers (epilogue overlaps the next row)
 constexpr int A_BYTES = PATCH_PANEL_BYTES;
-constexpr int X_BYTES = BT * 64 * 2;     // one 64-k slice of X (16 token rows)
+constexpr int X_BYTES = BT * 64 * 2;     // one 64-k slice of X (room for 16 token rows)
 constexpr int E_BYTES = PATCH_META_TILE_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 128;
@@ -51,7 +51,7 @@ constexpr uint32_t META_COL0 = NACC * BT;  // 4 metadata columns per stage after
 static_assert(META_COL0 + 4 * NS <= TMEM_COLS, "TMEM layout");
 constexpr uint32_t IDESC_DENSE = idesc_bf16(BM, BT, false);
 constexpr uint32_t IDESC_SPARSE = idesc_bf16(BM, BT, true);
-constexpr int WS_FLOATS_PER_CTA = 2 * BT * BM;  // [2 slots][16 tokens][128 rows]
+constexpr int WS_FLOATS_PER_CTA = 2 * BT * BM;  // [2 slots][128 rows][16 tokens]
 constexpr int DCAP = 256;                       // descriptors of the CTA's tiles staged in shared memory
 
 // stage info word written by the producer, read by the MMA thread
@@ -85,7 +85,7 @@ struct Args {
   const patch_tile_desc* desc;
   const uint8_t* meta;
   uint16_t* Y;
-  float* ws;           // [G][2][16][128] fp32 partials
+  float* ws;           // [G][2][128][16] fp32 partials
   uint32_t* counters;  // [Tn][4] arrivals per tile row and TMEM lane quarter (zero between calls)
   int M, N, Tk, Tn;
   int64_t P;  // panels in the values blob
@@ -197,7 +197,8 @@ __device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap
     if (p + 1 == p1 || (kt == a.Tk - 1 && last_panel_of_tile)) info |= INFO_SEG_END;
     s.info[st] = info;  // published to the MMA thread by the barrier's release
     Stage& g = s.st[st];
-    const uint32_t rest = sparse ? 2 * X_BYTES + E_BYTES : X_BYTES;
+    const uint32_t xb = uint32_t(a.M) * 128;  // an X slice holds M token rows (rows M..15 of the slot are never read back)
+    const uint32_t rest = sparse ? 2 * xb + E_BYTES : xb;
     mbar_expect_tx(&s.full[st], early ? rest : A_BYTES + rest);
     if (!early) tma_load_2d(g.a, tmap_w, &s.full[st], 0, int(p * 128));
     if (sparse) bulk_load(g.e, a.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.full[st]);
@@ -294,10 +295,14 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, in
     // A cut row: publish this warp's 32 rows (its TMEM lane quarter q) of
     // partial sums and count the arrival; the last covering CTA to arrive for
     // quarter q adds up that quarter's partials (in CTA order) and stores them.
-    float* mine = a.ws + int64_t(blockIdx.x) * WS_FLOATS_PER_CTA + (tn == tn_first ? 0 : BT * BM);
+    // partial sums of row r: 16 consecutive floats (all 16 MMA columns)
+    float4* mine = reinterpret_cast<float4*>(a.ws + int64_t(blockIdx.x) * WS_FLOATS_PER_CTA +
+                                             (tn == tn_first ? 0 : BT * BM) + r * BT);
 #pragma unroll
-    for (int m = 0; m < BT; ++m)
-      if (m < a.M) mine[m * BM + r] = __uint_as_float(v[m]);
+    for (int k = 0; k < BT / 4; ++k)
+      if (4 * k < a.M)
+        mine[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                              __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
     const int64_t rb = tn == tn_first ? s.row_lo[0] : s.row_hi[0];
     const int64_t re = tn == tn_first ? s.row_lo[1] : s.row_hi[1];
     const int64_t c_lo = cta_of_panel(rb, a.P, G), c_hi = cta_of_panel(re - 1, a.P, G);
@@ -310,16 +315,34 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, in
     old = __shfl_sync(0xFFFFFFFFu, old, 0);
     if (old != uint32_t(c_hi - c_lo)) continue;
     __syncwarp();  // orders lane 0's acquire before every lane's loads
+    // only the first covering CTA can have started before the row (its "last row" slot)
+    const int slot_lo = range_begin(c_lo, a.P, G) < rb ? 1 : 0;
+    const int nv = (a.M + 3) / 4;  // float4s per row that carry real tokens
     float sum[BT];
 #pragma unroll
     for (int m = 0; m < BT; ++m) sum[m] = 0.0f;
-    for (int64_t c = c_lo; c <= c_hi; ++c) {
-      // only the first covering CTA can have started before the row (its "last row" slot)
-      const int slot = (c == c_lo && range_begin(c, a.P, G) < rb) ? 1 : 0;
-      const float* src = a.ws + c * WS_FLOATS_PER_CTA + slot * BT * BM + r;
+    // covering CTAs 4 at a time: all their loads are issued before the
+    // additions, which run in CTA order (deterministic)
+    for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 4) {
+      float4 part[4][BT / 4];
 #pragma unroll
-      for (int m = 0; m < BT; ++m)
-        if (m < a.M) sum[m] += __ldcg(src + m * BM);
+      for (int j = 0; j < 4; ++j) {
+        const int64_t c = c0 + j;
+        const float4* src = reinterpret_cast<const float4*>(
+            a.ws + c * WS_FLOATS_PER_CTA + (c == c_lo ? slot_lo : 0) * BT * BM + r * BT);
+#pragma unroll
+        for (int k = 0; k < BT / 4; ++k)
+          part[j][k] = (c <= c_hi && k < nv) ? __ldcg(src + k) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int k = 0; k < BT / 4; ++k) {
+          sum[4 * k] += part[j][k].x;
+          sum[4 * k + 1] += part[j][k].y;
+          sum[4 * k + 2] += part[j][k].z;
+          sum[4 * k + 3] += part[j][k].w;
+        }
     }
 #pragma unroll
     for (int m = 0; m < BT; ++m)
@@ -435,7 +458,10 @@ cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W
   using namespace decode_tc;
   const Plan pl = plan(W, num_sms);
   CUtensorMap tmap_x, tmap_w;
-  if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, BT)) return cudaErrorUnknown;
+  // X boxes carry exactly the M token rows: the MMA still reads 16 rows (N = 16),
+  // but accumulator columns >= M are never stored, so rows >= M may hold anything
+  if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, uint32_t(M)))
+    return cudaErrorUnknown;
   if (!make_map_2d_bf16(&tmap_w, W.values, 64, uint64_t(pl.P) * 128, 128, 64, 128)) return cudaErrorUnknown;
   Args a;
   a.desc = W.desc;
