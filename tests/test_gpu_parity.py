@@ -239,13 +239,23 @@ def test_prefill_path_small_m_matches_decode(M):
 
 
 def test_prefill_many_output_tiles():
-    """More output tiles than SMs: the persistent schedule wraps around."""
-    N, K, M = 128 * 40, 256, 1100
+    """More work units (row pairs x token blocks) than SMs: the persistent schedule wraps around."""
+    N, K, M = 128 * 80, 256, 1100
     x, w, bm, ids = _layer(N, K, M, "exact", 0.5, cfg=5)
     rows = np.array([0, 1, 255, 256, 511, 700, 1023, 1099])
     ref = oracle.hybrid_gemm(x, w, bm, ids, rows=rows)
     y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids), tsg.PATH_PREFILL)
     check_gemm(y[rows], ref, "prefill wrap")
+
+
+def test_prefill_long_k_reads_descriptors_from_global():
+    """More K-tiles per row than the kernel stages in shared memory (K > 16384),
+    odd tile-row count (the last row pair has one row)."""
+    N, K, M = 384, 128 * 130, 40
+    x, w, bm, ids = _layer(N, K, M, "exact", 0.5, cfg=10)
+    ref = oracle.hybrid_gemm(x, w, bm, ids)
+    y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids), tsg.PATH_PREFILL)
+    check_gemm(y, ref, "prefill long K")
 
 
 def test_gemm_all_sparse_equals_24_and_all_dense_equals_dense():

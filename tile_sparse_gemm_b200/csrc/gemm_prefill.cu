@@ -1,7 +1,7 @@
 // Prefill path of patch_gemm (M > 16): a persistent, warp-specialised
 // TMA + tcgen05 kernel for sm_100a in which dense tiles run on the dense
 // tensor-core MMA and 2:4 sparse tiles on the structured-sparse MMA, both
-// accumulating into one fp32 tile in tensor memory.
+// accumulating into fp32 tiles in tensor memory.
 //
 // "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs", section 2
 // "Methodology: PATCH", "Inference & Deployment": hybrid execution over
@@ -12,21 +12,36 @@
 // computes Y^T = W_eff * X^T: the MMA's M = 128 rows of W (one tile row), its
 // N = BT tokens, K streams over the tiles of the row.
 //
-// CTA = 6 warps, one CTA per SM, static round-robin over output tiles
-// (tile row tn, token block tb):
-//   warp 0  producer: per K-tile reads the descriptor; TMA-loads a dense tile's
-//           2 panels (or a sparse tile's 1 value panel + its 2 KB of metadata
-//           by bulk copy) into the A ring and the 2 matching 64-k panels of X
-//           into the B ring.
-//   warp 1  MMA issuer (one thread) and TMEM owner: dense panel -> 4 x
-//           tcgen05.mma kind::f16 (K = 16); sparse tile -> tcgen05.cp of the
-//           metadata into TMEM, then 4 x tcgen05.mma.sp kind::f16 (K = 32
-//           logical); tcgen05.commit releases ring slots and, per output tile,
-//           signals the epilogue.
-//   warps 2-5 epilogue: tcgen05.ld of the 128 x BT fp32 accumulator, one
-//           round to bf16 (nearest even), stores to Y[m][n]; two TMEM
-//           accumulators let it drain one output tile while the MMAs of the
-//           next one run.
+// Work unit = two tile rows (2 x 128 output features) x BT tokens.  Both rows
+// multiply the same X panels, so one 30 KiB X panel in shared memory feeds
+// two MMA chains; each row keeps its own kind per K-tile (dense or sparse),
+// so the two rows of a unit never need to agree.  Per byte brought in from L2
+// this does 1.5x (dense) to 1.6x (sparse) the tensor-core work of a one-row
+// tile, which is what bounds a 128-row tile on this GPU.
+//
+// CTA = 16 warps, one CTA per SM, static round-robin over units
+// (row pair rp, token block tb):
+//   warps 0, 2  W producers of rows 0 and 1: per K-tile the row's descriptor
+//           (staged in shared memory); a sparse tile's 2 KiB of metadata by
+//           bulk copy; the W panels (2 per dense tile, 1 per sparse tile) by
+//           TMA into the row's A ring.
+//   warps 1, 3  MMA issuers of rows 0 and 1 (one thread each; warp 1 owns
+//           TMEM): dense panel -> 4 x tcgen05.mma kind::f16 (K = 16); sparse
+//           tile -> tcgen05.cp of the metadata into TMEM, then 4 x
+//           tcgen05.mma.sp kind::f16 (K = 32 logical); tcgen05.commit
+//           releases ring slots and, per unit, signals the row's epilogue.
+//           One issuing thread for both rows cannot keep the tensor core
+//           busy: every wait, commit and MMA issue is a long-latency
+//           instruction in one serial chain.
+//   warp 4  X producer: TMA-loads the 2 matching 64-k panels of X per K-tile
+//           into the B ring shared by both rows.
+//   warps 8-15 epilogue: warps 8-11 drain row 0's accumulator, 12-15 row 1's
+//           (each warp its TMEM lane quarter): tcgen05.ld, one round to bf16
+//           (nearest even), stores to Y[m][n].
+// Tensor memory: row 0's accumulator at columns 0..BT-1, row 1's at 256..,
+// metadata slots of 4 columns after each.  The two accumulators use all of
+// it, so a unit's epilogue does not overlap the next unit's MMAs; the
+// producer keeps loading meanwhile, so the rings are full when they restart.
 // Every mbarrier wait is bounded in time; when one runs out the kernel sets
 // PATCH_DEV_TIMEOUT, the other roles stop at their next wait, the producer
 // waits for its copies in flight, the MMA thread for its MMAs, and TMEM is
@@ -42,241 +57,261 @@ namespace prefill {
 
 using namespace tc;
 
-constexpr int BM = 128;                  // W rows per output tile (MMA M)
-constexpr int BT = 240;                  // tokens per output tile (MMA N; 2 x 240 + metadata fit TMEM)
-constexpr int NA = 5;                    // A ring: W panels of 128 x 64 bf16
-constexpr int NB = 4;                    // B ring: X panels of BT x 64 bf16
-constexpr int NE = 4;                    // metadata ring
+constexpr int BM = 128;                  // W rows per tile row (MMA M)
+constexpr int ROWS = 2;                  // tile rows per unit, sharing the X panels
+constexpr int BT = 240;                  // most tokens per unit (MMA N); each launch picks bt <= BT
+constexpr int NA = 3;                    // A ring per row: W panels of 128 x 64 bf16
+constexpr int NB = 3;                    // B ring: X panels of BT x 64 bf16
+constexpr int NE = 2;                    // metadata ring per row
 constexpr int A_BYTES = PATCH_PANEL_BYTES;
 constexpr int B_BYTES = BT * 64 * 2;
 constexpr int E_BYTES = PATCH_META_TILE_BYTES;
-constexpr int THREADS = 192;
-constexpr int MAXTK = 256;               // descriptors of one tile row staged in shared memory
-constexpr int NACC = 2;                  // accumulators: the epilogue of one tile overlaps the next
-constexpr uint32_t TMEM_COLS = 512;      // accumulators at columns 0 and 256, metadata slots at BT..
-constexpr uint32_t ACC_STRIDE = 256;
-constexpr uint32_t META_COL0 = BT;
-static_assert(META_COL0 + 4 * 4 <= ACC_STRIDE && ACC_STRIDE + BT <= TMEM_COLS, "TMEM layout");
+constexpr int EPI_WARP0 = 8;             // warps 8-11 drain row 0, 12-15 row 1
+constexpr int THREADS = 32 * (EPI_WARP0 + 4 * ROWS);
+constexpr int MAXTK = 128;               // descriptors of one tile row staged in shared memory (K <= 16384)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_STRIDE = 256;     // row r's accumulator at column 256 r
+constexpr uint32_t META_COL0 = BT;       // row r's metadata slot e at column 256 r + BT + 4 e
+static_assert(META_COL0 + 4 * NE <= ACC_STRIDE && ACC_STRIDE + BT <= TMEM_COLS, "TMEM layout");
+static_assert(B_BYTES % 1024 == 0, "X panels keep the 1024-byte alignment of the 128-byte swizzle");
 
-constexpr uint32_t IDESC_DENSE = tc::idesc_bf16(BM, BT, false);
-constexpr uint32_t IDESC_SPARSE = tc::idesc_bf16(BM, BT, true);
 
 struct Shared {
-  alignas(1024) uint8_t a[NA][A_BYTES];
+  alignas(1024) uint8_t a[ROWS][NA][A_BYTES];
   alignas(1024) uint8_t b[NB][B_BYTES];
-  alignas(128) uint8_t e[NE][E_BYTES];
-  uint64_t a_full[NA], a_empty[NA], b_full[NB], b_empty[NB], e_full[NE], e_empty[NE];
-  uint64_t acc_full[NACC], acc_empty[NACC], drain;
-  uint64_t pdesc_full[2];             // descriptor rows, bulk-copied by the producer
-  alignas(16) patch_tile_desc pdesc[2][MAXTK];
-  uint32_t a_kind[NA];                // tile kind of the panel in each A slot (producer -> MMA)
+  alignas(128) uint8_t e[ROWS][NE][E_BYTES];
+  uint64_t a_full[ROWS][NA], a_empty[ROWS][NA], e_full[ROWS][NE], e_empty[ROWS][NE];
+  uint64_t b_full[NB], b_empty[NB];   // b_empty: one arrival per row's MMA thread
+  uint64_t acc_full[ROWS], acc_empty[ROWS], drain[ROWS];
+  uint64_t pdesc_full[ROWS][2];       // descriptor rows, bulk-copied by each row's producer
+  alignas(16) patch_tile_desc pdesc[ROWS][2][MAXTK];
+  uint32_t a_kind[ROWS][NA];          // tile kind of the panel in each A slot (producer -> MMA)
   uint32_t tmem_base;
   int abort_flag;
 };
 constexpr size_t SMEM_BYTES = sizeof(Shared) + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
-// ---------------------------------------------------------------- roles
-
 struct Args {
   const uint8_t* meta;
   const patch_tile_desc* desc;
   uint16_t* Y;
-  int M, N, Tk, n_items;
+  int M, N, Tn, Tk, n_pairs, n_items;
+  int bt;                      // tokens per unit: a multiple of 16, at most BT
+  uint32_t idesc_dense, idesc_sparse;
   uint64_t limit_ns;
   int32_t* status;
-  int inject;  // 1: producer stops after the first K-tile (exercises the timeout path)
+  int inject;  // 1: row 0's producer stops after the first K-tile (exercises the timeout path)
 };
 
-// Descriptor of tile (tn, kt): from the staged row when it fits, else from global memory.
-__device__ __forceinline__ patch_tile_desc row_desc(const Shared& s, const Args& p, bool staged, int buf, int tn,
-                                                    int kt) {
-  return staged ? s.pdesc[buf][kt] : p.desc[int64_t(tn) * p.Tk + kt];
-}
+// tile rows in row pair rp (the last pair of an odd Tn has one)
+__device__ __forceinline__ int rows_of(int rp, int Tn) { return Tn - ROWS * rp < ROWS ? Tn - ROWS * rp : ROWS; }
 
-__device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap* tmap_w, const Args& p) {
-  const int Tn = p.N / BM;
+// Units that share an X block (same tb) or W rows (same rp) start their K loop
+// at different tiles, so they do not all hit the same L2 lines at the same
+// moment; only the order of the fp32 sum changes.
+__device__ __forceinline__ int k_rotation(int rp, int tb, int Tk) { return (rp + 7 * tb) % Tk; }
+
+// ---------------------------------------------------------------- roles
+
+// W producer of row r: the row's descriptors, metadata and W panels.  It never
+// touches X, so it may run ahead of the previous kernel in the stream (W, the
+// metadata and the descriptors are inputs that no kernel triggering an early
+// launch writes).
+__device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, int r) {
   const bool staged = p.Tk <= MAXTK;
-  uint32_t a_i = 0, b_i = 0, e_i = 0, d_i = 0;  // loads issued per ring / descriptor rows staged
-  bool ok = true, waited = false;
-  // stage the first item's descriptor row
-  if (staged && int(blockIdx.x) < p.n_items) {
-    const int tn0 = int(blockIdx.x) % Tn;
-    mbar_expect_tx(&s.pdesc_full[0], uint32_t(p.Tk * sizeof(patch_tile_desc)));
-    bulk_load(s.pdesc[0], p.desc + int64_t(tn0) * p.Tk, uint32_t(p.Tk * sizeof(patch_tile_desc)), &s.pdesc_full[0]);
+  const uint32_t row_bytes = uint32_t(p.Tk * sizeof(patch_tile_desc));
+  uint32_t a_i = 0, e_i = 0, d_i = 0;  // loads issued per ring / descriptor rows staged
+  bool ok = true;
+  // stage (or, for a pair without row r, complete with no bytes) the descriptor row of an item
+  auto stage_row = [&](int item, int buf) {
+    const int rp = item % p.n_pairs;
+    const bool has = r < rows_of(rp, p.Tn);
+    mbar_expect_tx(&s.pdesc_full[r][buf], has ? row_bytes : 0u);
+    if (has) bulk_load(s.pdesc[r][buf], p.desc + int64_t(ROWS * rp + r) * p.Tk, row_bytes, &s.pdesc_full[r][buf]);
     ++d_i;
-  }
+  };
+  if (staged && int(blockIdx.x) < p.n_items) stage_row(blockIdx.x, 0);
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const int tn = item % Tn, tb = item / Tn;
+    const int rp = item % p.n_pairs, tb = item / p.n_pairs, tn = ROWS * rp + r;
     const int buf = it & 1;
     if (staged) {
-      if (!(ok = wait_bounded(&s.pdesc_full[buf], (it >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
+      if (!(ok = wait_bounded(&s.pdesc_full[r][buf], (it >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
         break;
-      // prefetch the next item's row into the other buffer (its previous row is done)
-      const int next = item + gridDim.x;
-      if (next < p.n_items) {
-        mbar_expect_tx(&s.pdesc_full[buf ^ 1], uint32_t(p.Tk * sizeof(patch_tile_desc)));
-        bulk_load(s.pdesc[buf ^ 1], p.desc + int64_t(next % Tn) * p.Tk, uint32_t(p.Tk * sizeof(patch_tile_desc)),
-                  &s.pdesc_full[buf ^ 1]);
-        ++d_i;
-      }
+      // prefetch the next unit's row into the other buffer (its previous row is done)
+      if (item + int(gridDim.x) < p.n_items) stage_row(item + gridDim.x, buf ^ 1);
     }
-    // CTAs that share an X block (same tb) or a W tile row (same tn) start
-    // their K loop at different tiles, so they do not all hit the same L2 lines
-    // at the same moment; the sum order is the only thing that changes
-    const int rot = (tn + 7 * tb) % p.Tk;
-    for (int j = 0; ok && j < p.Tk; ++j) {
-      const int kt = (j + rot) % p.Tk;
-      if (p.inject && (item != int(blockIdx.x) || j > 0)) {
+    if (r >= rows_of(rp, p.Tn)) continue;
+    int kt = k_rotation(rp, tb, p.Tk);
+    for (int j = 0; ok && j < p.Tk; ++j, kt = (kt + 1 == p.Tk ? 0 : kt + 1)) {
+      if (p.inject && r == 0 && (item != int(blockIdx.x) || j > 0)) {
         ok = false;
         break;
       }
-      const patch_tile_desc d = row_desc(s, p, staged, buf, tn, kt);
-      const int panel = int(d.val_offset / A_BYTES);
+      const patch_tile_desc d = staged ? s.pdesc[r][buf][kt] : p.desc[int64_t(tn) * p.Tk + kt];
       if (d.kind) {
         const uint32_t es = e_i % NE;
-        if (!(ok = wait_bounded(&s.e_empty[es], ((e_i / NE) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
-        mbar_expect_tx(&s.e_full[es], E_BYTES);
-        bulk_load(s.e[es], p.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.e_full[es]);
+        if (!(ok = wait_bounded(&s.e_empty[r][es], ((e_i / NE) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
+          break;
+        mbar_expect_tx(&s.e_full[r][es], E_BYTES);
+        bulk_load(s.e[r][es], p.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.e_full[r][es]);
         ++e_i;
       }
-      const int n_a = d.kind ? 1 : 2;
-      for (int h = 0; h < n_a; ++h) {
+      // a dense tile's 2 panels (one per 64-k half), a sparse tile's one
+      const int panel = int(d.val_offset / A_BYTES);
+      for (int h = 0; h < (d.kind ? 1 : 2); ++h) {
         const uint32_t as = a_i % NA;
-        if (!(ok = wait_bounded(&s.a_empty[as], ((a_i / NA) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
+        if (!(ok = wait_bounded(&s.a_empty[r][as], ((a_i / NA) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
           break;
-        s.a_kind[as] = d.kind;  // published to the MMA thread by the barrier's release
-        mbar_expect_tx(&s.a_full[as], A_BYTES);
-        tma_load_2d(s.a[as], tmap_w, &s.a_full[as], 0, (panel + h) * 128);
+        s.a_kind[r][as] = d.kind;  // published to the MMA thread by the barrier's release
+        mbar_expect_tx(&s.a_full[r][as], A_BYTES);
+        tma_load_2d(s.a[r][as], tmap_w, &s.a_full[r][as], 0, (panel + h) * 128);
         ++a_i;
-      }
-      if (!ok) break;
-      // X may be the previous kernel's output: wait for it before the first X load
-      if (!waited) {
-        pdl_wait_previous();
-        waited = true;
-      }
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t bs = b_i % NB;
-        if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
-          break;
-        mbar_expect_tx(&s.b_full[bs], B_BYTES);
-        tma_load_2d(s.b[bs], tmap_x, &s.b_full[bs], kt * kTile + 64 * h, tb * BT);
-        ++b_i;
       }
     }
   }
   // every copy issued must have landed before the CTA may exit
   for (uint32_t i = (a_i > NA ? a_i - NA : 0); i < a_i; ++i)
-    wait_bounded(&s.a_full[i % NA], (i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, true);
-  for (uint32_t i = (b_i > NB ? b_i - NB : 0); i < b_i; ++i)
-    wait_bounded(&s.b_full[i % NB], (i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+    wait_bounded(&s.a_full[r][i % NA], (i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, true);
   for (uint32_t i = (e_i > NE ? e_i - NE : 0); i < e_i; ++i)
-    wait_bounded(&s.e_full[i % NE], (i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+    wait_bounded(&s.e_full[r][i % NE], (i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, true);
   for (uint32_t i = (d_i > 2 ? d_i - 2 : 0); i < d_i; ++i)
-    wait_bounded(&s.pdesc_full[i & 1], (i >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+    wait_bounded(&s.pdesc_full[r][i & 1], (i >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, true);
 }
 
-__device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p) {
+// X producer: the two 64-k panels of X per K-tile, in the same rotated K order.
+__device__ void producer_x(Shared& s, const CUtensorMap* tmap_x, const Args& p) {
+  uint32_t b_i = 0;
+  bool ok = true;
+  // X may be the previous kernel's output: wait for it before the first X load
+  pdl_wait_previous();
+  for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+    const int rp = item % p.n_pairs, tb = item / p.n_pairs;
+    int kt = k_rotation(rp, tb, p.Tk);
+    for (int j = 0; ok && j < p.Tk; ++j, kt = (kt + 1 == p.Tk ? 0 : kt + 1)) {
+      for (int h = 0; ok && h < 2; ++h) {
+        const uint32_t bs = b_i % NB;
+        if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
+          break;
+        mbar_expect_tx(&s.b_full[bs], uint32_t(p.bt) * 128u);
+        tma_load_2d(s.b[bs], tmap_x, &s.b_full[bs], kt * kTile + 64 * h, tb * p.bt);
+        ++b_i;
+      }
+    }
+  }
+  for (uint32_t i = (b_i > NB ? b_i - NB : 0); i < b_i; ++i)
+    wait_bounded(&s.b_full[i % NB], (i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+}
+
+// MMA issuer of row r (one thread): each row has its own issuing thread, so
+// the two chains' barrier waits, commits and bookkeeping overlap and the
+// tensor core, shared by both, stays fed.  Both consume the same X slots; a
+// slot is free once both rows' MMAs on it are complete (two commits).
+__device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
+  const uint32_t acc = tmem + ACC_STRIDE * r;
   uint32_t a_i = 0, b_i = 0, e_i = 0;
   bool ok = true;
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const int buf = it % NACC;
-    if (!(ok = wait_bounded(&s.acc_empty[buf], ((it / NACC) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
-      break;
+    const bool active = r < rows_of(item % p.n_pairs, p.Tn);
+    if (!(ok = wait_bounded(&s.acc_empty[r], (it & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
     tc_fence_after();
-    const uint32_t acc = tmem + ACC_STRIDE * buf;
     uint32_t accumulate = 0;
     for (int kt = 0; ok && kt < p.Tk; ++kt) {
-      // the tile's kind arrives with its first A panel
-      uint32_t as = a_i % NA;
-      if (!(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
-      const uint32_t kind = *reinterpret_cast<volatile uint32_t*>(&s.a_kind[as]);
-      if (kind) {
-        const uint32_t es = e_i % NE;
-        if (!(ok = wait_bounded(&s.e_full[es], (e_i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+      uint32_t kind = 0, as = 0, es = 0;
+      for (int h = 0; h < 2; ++h) {
+        // the tile's kind arrives with its first panel; a sparse tile's one
+        // panel serves both halves and its metadata goes to TMEM first
+        if (active && (h == 0 || !kind)) {
+          as = a_i % NA;
+          if (!(ok = wait_bounded(&s.a_full[r][as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
+            break;
+          ++a_i;
+          if (h == 0) kind = *reinterpret_cast<volatile uint32_t*>(&s.a_kind[r][as]);
+          if (h == 0 && kind) {
+            es = e_i % NE;
+            if (!(ok = wait_bounded(&s.e_full[r][es], (e_i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
+              break;
+            ++e_i;
+            tc_fence_after();
+            tmem_cp_128x128b(acc + META_COL0 + 4 * es, meta_desc(smem_u32(s.e[r][es])));
+          }
+        }
+        const uint32_t bs = b_i % NB;
+        if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+        ++b_i;
+        if (!active) {  // the pair's missing row only paces the X ring
+          mbar_arrive(&s.b_empty[bs]);
+          continue;
+        }
         tc_fence_after();
-        const uint32_t e_tmem = tmem + META_COL0 + 4 * es;
-        tmem_cp_128x128b(e_tmem, meta_desc(smem_u32(s.e[es])));
-        const uint64_t a0 = sw128_desc(smem_u32(s.a[as]));
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t bs = b_i % NB;
-          if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
-          tc_fence_after();
-          const uint64_t b0 = sw128_desc(smem_u32(s.b[bs]));
+        const uint64_t a0 = sw128_desc(smem_u32(s.a[r][as]));
+        const uint64_t b0 = sw128_desc(smem_u32(s.b[bs]));
+        if (kind) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const uint32_t kb = 2 * h + j;  // 32-k block of the tile: 16 kept values = 32 B of A
-            mma_sparse(acc, a0 + (kb * 32 >> 4), b0 + (j * 64 >> 4), e_tmem + (kb & 2u),
-                       IDESC_SPARSE | (kb & 1u), accumulate);
+            mma_sparse(acc, a0 + (kb * 32 >> 4), b0 + (j * 64 >> 4), acc + META_COL0 + 4 * es + (kb & 2u),
+                       p.idesc_sparse | (kb & 1u), accumulate);
             accumulate = 1;
           }
-          tc_commit(&s.b_empty[bs]);
-          ++b_i;
-        }
-        if (!ok) break;
-        tc_commit(&s.a_empty[as]);
-        ++a_i;
-        tc_commit(&s.e_empty[es]);
-        ++e_i;
-      } else {
-        for (int h = 0; h < 2; ++h) {
-          as = a_i % NA;
-          const uint32_t bs = b_i % NB;
-          if (h == 1 &&
-              !(ok = wait_bounded(&s.a_full[as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
-            break;
-          if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
-          tc_fence_after();
-          const uint64_t a0 = sw128_desc(smem_u32(s.a[as]));
-          const uint64_t b0 = sw128_desc(smem_u32(s.b[bs]));
+        } else {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {  // K = 16 per MMA = 32 B along the swizzled row
-            mma_dense(acc, a0 + (j * 32 >> 4), b0 + (j * 32 >> 4), IDESC_DENSE, accumulate);
+            mma_dense(acc, a0 + (j * 32 >> 4), b0 + (j * 32 >> 4), p.idesc_dense, accumulate);
             accumulate = 1;
           }
-          tc_commit(&s.a_empty[as]);
-          ++a_i;
-          tc_commit(&s.b_empty[bs]);
-          ++b_i;
+        }
+        tc_commit(&s.b_empty[bs]);
+        if (!kind) {
+          tc_commit(&s.a_empty[r][as]);
+        } else if (h == 1) {
+          tc_commit(&s.a_empty[r][as]);
+          tc_commit(&s.e_empty[r][es]);
         }
       }
     }
-    if (ok) tc_commit(&s.acc_full[buf]);
+    if (ok) {
+      if (active)
+        tc_commit(&s.acc_full[r]);
+      else
+        mbar_arrive(&s.acc_full[r]);
+    }
   }
   // all MMAs and copies issued must be complete before TMEM is freed
-  tc_commit(&s.drain);
-  wait_bounded(&s.drain, 0, &s.abort_flag, p.limit_ns, p.status, true);
+  tc_commit(&s.drain[r]);
+  wait_bounded(&s.drain[r], 0, &s.abort_flag, p.limit_ns, p.status, true);
 }
 
+// Epilogue warp: drains its TMEM lane quarter of one row's accumulator.
 __device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
-  const int Tn = p.N / BM;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = warp & 3;  // the TMEM lane quarter this warp may access
+  const int q = warp & 3;                  // the TMEM lane quarter this warp may access
+  const int r = (warp - EPI_WARP0) >> 2;   // the row of the pair it drains
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
-    const int tn = item % Tn, tb = item / Tn;
-    const int buf = it % NACC;
-    if (!wait_bounded(&s.acc_full[buf], (it / NACC) & 1, &s.abort_flag, p.limit_ns, p.status, false)) break;
+    const int rp = item % p.n_pairs, tb = item / p.n_pairs;
+    if (!wait_bounded(&s.acc_full[r], it & 1, &s.abort_flag, p.limit_ns, p.status, false)) break;
     tc_fence_after();
-    const int64_t n = int64_t(tn) * BM + 32 * q + lane;
-    const int m0 = tb * BT;
-    const uint32_t acc = tmem + (uint32_t(32 * q) << 16) + ACC_STRIDE * buf;
-    for (int c = 0; c < BT / 16; ++c) {
-      if (m0 + 16 * c >= p.M) break;  // warp-uniform
-      uint32_t v[16];
-      tmem_ld_16cols(acc + uint32_t(16 * c), v);
+    if (r < rows_of(rp, p.Tn)) {
+      const int64_t n = int64_t(ROWS * rp + r) * BM + 32 * q + lane;
+      const int m0 = tb * p.bt;
+      const uint32_t acc = tmem + (uint32_t(32 * q) << 16) + ACC_STRIDE * r;
+      for (int c = 0; c < p.bt / 16; ++c) {
+        if (m0 + 16 * c >= p.M) break;  // warp-uniform
+        uint32_t v[16];
+        tmem_ld_16cols(acc + uint32_t(16 * c), v);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int m = m0 + 16 * c + j;
-        if (m < p.M) p.Y[int64_t(m) * p.N + n] = f32_to_bf16_rne(__uint_as_float(v[j]));
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + 16 * c + j;
+          if (m < p.M) p.Y[int64_t(m) * p.N + n] = f32_to_bf16_rne(__uint_as_float(v[j]));
+        }
       }
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.acc_empty[buf]);
+    if (lane == 0) mbar_arrive(&s.acc_empty[r]);
   }
 }
 
@@ -289,29 +324,29 @@ __global__ void __launch_bounds__(THREADS, 1)
   pdl_launch_dependents();  // the next kernel may run its prologue as our CTAs finish
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NA; ++i) {
-      mbar_init(&s.a_full[i], 1);
-      mbar_init(&s.a_empty[i], 1);
+    for (int r = 0; r < ROWS; ++r) {
+      for (int i = 0; i < NA; ++i) {
+        mbar_init(&s.a_full[r][i], 1);
+        mbar_init(&s.a_empty[r][i], 1);
+      }
+      for (int i = 0; i < NE; ++i) {
+        mbar_init(&s.e_full[r][i], 1);
+        mbar_init(&s.e_empty[r][i], 1);
+      }
+      mbar_init(&s.acc_full[r], 1);
+      mbar_init(&s.acc_empty[r], 4);
+      mbar_init(&s.drain[r], 1);
+      mbar_init(&s.pdesc_full[r][0], 1);
+      mbar_init(&s.pdesc_full[r][1], 1);
     }
     for (int i = 0; i < NB; ++i) {
       mbar_init(&s.b_full[i], 1);
-      mbar_init(&s.b_empty[i], 1);
+      mbar_init(&s.b_empty[i], ROWS);
     }
-    for (int i = 0; i < NE; ++i) {
-      mbar_init(&s.e_full[i], 1);
-      mbar_init(&s.e_empty[i], 1);
-    }
-    for (int i = 0; i < NACC; ++i) {
-      mbar_init(&s.acc_full[i], 1);
-      mbar_init(&s.acc_empty[i], 4);
-    }
-    mbar_init(&s.drain, 1);
-    mbar_init(&s.pdesc_full[0], 1);
-    mbar_init(&s.pdesc_full[1], 1);
     s.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+    prefetch_tensormap(&tmap_x);
+    prefetch_tensormap(&tmap_w);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -325,13 +360,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 0) {
-    if (lane == 0) producer(s, &tmap_x, &tmap_w, p);
+  // warps 0/2: W producers of rows 0/1; 1/3: MMA issuers of rows 0/1; 4: X producer
+  if (warp < 4) {
+    if (lane == 0) {
+      if (warp & 1)
+        mma_issuer(s, tmem, p, warp >> 1);
+      else
+        producer_w(s, &tmap_w, p, warp >> 1);
+    }
     __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) mma_issuer(s, tmem, p);
+  } else if (warp == 4) {
+    if (lane == 0) producer_x(s, &tmap_x, p);
     __syncwarp();
-  } else {
+  } else if (warp >= EPI_WARP0) {
     epilogue(s, tmem, p);
   }
 
@@ -379,14 +420,39 @@ bool make_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tokens per unit: the multiple of 16 in [64, BT] that minimises the time of
+// the slowest CTA, modelled as (units per CTA, rounded up) x (unit time).  A
+// unit's K-tile costs the larger of its tensor-core cycles (8 bt: 2 rows x
+// 128 K at 8192 FLOP per cycle) and the cycles to bring its 64 KiB of W plus
+// 256 bt bytes of X from L2 at about 64 B per cycle; a unit adds ~4000 cycles
+// of pipeline fill and epilogue.  Ties go to the larger bt.
+static int pick_bt(int64_t M, int64_t n_pairs, int64_t Tk, int num_sms) {
+  using prefill::BT;
+  int best = BT;
+  int64_t best_cost = -1;
+  for (int bt = BT; bt >= 64; bt -= 16) {
+    const int64_t units = n_pairs * ((M + bt - 1) / bt);
+    const int64_t mma = 8 * bt, feed = 1024 + 4 * bt;
+    const int64_t cost = (units + num_sms - 1) / num_sms * (Tk * (mma > feed ? mma : feed) + 4000);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bt;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
                            int32_t* status, int num_sms, uint64_t limit_ns, int inject,
                            cudaStream_t stream) {
   using namespace prefill;
   const int64_t Tn = W.N / BM, Tk = W.K / kTile, T = Tn * Tk;
   const uint64_t n_panels = uint64_t(2 * (T - W.n_sparse) + W.n_sparse);
+  const int64_t n_pairs = (Tn + ROWS - 1) / ROWS;
+  const int bt = pick_bt(M, n_pairs, Tk, num_sms);
   CUtensorMap tmap_x, tmap_w;
-  if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, BT)) return cudaErrorUnknown;
+  if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, uint32_t(bt)))
+    return cudaErrorUnknown;
   if (!make_map_2d_bf16(&tmap_w, W.values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
   Args p;
   p.meta = static_cast<const uint8_t*>(W.meta);
@@ -394,8 +460,13 @@ cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, 
   p.Y = Y;
   p.M = int(M);
   p.N = int(W.N);
+  p.Tn = int(Tn);
   p.Tk = int(Tk);
-  p.n_items = int(Tn * ((M + BT - 1) / BT));
+  p.n_pairs = int(n_pairs);
+  p.n_items = int(n_pairs * ((M + bt - 1) / bt));
+  p.bt = bt;
+  p.idesc_dense = tc::idesc_bf16(BM, bt, false);
+  p.idesc_sparse = tc::idesc_bf16(BM, bt, true);
   p.limit_ns = limit_ns;
   p.status = status;
   p.inject = inject;
