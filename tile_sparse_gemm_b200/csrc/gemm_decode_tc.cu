@@ -23,10 +23,11 @@
 // One pipeline stage per panel holds the 16 KiB weight panel, the 64-k
 // slices of X it multiplies (1 for a dense panel, 2 for a sparse one) and,
 // for a sparse tile, its 2 KiB of metadata, all landing on one mbarrier.
-// Roles per CTA (6 warps): warp 0 TMA producer, warp 1 MMA issuer and TMEM
-// owner (dense panel: 4 x kind::f16 K = 16; sparse tile: tcgen05.cp of the
-// metadata, then 4 x kind::f16 .sp K = 32), warps 2-5 epilogue.  Every wait
-// is bounded in time as in the prefill kernel.
+// Roles per CTA (7 warps): warp 0 W producer (weight panels, the stage's
+// info word), warp 6 X producer (X slices, metadata), warp 1 MMA issuer and
+// TMEM owner (dense panel: 4 x kind::f16 K = 16; sparse tile: tcgen05.cp of
+// the metadata, then 4 x kind::f16 .sp K = 32), warps 2-5 epilogue.  Every
+// wait is bounded in time as in the prefill kernel.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -45,7 +46,7 @@ constexpr int NACC = 2;                  // accumulator buffers (epilogue overla
 constexpr int A_BYTES = PATCH_PANEL_BYTES;
 constexpr int X_BYTES = BT * 64 * 2;     // one 64-k slice of X (room for 16 token rows)
 constexpr int E_BYTES = PATCH_META_TILE_BYTES;
-constexpr int THREADS = 192;
+constexpr int THREADS = 224;  // warps: 0 W producer, 1 MMA, 2-5 epilogue, 6 X producer
 constexpr uint32_t TMEM_COLS = 128;
 constexpr uint32_t META_COL0 = NACC * BT;  // 4 metadata columns per stage after the accumulators
 static_assert(META_COL0 + 4 * NS <= TMEM_COLS, "TMEM layout");
@@ -163,62 +164,102 @@ __device__ __forceinline__ void load_x(Stage& g, uint64_t* full, const CUtensorM
   }
 }
 
-// The weight panels of the first NS stages are requested at kernel entry and
-// their metadata before this kernel waits for the previous kernel in the
-// stream (neither depends on it); the X slices of those stages, which may be
-// that kernel's output, are requested once it has completed.
-__device__ void producer(Shared& s, const CUtensorMap* tmap_x, const CUtensorMap* tmap_w, const Args& a,
-                         int64_t p0, int64_t p1) {
-  int t = s.t_first;
-  patch_tile_desc d = tile_desc(s, a, t);
-  int h = int(p0 - panel_of(d));
-  int kt = t % a.Tk;
-  uint32_t i = 0;
-  bool waited = false;
-  uint32_t deferred[NS];
-  auto release_deferred = [&]() {
-    pdl_wait_previous();
-    waited = true;
-    const uint32_t n = i < NS ? i : NS;
-#pragma unroll
-    for (uint32_t j = 0; j < NS; ++j)
-      if (j < n) load_x(s.st[j], &s.full[j], tmap_x, deferred[j]);
-  };
-  for (int64_t p = p0; p < p1; ++p, ++i) {
-    const uint32_t st = i % NS;
-    if (i == NS && !waited) release_deferred();  // stage 0 must be consumable before it is reused
-    const bool early = i < NS;  // weight panel already requested at kernel entry
-    if (!early && !wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false))
-      break;
-    const bool sparse = d.kind != 0;
-    const bool last_panel_of_tile = sparse || h == 1;
-    uint32_t info = sparse ? INFO_SPARSE : 0u;
-    if (p == p0 || (kt == 0 && h == 0)) info |= INFO_SEG_START;
-    if (p + 1 == p1 || (kt == a.Tk - 1 && last_panel_of_tile)) info |= INFO_SEG_END;
-    s.info[st] = info;  // published to the MMA thread by the barrier's release
-    Stage& g = s.st[st];
-    const uint32_t xb = uint32_t(a.M) * 128;  // an X slice holds M token rows (rows M..15 of the slot are never read back)
-    const uint32_t rest = sparse ? 2 * xb + E_BYTES : xb;
-    mbar_expect_tx(&s.full[st], early ? rest : A_BYTES + rest);
-    if (!early) tma_load_2d(g.a, tmap_w, &s.full[st], 0, int(p * 128));
-    if (sparse) bulk_load(g.e, a.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.full[st]);
-    const uint32_t xinfo = uint32_t(kt) << 2 | uint32_t(h) << 1 | (sparse ? 1u : 0u);
-#pragma unroll
-    for (uint32_t j = 0; j < NS; ++j)
-      if (!waited && j == i) deferred[j] = xinfo;
-    if (waited) load_x(g, &s.full[st], tmap_x, xinfo);
-    // next panel: second half of a dense tile, or the next tile
-    if (last_panel_of_tile) {
+// Walks a CTA's panels in order: tile t, K-tile kt, half h of a dense tile.
+struct PanelWalk {
+  int t, h, kt;
+  patch_tile_desc d;
+  __device__ __forceinline__ void start(const Shared& s, const Args& a, int64_t p0) {
+    t = s.t_first;
+    d = tile_desc(s, a, t);
+    h = int(p0 - panel_of(d));
+    kt = t % a.Tk;
+  }
+  __device__ __forceinline__ bool sparse() const { return d.kind != 0; }
+  __device__ __forceinline__ bool last_of_tile() const { return d.kind != 0 || h == 1; }
+  // X slices of this panel: K-tile, half, both halves for a sparse tile
+  __device__ __forceinline__ uint32_t xinfo() const {
+    return uint32_t(kt) << 2 | uint32_t(h) << 1 | (sparse() ? 1u : 0u);
+  }
+  __device__ __forceinline__ void next(const Shared& s, const Args& a, bool more) {
+    if (last_of_tile()) {
       h = 0;
       ++t;
       if (++kt == a.Tk) kt = 0;
-      if (p + 1 < p1) d = tile_desc(s, a, t);
+      if (more) d = tile_desc(s, a, t);
     } else {
       h = 1;
     }
   }
-  if (!waited) release_deferred();
+};
+
+// Two producer threads fill each stage; the stage barrier counts one arrival
+// from each.  One thread issuing every copy spends about as long per panel as
+// HBM takes to deliver it.
+//
+// W producer: the weight panel and the stage's info word.  The panels of the
+// first NS stages were requested at kernel entry; for those it only arrives.
+__device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& a, int64_t p0, int64_t p1) {
+  PanelWalk w;
+  w.start(s, a, p0);
+  uint32_t i = 0;
+  for (int64_t p = p0; p < p1; ++p, ++i) {
+    const uint32_t st = i % NS;
+    const bool early = i < NS;
+    if (!early && !wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false))
+      break;
+    uint32_t info = w.sparse() ? INFO_SPARSE : 0u;
+    if (p == p0 || (w.kt == 0 && w.h == 0)) info |= INFO_SEG_START;
+    if (p + 1 == p1 || (w.kt == a.Tk - 1 && w.last_of_tile())) info |= INFO_SEG_END;
+    s.info[st] = info;  // published to the MMA thread by this thread's arrival
+    if (early) {
+      mbar_arrive(&s.full[st]);
+    } else {
+      mbar_expect_tx(&s.full[st], A_BYTES);
+      tma_load_2d(s.st[st].a, tmap_w, &s.full[st], 0, int(p * 128));
+    }
+    w.next(s, a, p + 1 < p1);
+  }
   // every copy issued must have landed before the CTA may exit
+  for (uint32_t j = (i > NS ? i - NS : 0); j < i; ++j)
+    wait_bounded(&s.full[j % NS], (j / NS) & 1, &s.abort_flag, a.limit_ns, a.status, true);
+}
+
+// X producer: a sparse tile's metadata and the panel's X slices (M token rows
+// x 64 k each).  The metadata of the first NS stages is requested before this
+// kernel waits for the previous kernel in the stream; X, which may be that
+// kernel's output, only after it has completed.
+__device__ void producer_x(Shared& s, const CUtensorMap* tmap_x, const Args& a, int64_t p0, int64_t p1) {
+  PanelWalk w;
+  w.start(s, a, p0);
+  const uint32_t xb = uint32_t(a.M) * 128;  // an X slice holds M token rows (rows M..15 of the slot are never read back)
+  const int64_t n0 = p1 - p0 < NS ? p1 - p0 : NS;
+  uint32_t first[NS];
+  uint32_t i = 0;
+  int64_t p = p0;
+#pragma unroll
+  for (int j = 0; j < NS; ++j) {
+    if (j >= n0) break;
+    const bool sparse = w.sparse();
+    mbar_expect_tx(&s.full[j], sparse ? 2 * xb + E_BYTES : xb);
+    if (sparse) bulk_load(s.st[j].e, a.meta + uint64_t(w.d.sparse_ordinal) * E_BYTES, E_BYTES, &s.full[j]);
+    first[j] = w.xinfo();
+    w.next(s, a, p + 1 < p1);
+    ++p;
+    ++i;
+  }
+  pdl_wait_previous();
+#pragma unroll
+  for (int j = 0; j < NS; ++j)
+    if (j < n0) load_x(s.st[j], &s.full[j], tmap_x, first[j]);
+  for (; p < p1; ++p, ++i) {
+    const uint32_t st = i % NS;
+    if (!wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false)) break;
+    const bool sparse = w.sparse();
+    mbar_expect_tx(&s.full[st], sparse ? 2 * xb + E_BYTES : xb);
+    if (sparse) bulk_load(s.st[st].e, a.meta + uint64_t(w.d.sparse_ordinal) * E_BYTES, E_BYTES, &s.full[st]);
+    load_x(s.st[st], &s.full[st], tmap_x, w.xinfo());
+    w.next(s, a, p + 1 < p1);
+  }
   for (uint32_t j = (i > NS ? i - NS : 0); j < i; ++j)
     wait_bounded(&s.full[j % NS], (j / NS) & 1, &s.abort_flag, a.limit_ns, a.status, true);
 }
@@ -264,6 +305,37 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& a, int64_t p0, 
   }
   tc_commit(&s.drain);
   wait_bounded(&s.drain, 0, &s.abort_flag, a.limit_ns, a.status, true);
+}
+
+// Sum of the partial rows (row r of the tile row) of covering CTAs c_lo..c_hi,
+// in CTA order (deterministic).  B CTAs at a time: all their loads are issued
+// before the additions; NV float4s (4 tokens each) per partial row at most.
+template <int B, int NV>
+__device__ __forceinline__ void sum_partials(const Args& a, int r, int64_t c_lo, int64_t c_hi, int slot_lo, int nv,
+                                             float (&sum)[BT]) {
+#pragma unroll
+  for (int m = 0; m < BT; ++m) sum[m] = 0.0f;
+  for (int64_t c0 = c_lo; c0 <= c_hi; c0 += B) {
+    float4 part[B][NV];
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      const int64_t c = c0 + j;
+      const float4* src = reinterpret_cast<const float4*>(
+          a.ws + c * WS_FLOATS_PER_CTA + (c == c_lo ? slot_lo : 0) * BT * BM + r * BT);
+#pragma unroll
+      for (int k = 0; k < NV; ++k)
+        part[j][k] = (c <= c_hi && k < nv) ? __ldcg(src + k) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+#pragma unroll
+    for (int j = 0; j < B; ++j)
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        sum[4 * k] += part[j][k].x;
+        sum[4 * k + 1] += part[j][k].y;
+        sum[4 * k + 2] += part[j][k].z;
+        sum[4 * k + 3] += part[j][k].w;
+      }
+  }
 }
 
 __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, int64_t p1) {
@@ -319,31 +391,10 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, in
     const int slot_lo = range_begin(c_lo, a.P, G) < rb ? 1 : 0;
     const int nv = (a.M + 3) / 4;  // float4s per row that carry real tokens
     float sum[BT];
-#pragma unroll
-    for (int m = 0; m < BT; ++m) sum[m] = 0.0f;
-    // covering CTAs 4 at a time: all their loads are issued before the
-    // additions, which run in CTA order (deterministic)
-    for (int64_t c0 = c_lo; c0 <= c_hi; c0 += 4) {
-      float4 part[4][BT / 4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t c = c0 + j;
-        const float4* src = reinterpret_cast<const float4*>(
-            a.ws + c * WS_FLOATS_PER_CTA + (c == c_lo ? slot_lo : 0) * BT * BM + r * BT);
-#pragma unroll
-        for (int k = 0; k < BT / 4; ++k)
-          part[j][k] = (c <= c_hi && k < nv) ? __ldcg(src + k) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int k = 0; k < BT / 4; ++k) {
-          sum[4 * k] += part[j][k].x;
-          sum[4 * k + 1] += part[j][k].y;
-          sum[4 * k + 2] += part[j][k].z;
-          sum[4 * k + 3] += part[j][k].w;
-        }
-    }
+    if (nv <= 2)  // up to 8 tokens: 8 covering CTAs' partials per round of loads
+      sum_partials<8, 2>(a, r, c_lo, c_hi, slot_lo, nv, sum);
+    else
+      sum_partials<4, BT / 4>(a, r, c_lo, c_hi, slot_lo, nv, sum);
 #pragma unroll
     for (int m = 0; m < BT; ++m)
       if (m < a.M) a.Y[int64_t(m) * a.N + n] = f32_to_bf16_rne(sum[m]);
@@ -363,7 +414,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
-      mbar_init(&s.full[i], 1);
+      mbar_init(&s.full[i], 2);  // one arrival per producer thread
       mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < NACC; ++i) {
@@ -412,10 +463,13 @@ __global__ void __launch_bounds__(THREADS, 2)
   const uint32_t tmem = s.tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) producer(s, &tmap_x, &tmap_w, a, p0, p1);
+    if (lane == 0) producer_w(s, &tmap_w, a, p0, p1);
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) mma_issuer(s, tmem, a, p0, p1);
+    __syncwarp();
+  } else if (warp == 6) {
+    if (lane == 0) producer_x(s, &tmap_x, a, p0, p1);
     __syncwarp();
   } else {
     epilogue(s, tmem, a, p0, p1);
