@@ -67,6 +67,7 @@ constexpr int A_BYTES = PATCH_PANEL_BYTES;
 constexpr int B_BYTES = BT * 64 * 2;
 constexpr int E_BYTES = PATCH_META_TILE_BYTES;
 constexpr int EPI_WARP0 = 8;             // warps 8-11 drain row 0, 12-15 row 1
+constexpr int YT = 16;                   // tokens per Y chunk the epilogue stores with one TMA store
 constexpr int THREADS = 32 * (EPI_WARP0 + 4 * ROWS);
 constexpr int MAXTK = 128;               // descriptors of one tile row staged in shared memory (K <= 16384)
 constexpr uint32_t TMEM_COLS = 512;
@@ -80,6 +81,7 @@ struct Shared {
   alignas(1024) uint8_t a[ROWS][NA][A_BYTES];
   alignas(1024) uint8_t b[NB][B_BYTES];
   alignas(128) uint8_t e[ROWS][NE][E_BYTES];
+  alignas(128) uint16_t y[ROWS][2][YT][BM];  // epilogue: bf16 Y chunks (YT tokens x 128 features) per row, 2 buffers
   uint64_t a_full[ROWS][NA], a_empty[ROWS][NA], e_full[ROWS][NE], e_empty[ROWS][NE];
   uint64_t b_full[NB], b_empty[NB];   // b_empty: one arrival per row's MMA thread
   uint64_t acc_full[ROWS], acc_empty[ROWS], drain[ROWS];
@@ -96,7 +98,7 @@ struct Args {
   const uint8_t* meta;
   const patch_tile_desc* desc;
   uint16_t* Y;
-  int M, N, Tn, Tk, n_pairs, n_items;
+  int M, N, Tn, Tk, n_pairs, n_tb, n_items;  // units: row pair rp = item / n_tb, token block tb = item % n_tb
   int bt;                      // tokens per unit: a multiple of 16, at most BT
   uint32_t idesc_dense, idesc_sparse;
   uint64_t limit_ns;
@@ -107,6 +109,9 @@ struct Args {
 // tile rows in row pair rp (the last pair of an odd Tn has one)
 __device__ __forceinline__ int rows_of(int rp, int Tn) { return Tn - ROWS * rp < ROWS ? Tn - ROWS * rp : ROWS; }
 
+// Units run row pair by row pair (all token blocks of a pair are consecutive
+// items), so the CTAs of one wave read a few row pairs' W, which stays in L2
+// while every token block uses it, instead of every wave reading all of W.
 // Units that share an X block (same tb) or W rows (same rp) start their K loop
 // at different tiles, so they do not all hit the same L2 lines at the same
 // moment; only the order of the fp32 sum changes.
@@ -125,7 +130,7 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
   bool ok = true;
   // stage (or, for a pair without row r, complete with no bytes) the descriptor row of an item
   auto stage_row = [&](int item, int buf) {
-    const int rp = item % p.n_pairs;
+    const int rp = item / p.n_tb;
     const bool has = r < rows_of(rp, p.Tn);
     mbar_expect_tx(&s.pdesc_full[r][buf], has ? row_bytes : 0u);
     if (has) bulk_load(s.pdesc[r][buf], p.desc + int64_t(ROWS * rp + r) * p.Tk, row_bytes, &s.pdesc_full[r][buf]);
@@ -134,7 +139,7 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
   if (staged && int(blockIdx.x) < p.n_items) stage_row(blockIdx.x, 0);
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const int rp = item % p.n_pairs, tb = item / p.n_pairs, tn = ROWS * rp + r;
+    const int rp = item / p.n_tb, tb = item % p.n_tb, tn = ROWS * rp + r;
     const int buf = it & 1;
     if (staged) {
       if (!(ok = wait_bounded(&s.pdesc_full[r][buf], (it >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
@@ -187,7 +192,7 @@ __device__ void producer_x(Shared& s, const CUtensorMap* tmap_x, const Args& p) 
   // X may be the previous kernel's output: wait for it before the first X load
   pdl_wait_previous();
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-    const int rp = item % p.n_pairs, tb = item / p.n_pairs;
+    const int rp = item / p.n_tb, tb = item % p.n_tb;
     int kt = k_rotation(rp, tb, p.Tk);
     for (int j = 0; ok && j < p.Tk; ++j, kt = (kt + 1 == p.Tk ? 0 : kt + 1)) {
       for (int h = 0; ok && h < 2; ++h) {
@@ -214,7 +219,7 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
   bool ok = true;
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const bool active = r < rows_of(item % p.n_pairs, p.Tn);
+    const bool active = r < rows_of(item / p.n_tb, p.Tn);
     if (!(ok = wait_bounded(&s.acc_empty[r], (it & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
     tc_fence_after();
     uint32_t accumulate = 0;
@@ -284,28 +289,43 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
   wait_bounded(&s.drain[r], 0, &s.abort_flag, p.limit_ns, p.status, true);
 }
 
-// Epilogue warp: drains its TMEM lane quarter of one row's accumulator.
-__device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
+// Epilogue warps of row r (4 warps, one per TMEM lane quarter): per chunk of
+// YT tokens, each warp loads its 32 features x YT tokens from TMEM, rounds to
+// bf16 and writes them into a shared [YT][128] chunk; one thread then stores
+// the chunk to Y with a TMA store (full 256-byte rows of Y instead of 64-byte
+// pieces).  Two chunk buffers: a buffer is rewritten only after the store
+// that read it has finished reading.
+__device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, const Args& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3;                  // the TMEM lane quarter this warp may access
   const int r = (warp - EPI_WARP0) >> 2;   // the row of the pair it drains
+  const uint32_t bar_id = 1 + r;           // named barrier of the row's 128 epilogue threads
+  const bool leader = warp == EPI_WARP0 + 4 * r && lane == 0;
+  uint32_t chunk = 0;                      // chunks stored by this row so far (buffer = chunk & 1)
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
-    const int rp = item % p.n_pairs, tb = item / p.n_pairs;
-    if (!wait_bounded(&s.acc_full[r], it & 1, &s.abort_flag, p.limit_ns, p.status, false)) break;
+    const int rp = item / p.n_tb, tb = item % p.n_tb;
+    // the four warps of a row take the same decision, so none is left at a barrier
+    const bool ok = wait_bounded(&s.acc_full[r], it & 1, &s.abort_flag, p.limit_ns, p.status, false);
+    if (!named_bar_and(bar_id, 128, ok)) break;
     tc_fence_after();
     if (r < rows_of(rp, p.Tn)) {
-      const int64_t n = int64_t(ROWS * rp + r) * BM + 32 * q + lane;
-      const int m0 = tb * p.bt;
+      const int n0 = (ROWS * rp + r) * BM, m0 = tb * p.bt;
+      const int valid = p.M - m0 < p.bt ? p.M - m0 : p.bt;  // tokens of this unit inside X
       const uint32_t acc = tmem + (uint32_t(32 * q) << 16) + ACC_STRIDE * r;
-      for (int c = 0; c < p.bt / 16; ++c) {
-        if (m0 + 16 * c >= p.M) break;  // warp-uniform
-        uint32_t v[16];
-        tmem_ld_16cols(acc + uint32_t(16 * c), v);
+      for (int c = 0; c * YT < valid; ++c, ++chunk) {
+        uint32_t v[YT];
+        tmem_ld_16cols(acc + uint32_t(YT * c), v);
+        uint16_t(*buf)[BM] = s.y[r][chunk & 1];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = m0 + 16 * c + j;
-          if (m < p.M) p.Y[int64_t(m) * p.N + n] = f32_to_bf16_rne(__uint_as_float(v[j]));
+        for (int j = 0; j < YT; ++j) buf[j][32 * q + lane] = f32_to_bf16_rne(__uint_as_float(v[j]));
+        fence_proxy_async_smem();
+        if (leader) bulk_wait_read_all();  // the previous chunk's store has read the other buffer
+        named_bar_sync(bar_id, 128);
+        // token rows past M are clipped by the store
+        if (leader) {
+          tma_store_2d(tmap_y, buf, n0, m0 + YT * c);
+          bulk_commit_group();
         }
       }
     }
@@ -313,11 +333,12 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.acc_empty[r]);
   }
+  if (leader) bulk_wait_all();  // Y written before the CTA exits
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   const Args p) {
+                   const __grid_constant__ CUtensorMap tmap_y, const Args p) {
   extern __shared__ uint8_t smem_raw[];
   Shared& s = *reinterpret_cast<Shared*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -347,6 +368,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tensormap(&tmap_x);
     prefetch_tensormap(&tmap_w);
+    prefetch_tensormap(&tmap_y);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -373,7 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) producer_x(s, &tmap_x, p);
     __syncwarp();
   } else if (warp >= EPI_WARP0) {
-    epilogue(s, tmem, p);
+    epilogue(s, tmem, &tmap_y, p);
   }
 
   tc_fence_before();
@@ -420,6 +442,19 @@ bool make_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Y [M][N] bf16 as a TMA store target: boxes of 16 token rows x 128 features,
+// no swizzle (the epilogue writes the chunk row-major).
+static bool make_map_y(CUtensorMap* map, void* Y, uint64_t N, uint64_t M) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {N, M};
+  const cuuint64_t strides[1] = {N * 2};
+  const cuuint32_t box[2] = {uint32_t(prefill::BM), uint32_t(prefill::YT)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tokens per unit: the multiple of 16 in [64, BT] that minimises the time of
 // the slowest CTA, modelled as (units per CTA, rounded up) x (unit time).  A
 // unit's K-tile costs the larger of its tensor-core cycles (8 bt: 2 rows x
@@ -450,10 +485,11 @@ cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, 
   const uint64_t n_panels = uint64_t(2 * (T - W.n_sparse) + W.n_sparse);
   const int64_t n_pairs = (Tn + ROWS - 1) / ROWS;
   const int bt = pick_bt(M, n_pairs, Tk, num_sms);
-  CUtensorMap tmap_x, tmap_w;
+  CUtensorMap tmap_x, tmap_w, tmap_y;
   if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, uint32_t(bt)))
     return cudaErrorUnknown;
   if (!make_map_2d_bf16(&tmap_w, W.values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
+  if (!make_map_y(&tmap_y, Y, uint64_t(W.N), uint64_t(M))) return cudaErrorUnknown;
   Args p;
   p.meta = static_cast<const uint8_t*>(W.meta);
   p.desc = W.desc;
@@ -463,7 +499,8 @@ cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, 
   p.Tn = int(Tn);
   p.Tk = int(Tk);
   p.n_pairs = int(n_pairs);
-  p.n_items = int(n_pairs * ((M + bt - 1) / bt));
+  p.n_tb = int((M + bt - 1) / bt);
+  p.n_items = int(n_pairs) * p.n_tb;
   p.bt = bt;
   p.idesc_dense = tc::idesc_bf16(BM, bt, false);
   p.idesc_sparse = tc::idesc_bf16(BM, bt, true);
@@ -473,7 +510,8 @@ cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, 
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES));
   if (e != cudaSuccess) return e;
-  return launch_pdl(prefill_kernel, dim3(unsigned(grid)), dim3(THREADS), SMEM_BYTES, stream, tmap_x, tmap_w, p);
+  return launch_pdl(prefill_kernel, dim3(unsigned(grid)), dim3(THREADS), SMEM_BYTES, stream, tmap_x, tmap_w, tmap_y,
+                    p);
 }
 
 }  // namespace patch
