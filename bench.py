@@ -295,6 +295,24 @@ def offline_steps(layers, dev, pk, reps=5):
 # ------------------------------------------------------------ GPU arm
 
 
+def job_times(ms, e2e_ms, world, dev=None):
+    """Timed-region and end-to-end times (ms) of the whole job: the maximum over
+    ranks, since the job ends when its slowest rank does."""
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    return ms, e2e_ms
+
+
+def job_throughput(per_step_units, steps, world, ms):
+    """Whole-job throughput of `world` replicas that each process per_step_units
+    per step (weak scaling): all ranks' units over the job's time."""
+    return per_step_units * steps * world / (ms / 1e3)
+
+
 def run_ours(args, rank, world):
     import torch
     import torch.distributed as dist
@@ -421,10 +439,7 @@ def run_ours(args, rank, world):
     barrier()
     e2e_ms = e0.elapsed_time(e1)
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = job_times(ms, e2e_ms, world, dev)
 
     if args.workload == "decode":
         unit, per_step = "GB/s", sum(call_bytes(layers[li], M) for li, M in calls) / 1e9
@@ -432,8 +447,8 @@ def run_ours(args, rank, world):
     else:
         unit, per_step = "TFLOP/s", sum(call_flops(layers[li], M) for li, M in calls) / 1e12
         metric = "hybrid GEMM TFLOP/s, dense-equivalent (prefill)"
-    value = per_step * args.steps * world / (ms / 1e3)
-    e2e_value = per_step * args.steps * world / (e2e_ms / 1e3)
+    value = job_throughput(per_step, args.steps, world, ms)
+    e2e_value = job_throughput(per_step, args.steps, world, e2e_ms)
 
     # roofline of the dominant kernel: algorithmic bytes (or FLOPs) per launch / mean launch time.
     # Every call of the step is one launch of that kernel, so the mean over the
