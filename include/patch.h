@@ -190,13 +190,19 @@ PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight
  *     leaves it zero-filled again (the decode path keeps per-row arrival
  *     counters there), so one zero-fill at allocation suffices.  After a call
  *     that reported an error, zero it again.
- * M <= 16 runs the decode path: one CTA per SM streams an equal share of
- * the stored panels through a TMA ring (stream-K), the tensor cores reduce
+ * M <= 16 runs the decode path: 1.5 CTAs per SM each stream an equal share
+ * of the stored panels through a TMA ring (stream-K), the tensor cores reduce
  * them (N = 16 tokens, zero-padded); a tile row cut between CTAs is finished
  * by the last CTA to reach it, which adds the fp32 partials in the
  * workspace in CTA order (deterministic).
- * Larger M runs the prefill path (TMA-fed tcgen05 kernel, dense and sparse
- * MMAs into one TMEM fp32 tile per 128 x 256 output tile).
+ * Larger M runs the prefill path (TMA-fed tcgen05 kernel: each CTA takes two
+ * tile rows x up to 240 tokens at a time, dense and sparse MMAs into one TMEM
+ * fp32 accumulator per tile row).
+ * The kernels are launched with programmatic dependent launch: they read W,
+ * its metadata and descriptors before the previous kernel in the stream has
+ * completed, and X only after.  X may therefore be that kernel's output; the
+ * packed weight must not be written by a kernel that allows an early launch
+ * of its successor (patch_pack does not).
  * A bounded wait that runs out sets PATCH_DEV_TIMEOUT (Y is then undefined).
  */
 PATCH_API patch_status_t patch_gemm(const uint16_t *X, int64_t M, const patch_weight *W, uint16_t *Y,
