@@ -246,15 +246,16 @@ def cpu_baseline(workload, budget_s=15.0, min_s=0.0):
 
 def offline_steps(layers, dev, pk, reps=5):
     """HBM throughput of the once-per-model steps on the step's layers: the hard
-    mask (argmax of tile and pattern logits, masked W) and the packer."""
+    mask (argmax of tile and pattern logits, masked W), the packer, and the
+    fused path (tile kinds, then a pack that takes the pattern argmax itself)."""
     import torch
 
     import tile_sparse_gemm_b200 as tsg
 
     out = {}
     status = tsg.new_status(dev)
-    mask_bytes = pack_bytes = 0
-    mask_ms = pack_ms = 0.0
+    mask_bytes = pack_bytes = fused_bytes = 0
+    mask_ms = pack_ms = fused_ms = 0.0
     for i, L in enumerate(layers):
         N, K = L["N"], L["K"]
         w = torch.from_numpy(L["w"].view(np.int16)).view(torch.bfloat16).to(dev)
@@ -266,7 +267,10 @@ def offline_steps(layers, dev, pk, reps=5):
         for _ in range(2):
             tsg.patch_hard_mask(w, tl, pl, status=status)
             tsg.patch_pack(w, bm, ids, ns, status=status)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        fbm, fns = tsg.patch_tile_kinds(tl)
+        fns = int(fns.item())
+        tsg.patch_pack_from_logits(w, fbm, pl, fns, status=status)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         torch.cuda.synchronize()
         e[0].record()
         for _ in range(reps):
@@ -275,9 +279,17 @@ def offline_steps(layers, dev, pk, reps=5):
         for _ in range(reps):
             tsg.patch_pack(w, bm, ids, ns, status=status)
         e[2].record()
+        for _ in range(reps):  # fused: tile kinds, then pack with the pattern argmax inside
+            tsg.patch_tile_kinds(tl)
+            tsg.patch_pack_from_logits(w, fbm, pl, fns, status=status)
+        e[3].record()
         torch.cuda.synchronize()
         mask_ms += e[0].elapsed_time(e[1]) / reps
         pack_ms += e[1].elapsed_time(e[2]) / reps
+        fused_ms += e[2].elapsed_time(e[3]) / reps
+        T = (N // 128) * (K // 128)
+        # reads W, the tile logits and the pattern logits of sparse tiles; writes the bitmap and the blobs
+        fused_bytes += 2 * N * K + 8 * T + 6 * fns * 128 * 128 + T + stored_bytes(N, K, fns)
         mask_bytes += N * K * (2 + 6 + 2) + N * K // 4 + (N // 128) * (K // 128) * 9
         # reads W (dense tiles whole, sparse tiles whole 16 B rows) + ids of sparse tiles + bitmap; writes the blobs
         pack_bytes += 2 * N * K + ns * 128 * 32 + (N // 128) * (K // 128) + stored_bytes(N, K, ns)
@@ -285,7 +297,8 @@ def offline_steps(layers, dev, pk, reps=5):
     code, bits = tsg.patch_read_status(status)
     if code != 0:
         raise RuntimeError(f"offline steps: device status {code} bits {bits}")
-    for name, b, ms in (("hard_mask", mask_bytes, mask_ms), ("pack", pack_bytes, pack_ms)):
+    for name, b, ms in (("hard_mask", mask_bytes, mask_ms), ("pack", pack_bytes, pack_ms),
+                        ("tile_kinds+pack_from_logits", fused_bytes, fused_ms)):
         gbs = b / 1e9 / (ms / 1e3)
         out[name] = {"GB/s": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4), "ms_total": round(ms, 3),
                      "bytes": int(b), "note": "7 LLaMA-2-7B layers, mean of %d calls each (eager launches)" % reps}

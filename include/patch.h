@@ -172,6 +172,39 @@ PATCH_API patch_status_t patch_pack(const uint16_t *W, int64_t N, int64_t K, con
                           patch_tile_desc *desc, int32_t *dev_status, void *stream);
 
 /*
+ * patch_tile_kinds: the tile half of the hard mask alone ("Learnable
+ * Distributions", item 1: a 2-way logit per tile chooses dense or 2:4 sparse).
+ *   tile_logits fp32 [Tn][Tk][2] (index 0 = dense, 1 = sparse);
+ *   bitmap      u8 [Tn][Tk] out: 1 where logit[1] > logit[0] (ties -> dense),
+ *               the same decision patch_hard_mask takes;
+ *   n_sparse    one int64 on the DEVICE out: the number of sparse tiles (the
+ *               caller reads it to size the packed blobs with patch_pack_sizes).
+ * One launch, no other memory touched.  Errors: PATCH_ERR_INVALID_ARG (NULL),
+ * PATCH_ERR_SHAPE, PATCH_ERR_ALIGN (tile_logits or n_sparse not 8-byte aligned),
+ * PATCH_ERR_DEVICE.
+ */
+PATCH_API patch_status_t patch_tile_kinds(const float *tile_logits, int64_t N, int64_t K, uint8_t *bitmap,
+                                          int64_t *n_sparse, void *stream);
+
+/*
+ * patch_pack_from_logits: hard mask and pack in one pass, without the masked
+ * weight or the pattern ids in memory.  Same output as patch_hard_mask
+ * followed by patch_pack: every sparse tile's pattern ids are the argmax of
+ * its 6 pattern logits per group (first maximum wins, as in patch_hard_mask),
+ * taken inside the pack kernel; the pattern logits of dense tiles are never
+ * read.  (Frozen pattern ids, as in the paper's tile-only variant, go through
+ * patch_pack with pat_id instead.)
+ *   W bf16 [N][K]; bitmap u8 [Tn][Tk] (from patch_tile_kinds or patch_hard_mask);
+ *   pattern_logits fp32 [N][K/4][6] (16-byte aligned); n_sparse, values,
+ *   meta, desc, dev_status as for patch_pack (PATCH_DEV_COUNT on a count
+ *   mismatch, nothing written past the blob sizes).
+ */
+PATCH_API patch_status_t patch_pack_from_logits(const uint16_t *W, int64_t N, int64_t K, const uint8_t *bitmap,
+                                                const float *pattern_logits, int64_t n_sparse, void *values,
+                                                void *meta, patch_tile_desc *desc, int32_t *dev_status,
+                                                void *stream);
+
+/*
  * patch_gemm_workspace_size: device scratch bytes patch_gemm needs for M rows
  * of X and this weight (0 when none is needed; for M <= 16 enough for either
  * decode kernel).  Host only, but queries the current device's SM count.

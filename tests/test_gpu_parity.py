@@ -116,6 +116,89 @@ def test_pack_of_masked_and_random_patterns():
     assert np.array_equal(pw.desc.cpu().numpy(), d_ref)
 
 
+# ------------------------------------------------- fused hard mask -> pack
+
+
+@pytest.mark.parametrize("N,K,cfg", [(512, 512, 1), (128, 128, 0), (384, 640, 7), (1024, 256, 8)])
+def test_tile_kinds_and_pack_from_logits_bit_exact(N, K, cfg):
+    """Tile kinds from the tile logits and a pack that takes each sparse tile's
+    pattern ids as the argmax of its pattern logits: the oracle's hard mask
+    followed by its pack, byte for byte, without the masked W or the ids."""
+    w = si.gen_w(N, K, cfg, 1)
+    tl = si.gen_tile_logits(N, K, cfg, 1)
+    pl = si.gen_pattern_logits(N, K, cfg, 1)
+    _, bm_ref, id_ref = oracle.hard_mask(w, tl, pl)
+    v_ref, m_ref, d_ref = oracle.pack(w, bm_ref, id_ref)
+    bitmap, n_dev = tsg.patch_tile_kinds(to_dev(tl))
+    assert np.array_equal(bitmap.cpu().numpy(), bm_ref)
+    assert int(n_dev.item()) == int(bm_ref.sum())
+    status = tsg.new_status()
+    pw = tsg.patch_pack_from_logits(to_dev_bf16(w), bitmap, to_dev(pl), int(n_dev.item()), status=status)
+    assert tsg.patch_read_status(status)[0] == 0
+    assert np.array_equal(pw.desc.cpu().numpy(), d_ref)
+    assert np.array_equal(pw.values.cpu().numpy(), v_ref)
+    assert np.array_equal(pw.meta.cpu().numpy(), m_ref)
+
+
+def test_pack_from_logits_ties_and_nan_match_the_hard_mask():
+    N = K = 256
+    w = si.gen_w(N, K, 6, 0)
+    tl = np.array([[[0.0, 0.0], [0.0, 1.0]], [[np.nan, 1.0], [-1.0, 2.0]]], np.float32)
+    rng = np.random.default_rng(3)
+    pl = rng.integers(-2, 3, (N, K // 4, 6)).astype(np.float32)  # many ties
+    pl[::7, ::5, 3] = np.nan
+    pl[::11, ::3, 0] = np.nan
+    _, bm_ref, id_ref = oracle.hard_mask(w, tl, pl)
+    v_ref, m_ref, d_ref = oracle.pack(w, bm_ref, id_ref)
+    bitmap, n_dev = tsg.patch_tile_kinds(to_dev(tl))
+    pw = tsg.patch_pack_from_logits(to_dev_bf16(w), bitmap, to_dev(pl), int(n_dev.item()))
+    assert bm_ref.tolist() == [[0, 1], [0, 1]]
+    assert np.array_equal(pw.values.cpu().numpy(), v_ref)
+    assert np.array_equal(pw.meta.cpu().numpy(), m_ref)
+    assert np.array_equal(pw.desc.cpu().numpy(), d_ref)
+
+
+def test_fused_and_two_step_mask_pack_agree_and_multiply_alike():
+    """hard mask -> pack and tile kinds -> pack-from-logits give the same blobs,
+    and a GEMM on them matches the oracle."""
+    N, K, M = 384, 512, 8
+    w = si.gen_w(N, K, 9, 2)
+    tl = si.gen_tile_logits(N, K, 9, 2)
+    pl = si.gen_pattern_logits(N, K, 9, 2)
+    _, bm2, ids2 = tsg.patch_hard_mask(to_dev_bf16(w), to_dev(tl), to_dev(pl), want_masked=False)
+    two = tsg.patch_pack(to_dev_bf16(w), bm2, ids2)
+    bitmap, n_dev = tsg.patch_tile_kinds(to_dev(tl))
+    one = tsg.patch_pack_from_logits(to_dev_bf16(w), bitmap, to_dev(pl), int(n_dev.item()))
+    for a, b in ((one.values, two.values), (one.meta, two.meta), (one.desc, two.desc)):
+        assert torch.equal(a, b)
+    x = si.gen_x(M, K, 9, 2)
+    _, bm_ref, id_ref = oracle.hard_mask(w, tl, pl)
+    check_gemm(gemm_on_gpu(x, one), oracle.hybrid_gemm(x, w, bm_ref, id_ref), "fused mask-pack GEMM")
+
+
+def test_pack_from_logits_count_mismatch_flagged_without_overrun():
+    import ctypes
+    N = K = 256
+    w = si.gen_w(N, K, 4, 0)
+    pl = si.gen_pattern_logits(N, K, 4, 0)
+    bm = np.array([[1, 1], [0, 1]], np.uint8)  # 3 sparse tiles
+    vb, mb, db = tsg.patch_pack_sizes(N, K, 2)
+    guard = 4096
+    values = torch.full((vb + guard,), 0xAB, dtype=torch.uint8, device="cuda")
+    meta = torch.full((mb + guard,), 0xCD, dtype=torch.uint8, device="cuda")
+    desc = torch.zeros(db, dtype=torch.uint8, device="cuda")
+    status = tsg.new_status()
+    rc = tsg.lib().patch_pack_from_logits(
+        ctypes.c_void_p(to_dev_bf16(w).data_ptr()), N, K, ctypes.c_void_p(to_dev(bm).data_ptr()),
+        ctypes.c_void_p(to_dev(pl).data_ptr()), 2, ctypes.c_void_p(values.data_ptr()),
+        ctypes.c_void_p(meta.data_ptr()), ctypes.c_void_p(desc.data_ptr()), ctypes.c_void_p(status.data_ptr()),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    code, bits = tsg.patch_read_status(status)
+    assert code == 9 and bits & tsg.DEV_COUNT
+    assert torch.all(values[vb:] == 0xAB) and torch.all(meta[mb:] == 0xCD)
+
+
 def test_pack_flags_bad_pattern_id():
     N = K = 256
     w = si.gen_w(N, K, 6, 0)

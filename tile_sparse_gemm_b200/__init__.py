@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
             "patch_pack_sizes": [I64, I64, I64, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)],
             "patch_hard_mask": [P, I64, I64, P, P, P, P, P, P, P],
             "patch_pack": [P, I64, I64, P, P, I64, P, P, P, P, P],
+            "patch_tile_kinds": [P, I64, I64, P, P, P],
+            "patch_pack_from_logits": [P, I64, I64, P, P, I64, P, P, P, P, P],
             "patch_gemm_workspace_size": [I64, WP, ctypes.POINTER(SZ)],
             "patch_gemm": [P, I64, WP, P, P, SZ, P, P],
             "patch_gemm_ex": [P, I64, WP, P, P, SZ, P, P, I32, ctypes.c_uint64],
@@ -172,6 +174,42 @@ def patch_pack(W: torch.Tensor, bitmap: torch.Tensor, pat_id: torch.Tensor, n_sp
     _check(lib().patch_pack(_dev(W, "W"), N, K, _dev(bitmap, "bitmap"), _dev(pat_id, "pat_id"), n_sparse,
                             _dev(values, "values"), _dev(meta, "meta") if mb else None, _dev(desc, "desc"),
                             _dev(status, "status"), _stream(stream)), "patch_pack")
+    return PackedWeight(N, K, n_sparse, values, meta, desc)
+
+
+def patch_tile_kinds(tile_logits: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Tile kinds (argmax of the 2 tile logits, ties -> dense) of fp32
+    tile_logits [Tn][Tk][2]: (bitmap u8 [Tn][Tk], n_sparse int64 [1]), both on
+    the device."""
+    Tn, Tk, two = tile_logits.shape
+    if two != 2:
+        raise ValueError("tile_logits must be [Tn][Tk][2]")
+    dev = tile_logits.device
+    bitmap = torch.empty((Tn, Tk), dtype=torch.uint8, device=dev)
+    n_sparse = torch.empty(1, dtype=torch.int64, device=dev)
+    _check(lib().patch_tile_kinds(_dev(tile_logits, "tile_logits"), Tn * 128, Tk * 128, _dev(bitmap, "bitmap"),
+                                  _dev(n_sparse, "n_sparse"), _stream(stream)), "patch_tile_kinds")
+    return bitmap, n_sparse
+
+
+def patch_pack_from_logits(W: torch.Tensor, bitmap: torch.Tensor, pattern_logits: torch.Tensor,
+                           n_sparse: int | None = None, status: torch.Tensor | None = None,
+                           stream=None) -> PackedWeight:
+    """Hard mask and pack in one pass: like patch_pack, with each sparse tile's
+    pattern ids the argmax of its pattern logits (fp32 [N][K/4][6])."""
+    N, K = W.shape
+    if n_sparse is None:
+        n_sparse = int(torch.count_nonzero(bitmap).item())
+    vb, mb, db = patch_pack_sizes(N, K, n_sparse)
+    dev = W.device
+    status = new_status(dev) if status is None else status
+    values = torch.empty(vb, dtype=torch.uint8, device=dev)
+    meta = torch.empty(mb, dtype=torch.uint8, device=dev)
+    desc = torch.empty(db, dtype=torch.uint8, device=dev)
+    _check(lib().patch_pack_from_logits(_dev(W, "W"), N, K, _dev(bitmap, "bitmap"),
+                                        _dev(pattern_logits, "pattern_logits"), n_sparse, _dev(values, "values"),
+                                        _dev(meta, "meta") if mb else None, _dev(desc, "desc"),
+                                        _dev(status, "status"), _stream(stream)), "patch_pack_from_logits")
     return PackedWeight(N, K, n_sparse, values, meta, desc)
 
 

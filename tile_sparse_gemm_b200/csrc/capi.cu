@@ -102,7 +102,41 @@ patch_status_t patch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t
   int sms = 0;
   patch_status_t st = device_sms(&sms);
   if (st != PATCH_OK) return st;
-  if (launch_pack(W, N, K, bitmap, pat_id, n_sparse, values, meta, desc, dev_status, sms,
+  if (launch_pack(W, N, K, bitmap, pat_id, nullptr, n_sparse, values, meta, desc, dev_status, sms,
+                  static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
+patch_status_t patch_tile_kinds(const float* tile_logits, int64_t N, int64_t K, uint8_t* bitmap,
+                                int64_t* n_sparse, void* stream) {
+  if (!tile_logits || !bitmap || !n_sparse) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return PATCH_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(tile_logits) % 8 || reinterpret_cast<uintptr_t>(n_sparse) % 8)
+    return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_tile_kinds(tile_logits, N, K, bitmap, n_sparse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
+patch_status_t patch_pack_from_logits(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap,
+                                      const float* pattern_logits, int64_t n_sparse, void* values, void* meta,
+                                      patch_tile_desc* desc, int32_t* dev_status, void* stream) {
+  if (!W || !bitmap || !pattern_logits || !values || !desc || !dev_status) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return PATCH_ERR_SHAPE;
+  const int64_t T = (N / kTile) * (K / kTile);
+  if (n_sparse < 0 || n_sparse > T) return PATCH_ERR_INVALID_ARG;
+  if (n_sparse > 0 && !meta) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(pattern_logits) || !aligned16(values) || !aligned16(desc) ||
+      (meta && !aligned16(meta)))
+    return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_pack(W, N, K, bitmap, nullptr, pattern_logits, n_sparse, values, meta, desc, dev_status, sms,
                   static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return PATCH_ERR_CUDA;
   return PATCH_OK;

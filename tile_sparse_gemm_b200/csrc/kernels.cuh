@@ -14,9 +14,13 @@ cudaError_t launch_hard_mask(const uint16_t* W, int64_t N, int64_t K, const floa
                              const float* pattern_logits, uint16_t* W_masked, uint8_t* bitmap,
                              uint8_t* pat_id, int num_sms, cudaStream_t stream);
 
+// pattern ids from pat_id, or (pattern_logits != NULL) from the argmax of the pattern logits
 cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap,
-                        const uint8_t* pat_id, int64_t n_sparse, void* values, void* meta,
-                        patch_tile_desc* desc, int32_t* status, int num_sms, cudaStream_t stream);
+                        const uint8_t* pat_id, const float* pattern_logits, int64_t n_sparse, void* values,
+                        void* meta, patch_tile_desc* desc, int32_t* status, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_tile_kinds(const float* tile_logits, int64_t N, int64_t K, uint8_t* bitmap, int64_t* n_sparse,
+                              cudaStream_t stream);
 
 // Decode split: L K-tiles per unit, S K-splits, units CTAs, smem bytes, fp32 workspace bytes.
 struct DecodePlan {

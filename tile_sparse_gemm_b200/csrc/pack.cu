@@ -9,7 +9,9 @@
 // order -> descriptors {kind, sparse ordinal, byte offset}.
 // Launch 2 (one CTA per tile): dense tile -> 2 panels of 128 x 64 bf16;
 // sparse tile -> 1 panel of kept values + 2048 B of metadata in the order the
-// tensor-core sparse MMA reads it.  Integer/bit work only; HBM-bound.
+// tensor-core sparse MMA reads it.  HBM-bound.  The pattern ids come either
+// from pat_id or, fused with the hard mask, from the argmax of the pattern
+// logits of sparse tiles only ("Learnable Distributions", item 2).
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -64,10 +66,29 @@ __global__ void __launch_bounds__(kScanThreads) pack_scan_kernel(
   if (threadIdx.x == 0 && carry_s != uint64_t(n_sparse)) set_status(status, PATCH_DEV_COUNT);
 }
 
+// Index of the first maximum of 6 logits (a later value wins only when
+// strictly greater): the pattern decision of patch_hard_mask.
+__device__ __forceinline__ uint32_t argmax6_first(const float* v) {
+  uint32_t best = 0;
+  float bv = v[0];
+#pragma unroll
+  for (uint32_t j = 1; j < 6; ++j) {
+    if (v[j] > bv) {
+      bv = v[j];
+      best = j;
+    }
+  }
+  return best;
+}
+
+// FROM_LOGITS: a sparse tile's pattern ids are the argmax of its pattern
+// logits (fused hard mask); otherwise they are read from pat_id.
+template <bool FROM_LOGITS>
 __global__ void __launch_bounds__(256) pack_tiles_kernel(
     const uint16_t* __restrict__ W, int64_t K, const uint8_t* __restrict__ pat_id,
-    const patch_tile_desc* __restrict__ desc, int64_t T, int64_t n_sparse, uint64_t values_bytes,
-    uint8_t* __restrict__ values, uint8_t* __restrict__ meta, int32_t* status) {
+    const float4* __restrict__ pattern_logits, const patch_tile_desc* __restrict__ desc, int64_t T,
+    int64_t n_sparse, uint64_t values_bytes, uint8_t* __restrict__ values, uint8_t* __restrict__ meta,
+    int32_t* status) {
   __shared__ __align__(16) uint8_t meta_s[PATCH_META_TILE_BYTES];
   const int64_t Tk = K / kTile;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
@@ -91,13 +112,31 @@ __global__ void __launch_bounds__(256) pack_tiles_kernel(
       for (int c = threadIdx.x; c < 2048; c += blockDim.x) {
         const int r = c >> 4, p = c & 15;
         const uint4 w = __ldcs(reinterpret_cast<const uint4*>(wt + int64_t(r) * K + p * 8));
-        const uint16_t ids2 = *reinterpret_cast<const uint16_t*>(
-            pat_id + (tn * kTile + r) * (K / 4) + tk * 32 + 2 * p);
-        uint32_t id0 = ids2 & 0xFF, id1 = ids2 >> 8;
-        if (id0 > 5 || id1 > 5) {
-          set_status(status, PATCH_DEV_BAD_PATTERN);
-          if (id0 > 5) id0 = 0;
-          if (id1 > 5) id1 = 0;
+        // groups 2p, 2p+1 of row r of the tile
+        const int64_t group = (tn * kTile + r) * (K / 4) + tk * 32 + 2 * p;
+        uint32_t id0, id1;
+        if constexpr (FROM_LOGITS) {
+          // 2 groups x 6 logits = 48 contiguous bytes, 16-byte aligned
+          float lg[12];
+#pragma unroll
+          for (int q = 0; q < 3; ++q) {
+            const float4 v = __ldcs(pattern_logits + group * 6 / 4 + q);
+            lg[4 * q] = v.x;
+            lg[4 * q + 1] = v.y;
+            lg[4 * q + 2] = v.z;
+            lg[4 * q + 3] = v.w;
+          }
+          id0 = argmax6_first(lg);
+          id1 = argmax6_first(lg + 6);
+        } else {
+          const uint16_t ids2 = *reinterpret_cast<const uint16_t*>(pat_id + group);
+          id0 = ids2 & 0xFF;
+          id1 = ids2 >> 8;
+          if (id0 > 5 || id1 > 5) {
+            set_status(status, PATCH_DEV_BAD_PATTERN);
+            if (id0 > 5) id0 = 0;
+            if (id1 > 5) id1 = 0;
+          }
         }
         const uint32_t c0 = pattern_code(id0), c1 = pattern_code(id1);
         // the 4 bf16 of each group as one 64-bit word; position i is bits 16i..16i+15
@@ -118,9 +157,8 @@ __global__ void __launch_bounds__(256) pack_tiles_kernel(
 }
 
 cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap,
-                        const uint8_t* pat_id, int64_t n_sparse, void* values, void* meta,
-                        patch_tile_desc* desc, int32_t* status, int num_sms,
-                        cudaStream_t stream) {
+                        const uint8_t* pat_id, const float* pattern_logits, int64_t n_sparse, void* values,
+                        void* meta, patch_tile_desc* desc, int32_t* status, int num_sms, cudaStream_t stream) {
   const int64_t T = (N / kTile) * (K / kTile);
   const uint64_t values_bytes =
       uint64_t(T - n_sparse) * PATCH_DENSE_TILE_BYTES + uint64_t(n_sparse) * PATCH_SPARSE_TILE_BYTES;
@@ -128,9 +166,41 @@ cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   int64_t blocks = T < int64_t(num_sms) * 16 ? T : int64_t(num_sms) * 16;
-  pack_tiles_kernel<<<int(blocks), 256, 0, stream>>>(W, K, pat_id, desc, T, n_sparse, values_bytes,
-                                                     static_cast<uint8_t*>(values),
-                                                     static_cast<uint8_t*>(meta), status);
+  if (pattern_logits)
+    pack_tiles_kernel<true><<<int(blocks), 256, 0, stream>>>(
+        W, K, nullptr, reinterpret_cast<const float4*>(pattern_logits), desc, T, n_sparse, values_bytes,
+        static_cast<uint8_t*>(values), static_cast<uint8_t*>(meta), status);
+  else
+    pack_tiles_kernel<false><<<int(blocks), 256, 0, stream>>>(W, K, pat_id, nullptr, desc, T, n_sparse,
+                                                              values_bytes, static_cast<uint8_t*>(values),
+                                                              static_cast<uint8_t*>(meta), status);
+  return cudaGetLastError();
+}
+
+// Tile kinds from the tile logits (argmax of 2, ties -> dense) and their count.
+__global__ void __launch_bounds__(kScanThreads) tile_kinds_kernel(const float2* __restrict__ tile_logits, int64_t T,
+                                                                  uint8_t* __restrict__ bitmap,
+                                                                  int64_t* __restrict__ n_sparse) {
+  __shared__ int64_t total;
+  if (threadIdx.x == 0) total = 0;
+  __syncthreads();
+  int64_t mine = 0;
+  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
+    const float2 l = tile_logits[t];
+    const uint8_t sparse = l.y > l.x ? 1 : 0;
+    bitmap[t] = sparse;
+    mine += sparse;
+  }
+  atomicAdd(reinterpret_cast<unsigned long long*>(&total), static_cast<unsigned long long>(mine));
+  __syncthreads();
+  if (threadIdx.x == 0) *n_sparse = total;
+}
+
+cudaError_t launch_tile_kinds(const float* tile_logits, int64_t N, int64_t K, uint8_t* bitmap, int64_t* n_sparse,
+                              cudaStream_t stream) {
+  const int64_t T = (N / kTile) * (K / kTile);
+  tile_kinds_kernel<<<1, kScanThreads, 0, stream>>>(reinterpret_cast<const float2*>(tile_logits), T, bitmap,
+                                                    n_sparse);
   return cudaGetLastError();
 }
 
