@@ -160,11 +160,35 @@ class ClockSampler:
 # ------------------------------------------------------------ workloads
 
 
+def is_decode(workload):
+    return workload in ("decode", "decode_fused")
+
+
 def build_layers(workload, only=None, fracs=None, tokens=None):
     """Host inputs of every layer in the step: list of dicts.  `only`, `fracs` and
     `tokens` select a subset (profiling runs); the default is the whole workload."""
     layers = []
-    ms = tuple(tokens) if tokens else (DECODE_MS if workload == "decode" else (PREFILL_M,))
+    ms = tuple(tokens) if tokens else (DECODE_MS if is_decode(workload) else (PREFILL_M,))
+    if workload == "decode_fused":
+        # q|k|v and gate|up as single GEMMs over row-concatenated weights (the
+        # usual fused projections; tiles stay whole), o and down alone; the same
+        # weights, tile choices and patterns as the "decode" workload
+        members = {}
+        for i, (name, N, K) in enumerate(si.LLAMA2_7B):
+            w = si.gen_w(N, K, DECODE_CONFIG, i)
+            f = fracs[0] if fracs else 0.5
+            members[name] = (i, w, si.tiles_exact(N, K, f, DECODE_CONFIG, i), si.patterns_top2(w), f)
+        for name, parts in (("qkv", ("q", "k", "v")), ("o", ("o",)), ("gate_up", ("gate", "up")), ("down", ("down",))):
+            if only and name not in only:
+                continue
+            i0, _, _, _, f = members[parts[0]]
+            w = np.concatenate([members[m][1] for m in parts])
+            bm = np.concatenate([members[m][2] for m in parts])
+            ids = np.concatenate([members[m][3] for m in parts])
+            N, K = w.shape
+            layers.append(dict(name=name, N=N, K=K, w=w, bm=bm, ids=ids, frac=f,
+                               xs={M: si.gen_x(M, K, DECODE_CONFIG, i0) for M in ms}))
+        return layers
     if workload == "decode":
         for i, (name, N, K) in enumerate(si.LLAMA2_7B):
             if only and name not in only:
@@ -223,7 +247,7 @@ def cpu_baseline(workload, budget_s=15.0, min_s=0.0):
             oracle.hybrid_gemm(x, L["w"], L["bm"], L["ids"], rows=rows)
             dt = time.perf_counter() - t0
             spent += dt
-            if workload == "decode":
+            if is_decode(workload):
                 done_units += call_bytes(L, M) / 1e9
                 if passes == 1:
                     what.append(f"{L['name']}@M={M}")
@@ -235,9 +259,9 @@ def cpu_baseline(workload, budget_s=15.0, min_s=0.0):
                 break
         if spent >= budget_s or spent >= min_s:
             break
-    return {"value": done_units / spent, "unit": "GB/s" if workload == "decode" else "TFLOP/s",
+    return {"value": done_units / spent, "unit": "GB/s" if is_decode(workload) else "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle", "seconds": round(spent, 3), "passes": passes,
-            "sample": ("decode GEMMs " if workload == "decode" else "prefill GEMMs, 16 of 2048 token rows each: ")
+            "sample": ("decode GEMMs " if is_decode(workload) else "prefill GEMMs, 16 of 2048 token rows each: ")
             + ", ".join(what[:8]) + (" ..." if len(what) > 8 else "") + f" ({len(what)} calls per pass)"}
 
 
@@ -454,9 +478,11 @@ def run_ours(args, rank, world):
 
     ms, e2e_ms = job_times(ms, e2e_ms, world, dev)
 
-    if args.workload == "decode":
+    if is_decode(args.workload):
         unit, per_step = "GB/s", sum(call_bytes(layers[li], M) for li, M in calls) / 1e9
         metric = "hybrid GEMM HBM GB/s over stored bytes (decode)"
+        if args.workload == "decode_fused":
+            metric = "hybrid GEMM HBM GB/s over stored bytes (decode, fused q|k|v and gate|up projections)"
     else:
         unit, per_step = "TFLOP/s", sum(call_flops(layers[li], M) for li, M in calls) / 1e12
         metric = "hybrid GEMM TFLOP/s, dense-equivalent (prefill)"
@@ -467,7 +493,7 @@ def run_ours(args, rank, world):
     # Every call of the step is one launch of that kernel, so the mean over the
     # timed region is the step's bytes (FLOPs) over the step's time; the per-call
     # split below comes from the event-instrumented graph.
-    w_ = np.array([call_bytes(layers[li], M) if args.workload == "decode" else call_flops(layers[li], M)
+    w_ = np.array([call_bytes(layers[li], M) if is_decode(args.workload) else call_flops(layers[li], M)
                    for li, M in calls], dtype=np.float64)
     step_ms = ms / args.steps
     if call_ms is None:
@@ -475,7 +501,7 @@ def run_ours(args, rank, world):
     else:
         split_ms = call_ms.mean(axis=0)
     mean_call_ms = split_ms * (step_ms / split_ms.sum())  # scaled to the event-free step time
-    if args.workload == "decode":
+    if is_decode(args.workload):
         alg = np.array([call_bytes(layers[li], M) for li, M in calls]) / 1e9
         achieved = float(alg.sum() / (mean_call_ms.sum() / 1e3))
         traffic = measured_traffic("decode", [f"{layers[li]['name']}@M={M}" for li, M in calls])
@@ -516,7 +542,8 @@ def run_ours(args, rank, world):
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"LLaMA-2-7B linear layers ({args.workload})",
-                   "shapes": [f"{n}:{N}x{K}" for n, N, K in si.LLAMA2_7B],
+                   "shapes": [f"{L['name']}:{L['N']}x{L['K']}" for L in layers] if args.workload == "decode_fused"
+                   else [f"{n}:{N}x{K}" for n, N, K in si.LLAMA2_7B],
                    "tokens": sorted({M for _, M in calls}),
                    "sparse_tile_fraction": sorted({L["frac"] for L in layers}),
                    "resident_weight_bytes": resident,
@@ -538,7 +565,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "decode_fused", "prefill"], default="decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed calls eagerly instead of one CUDA graph")
@@ -564,7 +591,7 @@ def main():
         value = statistics.median(steps)
         cb = dict(cb, value=round(value, 4))
         print(json.dumps({"impl": "reference", "metric": "hybrid GEMM HBM GB/s over stored bytes (decode)"
-                          if args.workload == "decode" else "hybrid GEMM TFLOP/s, dense-equivalent (prefill)",
+                          if is_decode(args.workload) else "hybrid GEMM TFLOP/s, dense-equivalent (prefill)",
                           "value": round(value, 4), "unit": cb["unit"], "n_gpus": args.gpus, "steps": args.steps,
                           "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                           "dtype": "f64", "data": "synthetic",

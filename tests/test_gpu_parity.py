@@ -331,6 +331,28 @@ def test_prefill_many_output_tiles():
     check_gemm(y[rows], ref, "prefill wrap")
 
 
+@pytest.mark.parametrize("M", [1, 16, 40])
+def test_fused_projection_is_a_gemm_on_row_concatenated_weights(M):
+    """q|k|v (or gate|up) fused: one GEMM over the row-concatenated packed
+    weight gives the concatenation of the separate layers' outputs."""
+    K = 384
+    parts = [(256, 0.5), (128, 0.0), (384, 1.0)]
+    ws, bms, idss = [], [], []
+    for j, (N, f) in enumerate(parts):
+        w = si.gen_w(N, K, 11, j)
+        ws.append(w)
+        bms.append(si.tiles_exact(N, K, f, 11, j))
+        idss.append(si.patterns_top2(w))
+    x = si.gen_x(M, K, 11, 0)
+    w_cat, bm_cat, ids_cat = np.concatenate(ws), np.concatenate(bms), np.concatenate(idss)
+    y = gemm_on_gpu(x, pack_on_gpu(w_cat, bm_cat, ids_cat))
+    check_gemm(y, oracle.hybrid_gemm(x, w_cat, bm_cat, ids_cat), f"fused projection M={M}")
+    n0 = 0
+    for w, bm, ids in zip(ws, bms, idss):
+        check_gemm(y[:, n0:n0 + w.shape[0]], oracle.hybrid_gemm(x, w, bm, ids), "part")
+        n0 += w.shape[0]
+
+
 def test_prefill_long_k_reads_descriptors_from_global():
     """More K-tiles per row than the kernel stages in shared memory (K > 16384),
     odd tile-row count (the last row pair has one row)."""
