@@ -3,7 +3,9 @@
 Only the test suite, the package smoke check and the benchmark's CPU-baseline
 leg may import this package.  The arithmetic lives in ``patch_oracle.c``
 (plain C, fp64, OpenMP over output elements); this module only compiles it
-with gcc and marshals numpy arrays.  It shares no code with the CUDA library.
+with gcc and marshals numpy arrays, except the gated MLP's SiLU and product
+(``hybrid_mlp``), written here in fp64 numpy on top of the C GEMM.  It shares
+no code with the CUDA library.
 """
 from __future__ import annotations
 
@@ -157,3 +159,21 @@ def hybrid_gemm(x: np.ndarray, w: np.ndarray, bitmap: np.ndarray, pat_id: np.nda
                                       _ptr(np.ascontiguousarray(pat_id, np.uint8)), _ptr(y)),
            "hybrid_gemm")
     return y
+
+
+def silu(z):
+    """SiLU, z * sigmoid(z), in fp64: the gate activation of LLaMA's gated MLP
+    (the linears of the pages' LLaMA-2 7B end-to-end runs, "Experimental
+    Results" -> "Speedup & Efficiency"; the activation itself is LLaMA's, the
+    pages do not state it)."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def hybrid_mlp(x: np.ndarray, gate, up, rows: np.ndarray | None = None) -> np.ndarray:
+    """H = silu(X W_gate_eff^T) * (X W_up_eff^T) in fp64, the gated MLP's first
+    half on two hybrid weights; gate and up are (w, bitmap, pat_id)."""
+    g = hybrid_gemm(x, *gate, rows=rows)
+    u = hybrid_gemm(x, *up, rows=rows)
+    return silu(g) * u

@@ -7,6 +7,7 @@ library matmul / argmax, closed-form sizes, and the pattern table under
 tests/golden/.
 """
 import itertools
+import math
 import os
 
 import numpy as np
@@ -14,6 +15,7 @@ import pytest
 
 import oracle
 import synth_inputs as si
+from _util import bf16_to_f64
 
 TILE = 128
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pattern_codes.txt")
@@ -313,3 +315,40 @@ def test_bf16_rounding_is_rne():
     b = si.f32_to_bf16_bits(f)
     assert b.tolist()[:4] == [0x3F80, 0x3F80, 0x3F82, 0xC020]  # ties go to even
     assert abs(si.bf16_bits_to_f32(b)[4] - 3.0e-3) < 3.0e-3 * 2 ** -8
+
+
+# ---------------------------------------------------------------- gated MLP
+
+
+def test_silu_closed_forms_and_identities():
+    """silu against an independent form: z * (1 + tanh(z / 2)) / 2, plus
+    silu(0) = 0, silu(1) = e / (1 + e), silu(z) - silu(-z) = z and the limits."""
+    z = np.linspace(-30.0, 30.0, 2001)
+    tanh_form = z * (1.0 + np.tanh(z / 2.0)) / 2.0
+    # (the tanh form loses relative accuracy to cancellation for very negative z)
+    assert np.allclose(oracle.silu(z), tanh_form, rtol=1e-12, atol=1e-14)
+    assert oracle.silu(0.0) == 0.0
+    assert oracle.silu(1.0) == pytest.approx(math.e / (1.0 + math.e), rel=1e-15)
+    assert np.allclose(oracle.silu(z) - oracle.silu(-z), z, rtol=1e-13, atol=1e-12)
+    assert oracle.silu(800.0) == 800.0 and oracle.silu(-800.0) == 0.0
+
+
+def test_hybrid_mlp_on_one_hot_inputs():
+    """Brute force on a one-hot X column: H[m][n] = silu(Wg_eff[n][k]) * Wu_eff[n][k]
+    for every kept k, with the activation evaluated through tanh instead."""
+    N, K = 128, 256
+    wg = si.gen_w(N, K, 0, 5, std=0.5)
+    wu = si.gen_w(N, K, 0, 6, std=0.5)
+    bmg = np.array([[0, 1]], np.uint8)
+    bmu = np.array([[1, 0]], np.uint8)
+    idg, idu = si.patterns_top2(wg), si.patterns_top2(wu)
+    ks = [0, 5, 130, 255]
+    x = np.zeros((len(ks), K), np.uint16)
+    for m, k in enumerate(ks):
+        x[m, k] = 0x3F80  # 1.0
+    h = oracle.hybrid_mlp(x, (wg, bmg, idg), (wu, bmu, idu))
+    geff = bf16_to_f64(oracle.apply_mask(wg, bmg, idg))
+    ueff = bf16_to_f64(oracle.apply_mask(wu, bmu, idu))
+    for m, k in enumerate(ks):
+        g, u = geff[:, k], ueff[:, k]
+        assert np.allclose(h[m], g * (1.0 + np.tanh(g / 2.0)) / 2.0 * u, rtol=1e-12, atol=1e-15)
