@@ -329,6 +329,69 @@ def offline_steps(layers, dev, pk, reps=5):
     return out
 
 
+# ------------------------------------------------------------ gated MLP
+
+
+def mlp_steps(dev, pk, reps=10):
+    """The gated MLP's first half H = silu(X Wg^T) * (X Wu^T) on LLaMA-2-7B's
+    gate and up (11008 x 4096, 50% sparse tiles): one fused launch against two
+    separate GEMMs, at M = 2048 (prefill) and M = 16 (decode)."""
+    import torch
+
+    import tile_sparse_gemm_b200 as tsg
+
+    status = tsg.new_status(dev)
+    packed = []
+    for i in (4, 5):  # gate, up
+        name, N, K = si.LLAMA2_7B[i]
+        w = si.gen_w(N, K, PREFILL_CONFIG, i)
+        bm = si.tiles_exact(N, K, 0.5, PREFILL_CONFIG, i)
+        packed.append(tsg.patch_pack(torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev),
+                                     torch.from_numpy(bm).to(dev), torch.from_numpy(si.patterns_top2(w)).to(dev),
+                                     int(bm.sum()), status=status))
+    g, u = packed
+    out = {}
+    for M in (PREFILL_M, 16):
+        x = torch.from_numpy(si.gen_x(M, g.K, PREFILL_CONFIG, 4).view(np.int16)).view(torch.bfloat16).to(dev)
+        h = torch.empty((M, g.N), dtype=torch.bfloat16, device=dev)
+        y1, y2 = torch.empty_like(h), torch.empty_like(h)
+        ws = torch.zeros(max(tsg.patch_gemm_workspace_size(M, g), 16), dtype=torch.uint8, device=dev)
+        import ctypes
+        b = ctypes.c_size_t()
+        sg, su = g.struct(), u.struct()
+        tsg.lib().patch_gemm_mlp_workspace_size(M, ctypes.byref(sg), ctypes.byref(su), ctypes.byref(b))
+        wsm = torch.zeros(max(b.value, 16), dtype=torch.uint8, device=dev)
+
+        def fused():
+            tsg.patch_gemm_mlp(x, g, u, H=h, workspace=wsm, status=status)
+
+        def separate():
+            tsg.patch_gemm(x, g, Y=y1, workspace=ws, status=status)
+            tsg.patch_gemm(x, u, Y=y2, workspace=ws, status=status)
+
+        res = {}
+        for name, fn in (("fused", fused), ("two_gemms", separate)):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            res[name] = e0.elapsed_time(e1) / reps * 1e3  # us
+        flops = 2 * 2.0 * M * g.N * g.K
+        out[f"M={M}"] = {"fused_us": round(res["fused"], 1), "two_gemms_us": round(res["two_gemms"], 1),
+                         "fused_TFLOP/s": round(flops / (res["fused"] * 1e-6) / 1e12, 1),
+                         "note": "fused = one prefill launch with silu(gate)*up in the epilogue" if M > 16
+                         else "fused = two decode GEMMs + one elementwise launch"}
+    code, bits = tsg.patch_read_status(status)
+    if code != 0:
+        raise RuntimeError(f"gated MLP: device status {code} bits {bits}")
+    return out
+
+
 # ------------------------------------------------------------ GPU arm
 
 
@@ -556,6 +619,7 @@ def run_ours(args, rank, world):
         "per_call": detail,
         "per_call_note": "split of the event-free step time in proportion to an event-instrumented replay",
         "offline": offline_steps(layers, dev, pk) if args.workload == "decode" and not (args.layers or args.fracs) else None,
+        "gated_mlp": mlp_steps(dev, pk) if args.workload == "prefill" and not (args.layers or args.fracs) else None,
     }
     return out
 

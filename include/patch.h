@@ -285,6 +285,30 @@ PATCH_API patch_status_t patch_gemm_decode_noalloc(const uint16_t *X, int64_t M,
                                                    uint16_t *Y, int32_t *dev_status, void *stream);
 
 /*
+ * patch_gemm_mlp_workspace_size / patch_gemm_mlp: the first half of LLaMA's
+ * gated MLP on two hybrid weights of the same shape,
+ *   H[m][n] = silu(G[m][n]) * U[m][n],  G = X W_gate_eff^T,  U = X W_up_eff^T,
+ * silu(z) = z / (1 + e^-z), fp32 accumulation, one round to bf16 at the end
+ * (the linears of the pages' LLaMA-2 7B end-to-end runs, "Experimental
+ * Results" -> "Speedup & Efficiency"; the gated SiLU is LLaMA's, not stated
+ * by the pages).
+ *   X bf16 [M][K]; W_gate, W_up packed [N][K] each; H bf16 [M][N] (16-byte aligned).
+ * M > 16: one prefill launch in which each unit multiplies a gate tile row and
+ * the up tile row of the same 128 features against the same X panels and the
+ * epilogue writes H directly (G and U never reach memory).
+ * M <= 16: two decode GEMMs write G and U (bf16) into the workspace, then one
+ * elementwise launch forms H.
+ * workspace: patch_gemm_mlp_workspace_size bytes, zero-filled before its first
+ * use and left so by every successful call (as for patch_gemm).
+ * Errors as patch_gemm; PATCH_ERR_SHAPE also when the two weights differ in shape.
+ */
+PATCH_API patch_status_t patch_gemm_mlp_workspace_size(int64_t M, const patch_weight *W_gate, const patch_weight *W_up,
+                                                       size_t *bytes);
+PATCH_API patch_status_t patch_gemm_mlp(const uint16_t *X, int64_t M, const patch_weight *W_gate,
+                                        const patch_weight *W_up, uint16_t *H, void *workspace, size_t workspace_bytes,
+                                        int32_t *dev_status, void *stream);
+
+/*
  * patch_read_status: synchronise `stream`, copy *dev_status to *host_bits and
  * return the first error it encodes (PATCH_ERR_TIMEOUT, then BAD_PATTERN,
  * then COUNT) or PATCH_OK.  host_bits may be NULL.

@@ -353,6 +353,43 @@ def test_fused_projection_is_a_gemm_on_row_concatenated_weights(M):
         n0 += w.shape[0]
 
 
+@pytest.mark.parametrize("M", [1, 7, 16, 17, 300, 1100])
+@pytest.mark.parametrize("N,K", [(384, 640), (256, 256)])
+def test_gated_mlp(M, N, K):
+    """H = silu(X Wg^T) * (X Wu^T): decode path (two GEMMs + elementwise) for
+    M <= 16, one prefill launch with the product in the epilogue above."""
+    wg, wu = si.gen_w(N, K, 12, 0, std=0.05), si.gen_w(N, K, 12, 1, std=0.05)
+    bmg, bmu = si.tiles_exact(N, K, 0.5, 12, 0), si.tiles_exact(N, K, 0.5, 12, 1)
+    idg, idu = si.patterns_top2(wg), si.patterns_top2(wu)
+    x = si.gen_x(M, K, 12, 2)
+    rows = None if M <= 300 else np.array([0, 1, 239, 240, 700, 1099])
+    ref = oracle.hybrid_mlp(x, (wg, bmg, idg), (wu, bmu, idu), rows=rows)
+    status = tsg.new_status()
+    h = tsg.patch_gemm_mlp(to_dev_bf16(x), pack_on_gpu(wg, bmg, idg), pack_on_gpu(wu, bmu, idu), status=status)
+    code, bits = tsg.patch_read_status(status)
+    assert code == 0, (code, bits)
+    hb = bits_of(h)
+    check_gemm(hb if rows is None else hb[rows], ref, f"gated MLP M={M}")
+
+
+def test_gated_mlp_rejects_mismatched_weights():
+    a = pack_on_gpu(si.gen_w(256, 256, 1, 0), np.zeros((2, 2), np.uint8), si.patterns_top2(si.gen_w(256, 256, 1, 0)))
+    b = pack_on_gpu(si.gen_w(384, 256, 1, 1), np.zeros((3, 2), np.uint8), si.patterns_top2(si.gen_w(384, 256, 1, 1)))
+    x = to_dev_bf16(si.gen_x(4, 256, 1, 0))
+    with pytest.raises(ValueError):
+        tsg.patch_gemm_mlp(x, a, b)
+    import ctypes
+    h = torch.empty((4, 256), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    status = tsg.new_status()
+    sa, sb = a.struct(), b.struct()
+    rc = tsg.lib().patch_gemm_mlp(ctypes.c_void_p(x.data_ptr()), 4, ctypes.byref(sa), ctypes.byref(sb),
+                                  ctypes.c_void_p(h.data_ptr()), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                  ctypes.c_void_p(status.data_ptr()),
+                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 2  # PATCH_ERR_SHAPE, before any launch
+
+
 def test_prefill_long_k_reads_descriptors_from_global():
     """More K-tiles per row than the kernel stages in shared memory (K > 16384),
     odd tile-row count (the last row pair has one row)."""

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "patch_gemm": [P, I64, WP, P, P, SZ, P, P],
             "patch_gemm_ex": [P, I64, WP, P, P, SZ, P, P, I32, ctypes.c_uint64],
             "patch_read_status": [P, P, ctypes.POINTER(ctypes.c_int32)],
+            "patch_gemm_mlp_workspace_size": [I64, WP, WP, ctypes.POINTER(SZ)],
+            "patch_gemm_mlp": [P, I64, WP, WP, P, P, SZ, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -248,6 +250,29 @@ def patch_gemm(X: torch.Tensor, weight: PackedWeight, Y: torch.Tensor | None = N
     Every call runs on the current stream and launches only libpatch kernels, so a
     sequence of calls can be captured in a CUDA graph (after one eager call)."""
     return patch_gemm_ex(X, weight, Y, workspace, status, PATH_AUTO, 0, stream)
+
+
+def patch_gemm_mlp(X: torch.Tensor, gate: PackedWeight, up: PackedWeight, H: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """H = silu(X W_gate^T) * (X W_up^T) (bf16 [M][N]) on two packed weights of one shape."""
+    M, K = X.shape
+    if K != gate.K or (gate.N, gate.K) != (up.N, up.K):
+        raise ValueError("X, gate and up shapes disagree")
+    dev = X.device
+    if H is None:
+        H = torch.empty((M, gate.N), dtype=torch.bfloat16, device=dev)
+    status = new_status(dev) if status is None else status
+    sg, su = gate.struct(), up.struct()
+    if workspace is None:
+        b = ctypes.c_size_t()
+        _check(lib().patch_gemm_mlp_workspace_size(M, ctypes.byref(sg), ctypes.byref(su), ctypes.byref(b)),
+               "patch_gemm_mlp_workspace_size")
+        workspace = torch.zeros(max(b.value, 16), dtype=torch.uint8, device=dev)  # must start zero-filled
+    _check(lib().patch_gemm_mlp(_dev(X, "X"), M, ctypes.byref(sg), ctypes.byref(su), _dev(H, "H"),
+                                _dev(workspace, "workspace"), workspace.numel(), _dev(status, "status"),
+                                _stream(stream)), "patch_gemm_mlp")
+    return H
 
 
 def patch_read_status(status: torch.Tensor, stream=None) -> tuple[int, int]:

@@ -201,6 +201,65 @@ patch_status_t patch_gemm(const uint16_t* X, int64_t M, const patch_weight* W, u
   return patch_gemm_ex(X, M, W, Y, workspace, workspace_bytes, dev_status, stream, PATCH_PATH_AUTO, 0);
 }
 
+// decode scratch for the gated MLP: [decode GEMM workspace][G][U], 256-byte aligned parts
+static size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+
+patch_status_t patch_gemm_mlp_workspace_size(int64_t M, const patch_weight* W_gate, const patch_weight* W_up,
+                                             size_t* bytes) {
+  if (!bytes || !W_gate || !W_up) return PATCH_ERR_INVALID_ARG;
+  if (W_gate->N != W_up->N || W_gate->K != W_up->K) return PATCH_ERR_SHAPE;
+  size_t a = 0, b = 0;
+  patch_status_t st = patch_gemm_workspace_size(M, W_gate, &a);
+  if (st != PATCH_OK) return st;
+  st = patch_gemm_workspace_size(M, W_up, &b);
+  if (st != PATCH_OK) return st;
+  *bytes = 0;
+  if (M == 0 || M > PATCH_DECODE_MAX_M) return PATCH_OK;
+  *bytes = round256(a > b ? a : b) + 2 * round256(size_t(M) * size_t(W_gate->N) * 2);
+  return PATCH_OK;
+}
+
+patch_status_t patch_gemm_mlp(const uint16_t* X, int64_t M, const patch_weight* W_gate, const patch_weight* W_up,
+                              uint16_t* H, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                              void* stream) {
+  if (M < 0 || !dev_status || !W_gate || !W_up) return PATCH_ERR_INVALID_ARG;
+  if (W_gate->N != W_up->N || W_gate->K != W_up->K) return PATCH_ERR_SHAPE;
+  patch_status_t st = check_weight(W_gate);
+  if (st != PATCH_OK) return st;
+  st = check_weight(W_up);
+  if (st != PATCH_OK) return st;
+  if (M == 0) return PATCH_OK;
+  if (!X || !H) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(H)) return PATCH_ERR_ALIGN;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint64_t limit_ns = 2000000ull * 1000ull;
+  if (M > PATCH_DECODE_MAX_M) {
+    if (launch_prefill_mlp(X, M, *W_gate, *W_up, H, dev_status, sms, limit_ns, s) != cudaSuccess)
+      return PATCH_ERR_CUDA;
+    return PATCH_OK;
+  }
+  size_t need = 0;
+  st = patch_gemm_mlp_workspace_size(M, W_gate, W_up, &need);
+  if (st != PATCH_OK) return st;
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PATCH_ERR_WORKSPACE;
+  size_t ws = 0;
+  patch_gemm_workspace_size(M, W_gate, &ws);
+  size_t wu = 0;
+  patch_gemm_workspace_size(M, W_up, &wu);
+  const size_t gemm_ws = round256(ws > wu ? ws : wu), yb = round256(size_t(M) * size_t(W_gate->N) * 2);
+  uint16_t* G = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + gemm_ws);
+  uint16_t* U = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + gemm_ws + yb);
+  st = patch_gemm(X, M, W_gate, G, workspace, gemm_ws, dev_status, stream);
+  if (st != PATCH_OK) return st;
+  st = patch_gemm(X, M, W_up, U, workspace, gemm_ws, dev_status, stream);
+  if (st != PATCH_OK) return st;
+  if (launch_silu_mul(G, U, H, M * W_gate->N, sms, s) != cudaSuccess) return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
 patch_status_t patch_read_status(const int32_t* dev_status, void* stream, int32_t* host_bits) {
   if (!dev_status) return PATCH_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -95,8 +95,9 @@ constexpr size_t SMEM_BYTES = sizeof(Shared) + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 struct Args {
-  const uint8_t* meta;
-  const patch_tile_desc* desc;
+  const uint8_t* meta[ROWS];          // row r of a unit reads weight r (the same weight unless mlp)
+  const patch_tile_desc* desc[ROWS];
+  int mlp;                            // 1: row 0 = gate, row 1 = up tile row rp; Y = silu(gate) * up
   uint16_t* Y;
   int M, N, Tn, Tk, n_pairs, n_tb, n_items;  // units: row pair rp = item / n_tb, token block tb = item % n_tb
   int bt;                      // tokens per unit: a multiple of 16, at most BT
@@ -106,8 +107,12 @@ struct Args {
   int inject;  // 1: row 0's producer stops after the first K-tile (exercises the timeout path)
 };
 
-// tile rows in row pair rp (the last pair of an odd Tn has one)
-__device__ __forceinline__ int rows_of(int rp, int Tn) { return Tn - ROWS * rp < ROWS ? Tn - ROWS * rp : ROWS; }
+// tile rows in unit row pair rp (the last pair of an odd Tn has one; a gated-MLP unit always has both)
+__device__ __forceinline__ int rows_of(const Args& p, int rp) {
+  return p.mlp ? ROWS : (p.Tn - ROWS * rp < ROWS ? p.Tn - ROWS * rp : ROWS);
+}
+// the tile row of its weight that row r of unit row pair rp reads
+__device__ __forceinline__ int tile_row(const Args& p, int rp, int r) { return p.mlp ? rp : ROWS * rp + r; }
 
 // Units run row pair by row pair (all token blocks of a pair are consecutive
 // items), so the CTAs of one wave read a few row pairs' W, which stays in L2
@@ -124,6 +129,8 @@ __device__ __forceinline__ int k_rotation(int rp, int tb, int Tk) { return (rp +
 // metadata and the descriptors are inputs that no kernel triggering an early
 // launch writes).
 __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, int r) {
+  const patch_tile_desc* desc = r ? p.desc[1] : p.desc[0];
+  const uint8_t* meta = r ? p.meta[1] : p.meta[0];
   const bool staged = p.Tk <= MAXTK;
   const uint32_t row_bytes = uint32_t(p.Tk * sizeof(patch_tile_desc));
   uint32_t a_i = 0, e_i = 0, d_i = 0;  // loads issued per ring / descriptor rows staged
@@ -131,15 +138,15 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
   // stage (or, for a pair without row r, complete with no bytes) the descriptor row of an item
   auto stage_row = [&](int item, int buf) {
     const int rp = item / p.n_tb;
-    const bool has = r < rows_of(rp, p.Tn);
+    const bool has = r < rows_of(p, rp);
     mbar_expect_tx(&s.pdesc_full[r][buf], has ? row_bytes : 0u);
-    if (has) bulk_load(s.pdesc[r][buf], p.desc + int64_t(ROWS * rp + r) * p.Tk, row_bytes, &s.pdesc_full[r][buf]);
+    if (has) bulk_load(s.pdesc[r][buf], desc + int64_t(tile_row(p, rp, r)) * p.Tk, row_bytes, &s.pdesc_full[r][buf]);
     ++d_i;
   };
   if (staged && int(blockIdx.x) < p.n_items) stage_row(blockIdx.x, 0);
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const int rp = item / p.n_tb, tb = item % p.n_tb, tn = ROWS * rp + r;
+    const int rp = item / p.n_tb, tb = item % p.n_tb, tn = tile_row(p, rp, r);
     const int buf = it & 1;
     if (staged) {
       if (!(ok = wait_bounded(&s.pdesc_full[r][buf], (it >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
@@ -147,20 +154,20 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
       // prefetch the next unit's row into the other buffer (its previous row is done)
       if (item + int(gridDim.x) < p.n_items) stage_row(item + gridDim.x, buf ^ 1);
     }
-    if (r >= rows_of(rp, p.Tn)) continue;
+    if (r >= rows_of(p, rp)) continue;
     int kt = k_rotation(rp, tb, p.Tk);
     for (int j = 0; ok && j < p.Tk; ++j, kt = (kt + 1 == p.Tk ? 0 : kt + 1)) {
       if (p.inject && r == 0 && (item != int(blockIdx.x) || j > 0)) {
         ok = false;
         break;
       }
-      const patch_tile_desc d = staged ? s.pdesc[r][buf][kt] : p.desc[int64_t(tn) * p.Tk + kt];
+      const patch_tile_desc d = staged ? s.pdesc[r][buf][kt] : desc[int64_t(tn) * p.Tk + kt];
       if (d.kind) {
         const uint32_t es = e_i % NE;
         if (!(ok = wait_bounded(&s.e_empty[r][es], ((e_i / NE) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
           break;
         mbar_expect_tx(&s.e_full[r][es], E_BYTES);
-        bulk_load(s.e[r][es], p.meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.e_full[r][es]);
+        bulk_load(s.e[r][es], meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.e_full[r][es]);
         ++e_i;
       }
       // a dense tile's 2 panels (one per 64-k half), a sparse tile's one
@@ -219,7 +226,7 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
   bool ok = true;
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const bool active = r < rows_of(item / p.n_tb, p.Tn);
+    const bool active = r < rows_of(p, item / p.n_tb);
     if (!(ok = wait_bounded(&s.acc_empty[r], (it & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
     tc_fence_after();
     uint32_t accumulate = 0;
@@ -289,34 +296,52 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
   wait_bounded(&s.drain[r], 0, &s.abort_flag, p.limit_ns, p.status, true);
 }
 
-// Epilogue warps of row r (4 warps, one per TMEM lane quarter): per chunk of
-// YT tokens, each warp loads its 32 features x YT tokens from TMEM, rounds to
-// bf16 and writes them into a shared [YT][128] chunk; one thread then stores
-// the chunk to Y with a TMA store (full 256-byte rows of Y instead of 64-byte
-// pieces).  Two chunk buffers: a buffer is rewritten only after the store
-// that read it has finished reading.
+// Epilogue warp groups (4 warps each, one per TMEM lane quarter): per chunk
+// of YT tokens, each warp loads its 32 features x YT tokens from TMEM, rounds
+// to bf16 and writes them into a shared [YT][128] chunk; one thread then
+// stores the chunk to Y with a TMA store (full 256-byte rows of Y instead of
+// 64-byte pieces).  Two chunk buffers per group: a buffer is rewritten only
+// after the store that read it has finished reading.  Group g drains row g of
+// the pair; for the gated MLP both groups read both rows (gate and up of the
+// same 128 features) and take every other chunk: Y = silu(gate) * up.
 __device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, const Args& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3;                  // the TMEM lane quarter this warp may access
-  const int r = (warp - EPI_WARP0) >> 2;   // the row of the pair it drains
-  const uint32_t bar_id = 1 + r;           // named barrier of the row's 128 epilogue threads
-  const bool leader = warp == EPI_WARP0 + 4 * r && lane == 0;
-  uint32_t chunk = 0;                      // chunks stored by this row so far (buffer = chunk & 1)
+  const int g = (warp - EPI_WARP0) >> 2;   // warp group
+  const uint32_t bar_id = 1 + g;           // named barrier of the group's 128 threads
+  const bool leader = warp == EPI_WARP0 + 4 * g && lane == 0;
+  uint32_t chunk = 0;                      // chunks stored by this group so far (buffer = chunk & 1)
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
     const int rp = item / p.n_tb, tb = item % p.n_tb;
-    // the four warps of a row take the same decision, so none is left at a barrier
-    const bool ok = wait_bounded(&s.acc_full[r], it & 1, &s.abort_flag, p.limit_ns, p.status, false);
+    // the four warps of a group take the same decision, so none is left at a barrier
+    bool ok = wait_bounded(&s.acc_full[g], it & 1, &s.abort_flag, p.limit_ns, p.status, false);
+    if (p.mlp) ok = ok && wait_bounded(&s.acc_full[g ^ 1], it & 1, &s.abort_flag, p.limit_ns, p.status, false);
     if (!named_bar_and(bar_id, 128, ok)) break;
     tc_fence_after();
-    if (r < rows_of(rp, p.Tn)) {
-      const int n0 = (ROWS * rp + r) * BM, m0 = tb * p.bt;
+    if (p.mlp || g < rows_of(p, rp)) {
+      const int n0 = (p.mlp ? rp : ROWS * rp + g) * BM, m0 = tb * p.bt;
       const int valid = p.M - m0 < p.bt ? p.M - m0 : p.bt;  // tokens of this unit inside X
-      const uint32_t acc = tmem + (uint32_t(32 * q) << 16) + ACC_STRIDE * r;
-      for (int c = 0; c * YT < valid; ++c, ++chunk) {
+      const uint32_t lanes = tmem + (uint32_t(32 * q) << 16);
+      const int c0 = p.mlp ? g : 0, dc = p.mlp ? 2 : 1;
+      for (int c = c0; c * YT < valid; c += dc, ++chunk) {
         uint32_t v[YT];
-        tmem_ld_16cols(acc + uint32_t(YT * c), v);
-        uint16_t(*buf)[BM] = s.y[r][chunk & 1];
+        if (p.mlp) {
+          uint32_t u[YT];
+          tmem_ld_16cols(lanes + uint32_t(YT * c), v);               // gate
+          tmem_ld_16cols(lanes + ACC_STRIDE + uint32_t(YT * c), u);  // up
+#pragma unroll
+          for (int j = 0; j < YT; ++j) {
+            // silu(gate) = gate / (1 + e^-gate), with CUDA's fast exponential and
+            // division (relative error ~1e-6, far below the bf16 rounding of H);
+            // a huge denominator gives -0 for a very negative gate
+            const float gate = __uint_as_float(v[j]);
+            v[j] = __float_as_uint(__fdividef(gate, 1.0f + __expf(-gate)) * __uint_as_float(u[j]));
+          }
+        } else {
+          tmem_ld_16cols(lanes + ACC_STRIDE * g + uint32_t(YT * c), v);
+        }
+        uint16_t(*buf)[BM] = s.y[g][chunk & 1];
 #pragma unroll
         for (int j = 0; j < YT; ++j) buf[j][32 * q + lane] = f32_to_bf16_rne(__uint_as_float(v[j]));
         fence_proxy_async_smem();
@@ -331,14 +356,18 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, co
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s.acc_empty[r]);
+    if (lane == 0) {
+      mbar_arrive(&s.acc_empty[g]);
+      if (p.mlp) mbar_arrive(&s.acc_empty[g ^ 1]);
+    }
   }
   if (leader) bulk_wait_all();  // Y written before the CTA exits
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   const __grid_constant__ CUtensorMap tmap_y, const Args p) {
+    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w0,
+                   const __grid_constant__ CUtensorMap tmap_w1, const __grid_constant__ CUtensorMap tmap_y,
+                   const Args p) {
   extern __shared__ uint8_t smem_raw[];
   Shared& s = *reinterpret_cast<Shared*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -355,7 +384,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(&s.e_empty[r][i], 1);
       }
       mbar_init(&s.acc_full[r], 1);
-      mbar_init(&s.acc_empty[r], 4);
+      mbar_init(&s.acc_empty[r], p.mlp ? 8 : 4);  // the gated MLP's groups both read both rows
       mbar_init(&s.drain[r], 1);
       mbar_init(&s.pdesc_full[r][0], 1);
       mbar_init(&s.pdesc_full[r][1], 1);
@@ -367,7 +396,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     s.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tensormap(&tmap_x);
-    prefetch_tensormap(&tmap_w);
+    prefetch_tensormap(&tmap_w0);
+    prefetch_tensormap(&tmap_w1);
     prefetch_tensormap(&tmap_y);
   }
   if (warp == 1) {
@@ -388,7 +418,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (warp & 1)
         mma_issuer(s, tmem, p, warp >> 1);
       else
-        producer_w(s, &tmap_w, p, warp >> 1);
+        producer_w(s, (warp >> 1) ? &tmap_w1 : &tmap_w0, p, warp >> 1);
     }
     __syncwarp();
   } else if (warp == 4) {
@@ -477,25 +507,35 @@ static int pick_bt(int64_t M, int64_t n_pairs, int64_t Tk, int num_sms) {
   return best;
 }
 
-cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
-                           int32_t* status, int num_sms, uint64_t limit_ns, int inject,
-                           cudaStream_t stream) {
+// Shared by the plain GEMM (w1 == w0, units of two consecutive tile rows) and
+// the gated MLP (w0 = gate, w1 = up, units of one tile row of each).
+static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch_weight& W0, const patch_weight& W1,
+                                       bool mlp, uint16_t* Y, int32_t* status, int num_sms, uint64_t limit_ns,
+                                       int inject, cudaStream_t stream) {
   using namespace prefill;
-  const int64_t Tn = W.N / BM, Tk = W.K / kTile, T = Tn * Tk;
-  const uint64_t n_panels = uint64_t(2 * (T - W.n_sparse) + W.n_sparse);
-  const int64_t n_pairs = (Tn + ROWS - 1) / ROWS;
+  const int64_t Tn = W0.N / BM, Tk = W0.K / kTile;
+  const int64_t n_pairs = mlp ? Tn : (Tn + ROWS - 1) / ROWS;
   const int bt = pick_bt(M, n_pairs, Tk, num_sms);
-  CUtensorMap tmap_x, tmap_w, tmap_y;
-  if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, uint32_t(bt)))
+  CUtensorMap tmap_x, tmap_w0, tmap_w1, tmap_y;
+  if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W0.K), uint64_t(M), uint64_t(W0.K) * 2, 64, uint32_t(bt)))
     return cudaErrorUnknown;
-  if (!make_map_2d_bf16(&tmap_w, W.values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
-  if (!make_map_y(&tmap_y, Y, uint64_t(W.N), uint64_t(M))) return cudaErrorUnknown;
+  const patch_weight* Ws[2] = {&W0, &W1};
+  CUtensorMap* maps[2] = {&tmap_w0, &tmap_w1};
+  for (int r = 0; r < 2; ++r) {
+    const int64_t T = (Ws[r]->N / BM) * Tk;
+    const uint64_t n_panels = uint64_t(2 * (T - Ws[r]->n_sparse) + Ws[r]->n_sparse);
+    if (!make_map_2d_bf16(maps[r], Ws[r]->values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
+  }
+  if (!make_map_y(&tmap_y, Y, uint64_t(Tn * BM), uint64_t(M))) return cudaErrorUnknown;
   Args p;
-  p.meta = static_cast<const uint8_t*>(W.meta);
-  p.desc = W.desc;
+  for (int r = 0; r < ROWS; ++r) {
+    p.meta[r] = static_cast<const uint8_t*>(Ws[r]->meta);
+    p.desc[r] = Ws[r]->desc;
+  }
+  p.mlp = mlp ? 1 : 0;
   p.Y = Y;
   p.M = int(M);
-  p.N = int(W.N);
+  p.N = int(Tn * BM);
   p.Tn = int(Tn);
   p.Tk = int(Tk);
   p.n_pairs = int(n_pairs);
@@ -510,8 +550,19 @@ cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, 
   const int grid = p.n_items < num_sms ? p.n_items : num_sms;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES));
   if (e != cudaSuccess) return e;
-  return launch_pdl(prefill_kernel, dim3(unsigned(grid)), dim3(THREADS), SMEM_BYTES, stream, tmap_x, tmap_w, tmap_y,
-                    p);
+  return launch_pdl(prefill_kernel, dim3(unsigned(grid)), dim3(THREADS), SMEM_BYTES, stream, tmap_x, tmap_w0, tmap_w1,
+                    tmap_y, p);
+}
+
+cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
+                           int32_t* status, int num_sms, uint64_t limit_ns, int inject,
+                           cudaStream_t stream) {
+  return launch_prefill_impl(X, M, W, W, false, Y, status, num_sms, limit_ns, inject, stream);
+}
+
+cudaError_t launch_prefill_mlp(const uint16_t* X, int64_t M, const patch_weight& W_gate, const patch_weight& W_up,
+                               uint16_t* H, int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream) {
+  return launch_prefill_impl(X, M, W_gate, W_up, true, H, status, num_sms, limit_ns, 0, stream);
 }
 
 }  // namespace patch

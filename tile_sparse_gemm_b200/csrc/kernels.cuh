@@ -36,7 +36,15 @@ cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, 
                            int32_t* status, int num_sms, uint64_t limit_ns, int inject,
                            cudaStream_t stream);
 
-// Tensor-core decode (stream-K over panels, M <= 16): main kernel + fixup.
+// Gated MLP first half, M > 16: H = silu(X W_gate^T) * (X W_up^T) in one prefill launch.
+cudaError_t launch_prefill_mlp(const uint16_t* X, int64_t M, const patch_weight& W_gate, const patch_weight& W_up,
+                               uint16_t* H, int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream);
+
+// H = silu(G) * U elementwise (bf16; count a multiple of 8).
+cudaError_t launch_silu_mul(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t count, int num_sms,
+                            cudaStream_t stream);
+
+// Tensor-core decode (stream-K over panels, M <= 16).
 size_t decode_tc_workspace_bytes(int64_t M, const patch_weight& W, int num_sms);
 cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
                              int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream);
