@@ -177,3 +177,61 @@ def hybrid_mlp(x: np.ndarray, gate, up, rows: np.ndarray | None = None) -> np.nd
     g = hybrid_gemm(x, *gate, rows=rows)
     u = hybrid_gemm(x, *up, rows=rows)
     return silu(g) * u
+
+
+# patterns as keep-position pairs, numbered lexicographically (the library's reading)
+_PAIRS = ((0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3))
+
+
+def soft_mask(w: np.ndarray, tile_logits: np.ndarray, pattern_logits: np.ndarray, tau: float,
+              tile_noise: np.ndarray | None = None, pattern_noise: np.ndarray | None = None):
+    """The training-time (soft) hybrid mask of "Core Mechanism" / "Learnable
+    Distributions", in fp64, following its steps:
+      1. tile choice:    p = softmax((tile_logits + tile_noise) / tau) over (dense, sparse);
+      2. pattern choice: q = softmax((pattern_logits + pattern_noise) / tau) over the 6 patterns;
+      3. hybrid mask:    M[n][k] = p_dense + p_sparse * sum_j q_j [k mod 4 in pattern j];
+      4. soft weight:    W_soft = W * M, rounded once to bf16 (nearest even).
+    The noise is the caller's (Gumbel samples; zero when None).  Returns
+    (W_soft bf16 bits [N][K], M fp64 [N][K])."""
+    N, K = w.shape
+    Tn, Tk = N // TILE, K // TILE
+    tl = tile_logits.astype(np.float64) + (0.0 if tile_noise is None else tile_noise.astype(np.float64))
+    pl = pattern_logits.astype(np.float64) + (0.0 if pattern_noise is None else pattern_noise.astype(np.float64))
+
+    def softmax(z):
+        z = z / tau
+        z = z - z.max(axis=-1, keepdims=True)
+        e = np.exp(z)
+        return e / e.sum(axis=-1, keepdims=True)
+
+    p = softmax(tl.reshape(Tn, Tk, 2))                         # [Tn][Tk][2]
+    q = softmax(pl.reshape(N, K // 4, 6))                      # [N][K/4][6]
+    keep = np.zeros((N, K // 4, 4))
+    for j, (a, b) in enumerate(_PAIRS):
+        keep[:, :, a] += q[:, :, j]
+        keep[:, :, b] += q[:, :, j]
+    keep = keep.reshape(N, K)
+    pd = np.repeat(np.repeat(p[:, :, 0], TILE, axis=0), TILE, axis=1)
+    ps = np.repeat(np.repeat(p[:, :, 1], TILE, axis=0), TILE, axis=1)
+    m = pd + ps * keep
+    wf = (w.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return _f64_to_bf16_rne(wf * m), m
+
+
+def _f64_to_bf16_rne(x: np.ndarray) -> np.ndarray:
+    """fp64 -> bf16 bits, round to nearest even.  Goes through fp32 (nearest
+    even); that double rounding can only go wrong when the fp32 value lands
+    exactly half way between two bf16 values, and those cases are settled by
+    comparing the fp64 value with that midpoint."""
+    f = np.asarray(x, np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    hi = u >> 16
+    r = ((u + 0x7FFF + (hi & 1)) >> 16).astype(np.uint16)
+    mid = (u & 0xFFFF) == 0x8000
+    if np.any(mid):
+        xm, fm = np.asarray(x, np.float64)[mid], f[mid].astype(np.float64)
+        res = r[mid]
+        res = np.where(np.abs(xm) > np.abs(fm), (hi[mid] + 1).astype(np.uint16), res)
+        res = np.where(np.abs(xm) < np.abs(fm), hi[mid].astype(np.uint16), res)
+        r[mid] = res
+    return r

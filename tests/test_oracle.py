@@ -352,3 +352,77 @@ def test_hybrid_mlp_on_one_hot_inputs():
     for m, k in enumerate(ks):
         g, u = geff[:, k], ueff[:, k]
         assert np.allclose(h[m], g * (1.0 + np.tanh(g / 2.0)) / 2.0 * u, rtol=1e-12, atol=1e-15)
+
+
+# ------------------------------------------------- soft (training-time) hybrid mask
+
+
+def _distinct_int_logits(shape, seed):
+    """Logits whose entries along the last axis are distinct integers (gaps >= 1)."""
+    rng = np.random.default_rng(seed)
+    n = shape[-1]
+    base = np.argsort(rng.random(shape), axis=-1).astype(np.float32)  # a permutation of 0..n-1
+    return base - n / 2
+
+
+def test_soft_mask_cold_limit_is_the_hard_mask():
+    """tau -> 0 with integer-separated logits: the soft mask becomes the
+    hard mask's 0/1 keep mask and W_soft to the hard-masked W, bit for bit."""
+    N, K = 256, 384
+    w = si.gen_w(N, K, 3, 0)
+    tl = _distinct_int_logits((N // TILE, K // TILE, 2), 1)
+    pl = _distinct_int_logits((N, K // 4, 6), 2)
+    ws, m = oracle.soft_mask(w, tl, pl, tau=1e-3)  # e^-(gap/tau) underflows to exactly 0
+    wm, bm, ids = oracle.hard_mask(w, tl, pl)
+    keep = np.zeros((N, K))
+    for n in range(0, N, 37):
+        for g in range(K // 4):
+            t = bm[n // TILE, (4 * g) // TILE]
+            kept = PAIRS[ids[n, g]] if t else (0, 1, 2, 3)
+            for i in kept:
+                keep[n, 4 * g + i] = 1.0
+        assert np.allclose(m[n], keep[n], atol=1e-15)
+    # W * 0 is -0 for a negative weight (a product); the hard mask selects +0
+    assert np.array_equal(np.where(ws == 0x8000, np.uint16(0), ws), wm)
+
+
+def test_soft_mask_hot_limit_and_group_sums():
+    """tau -> infinity: p = 1/2, q = 1/6, each position lies in 3 of the 6
+    patterns, so M = 1/2 + 1/2 * 3/6 = 3/4.  At any tau the 4 entries of a
+    group sum to 4 p_dense + 2 p_sparse, with p_sparse = 1 / (1 + e^((l_d - l_s)/tau))."""
+    N, K = 128, 256
+    w = si.gen_w(N, K, 4, 0)
+    tl = si.gen_tile_logits(N, K, 4, 0)
+    pl = si.gen_pattern_logits(N, K, 4, 0)
+    _, m_hot = oracle.soft_mask(w, tl, pl, tau=1e12)
+    assert np.allclose(m_hot, 0.75, atol=1e-9)
+    tau = 0.7
+    _, m = oracle.soft_mask(w, tl, pl, tau=tau)
+    assert np.all(m >= 0.0) and np.all(m <= 1.0)
+    sums = m.reshape(N, K // 4, 4).sum(axis=2)
+    for n in (0, 63, 127):
+        for g in (0, 17, 63):
+            ld, ls = float(tl[n // TILE, (4 * g) // TILE, 0]), float(tl[n // TILE, (4 * g) // TILE, 1])
+            ps = 1.0 / (1.0 + math.exp((ld - ls) / tau))
+            assert sums[n, g] == pytest.approx(4.0 * (1.0 - ps) + 2.0 * ps, rel=1e-12)
+
+
+def test_soft_mask_noise_enters_as_a_sum_and_patterns_map_to_pairs():
+    N, K = 128, 128
+    w = si.gen_w(N, K, 5, 0)
+    rng = np.random.default_rng(7)
+    tl = rng.standard_normal((1, 1, 2)).astype(np.float32)
+    pl = rng.standard_normal((N, K // 4, 6)).astype(np.float32)
+    tg = rng.gumbel(size=(1, 1, 2)).astype(np.float32)
+    pg = rng.gumbel(size=(N, K // 4, 6)).astype(np.float32)
+    a = oracle.soft_mask(w, tl, pl, 0.5, tg, pg)
+    b = oracle.soft_mask(w, (tl.astype(np.float64) + tg), (pl.astype(np.float64) + pg), 0.5)
+    assert np.array_equal(a[0], b[0]) and np.allclose(a[1], b[1], rtol=1e-15)
+    # a sparse-only tile and one dominant pattern per group: M = its keep mask
+    tl1 = np.array([[[-1e3, 1e3]]], np.float32)
+    for j, pair in enumerate(PAIRS):
+        pl1 = np.zeros((N, K // 4, 6), np.float32)
+        pl1[:, :, j] = 1e3
+        _, m1 = oracle.soft_mask(w, tl1, pl1, 1.0)
+        expect = np.array([1.0 if i in pair else 0.0 for i in range(4)])
+        assert np.allclose(m1.reshape(N, K // 4, 4), expect, atol=1e-12)
