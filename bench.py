@@ -278,8 +278,8 @@ def offline_steps(layers, dev, pk, reps=5):
 
     out = {}
     status = tsg.new_status(dev)
-    mask_bytes = pack_bytes = fused_bytes = 0
-    mask_ms = pack_ms = fused_ms = 0.0
+    mask_bytes = pack_bytes = fused_bytes = soft_bytes = 0
+    mask_ms = pack_ms = fused_ms = soft_ms = 0.0
     for i, L in enumerate(layers):
         N, K = L["N"], L["K"]
         w = torch.from_numpy(L["w"].view(np.int16)).view(torch.bfloat16).to(dev)
@@ -307,7 +307,16 @@ def offline_steps(layers, dev, pk, reps=5):
             tsg.patch_tile_kinds(tl)
             tsg.patch_pack_from_logits(w, fbm, pl, fns, status=status)
         e[3].record()
+        # training-time soft mask with noise inputs and the mask output (the noise
+        # tensors' contents do not change the work: the logits stand in for them)
+        tsg.patch_soft_mask(w, tl, pl, 0.5, tl, pl)
+        e4 = torch.cuda.Event(enable_timing=True)
+        for _ in range(reps):
+            tsg.patch_soft_mask(w, tl, pl, 0.5, tl, pl)
+        e4.record()
         torch.cuda.synchronize()
+        soft_ms += e[3].elapsed_time(e4) / reps
+        soft_bytes += N * K * (2 + 6 + 6 + 2 + 4) + (N // 128) * (K // 128) * 16
         mask_ms += e[0].elapsed_time(e[1]) / reps
         pack_ms += e[1].elapsed_time(e[2]) / reps
         fused_ms += e[2].elapsed_time(e[3]) / reps
@@ -322,7 +331,8 @@ def offline_steps(layers, dev, pk, reps=5):
     if code != 0:
         raise RuntimeError(f"offline steps: device status {code} bits {bits}")
     for name, b, ms in (("hard_mask", mask_bytes, mask_ms), ("pack", pack_bytes, pack_ms),
-                        ("tile_kinds+pack_from_logits", fused_bytes, fused_ms)):
+                        ("tile_kinds+pack_from_logits", fused_bytes, fused_ms),
+                        ("soft_mask (training forward)", soft_bytes, soft_ms)):
         gbs = b / 1e9 / (ms / 1e3)
         out[name] = {"GB/s": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4), "ms_total": round(ms, 3),
                      "bytes": int(b), "note": "7 LLaMA-2-7B layers, mean of %d calls each (eager launches)" % reps}

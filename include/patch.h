@@ -172,6 +172,29 @@ PATCH_API patch_status_t patch_pack(const uint16_t *W, int64_t N, int64_t K, con
                           patch_tile_desc *desc, int32_t *dev_status, void *stream);
 
 /*
+ * patch_soft_mask: the training-time (soft) form of the hybrid mask ("Core
+ * Mechanism": a weighted combination of the dense and the 2:4 option;
+ * "Learnable Distributions": tile and pattern choices sampled with
+ * Gumbel-Softmax).  Per tile p = softmax((tile_logits + tile_noise) / tau) over
+ * (dense, sparse); per group of 4 q = softmax((pattern_logits + pattern_noise)
+ * / tau) over the 6 patterns; M[n][k] = p_dense + p_sparse * sum_j q_j
+ * [k mod 4 in pattern j]; W_soft = W * M rounded once to bf16 (nearest even).
+ * The pages give neither tau nor the noise: the Gumbel samples are the
+ * caller's (NULL = no noise) and tau > 0 is an argument.  As tau -> 0 the
+ * mask becomes patch_hard_mask's (pruned entries are then -0 for negative
+ * weights: a product, not a select).  fp32 arithmetic with CUDA's expf.
+ *   W bf16 [N][K]; tile_logits / tile_noise fp32 [Tn][Tk][2] (8-byte aligned);
+ *   pattern_logits / pattern_noise fp32 [N][K/4][6]; W_soft bf16 [N][K] out;
+ *   mask fp32 [N][K] out (nullable).  16-byte alignment otherwise.
+ * Errors: PATCH_ERR_INVALID_ARG (NULL input, tau not positive and finite),
+ * PATCH_ERR_SHAPE, PATCH_ERR_ALIGN, PATCH_ERR_DEVICE.
+ */
+PATCH_API patch_status_t patch_soft_mask(const uint16_t *W, int64_t N, int64_t K, const float *tile_logits,
+                                         const float *tile_noise, const float *pattern_logits,
+                                         const float *pattern_noise, float tau, uint16_t *W_soft, float *mask,
+                                         void *stream);
+
+/*
  * patch_tile_kinds: the tile half of the hard mask alone ("Learnable
  * Distributions", item 1: a 2-way logit per tile chooses dense or 2:4 sparse).
  *   tile_logits fp32 [Tn][Tk][2] (index 0 = dense, 1 = sparse);

@@ -116,6 +116,59 @@ def test_pack_of_masked_and_random_patterns():
     assert np.array_equal(pw.desc.cpu().numpy(), d_ref)
 
 
+# ------------------------------------------------- soft (training-time) mask
+
+
+def _bf16_close(gpu_bits, ref_bits):
+    """Equal up to one bf16 rounding step (the GPU multiplies in fp32, the oracle in fp64)."""
+    from _util import bf16_to_f64
+    g, r = bf16_to_f64(gpu_bits), bf16_to_f64(ref_bits)
+    return np.all(np.abs(g - r) <= np.abs(r) * 2.0 ** -7 + 1e-30)
+
+
+@pytest.mark.parametrize("tau", [0.5, 2.0])
+@pytest.mark.parametrize("N,K", [(256, 384), (128, 128)])
+def test_soft_mask_matches_oracle(N, K, tau):
+    w = si.gen_w(N, K, 13, 0)
+    tl = si.gen_tile_logits(N, K, 13, 0)
+    pl = si.gen_pattern_logits(N, K, 13, 0)
+    rng = np.random.default_rng(13)
+    tg = rng.gumbel(size=tl.shape).astype(np.float32)
+    pg = rng.gumbel(size=pl.shape).astype(np.float32)
+    ws_ref, m_ref = oracle.soft_mask(w, tl, pl, tau, tg, pg)
+    ws, m = tsg.patch_soft_mask(to_dev_bf16(w), to_dev(tl), to_dev(pl), tau, to_dev(tg), to_dev(pg))
+    m = m.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(m - m_ref) <= 2e-6 + 1e-5 * np.abs(m_ref))
+    assert _bf16_close(bits_of(ws), ws_ref)
+    # without noise and without the mask output
+    ws_ref0, _ = oracle.soft_mask(w, tl, pl, tau)
+    ws0, none = tsg.patch_soft_mask(to_dev_bf16(w), to_dev(tl), to_dev(pl), tau, want_mask=False)
+    assert none is None and _bf16_close(bits_of(ws0), ws_ref0)
+
+
+def test_soft_mask_cold_limit_is_the_hard_mask():
+    N, K = 256, 256
+    w = si.gen_w(N, K, 14, 0)
+    rng = np.random.default_rng(14)
+    tl = (np.argsort(rng.random((N // TILE, K // TILE, 2)), axis=-1) - 1.0).astype(np.float32)
+    pl = (np.argsort(rng.random((N, K // 4, 6)), axis=-1) - 3.0).astype(np.float32)
+    wm_ref, _, _ = oracle.hard_mask(w, tl, pl)
+    ws, m = tsg.patch_soft_mask(to_dev_bf16(w), to_dev(tl), to_dev(pl), 1e-3)
+    b = bits_of(ws)
+    assert np.array_equal(np.where(b == 0x8000, np.uint16(0), b), wm_ref)
+    mm = m.cpu().numpy()
+    assert np.all((mm == 0.0) | (mm == 1.0))
+
+
+def test_soft_mask_rejects_bad_temperature():
+    N = K = 128
+    w = to_dev_bf16(si.gen_w(N, K, 1, 0))
+    tl, pl = to_dev(si.gen_tile_logits(N, K, 1, 0)), to_dev(si.gen_pattern_logits(N, K, 1, 0))
+    for tau in (0.0, -1.0, float("inf"), float("nan")):
+        with pytest.raises(tsg.PatchError):
+            tsg.patch_soft_mask(w, tl, pl, tau)
+
+
 # ------------------------------------------------- fused hard mask -> pack
 
 

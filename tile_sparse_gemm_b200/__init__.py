@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
             "patch_hard_mask": [P, I64, I64, P, P, P, P, P, P, P],
             "patch_pack": [P, I64, I64, P, P, I64, P, P, P, P, P],
             "patch_tile_kinds": [P, I64, I64, P, P, P],
+            "patch_soft_mask": [P, I64, I64, P, P, P, P, ctypes.c_float, P, P, P],
             "patch_pack_from_logits": [P, I64, I64, P, P, I64, P, P, P, P, P],
             "patch_gemm_workspace_size": [I64, WP, ctypes.POINTER(SZ)],
             "patch_gemm": [P, I64, WP, P, P, SZ, P, P],
@@ -177,6 +178,21 @@ def patch_pack(W: torch.Tensor, bitmap: torch.Tensor, pat_id: torch.Tensor, n_sp
                             _dev(values, "values"), _dev(meta, "meta") if mb else None, _dev(desc, "desc"),
                             _dev(status, "status"), _stream(stream)), "patch_pack")
     return PackedWeight(N, K, n_sparse, values, meta, desc)
+
+
+def patch_soft_mask(W: torch.Tensor, tile_logits: torch.Tensor, pattern_logits: torch.Tensor, tau: float,
+                    tile_noise: torch.Tensor | None = None, pattern_noise: torch.Tensor | None = None,
+                    want_mask: bool = True, stream=None):
+    """Training-time hybrid mask: (W_soft bf16 [N][K], M fp32 [N][K] or None)."""
+    N, K = W.shape
+    dev = W.device
+    w_soft = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    mask = torch.empty((N, K), dtype=torch.float32, device=dev) if want_mask else None
+    _check(lib().patch_soft_mask(_dev(W, "W"), N, K, _dev(tile_logits, "tile_logits"),
+                                 _dev(tile_noise, "tile_noise"), _dev(pattern_logits, "pattern_logits"),
+                                 _dev(pattern_noise, "pattern_noise"), float(tau), _dev(w_soft, "W_soft"),
+                                 _dev(mask, "mask"), _stream(stream)), "patch_soft_mask")
+    return w_soft, mask
 
 
 def patch_tile_kinds(tile_logits: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:

@@ -108,6 +108,25 @@ patch_status_t patch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t
   return PATCH_OK;
 }
 
+patch_status_t patch_soft_mask(const uint16_t* W, int64_t N, int64_t K, const float* tile_logits,
+                               const float* tile_noise, const float* pattern_logits, const float* pattern_noise,
+                               float tau, uint16_t* W_soft, float* mask, void* stream) {
+  if (!W || !tile_logits || !pattern_logits || !W_soft) return PATCH_ERR_INVALID_ARG;
+  if (!(tau > 0.0f) || !(tau < 3.0e38f)) return PATCH_ERR_INVALID_ARG;  // positive and finite
+  if (!shape_ok(N, K)) return PATCH_ERR_SHAPE;
+  auto a8 = [](const void* q) { return reinterpret_cast<uintptr_t>(q) % 8 == 0; };
+  if (!aligned16(W) || !aligned16(pattern_logits) || (pattern_noise && !aligned16(pattern_noise)) ||
+      !aligned16(W_soft) || (mask && !aligned16(mask)) || !a8(tile_logits) || (tile_noise && !a8(tile_noise)))
+    return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_soft_mask(W, N, K, tile_logits, tile_noise, pattern_logits, pattern_noise, tau, W_soft, mask, sms,
+                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
 patch_status_t patch_tile_kinds(const float* tile_logits, int64_t N, int64_t K, uint8_t* bitmap,
                                 int64_t* n_sparse, void* stream) {
   if (!tile_logits || !bitmap || !n_sparse) return PATCH_ERR_INVALID_ARG;

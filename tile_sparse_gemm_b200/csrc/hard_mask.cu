@@ -99,3 +99,104 @@ cudaError_t launch_hard_mask(const uint16_t* W, int64_t N, int64_t K, const floa
 }
 
 }  // namespace patch
+
+namespace patch {
+
+// Training-time (soft) hybrid mask: the Gumbel-Softmax relaxation of the two
+// choices above ("Core Mechanism": the mask is a weighted combination of the
+// dense option and the 2:4 option).  Per tile p = softmax((l + g) / tau) over
+// (dense, sparse); per group q = softmax((l + g) / tau) over the 6 patterns;
+// M = p_dense + p_sparse * sum_j q_j [position in pattern j]; W_soft = W * M.
+// The Gumbel samples g are the caller's (NULL = none).  One thread per 8
+// groups of one row, as in the hard mask; HBM-bound.
+__global__ void __launch_bounds__(256) soft_mask_kernel(
+    const uint4* __restrict__ W, int64_t N, int64_t K, const float2* __restrict__ tile_logits,
+    const float2* __restrict__ tile_noise, const float4* __restrict__ pattern_logits,
+    const float4* __restrict__ pattern_noise, float inv_tau, uint4* __restrict__ W_soft,
+    float4* __restrict__ mask) {
+  const int64_t items_per_row = K / 32;  // 8 groups per item
+  const int64_t n_items = N * items_per_row;
+  const int64_t Tk = K / kTile;
+  for (int64_t it = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; it < n_items;
+       it += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t n = it / items_per_row;
+    const int64_t j = it - n * items_per_row;
+    const int64_t t = (n / kTile) * Tk + (32 * j) / kTile;
+    float2 tl = tile_logits[t];
+    if (tile_noise) {
+      const float2 g = tile_noise[t];
+      tl.x += g.x;
+      tl.y += g.y;
+    }
+    const float zd = tl.x * inv_tau, zs = tl.y * inv_tau, zm = fmaxf(zd, zs);
+    const float ed = expf(zd - zm), es = expf(zs - zm);
+    const float pd = ed / (ed + es), ps = es / (ed + es);
+
+    float lg[48];
+#pragma unroll
+    for (int q = 0; q < 12; ++q) {
+      float4 v = __ldcs(pattern_logits + it * 12 + q);
+      if (pattern_noise) {
+        const float4 g = __ldcs(pattern_noise + it * 12 + q);
+        v.x += g.x;
+        v.y += g.y;
+        v.z += g.z;
+        v.w += g.w;
+      }
+      lg[4 * q] = v.x;
+      lg[4 * q + 1] = v.y;
+      lg[4 * q + 2] = v.z;
+      lg[4 * q + 3] = v.w;
+    }
+    float m[32];
+#pragma unroll
+    for (int gi = 0; gi < 8; ++gi) {
+      const float* l = lg + 6 * gi;
+      float zmax = l[0] * inv_tau;
+#pragma unroll
+      for (int c = 1; c < 6; ++c) zmax = fmaxf(zmax, l[c] * inv_tau);
+      float e[6], sum = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 6; ++c) {
+        e[c] = expf(l[c] * inv_tau - zmax);
+        sum += e[c];
+      }
+      // patterns 0:(0,1) 1:(0,2) 2:(0,3) 3:(1,2) 4:(1,3) 5:(2,3): each position lies in 3
+      const float keep[4] = {e[0] + e[1] + e[2], e[0] + e[3] + e[4], e[1] + e[3] + e[5], e[2] + e[4] + e[5]};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m[4 * gi + i] = pd + ps * (keep[i] / sum);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // 16 B = 8 weights
+      const uint4 w = __ldcs(W + it * 4 + q);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      uint32_t out[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float a = bf16_lo(ww[h]) * m[8 * q + 2 * h], b = bf16_hi(ww[h]) * m[8 * q + 2 * h + 1];
+        out[h] = uint32_t(f32_to_bf16_rne(a)) | uint32_t(f32_to_bf16_rne(b)) << 16;
+      }
+      __stcs(W_soft + it * 4 + q, make_uint4(out[0], out[1], out[2], out[3]));
+    }
+    if (mask) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) __stcs(mask + it * 8 + q, make_float4(m[4 * q], m[4 * q + 1], m[4 * q + 2], m[4 * q + 3]));
+    }
+  }
+}
+
+cudaError_t launch_soft_mask(const uint16_t* W, int64_t N, int64_t K, const float* tile_logits,
+                             const float* tile_noise, const float* pattern_logits, const float* pattern_noise,
+                             float tau, uint16_t* W_soft, float* mask, int num_sms, cudaStream_t stream) {
+  const int64_t n_items = N * (K / 32);
+  int64_t blocks = (n_items + 255) / 256;
+  if (blocks > int64_t(num_sms) * 8) blocks = int64_t(num_sms) * 8;
+  soft_mask_kernel<<<int(blocks), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(W), N, K, reinterpret_cast<const float2*>(tile_logits),
+      reinterpret_cast<const float2*>(tile_noise), reinterpret_cast<const float4*>(pattern_logits),
+      reinterpret_cast<const float4*>(pattern_noise), 1.0f / tau, reinterpret_cast<uint4*>(W_soft),
+      reinterpret_cast<float4*>(mask));
+  return cudaGetLastError();
+}
+
+}  // namespace patch

@@ -22,6 +22,10 @@ cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* 
 cudaError_t launch_tile_kinds(const float* tile_logits, int64_t N, int64_t K, uint8_t* bitmap, int64_t* n_sparse,
                               cudaStream_t stream);
 
+cudaError_t launch_soft_mask(const uint16_t* W, int64_t N, int64_t K, const float* tile_logits,
+                             const float* tile_noise, const float* pattern_logits, const float* pattern_noise,
+                             float tau, uint16_t* W_soft, float* mask, int num_sms, cudaStream_t stream);
+
 // Decode split: L K-tiles per unit, S K-splits, units CTAs, smem bytes, fp32 workspace bytes.
 struct DecodePlan {
   int L, S, units;
