@@ -332,6 +332,25 @@ PATCH_API patch_status_t patch_gemm_mlp(const uint16_t *X, int64_t M, const patc
                                         int32_t *dev_status, void *stream);
 
 /*
+ * patch_shard_rows: column-parallel split of one layer over n_shards GPUs
+ * (output features are independent, so each GPU multiplies a contiguous range
+ * of tile rows and the full Y is the concatenation of the shards' Y along N).
+ * Balanced by stored bytes, not by rows: tile row r stores
+ *   bytes(r) = sum over its Tk tiles of (dense ? 32768 : 18432) + 16 * Tk,
+ * and shard i (0-based) is [row_begin[i], row_begin[i + 1]) where
+ * row_begin[0] = 0, row_begin[n_shards] = Tn and, for 0 < i < n_shards,
+ * row_begin[i] is the first row whose prefix sum of bytes (rows before it)
+ * reaches i / n_shards of the total, then moved, if needed, to keep every
+ * shard non-empty (row_begin[i - 1] < row_begin[i] <= Tn - (n_shards - i)).
+ *   bitmap    HOST u8 [Tn][Tk] (nonzero = sparse);
+ *   row_begin HOST int64 [n_shards + 1] out.
+ * Host only, no device work.  Errors: PATCH_ERR_INVALID_ARG (NULL, Tn or Tk < 1,
+ * n_shards < 1 or > Tn).
+ */
+PATCH_API patch_status_t patch_shard_rows(const uint8_t *bitmap, int64_t Tn, int64_t Tk, int64_t n_shards,
+                                          int64_t *row_begin);
+
+/*
  * patch_read_status: synchronise `stream`, copy *dev_status to *host_bits and
  * return the first error it encodes (PATCH_ERR_TIMEOUT, then BAD_PATTERN,
  * then COUNT) or PATCH_OK.  host_bits may be NULL.

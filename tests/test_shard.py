@@ -1,0 +1,93 @@
+"""Column-parallel sharding of a layer over several GPUs (host logic, CPU):
+the tile-row split balanced by stored bytes, and -- with two gloo ranks --
+that the shards' outputs concatenate to the whole layer's output."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+import oracle
+import synth_inputs as si
+import tile_sparse_gemm_b200 as tsg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+DENSE, SPARSE = 32768, 16384 + 2048
+
+
+def _row_bytes(bm):
+    return np.where(bm != 0, SPARSE, DENSE).sum(axis=1) + 16 * bm.shape[1]
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("kind", ["exact", "clustered", "bernoulli"])
+def test_shard_rows_definition_and_balance(n, kind):
+    N, K = 128 * 43, 128 * 8
+    bm = {"exact": si.tiles_exact, "clustered": si.tiles_clustered, "bernoulli": si.tiles_bernoulli}[kind](
+        N, K, 0.5, 3, n)
+    rows = tsg.shard_rows(bm, n)
+    rb = _row_bytes(bm)
+    prefix = np.concatenate([[0], np.cumsum(rb)])
+    total = prefix[-1]
+    assert rows[0][0] == 0 and rows[-1][1] == bm.shape[0]
+    for (b0, e0), (b1, e1) in zip(rows, rows[1:]):
+        assert e0 == b1  # contiguous
+    for i, (b, e) in enumerate(rows):
+        assert e > b  # never empty
+        if i > 0:  # the first row whose prefix reaches i/n of the total (no clamp needed at these sizes)
+            assert prefix[b] * n >= i * total and prefix[b - 1] * n < i * total
+    # balance: no shard exceeds its fair share by more than one row
+    worst = max(prefix[e] - prefix[b] for b, e in rows)
+    assert worst <= total / n + rb.max()
+
+
+def test_shard_rows_keeps_every_shard_non_empty():
+    bm = np.zeros((5, 3), np.uint8)
+    bm[0] = 1  # one light row, then heavy ones
+    assert tsg.shard_rows(bm, 5) == [(0, 1), (1, 2), (2, 3), (3, 4), (4, 5)]
+    with pytest.raises(tsg.PatchError):
+        tsg.shard_rows(bm, 6)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle as orc
+        import synth_inputs as s
+        import tile_sparse_gemm_b200 as t
+        N, K, M = 128 * 7, 256, 5
+        w, x = s.gen_w(N, K, 15, 0), s.gen_x(M, K, 15, 0)
+        bm, ids = s.tiles_clustered(N, K, 0.5, 15, 0), s.patterns_top2(w)
+        b, e = t.shard_rows(bm, world)[rank]
+        # this rank's shard of Y (the oracle stands in for the GPU GEMM on CPU)
+        y = orc.hybrid_gemm(x, w[b * 128:e * 128], bm[b:e], ids[b * 128:e * 128])
+        parts = [None] * world
+        dist.all_gather_object(parts, y)
+        out[rank] = np.concatenate(parts, axis=1)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_concatenate_to_the_whole_layer():
+    world = 2
+    out = mp.Manager().dict()
+    mp.start_processes(_rank, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+    N, K, M = 128 * 7, 256, 5
+    w, x = si.gen_w(N, K, 15, 0), si.gen_x(M, K, 15, 0)
+    ref = oracle.hybrid_gemm(x, w, si.tiles_clustered(N, K, 0.5, 15, 0), si.patterns_top2(w))
+    for r in range(world):
+        assert np.array_equal(out[r], ref)

@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "patch_pack": [P, I64, I64, P, P, I64, P, P, P, P, P],
             "patch_tile_kinds": [P, I64, I64, P, P, P],
             "patch_soft_mask": [P, I64, I64, P, P, P, P, ctypes.c_float, P, P, P],
+            "patch_shard_rows": [P, I64, I64, I64, P],
             "patch_pack_from_logits": [P, I64, I64, P, P, I64, P, P, P, P, P],
             "patch_gemm_workspace_size": [I64, WP, ctypes.POINTER(SZ)],
             "patch_gemm": [P, I64, WP, P, P, SZ, P, P],
@@ -289,6 +290,24 @@ def patch_gemm_mlp(X: torch.Tensor, gate: PackedWeight, up: PackedWeight, H: tor
                                 _dev(workspace, "workspace"), workspace.numel(), _dev(status, "status"),
                                 _stream(stream)), "patch_gemm_mlp")
     return H
+
+
+def shard_rows(bitmap, n_shards: int) -> list[tuple[int, int]]:
+    """Column-parallel split of a layer into n_shards contiguous tile-row ranges
+    balanced by stored bytes (host computation): [(row_begin, row_end), ...]."""
+    import numpy as np
+    bm = np.ascontiguousarray(bitmap.cpu().numpy() if isinstance(bitmap, torch.Tensor) else bitmap, dtype=np.uint8)
+    Tn, Tk = bm.shape
+    out = np.zeros(n_shards + 1, dtype=np.int64)
+    _check(lib().patch_shard_rows(bm.ctypes.data_as(ctypes.c_void_p), Tn, Tk, n_shards,
+                                  out.ctypes.data_as(ctypes.c_void_p)), "patch_shard_rows")
+    return [(int(out[i]), int(out[i + 1])) for i in range(n_shards)]
+
+
+def shard_of(W: torch.Tensor, bitmap: torch.Tensor, pat_id: torch.Tensor, rows: tuple[int, int]):
+    """Views of one shard's W rows, bitmap rows and pattern-id rows (no copy)."""
+    b, e = rows
+    return W[b * 128:e * 128], bitmap[b:e], pat_id[b * 128:e * 128]
 
 
 def patch_read_status(status: torch.Tensor, stream=None) -> tuple[int, int]:

@@ -279,6 +279,39 @@ patch_status_t patch_gemm_mlp(const uint16_t* X, int64_t M, const patch_weight* 
   return PATCH_OK;
 }
 
+patch_status_t patch_shard_rows(const uint8_t* bitmap, int64_t Tn, int64_t Tk, int64_t n_shards,
+                                int64_t* row_begin) {
+  if (!bitmap || !row_begin || Tn < 1 || Tk < 1 || n_shards < 1 || n_shards > Tn) return PATCH_ERR_INVALID_ARG;
+  // prefix sums of the stored bytes of the tile rows
+  int64_t total = 0;
+  for (int64_t r = 0; r < Tn; ++r) {
+    int64_t b = 16 * Tk;
+    for (int64_t k = 0; k < Tk; ++k)
+      b += bitmap[r * Tk + k] ? int64_t(PATCH_SPARSE_TILE_BYTES + PATCH_META_TILE_BYTES) : int64_t(PATCH_DENSE_TILE_BYTES);
+    total += b;
+  }
+  row_begin[0] = 0;
+  int64_t r = 0, before = 0;  // rows [0, r) hold `before` bytes
+  for (int64_t i = 1; i < n_shards; ++i) {
+    // first row whose prefix reaches i / n of the total (compared without rounding)
+    while (r < Tn && before * n_shards < i * total) {
+      int64_t b = 16 * Tk;
+      for (int64_t k = 0; k < Tk; ++k)
+        b += bitmap[r * Tk + k] ? int64_t(PATCH_SPARSE_TILE_BYTES + PATCH_META_TILE_BYTES)
+                                : int64_t(PATCH_DENSE_TILE_BYTES);
+      before += b;
+      ++r;
+    }
+    // strictly increasing, and leave at least one row for each later shard
+    int64_t v = r;
+    if (v <= row_begin[i - 1]) v = row_begin[i - 1] + 1;
+    if (v > Tn - (n_shards - i)) v = Tn - (n_shards - i);
+    row_begin[i] = v;
+  }
+  row_begin[n_shards] = Tn;
+  return PATCH_OK;
+}
+
 patch_status_t patch_read_status(const int32_t* dev_status, void* stream, int32_t* host_bits) {
   if (!dev_status) return PATCH_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
