@@ -126,6 +126,10 @@ LLAMA3_8B = [("q", 4096, 4096), ("k", 1024, 4096), ("v", 1024, 4096), ("o", 4096
              ("gate", 14336, 4096), ("up", 14336, 4096), ("down", 4096, 14336)]
 QWEN25_05B = [("q", 896, 896), ("k", 128, 896), ("v", 128, 896), ("o", 896, 896),
               ("gate", 4864, 896), ("up", 4864, 896), ("down", 896, 4864)]
+# Gemma-3-1B linears (hidden 1152, 4 query heads and 1 key/value head of 256, MLP 6912),
+# another of the model families the pages evaluate
+GEMMA3_1B = [("q", 1024, 1152), ("k", 256, 1152), ("v", 256, 1152), ("o", 1152, 1024),
+             ("gate", 6912, 1152), ("up", 6912, 1152), ("down", 1152, 6912)]
 
 
 def stack_fraction(layer: int, proj: str, n_layers: int = 32) -> float:

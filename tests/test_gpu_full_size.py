@@ -93,10 +93,10 @@ def test_llama2_stack_sampled_layers(group, M):
         check_gemm(y, ref, f"stack L{layer} {name} f={f} M={M}")
 
 
-@pytest.mark.parametrize("family", ["llama3", "qwen"])
+@pytest.mark.parametrize("family", ["llama3", "qwen", "gemma3"])
 def test_llama3_qwen_clustered(family):
-    shapes = si.LLAMA3_8B if family == "llama3" else si.QWEN25_05B
-    base = 0 if family == "llama3" else 7
+    shapes = {"llama3": si.LLAMA3_8B, "qwen": si.QWEN25_05B, "gemma3": si.GEMMA3_1B}[family]
+    base = {"llama3": 0, "qwen": 7, "gemma3": 14}[family]
     for j, (name, N, K) in enumerate(shapes):
         idx = base + j
         w, ids = weight(N, K, 5, idx)
