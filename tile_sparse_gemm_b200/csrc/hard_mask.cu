@@ -7,7 +7,10 @@
 // HBM-bound elementwise pass: per weight it reads 2 B of W and 6 B of pattern
 // logits and writes 2 B of masked W plus 1/4 B of pattern id.  One thread
 // handles 8 consecutive groups (32 weights) of one row: 4 x 16 B loads of W,
-// 12 x 16 B loads of logits, 4 x 16 B stores, one 8 B store of ids.
+// 12 x 16 B loads of logits, 4 x 16 B stores, one 8 B store of ids.  The
+// loads go through L1 (not the streaming hint): a warp's 16-byte pieces of
+// 192-byte items use half of each 32-byte sector per instruction, and the
+// next instruction finds the other half there.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -49,7 +52,7 @@ __global__ void __launch_bounds__(256) hard_mask_kernel(
     const float4* lp = pattern_logits + it * 12;
 #pragma unroll
     for (int q = 0; q < 12; ++q) {
-      float4 v = __ldcs(lp + q);
+      float4 v = __ldg(lp + q);
       lg[4 * q] = v.x;
       lg[4 * q + 1] = v.y;
       lg[4 * q + 2] = v.z;
@@ -66,7 +69,7 @@ __global__ void __launch_bounds__(256) hard_mask_kernel(
     if (W_masked) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {  // 16 B = 8 weights = groups 2q, 2q+1
-        uint4 w = __ldcs(W + it * 4 + q);
+        uint4 w = __ldg(W + it * 4 + q);
         if (sparse) {
           const uint32_t c0 = pattern_code(ids[2 * q]), c1 = pattern_code(ids[2 * q + 1]);
           // keep-masks of the 4 bf16 lanes of each group (bit i set = keep position i)
@@ -135,9 +138,9 @@ __global__ void __launch_bounds__(256) soft_mask_kernel(
     float lg[48];
 #pragma unroll
     for (int q = 0; q < 12; ++q) {
-      float4 v = __ldcs(pattern_logits + it * 12 + q);
+      float4 v = __ldg(pattern_logits + it * 12 + q);
       if (pattern_noise) {
-        const float4 g = __ldcs(pattern_noise + it * 12 + q);
+        const float4 g = __ldg(pattern_noise + it * 12 + q);
         v.x += g.x;
         v.y += g.y;
         v.z += g.z;
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(256) soft_mask_kernel(
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {  // 16 B = 8 weights
-      const uint4 w = __ldcs(W + it * 4 + q);
+      const uint4 w = __ldg(W + it * 4 + q);
       const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
       uint32_t out[4];
 #pragma unroll

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256) pack_tiles_kernel(
           float lg[12];
 #pragma unroll
           for (int q = 0; q < 3; ++q) {
-            const float4 v = __ldcs(pattern_logits + group * 6 / 4 + q);
+            const float4 v = __ldg(pattern_logits + group * 6 / 4 + q);
             lg[4 * q] = v.x;
             lg[4 * q + 1] = v.y;
             lg[4 * q + 2] = v.z;
