@@ -443,9 +443,20 @@ def run_ours(args, rank, world):
                             torch.from_numpy(L["bm"]).to(dev), torch.from_numpy(L["ids"]).to(dev),
                             int(L["bm"].sum()), status=status)
         packed.append(pw)
-    xs = {(li, M): torch.from_numpy(layers[li]["xs"][M].view(np.int16)).view(torch.bfloat16).to(dev)
-          for li, M in calls}
-    ys = {(li, M): torch.empty((M, layers[li]["N"]), dtype=torch.bfloat16, device=dev) for li, M in calls}
+    # every call's X (and Y) is a view into one device buffer, so that the
+    # end-to-end run moves a step's inputs and results with one copy each way
+    x_sizes = [M * layers[li]["K"] for li, M in calls]
+    y_sizes = [M * layers[li]["N"] for li, M in calls]
+    x_all = torch.empty(sum(x_sizes), dtype=torch.bfloat16, device=dev)
+    y_all = torch.empty(sum(y_sizes), dtype=torch.bfloat16, device=dev)
+    xs, ys = {}, {}
+    xo = yo = 0
+    for (li, M), xn, yn in zip(calls, x_sizes, y_sizes):  # sizes are multiples of 128: views stay 16-byte aligned
+        xs[(li, M)] = x_all[xo:xo + xn].view(M, layers[li]["K"])
+        xs[(li, M)].copy_(torch.from_numpy(layers[li]["xs"][M].view(np.int16)).view(torch.bfloat16))
+        ys[(li, M)] = y_all[yo:yo + yn].view(M, layers[li]["N"])
+        xo += xn
+        yo += yn
     ws_bytes = max(tsg.patch_gemm_workspace_size(M, packed[li]) for li, M in calls)
     ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)  # zero-filled once, left zeroed by each call
     launches_per_call = {c: 1 for c in calls}  # one kernel per patch_gemm call
@@ -526,29 +537,74 @@ def run_ours(args, rank, world):
     if code != 0:
         raise RuntimeError(f"device status {code} bits {bits} after timing")
 
-    # end to end through the public API with host buffers (pinned), copies inside the timed region
-    xh = {c: xs[c].cpu().pin_memory() for c in calls}
-    yh = {c: torch.empty(ys[c].shape, dtype=torch.bfloat16).pin_memory() for c in calls}
-    h2d = sum(xh[c].numel() * 2 for c in calls)
-    d2h = sum(yh[c].numel() * 2 for c in calls)
+    # End to end through the public API with host buffers.  Every step copies its
+    # inputs host -> device from pinned memory (one copy) and its results
+    # device -> host (one copy).  Two device buffer sets make a three-stage
+    # pipeline: while step s computes on set s%2, step s+1's inputs arrive in the
+    # other set and step s-1's results leave it, on two copy streams.  One stage
+    # (copy in, compute, copy out, joined) is one CUDA graph per set parity.  The
+    # timed region runs from before step 0's input copy to after step K-1's
+    # result copy; it carries K+1 copies each way for K steps (the first stage's
+    # result copy and the last stage's input copy are surplus).
+    x_host = x_all.cpu().pin_memory()
+    y_host = [torch.empty(y_all.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    h2d = x_host.numel() * 2
+    d2h = y_host[0].numel() * 2
+    x_sets, y_sets = [x_all, torch.empty_like(x_all)], [y_all, torch.empty_like(y_all)]
+    views = []
+    for bset in range(2):
+        xv, yv, xo, yo = {}, {}, 0, 0
+        for (li, M), xn, yn in zip(calls, x_sizes, y_sizes):
+            xv[(li, M)] = x_sets[bset][xo:xo + xn].view(M, layers[li]["K"])
+            yv[(li, M)] = y_sets[bset][yo:yo + yn].view(M, layers[li]["N"])
+            xo += xn
+            yo += yn
+        views.append((xv, yv))
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
+    def stage(p):
+        cur = torch.cuda.current_stream()
+        q = 1 - p
+        s_in.wait_stream(cur)
+        s_out.wait_stream(cur)
+        with torch.cuda.stream(s_in):
+            x_sets[q].copy_(x_host, non_blocking=True)  # inputs of the next step
+        with torch.cuda.stream(s_out):
+            y_host[q].copy_(y_sets[q], non_blocking=True)  # results of the previous step
+        xv, yv = views[p]
         for li, M in calls:
-            xs[(li, M)].copy_(xh[(li, M)], non_blocking=True)
-            tsg.patch_gemm(xs[(li, M)], packed[li], Y=ys[(li, M)], workspace=ws, status=status)
-            yh[(li, M)].copy_(ys[(li, M)], non_blocking=True)
+            tsg.patch_gemm(xv[(li, M)], packed[li], Y=yv[(li, M)], workspace=ws, status=status)
+        cur.wait_stream(s_in)
+        cur.wait_stream(s_out)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    stage_graphs = None
+    if not args.no_graph:
+        stage_graphs = []
+        for p in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                stage(p)
+            stage_graphs.append(g)
+
+    def run_e2e(n):
+        x_sets[0].copy_(x_host, non_blocking=True)
+        for st in range(n):
+            if stage_graphs is not None:
+                stage_graphs[st % 2].replay()
+            else:
+                stage(st % 2)
+        y_host[(n - 1) % 2].copy_(y_sets[(n - 1) % 2], non_blocking=True)
+
+    run_e2e(max(2, args.warmup))
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    run_e2e(args.steps)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    del stage_graphs
     e2e_ms = e0.elapsed_time(e1)
 
     ms, e2e_ms = job_times(ms, e2e_ms, world, dev)
