@@ -42,6 +42,8 @@ def _load():
         for name, args in {
             "oracle_apply_mask": [P, I64, I64, P, P, P],
             "oracle_hard_mask": [P, I64, I64, P, P, P, P, P],
+            "oracle_hard_mask_tiles": [P, I64, I64, I64, P, P, P, P, P],
+            "oracle_exec_tiles": [P, I64, I64, I64, P, P],
             "oracle_pack": [P, I64, I64, P, P, I64, P, P, P],
             "oracle_unpack": [P, P, P, I64, I64, P],
             "oracle_gemm_rows": [P, I64, P, I64, P, I64, I64, P],
@@ -99,6 +101,30 @@ def hard_mask(w: np.ndarray, tile_logits: np.ndarray, pattern_logits: np.ndarray
                                     _ptr(np.ascontiguousarray(pattern_logits, np.float32)),
                                     _ptr(wm), _ptr(bitmap), _ptr(pid)), "hard_mask")
     return wm, bitmap, pid
+
+
+def hard_mask_tiles(w: np.ndarray, tile_logits: np.ndarray, pattern_logits: np.ndarray, mask_tile: int):
+    """Hard mask with b x b mask tiles (b = mask_tile, 4..128): returns
+    (W_masked, bitmap [N/b][K/b] u8, pat_id [N][K/4] u8)."""
+    w = np.ascontiguousarray(w, np.uint16)
+    N, K = w.shape
+    b = int(mask_tile)
+    wm = np.empty_like(w)
+    bitmap = np.empty((N // b, K // b), np.uint8)
+    pid = np.empty((N, K // 4), np.uint8)
+    _check(_load().oracle_hard_mask_tiles(_ptr(w), N, K, b, _ptr(np.ascontiguousarray(tile_logits, np.float32)),
+                                          _ptr(np.ascontiguousarray(pattern_logits, np.float32)),
+                                          _ptr(wm), _ptr(bitmap), _ptr(pid)), "hard_mask_tiles")
+    return wm, bitmap, pid
+
+
+def exec_tiles(bitmap: np.ndarray, N: int, K: int, mask_tile: int):
+    """128 x 128 execution tiles of a b x b mask bitmap: (exec [N/128][K/128] u8, n_sparse)."""
+    bitmap = np.ascontiguousarray(bitmap, np.uint8)
+    ex = np.empty((N // TILE, K // TILE), np.uint8)
+    n = ctypes.c_int64()
+    _check(_load().oracle_exec_tiles(_ptr(bitmap), N, K, int(mask_tile), _ptr(ex), ctypes.byref(n)), "exec_tiles")
+    return ex, n.value
 
 
 def pack_sizes(N: int, K: int, n_sparse: int):

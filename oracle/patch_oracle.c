@@ -43,6 +43,11 @@
  *        ((g>>1)&1) | ((r>>3)&1)<<1 | (g>>3)<<2 | (r&7)<<4
  *        | ((g>>2)&1)<<7 | (r>>4)<<8 .
  *
+ * Mask tiles smaller than 128 x 128 (oracle_hard_mask_tiles,
+ * oracle_exec_tiles) follow "Ablation Studies" (tile size) with the reading
+ * that the execution tile stays 128 x 128 and runs sparse only when all its
+ * mask tiles are sparse.
+ *
  * Parity pins (tests/test_oracle.py): brute force over the 6 patterns with
  * one-hot logits, argmax ties, the exactly-2-of-4 invariant, global sparsity
  * = 0.5 x sparse-tile fraction, all-dense == numpy dense matmul, all-sparse
@@ -133,6 +138,75 @@ int oracle_hard_mask(const uint16_t *W, int64_t N, int64_t K, const float *tile_
         pat_id[i] = (uint8_t)argmax_first(pattern_logits + 6 * i, 6);
     if (W_masked)
         return oracle_apply_mask(W, N, K, bitmap, pat_id, W_masked);
+    return OK;
+}
+
+/*
+ * Mask tiles smaller than the execution tile ("Ablation Studies", tile size:
+ * the learned tile may be as small as 4 x 4, while hardware efficiency needs
+ * 128 x 128 execution tiles).  The mask tile is b x b, b a power of two from
+ * 4 to 128; tile logits are [N/b][K/b][2] and the bitmap [N/b][K/b].  Each
+ * choice is the argmax as above; position k of row n is kept when its b x b
+ * tile is dense, or when k mod 4 is in the pattern of its group.
+ */
+static int mask_tile_ok(int64_t b)
+{
+    return b == 4 || b == 8 || b == 16 || b == 32 || b == 64 || b == 128;
+}
+
+int oracle_hard_mask_tiles(const uint16_t *W, int64_t N, int64_t K, int64_t b, const float *tile_logits,
+                           const float *pattern_logits, uint16_t *W_masked, uint8_t *bitmap,
+                           uint8_t *pat_id)
+{
+    if (!shape_ok(N, K) || !mask_tile_ok(b))
+        return ERR_SHAPE;
+    int64_t Tnb = N / b, Tkb = K / b;
+    for (int64_t t = 0; t < Tnb * Tkb; ++t)
+        bitmap[t] = (uint8_t)argmax_first(tile_logits + 2 * t, 2);
+    int64_t G = N * (K / 4);
+    for (int64_t i = 0; i < G; ++i)
+        pat_id[i] = (uint8_t)argmax_first(pattern_logits + 6 * i, 6);
+    if (!W_masked)
+        return OK;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            int keep = 1;
+            if (bitmap[(n / b) * Tkb + k / b]) {
+                int id = pat_id[n * (K / 4) + k / 4];
+                int pos = (int)(k % 4);
+                keep = pos == KEEP[id][0] || pos == KEEP[id][1];
+            }
+            W_masked[n * K + k] = keep ? W[n * K + k] : (uint16_t)0x0000;
+        }
+    }
+    return OK;
+}
+
+/*
+ * Execution tiles of a b x b mask: the 128 x 128 execution tile (tn, tk) runs
+ * on the 2:4 sparse path only when every mask tile inside it is sparse; any
+ * dense mask tile makes it a dense execution tile (whose sparse mask tiles
+ * then carry their pruned zeros explicitly).  Writes exec [N/128][K/128] and
+ * returns the number of sparse execution tiles through *n_sparse.
+ */
+int oracle_exec_tiles(const uint8_t *bitmap, int64_t N, int64_t K, int64_t b, uint8_t *exec, int64_t *n_sparse)
+{
+    if (!shape_ok(N, K) || !mask_tile_ok(b))
+        return ERR_SHAPE;
+    int64_t Tn = N / TILE, Tk = K / TILE, Tkb = K / b, r = TILE / b;
+    int64_t count = 0;
+    for (int64_t tn = 0; tn < Tn; ++tn) {
+        for (int64_t tk = 0; tk < Tk; ++tk) {
+            int all_sparse = 1;
+            for (int64_t i = 0; i < r; ++i)
+                for (int64_t j = 0; j < r; ++j)
+                    if (!bitmap[(tn * r + i) * Tkb + tk * r + j])
+                        all_sparse = 0;
+            exec[tn * Tk + tk] = (uint8_t)all_sparse;
+            count += all_sparse;
+        }
+    }
+    *n_sparse = count;
     return OK;
 }
 

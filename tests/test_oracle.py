@@ -426,3 +426,109 @@ def test_soft_mask_noise_enters_as_a_sum_and_patterns_map_to_pairs():
         _, m1 = oracle.soft_mask(w, tl1, pl1, 1.0)
         expect = np.array([1.0 if i in pair else 0.0 for i in range(4)])
         assert np.allclose(m1.reshape(N, K // 4, 4), expect, atol=1e-12)
+
+
+# ---- mask tiles smaller than the 128 x 128 execution tile ("Ablation Studies", tile size)
+
+MASK_TILES = [4, 8, 16, 32, 64, 128]
+
+
+def test_mask_tiles_at_128_are_the_hard_mask():
+    """b = 128 reduces to the (separately pinned) 128 x 128 hard mask."""
+    N, K = 2 * TILE, 3 * TILE
+    w = si.gen_w(N, K, 5, 1)
+    tl = si.gen_tile_logits(N, K, 5, 1)
+    pl = si.gen_pattern_logits(N, K, 5, 1)
+    for a, b in zip(oracle.hard_mask(w, tl, pl), oracle.hard_mask_tiles(w, tl, pl, 128)):
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("b", [4, 8, 16, 32, 64])
+def test_mask_tiles_keep_exactly_what_each_tile_chose(b):
+    """All-ones W, one-hot logits drawn at random: every b x b block is fully kept
+    when its tile logit says dense, and keeps exactly its group's pair otherwise
+    (the pair read from the lexicographic enumeration of 2-subsets)."""
+    N, K = TILE, 2 * TILE
+    rng = np.random.default_rng(b)
+    choice = rng.integers(0, 2, (N // b, K // b))
+    ids = rng.integers(0, 6, (N, K // 4))
+    tl = np.zeros((N // b, K // b, 2), np.float32)
+    tl[..., 0] = 1.0 - choice
+    tl[..., 1] = choice
+    pl = np.zeros((N, K // 4, 6), np.float32)
+    np.put_along_axis(pl, ids[..., None], 1.0, axis=2)
+    w = np.full((N, K), ONE, np.uint16)
+    wm, bm, pid = oracle.hard_mask_tiles(w, tl, pl, b)
+    assert np.array_equal(bm, choice.astype(np.uint8))
+    assert np.array_equal(pid, ids.astype(np.uint8))
+    for n in range(0, N, 7):
+        for g in range(0, K // 4, 3):
+            kept_pos = set(PAIRS[ids[n, g]]) if choice[n // b, (4 * g) // b] else {0, 1, 2, 3}
+            row = wm[n, 4 * g:4 * g + 4]
+            assert {i for i in range(4) if row[i] == ONE} == kept_pos
+            assert all(row[i] == 0 for i in range(4) if i not in kept_pos)
+
+
+@pytest.mark.parametrize("b", MASK_TILES)
+def test_mask_tiles_global_sparsity_is_half_the_sparse_tile_fraction(b):
+    N, K = TILE, 2 * TILE
+    w = np.full((N, K), ONE, np.uint16)
+    rng = np.random.default_rng(100 + b)
+    tl = rng.standard_normal((N // b, K // b, 2)).astype(np.float32)
+    pl = rng.standard_normal((N, K // 4, 6)).astype(np.float32)
+    wm, bm, _ = oracle.hard_mask_tiles(w, tl, pl, b)
+    pruned = np.count_nonzero(wm == 0)
+    assert pruned * bm.size == N * K * int(bm.sum()) // 2  # pruned/NK == 0.5 * sparse tiles / tiles
+    groups = (wm.reshape(N, K // 4, 4) == ONE).sum(axis=2)
+    sparse_group = np.repeat(np.repeat(bm, b, axis=0), b // 4, axis=1)  # [N][K/4]: is the group's tile sparse
+    assert np.all(groups[sparse_group == 1] == 2) and np.all(groups[sparse_group == 0] == 4)
+
+
+def test_exec_tiles_all_sixteen_combinations_of_four_64_tiles():
+    """A 128 x 128 execution tile holding four 64 x 64 mask tiles is sparse only
+    in the one combination where all four are sparse."""
+    for combo in range(16):
+        bm = np.array([[combo & 1, (combo >> 1) & 1], [(combo >> 2) & 1, (combo >> 3) & 1]], np.uint8)
+        ex, n = oracle.exec_tiles(bm, TILE, TILE, 64)
+        assert ex.tolist() == [[1 if combo == 15 else 0]] and n == (1 if combo == 15 else 0)
+
+
+def test_exec_tiles_single_dense_4x4_tile_anywhere_makes_the_tile_dense():
+    N, K, b = 2 * TILE, 2 * TILE, 4
+    r = TILE // b
+    for (i, j) in [(0, 0), (r - 1, r - 1), (r // 2, 3), (r, r), (2 * r - 1, 0)]:
+        bm = np.ones((N // b, K // b), np.uint8)
+        bm[i, j] = 0
+        ex, n = oracle.exec_tiles(bm, N, K, b)
+        want = np.ones((2, 2), np.uint8)
+        want[i // r, j // r] = 0
+        assert np.array_equal(ex, want) and n == 3
+
+
+def test_exec_tiles_at_128_copy_the_bitmap():
+    bm = np.random.default_rng(7).integers(0, 2, (3, 5)).astype(np.uint8)
+    ex, n = oracle.exec_tiles(bm, 3 * TILE, 5 * TILE, 128)
+    assert np.array_equal(ex, bm) and n == int(bm.sum())
+
+
+@pytest.mark.parametrize("b", [4, 32, 64])
+def test_fine_mask_packs_and_multiplies_as_the_masked_weight(b):
+    """Packing W_masked with the execution bitmap loses nothing: the blobs unpack
+    to W_masked bit for bit (dense execution tiles carry the pruned zeros), and
+    the GEMM on them equals numpy's fp64 matmul of W_masked."""
+    N, K, M = 2 * TILE, 2 * TILE, 3
+    w = si.gen_w(N, K, 7, b)
+    rng = np.random.default_rng(b)
+    # mostly-sparse mask tiles, so that some execution tiles come out sparse
+    tl = np.zeros((N // b, K // b, 2), np.float32)
+    tl[..., 1] = 1.0
+    tl[: N // (2 * b), : K // (2 * b), 1] = rng.choice([1.0, -1.0], (N // (2 * b), K // (2 * b)))
+    pl = rng.standard_normal((N, K // 4, 6)).astype(np.float32)
+    wm, bm, pid = oracle.hard_mask_tiles(w, tl, pl, b)
+    ex, ns = oracle.exec_tiles(bm, N, K, b)
+    assert 1 <= ns < ex.size
+    v, m, d = oracle.pack(wm, ex, pid)
+    assert np.array_equal(oracle.unpack(v, m, d, N, K), wm)
+    x = si.gen_x(M, K, 7, b)
+    y = oracle.gemm(x, oracle.unpack(v, m, d, N, K))
+    assert np.allclose(y, f64(x) @ f64(wm).T, rtol=1e-12, atol=1e-12)
