@@ -407,6 +407,113 @@ def mlp_steps(dev, pk, reps=10):
 # ------------------------------------------------------------ GPU arm
 
 
+def tile_ablation(args):
+    """Mask tile size ablation ("Ablation Studies", tile size: performance holds
+    across learned tile sizes down to 4 x 4, while hardware efficiency needs
+    128 x 128 execution tiles).  For each mask tile b and layout (b x b tiles
+    sparse at seeded random positions, or as one band of tile rows), half of
+    the mask tiles sparse, the product path runs: patch_hard_mask_tiles ->
+    patch_exec_tiles -> patch_pack of W_masked; then patch_gemm is timed at
+    M = 1 (decode) and M = 2048 (prefill) against the same layer packed with
+    an all-dense bitmap.  Weights rotate over copies that exceed L2."""
+    import torch
+
+    import tile_sparse_gemm_b200 as tsg
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    status = tsg.new_status(dev)
+    shapes = [(n, N, K) for n, N, K in si.LLAMA2_7B if n in ("q", "gate")]
+    sizes = [128, 64, 32, 16, 8, 4]
+    l2_bytes = 126e6
+
+    def copies_of(pw):
+        n = max(2, int(np.ceil(3 * l2_bytes / (pw.values.numel() + pw.meta.numel() + pw.desc.numel()))))
+        return [pw] + [tsg.PackedWeight(pw.N, pw.K, pw.n_sparse, pw.values.clone(), pw.meta.clone(),
+                                        pw.desc.clone()) for _ in range(n - 1)]
+
+    def time_us(packs, M, reps):
+        K, N = packs[0].K, packs[0].N
+        x = torch.randn(M, K, device=dev).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(max(tsg.patch_gemm_workspace_size(M, packs[0]), 16), dtype=torch.uint8, device=dev)
+        for i in range(len(packs)):
+            tsg.patch_gemm(x, packs[i], Y=y, workspace=ws, status=status)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for r in range(reps):
+            tsg.patch_gemm(x, packs[r % len(packs)], Y=y, workspace=ws, status=status)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / reps
+
+    def paired(packs, dense_packs, M, reps, rounds=5):
+        """Medians over alternating rounds of (this layer, the all-dense layer)."""
+        a, d = [], []
+        for _ in range(rounds):
+            d.append(time_us(dense_packs, M, reps))
+            a.append(time_us(packs, M, reps))
+        return statistics.median(a), statistics.median(d)
+
+    rows = []
+    warm = torch.empty(2**28, dtype=torch.uint8, device=dev)
+    t_end = time.time() + 1.0
+    while time.time() < t_end:  # bring the clocks up before the first timing
+        warm.add_(1)
+        torch.cuda.synchronize()
+    del warm
+    for idx, (name, N, K) in enumerate(shapes):
+        w_np = si.gen_w(N, K, 2, idx)
+        ids = si.patterns_top2(w_np)
+        pl_np = np.zeros((N, K // 4, 6), np.float32)
+        np.put_along_axis(pl_np, ids[..., None].astype(np.int64), 1.0, axis=2)  # magnitude top-2 as logits
+        w = torch.from_numpy(w_np.view(np.int16)).view(torch.bfloat16).to(dev)
+        pl = torch.from_numpy(pl_np).to(dev)
+        del pl_np
+        dense = tsg.patch_pack(w, torch.zeros((N // 128, K // 128), dtype=torch.uint8, device=dev),
+                               torch.from_numpy(ids).to(dev), 0, status=status)
+        dense_packs = copies_of(dense)
+        dense_bytes = dense.values.numel() + dense.desc.numel()
+        base_all = {"decode": [], "prefill": []}
+        for clustered in (False, True):
+            for b in sizes:
+                kinds = si.mask_tiles(N, K, b, 0.5, clustered, 2, idx)
+                tl = torch.from_numpy(si.choice_logits(kinds)).to(dev)
+                wm, bm, pid = tsg.patch_hard_mask_tiles(w, tl, pl, b, status=status)
+                ex, n_dev = tsg.patch_exec_tiles(bm, N, K, b)
+                pw = tsg.patch_pack(wm, ex, pid, int(n_dev.item()), status=status)
+                packs = copies_of(pw)
+                stored = pw.values.numel() + pw.meta.numel() + pw.desc.numel()
+                t, base = {}, {}
+                for kind, M, reps in (("decode", 1, 300), ("prefill", 2048, 30)):
+                    t[kind], base[kind] = paired(packs, dense_packs, M, reps)
+                    base_all[kind].append(base[kind])
+                rows.append({"shape": f"{name} {N}x{K}", "mask_tile": b,
+                             "layout": "band of tile rows" if clustered else "random",
+                             "sparse_mask_tiles": 0.5,
+                             "sparse_exec_tiles": round(pw.n_sparse / ((N // 128) * (K // 128)), 4),
+                             "stored_vs_dense": round(stored / dense_bytes, 4),
+                             "decode_us": round(t["decode"], 2),
+                             "decode_GBps": round(stored / t["decode"] / 1e3, 1),
+                             "decode_speedup": round(base["decode"] / t["decode"], 3),
+                             "prefill_us": round(t["prefill"], 2),
+                             "prefill_speedup": round(base["prefill"] / t["prefill"], 3)})
+                del packs, pw, wm
+        del dense_packs
+        rows.append({"shape": f"{name} {N}x{K}", "mask_tile": None, "layout": "all dense",
+                     "decode_us": round(statistics.median(base_all["decode"]), 2),
+                     "prefill_us": round(statistics.median(base_all["prefill"]), 2)})
+    code, bits = tsg.patch_read_status(status)
+    if code != 0:
+        raise RuntimeError(f"device status {code} bits {bits}")
+    return {"metric": "mask tile-size ablation: speedup over the all-dense bitmap", "value": None, "unit": "x",
+            "n_gpus": 1, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "LLaMA-2-7B q and gate, mask tiles 128..4, half of them sparse",
+                       "l2": "weights rotate over copies holding 3x L2", "decode_M": 1, "prefill_M": 2048,
+                       "timing": "median of 5 rounds, each timing the all-dense layer then this one"},
+            "rows": rows}
+
+
 def job_times(ms, e2e_ms, world, dev=None):
     """Timed-region and end-to-end times (ms) of the whole job: the maximum over
     ranks, since the job ends when its slowest rank does."""
@@ -697,7 +804,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", choices=["decode", "decode_fused", "prefill"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "decode_fused", "prefill", "tile_ablation"], default="decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed calls eagerly instead of one CUDA graph")
@@ -731,6 +838,11 @@ def main():
                           "cpu_baseline": cb,
                           "e2e": {"value": round(value, 4), "unit": cb["unit"], "h2d_bytes_per_step": 0,
                                   "d2h_bytes_per_step": 0}}))
+        return
+
+    if args.workload == "tile_ablation":  # one GPU, rank 0 only
+        if rank == 0:
+            print(json.dumps(tile_ablation(args)))
         return
 
     if world > 1:

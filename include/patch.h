@@ -195,6 +195,40 @@ PATCH_API patch_status_t patch_soft_mask(const uint16_t *W, int64_t N, int64_t K
                                          void *stream);
 
 /*
+ * patch_hard_mask_tiles: patch_hard_mask with mask tiles of b x b, b =
+ * mask_tile in {4, 8, 16, 32, 64, 128} ("Ablation Studies", tile size: the
+ * learned tile can be as small as 4 x 4; hardware efficiency needs 128 x 128
+ * execution tiles).  Same decisions and outputs as patch_hard_mask except
+ *   tile_logits fp32 [N/b][K/b][2] (8-byte aligned), bitmap u8 [N/b][K/b],
+ *   and W_masked[n][k] keeps W when tile (n/b, k/b) is dense.
+ * mask_tile = 128 is patch_hard_mask.  To run a fine mask, pass its bitmap to
+ * patch_exec_tiles and pack W_MASKED (not W) with the execution bitmap and
+ * pat_id: dense execution tiles then carry the pruned zeros of their sparse
+ * mask tiles, so the packed weight multiplies exactly as W_masked.
+ * Errors: those of patch_hard_mask; PATCH_ERR_INVALID_ARG for another
+ * mask_tile.
+ */
+PATCH_API patch_status_t patch_hard_mask_tiles(const uint16_t *W, int64_t N, int64_t K, int64_t mask_tile,
+                                               const float *tile_logits, const float *pattern_logits,
+                                               uint16_t *W_masked, uint8_t *bitmap, uint8_t *pat_id,
+                                               int32_t *dev_status, void *stream);
+
+/*
+ * patch_exec_tiles: the 128 x 128 execution tiles of a b x b mask (b =
+ * mask_tile, 4..128): exec[tn][tk] = 1 (2:4 sparse execution) only when all
+ * (128/b)^2 mask tiles inside it are sparse, else 0 (dense execution).
+ *   bitmap   u8 [N/b][K/b] (patch_hard_mask_tiles' output);
+ *   exec     u8 [N/128][K/128] out, the bitmap patch_pack takes;
+ *   n_sparse one int64 on the DEVICE out (8-byte aligned): the number of sparse
+ *            execution tiles, for patch_pack_sizes.  It is zeroed on the stream
+ *            and then counted, so it needs no initial value.
+ * Errors: PATCH_ERR_INVALID_ARG (NULL, mask_tile), PATCH_ERR_SHAPE,
+ * PATCH_ERR_ALIGN, PATCH_ERR_DEVICE.
+ */
+PATCH_API patch_status_t patch_exec_tiles(const uint8_t *bitmap, int64_t N, int64_t K, int64_t mask_tile,
+                                          uint8_t *exec, int64_t *n_sparse, void *stream);
+
+/*
  * patch_tile_kinds: the tile half of the hard mask alone ("Learnable
  * Distributions", item 1: a 2-way logit per tile chooses dense or 2:4 sparse).
  *   tile_logits fp32 [Tn][Tk][2] (index 0 = dense, 1 = sparse);

@@ -93,6 +93,33 @@ def tiles_clustered(N: int, K: int, frac: float, config: int = 0, shape_idx: int
     return kinds.reshape(Tn, Tk)
 
 
+def mask_tiles(N: int, K: int, b: int, frac: float, clustered: bool, config: int = 0,
+               shape_idx: int = 0) -> np.ndarray:
+    """Kinds [N/b][K/b] uint8 of b x b mask tiles with exactly floor(frac*T_b + 0.5)
+    sparse: at seeded random positions, or as one contiguous run in row-major
+    tile order starting at a seeded offset (full-width bands of tile rows)."""
+    Tn, Tk = N // b, K // b
+    T = Tn * Tk
+    ns = exact_sparse_count(T, frac)
+    r = rng(config, shape_idx, STREAM_TILES)
+    kinds = np.zeros(T, dtype=np.uint8)
+    if clustered:
+        start = int(r.integers(0, T - ns + 1))
+        kinds[start:start + ns] = 1
+    else:
+        kinds[r.permutation(T)[:ns]] = 1
+    return kinds.reshape(Tn, Tk)
+
+
+def choice_logits(kinds: np.ndarray) -> np.ndarray:
+    """Tile logits [..][..][2] fp32 whose argmax is the given kind: (1, 0) for a
+    dense tile, (0, 1) for a sparse one."""
+    out = np.zeros(kinds.shape + (2,), np.float32)
+    out[..., 0] = (kinds == 0)
+    out[..., 1] = (kinds != 0)
+    return out
+
+
 def patterns_top2(w_bits: np.ndarray) -> np.ndarray:
     """Pattern ids [N][K/4] uint8: keep the two largest |w| of each group of 4 (ties -> lower index)."""
     N, K = w_bits.shape
@@ -107,9 +134,9 @@ def patterns_top2(w_bits: np.ndarray) -> np.ndarray:
     return table[lo, hi]
 
 
-def gen_tile_logits(N: int, K: int, config: int = 0, shape_idx: int = 0) -> np.ndarray:
+def gen_tile_logits(N: int, K: int, config: int = 0, shape_idx: int = 0, tile: int = TILE) -> np.ndarray:
     r = rng(config, shape_idx, STREAM_TILE_LOGITS)
-    return r.standard_normal((N // TILE, K // TILE, 2), dtype=np.float32)
+    return r.standard_normal((N // tile, K // tile, 2), dtype=np.float32)
 
 
 def gen_pattern_logits(N: int, K: int, config: int = 0, shape_idx: int = 0) -> np.ndarray:

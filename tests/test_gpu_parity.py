@@ -504,3 +504,82 @@ def test_decode_workspace_too_small_is_rejected():
     with pytest.raises(tsg.PatchError) as e:
         tsg.patch_gemm(to_dev_bf16(x), pw, workspace=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
     assert e.value.code == 8
+
+
+# ------------------------------------------- mask tiles finer than the execution tile
+
+
+@pytest.mark.parametrize("b", [4, 8, 16, 32, 64, 128])
+def test_hard_mask_tiles_bit_exact(b):
+    N, K = 256, 384  # K/b mask tiles per row: 3 times a power of two (odd at b = 128)
+    w = si.gen_w(N, K, 11, b)
+    tl = si.gen_tile_logits(N, K, 11, b, tile=b)
+    pl = si.gen_pattern_logits(N, K, 11, b)
+    pl[::5, ::7, 2] = pl[::5, ::7, 0]  # ties
+    pl[::13, ::3, 1] = np.nan
+    tl[::3, ::2, 1] = tl[::3, ::2, 0]  # tile ties -> dense
+    wm_ref, bm_ref, id_ref = oracle.hard_mask_tiles(w, tl, pl, b)
+    wm, bm, ids = tsg.patch_hard_mask_tiles(to_dev_bf16(w), to_dev(tl), to_dev(pl), b)
+    assert np.array_equal(bits_of(wm), wm_ref)
+    assert np.array_equal(bm.cpu().numpy(), bm_ref)
+    assert np.array_equal(ids.cpu().numpy(), id_ref)
+    _, bm2, ids2 = tsg.patch_hard_mask_tiles(to_dev_bf16(w), to_dev(tl), to_dev(pl), b, want_masked=False)
+    assert np.array_equal(bm2.cpu().numpy(), bm_ref) and np.array_equal(ids2.cpu().numpy(), id_ref)
+
+
+@pytest.mark.parametrize("b", [4, 16, 64, 128])
+@pytest.mark.parametrize("clustered", [False, True])
+def test_exec_tiles_bit_exact(b, clustered):
+    N, K = 512, 640
+    for frac in (0.5, 0.9, 1.0):
+        kinds = si.mask_tiles(N, K, b, frac, clustered, 12, b)
+        ex_ref, n_ref = oracle.exec_tiles(kinds, N, K, b)
+        ex, n = tsg.patch_exec_tiles(to_dev(kinds), N, K, b)
+        assert np.array_equal(ex.cpu().numpy(), ex_ref), (b, clustered, frac)
+        assert int(n.item()) == n_ref
+
+
+@pytest.mark.parametrize("b", [4, 32, 64])
+@pytest.mark.parametrize("M", [1, 16, 300])
+def test_fine_mask_pipeline_packs_and_multiplies_as_the_masked_weight(b, M):
+    """hard mask (b x b tiles) -> execution tiles -> pack of W_masked -> GEMM on
+    the GPU: blobs bit-exact with the oracle's, Y within tolerance of the oracle
+    GEMM on the oracle's W_masked."""
+    N, K = 384, 512
+    w = si.gen_w(N, K, 13, b)
+    kinds = si.mask_tiles(N, K, b, 0.8, True, 13, b)  # one band of 80% of the tile rows: some execution tiles sparse
+    tl = si.choice_logits(kinds)
+    pl = si.gen_pattern_logits(N, K, 13, b)
+    wm_ref, bm_ref, id_ref = oracle.hard_mask_tiles(w, tl, pl, b)
+    ex_ref, n_ref = oracle.exec_tiles(bm_ref, N, K, b)
+    assert 0 < n_ref < ex_ref.size
+    v_ref, m_ref, d_ref = oracle.pack(wm_ref, ex_ref, id_ref)
+    wm, bm, ids = tsg.patch_hard_mask_tiles(to_dev_bf16(w), to_dev(tl), to_dev(pl), b)
+    ex, n = tsg.patch_exec_tiles(bm, N, K, b)
+    status = tsg.new_status()
+    pw = tsg.patch_pack(wm, ex, ids, int(n.item()), status=status)
+    assert tsg.patch_read_status(status)[0] == 0
+    assert np.array_equal(pw.values.cpu().numpy(), v_ref)
+    assert np.array_equal(pw.meta.cpu().numpy(), m_ref)
+    assert np.array_equal(pw.desc.cpu().numpy(), d_ref)
+    x = si.gen_x(M, K, 13, b)
+    check_gemm(gemm_on_gpu(x, pw), oracle.gemm(x, wm_ref), f"mask tile {b}, M={M}")
+
+
+def test_mask_tile_arguments_are_checked():
+    import ctypes
+    N = K = 256
+    dev = torch.device("cuda")
+    w = torch.zeros((N, K), dtype=torch.bfloat16, device=dev)
+    pl = torch.zeros((N, K // 4, 6), dtype=torch.float32, device=dev)
+    tl = torch.zeros((N // 4, K // 4, 2), dtype=torch.float32, device=dev)
+    for bad in (0, 2, 3, 48, 256):
+        with pytest.raises(tsg.PatchError) as e:
+            tsg.patch_hard_mask_tiles(w, tl, pl, bad)
+        assert e.value.code == 1  # PATCH_ERR_INVALID_ARG, before any launch
+        with pytest.raises(tsg.PatchError) as e:
+            tsg.patch_exec_tiles(torch.zeros((N // 4, K // 4), dtype=torch.uint8, device=dev), N, K, bad)
+        assert e.value.code == 1
+    rc = tsg.lib().patch_exec_tiles(ctypes.c_void_p(tl.data_ptr()), N, K, 4, ctypes.c_void_p(tl.data_ptr()),
+                                    ctypes.c_void_p(tl.data_ptr() + 4), None)
+    assert rc == 3  # PATCH_ERR_ALIGN: n_sparse not 8-byte aligned

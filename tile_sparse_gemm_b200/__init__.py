@@ -29,6 +29,7 @@ _LIB_PATH = Path(__file__).resolve().parent / "libpatch.so"
 TILE = 128
 PANEL_BYTES = 16384
 DECODE_MAX_M = 16
+MASK_TILES = (4, 8, 16, 32, 64, 128)  # mask tile sizes patch_hard_mask_tiles takes
 
 PATCH_OK = 0
 STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_INVALID_ARG", 2: "PATCH_ERR_SHAPE", 3: "PATCH_ERR_ALIGN",
@@ -66,6 +67,8 @@ def lib() -> ctypes.CDLL:
             "patch_hard_mask": [P, I64, I64, P, P, P, P, P, P, P],
             "patch_pack": [P, I64, I64, P, P, I64, P, P, P, P, P],
             "patch_tile_kinds": [P, I64, I64, P, P, P],
+            "patch_hard_mask_tiles": [P, I64, I64, I64, P, P, P, P, P, P, P],
+            "patch_exec_tiles": [P, I64, I64, I64, P, P, P],
             "patch_soft_mask": [P, I64, I64, P, P, P, P, ctypes.c_float, P, P, P],
             "patch_shard_rows": [P, I64, I64, I64, P],
             "patch_pack_from_logits": [P, I64, I64, P, P, I64, P, P, P, P, P],
@@ -161,6 +164,39 @@ def patch_hard_mask(W: torch.Tensor | None, tile_logits: torch.Tensor, pattern_l
                                  _dev(bitmap, "bitmap"), _dev(pid, "pat_id"), _dev(status, "status"),
                                  _stream(stream)), "patch_hard_mask")
     return wm, bitmap, pid
+
+
+def patch_hard_mask_tiles(W: torch.Tensor | None, tile_logits: torch.Tensor, pattern_logits: torch.Tensor,
+                          mask_tile: int, status: torch.Tensor | None = None, want_masked: bool = True,
+                          stream=None):
+    """Argmax hard mask with b x b mask tiles (b = mask_tile, 4..128): tile_logits
+    fp32 [N/b][K/b][2].  Returns (W_masked or None, bitmap u8 [N/b][K/b], pat_id u8 [N][K/4])."""
+    N, K4, _ = pattern_logits.shape
+    K = 4 * K4
+    b = int(mask_tile)
+    dev = pattern_logits.device
+    status = new_status(dev) if status is None else status
+    wm = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if want_masked else None
+    shape = (N // b, K // b) if b in MASK_TILES else (1,)  # the library rejects other sizes
+    bitmap = torch.empty(shape, dtype=torch.uint8, device=dev)
+    pid = torch.empty((N, K // 4), dtype=torch.uint8, device=dev)
+    _check(lib().patch_hard_mask_tiles(_dev(W, "W"), N, K, b, _dev(tile_logits, "tile_logits"),
+                                       _dev(pattern_logits, "pattern_logits"), _dev(wm, "W_masked"),
+                                       _dev(bitmap, "bitmap"), _dev(pid, "pat_id"), _dev(status, "status"),
+                                       _stream(stream)), "patch_hard_mask_tiles")
+    return wm, bitmap, pid
+
+
+def patch_exec_tiles(bitmap: torch.Tensor, N: int, K: int, mask_tile: int,
+                     stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """128 x 128 execution tiles of a b x b mask bitmap (sparse only where every
+    mask tile inside is sparse): (exec u8 [N/128][K/128], n_sparse int64 [1]), on the device."""
+    dev = bitmap.device
+    ex = torch.empty((N // TILE, K // TILE), dtype=torch.uint8, device=dev)
+    n_sparse = torch.empty(1, dtype=torch.int64, device=dev)
+    _check(lib().patch_exec_tiles(_dev(bitmap, "bitmap"), N, K, int(mask_tile), _dev(ex, "exec"),
+                                  _dev(n_sparse, "n_sparse"), _stream(stream)), "patch_exec_tiles")
+    return ex, n_sparse
 
 
 def patch_pack(W: torch.Tensor, bitmap: torch.Tensor, pat_id: torch.Tensor, n_sparse: int | None = None,

@@ -89,6 +89,42 @@ patch_status_t patch_hard_mask(const uint16_t* W, int64_t N, int64_t K, const fl
   return PATCH_OK;
 }
 
+static bool mask_tile_ok(int64_t b) { return b == 4 || b == 8 || b == 16 || b == 32 || b == 64 || b == 128; }
+
+patch_status_t patch_hard_mask_tiles(const uint16_t* W, int64_t N, int64_t K, int64_t mask_tile,
+                                     const float* tile_logits, const float* pattern_logits, uint16_t* W_masked,
+                                     uint8_t* bitmap, uint8_t* pat_id, int32_t* dev_status, void* stream) {
+  if (!tile_logits || !pattern_logits || !bitmap || !pat_id || !dev_status) return PATCH_ERR_INVALID_ARG;
+  if (W_masked && !W) return PATCH_ERR_INVALID_ARG;
+  if (!mask_tile_ok(mask_tile)) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return PATCH_ERR_SHAPE;
+  if ((W && !aligned16(W)) || (W_masked && !aligned16(W_masked)) || !aligned16(pattern_logits) ||
+      !aligned16(pat_id) || reinterpret_cast<uintptr_t>(tile_logits) % 8)
+    return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_hard_mask_tiles(W, N, K, mask_tile, tile_logits, pattern_logits, W_masked, bitmap, pat_id, sms,
+                             static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
+patch_status_t patch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, uint8_t* exec,
+                                int64_t* n_sparse, void* stream) {
+  if (!bitmap || !exec || !n_sparse) return PATCH_ERR_INVALID_ARG;
+  if (!mask_tile_ok(mask_tile)) return PATCH_ERR_INVALID_ARG;
+  if (!shape_ok(N, K)) return PATCH_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(n_sparse) % 8) return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_exec_tiles(bitmap, N, K, mask_tile, exec, n_sparse, sms, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
 patch_status_t patch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap,
                           const uint8_t* pat_id, int64_t n_sparse, void* values, void* meta,
                           patch_tile_desc* desc, int32_t* dev_status, void* stream) {

@@ -48,6 +48,14 @@ cudaError_t launch_prefill_mlp(const uint16_t* X, int64_t M, const patch_weight&
 cudaError_t launch_silu_mul(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t count, int num_sms,
                             cudaStream_t stream);
 
+// Hard mask with b x b mask tiles (b = 4..128; 128 is launch_hard_mask).
+cudaError_t launch_hard_mask_tiles(const uint16_t* W, int64_t N, int64_t K, int64_t mask_tile,
+                                   const float* tile_logits, const float* pattern_logits, uint16_t* W_masked,
+                                   uint8_t* bitmap, uint8_t* pat_id, int num_sms, cudaStream_t stream);
+// 128 x 128 execution tiles of a b x b mask bitmap, and their sparse count (device int64).
+cudaError_t launch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, uint8_t* exec,
+                              int64_t* n_sparse, int num_sms, cudaStream_t stream);
+
 // Tensor-core decode (stream-K over panels, M <= 16).
 size_t decode_tc_workspace_bytes(int64_t M, const patch_weight& W, int num_sms);
 cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
