@@ -485,7 +485,7 @@ def tile_ablation(args):
                 packs = copies_of(pw)
                 stored = pw.values.numel() + pw.meta.numel() + pw.desc.numel()
                 t, base = {}, {}
-                for kind, M, reps in (("decode", 1, 300), ("prefill", 2048, 30)):
+                for kind, M, reps in (("decode", 1, 2000), ("prefill", 2048, 200)):
                     t[kind], base[kind] = paired(packs, dense_packs, M, reps)
                     base_all[kind].append(base[kind])
                 rows.append({"shape": f"{name} {N}x{K}", "mask_tile": b,

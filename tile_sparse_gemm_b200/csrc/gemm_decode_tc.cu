@@ -149,6 +149,53 @@ __device__ void find_tiles(const patch_tile_desc* desc, int T, int64_t P, int64_
   tb = lo_b;
 }
 
+// One-round form of the CTA's set-up: every thread loads one descriptor of a
+// window of blockDim.x tiles starting one tile row before the proportional
+// estimate of the CTA's first tile.  When the window holds the CTA's tiles and
+// the first tile of every tile row the epilogue needs (the rows holding the
+// CTA's first and last tile, and the rows after them), the tile range, the
+// staged descriptors and the row boundaries all come from those registers: one
+// global round trip instead of the three of find_tiles, the staging loop and
+// the boundary loads.  That is the usual case (even sparse tiles, Tk up to
+// about 100); otherwise it writes nothing and returns false (block-uniform).
+__device__ bool locate_one_round(Shared& s, const Args& a, int64_t pa, int64_t pb) {
+  const int n = blockDim.x, i = threadIdx.x;
+  const int T = a.Tn * a.Tk;
+  int64_t w64 = pa * T / a.P - a.Tk;
+  if (w64 > T - n) w64 = T - n;
+  if (w64 < 0) w64 = 0;
+  const int w = int(w64), t = w + i;
+  const bool in = t < T;
+  patch_tile_desc d = {};
+  if (in) d = a.desc[t];
+  const int64_t pm = in ? panel_of(d) : 0;
+  const int ca = __syncthreads_count(in && pm <= pa);
+  const int cb = __syncthreads_count(in && pm <= pb);
+  const int nv = T - w < n ? T - w : n;  // window entries inside the table
+  if (ca < 1 || cb < 1 || ((ca == nv || cb == nv) && w + nv != T)) return false;
+  const int ta = w + ca - 1, tb = w + cb - 1;
+  const int row_first = ta / a.Tk * a.Tk, row_after = (tb / a.Tk + 1) * a.Tk;
+  if (row_first < w || (row_after < T && row_after >= w + nv) || tb - ta + 1 > DCAP) return false;
+  if (in && t >= ta && t <= tb) s.dcache[t - ta] = d;
+  // first panel of: the first row, the row after it, the last row, the row after that (P past the end)
+  const int want[4] = {row_first, row_first + a.Tk, tb / a.Tk * a.Tk, row_after};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    int64_t* dst = k < 2 ? &s.row_lo[k] : &s.row_hi[k - 2];
+    if (want[k] >= T) {
+      if (i == 0) *dst = a.P;
+    } else if (in && t == want[k]) {
+      *dst = pm;
+    }
+  }
+  if (i == 0) {
+    s.t_first = ta;
+    s.t_last = tb;
+    s.cached = 1;
+  }
+  return true;
+}
+
 // Descriptor of tile t (staged in shared memory when the CTA's tiles fit).
 __device__ __forceinline__ patch_tile_desc tile_desc(const Shared& s, const Args& a, int t) {
   return s.cached ? s.dcache[t - s.t_first] : a.desc[t];
@@ -436,26 +483,28 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     prefetch_tensormap(&tmap_x);
   }
-  // locate the CTA's first and last tile, then stage their descriptors
-  // (G <= P, so every CTA has at least one panel)
-  int ta, tb;
-  find_tiles(a.desc, a.Tn * a.Tk, a.P, p0, p1 - 1, ta, tb);
-  const int count = tb - ta + 1;
-  if (threadIdx.x == 0) {
-    s.t_first = ta;
-    s.t_last = tb;
-    s.cached = count <= DCAP;
-  }
-  if (count <= DCAP)
-    for (int i = threadIdx.x; i < count; i += blockDim.x) s.dcache[i] = a.desc[ta + i];
+  // locate the CTA's first and last tile, stage their descriptors and the
   // tile-row boundaries the epilogue needs for rows cut by this CTA's range
-  if (threadIdx.x < 4) {
-    const int tn = (threadIdx.x < 2 ? ta : tb) / a.Tk + (threadIdx.x & 1);
-    const int64_t v = tn < a.Tn ? panel_of(a.desc[int64_t(tn) * a.Tk]) : a.P;
-    if (threadIdx.x < 2)
-      s.row_lo[threadIdx.x] = v;
-    else
-      s.row_hi[threadIdx.x - 2] = v;
+  // (G <= P, so every CTA has at least one panel)
+  if (!locate_one_round(s, a, p0, p1 - 1)) {
+    int ta, tb;
+    find_tiles(a.desc, a.Tn * a.Tk, a.P, p0, p1 - 1, ta, tb);
+    const int count = tb - ta + 1;
+    if (threadIdx.x == 0) {
+      s.t_first = ta;
+      s.t_last = tb;
+      s.cached = count <= DCAP;
+    }
+    if (count <= DCAP)
+      for (int i = threadIdx.x; i < count; i += blockDim.x) s.dcache[i] = a.desc[ta + i];
+    if (threadIdx.x < 4) {
+      const int tn = (threadIdx.x < 2 ? ta : tb) / a.Tk + (threadIdx.x & 1);
+      const int64_t v = tn < a.Tn ? panel_of(a.desc[int64_t(tn) * a.Tk]) : a.P;
+      if (threadIdx.x < 2)
+        s.row_lo[threadIdx.x] = v;
+      else
+        s.row_hi[threadIdx.x - 2] = v;
+    }
   }
   if (warp == 1) tmem_alloc(&s.tmem_base, TMEM_COLS);
   tc_fence_before();

@@ -12,7 +12,8 @@
 // computes Y^T = W_eff * X^T: the MMA's M = 128 rows of W (one tile row), its
 // N = BT tokens, K streams over the tiles of the row.
 //
-// Work unit = two tile rows (2 x 128 output features) x BT tokens.  Both rows
+// Work unit = two tile rows (2 x 128 output features, rows rp and rp + Tn/2)
+// x BT tokens.  Both rows
 // multiply the same X panels, so one 30 KiB X panel in shared memory feeds
 // two MMA chains; each row keeps its own kind per K-tile (dense or sparse),
 // so the two rows of a unit never need to agree.  Per byte brought in from L2
@@ -107,12 +108,18 @@ struct Args {
   int inject;  // 1: row 0's producer stops after the first K-tile (exercises the timeout path)
 };
 
-// tile rows in unit row pair rp (the last pair of an odd Tn has one; a gated-MLP unit always has both)
+// Row pair rp holds tile rows rp and rp + n_pairs (n_pairs = ceil(Tn / 2);
+// the last pair of an odd Tn has one row).  A unit costs the sum of its two
+// rows' MMA time, so pairing each row with the one half the layer away keeps
+// unit costs even when sparse tiles come in bands of tile rows (a band of half
+// the rows puts exactly one row of every pair inside it), where neighbouring
+// rows would pair dense with dense and sparse with sparse and a one-wave grid
+// would wait for the dense pairs.  A gated-MLP unit is gate and up tile row rp.
 __device__ __forceinline__ int rows_of(const Args& p, int rp) {
-  return p.mlp ? ROWS : (p.Tn - ROWS * rp < ROWS ? p.Tn - ROWS * rp : ROWS);
+  return p.mlp ? ROWS : (rp + p.n_pairs < p.Tn ? ROWS : 1);
 }
 // the tile row of its weight that row r of unit row pair rp reads
-__device__ __forceinline__ int tile_row(const Args& p, int rp, int r) { return p.mlp ? rp : ROWS * rp + r; }
+__device__ __forceinline__ int tile_row(const Args& p, int rp, int r) { return p.mlp ? rp : rp + r * p.n_pairs; }
 
 // Units run row pair by row pair (all token blocks of a pair are consecutive
 // items), so the CTAs of one wave read a few row pairs' W, which stays in L2
@@ -320,7 +327,7 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, co
     if (!named_bar_and(bar_id, 128, ok)) break;
     tc_fence_after();
     if (p.mlp || g < rows_of(p, rp)) {
-      const int n0 = (p.mlp ? rp : ROWS * rp + g) * BM, m0 = tb * p.bt;
+      const int n0 = tile_row(p, rp, g) * BM, m0 = tb * p.bt;
       const int valid = p.M - m0 < p.bt ? p.M - m0 : p.bt;  // tokens of this unit inside X
       const uint32_t lanes = tmem + (uint32_t(32 * q) << 16);
       const int c0 = p.mlp ? g : 0, dc = p.mlp ? 2 : 1;
