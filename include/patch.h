@@ -96,8 +96,8 @@ typedef enum {
 #define PATCH_DEV_COUNT 0x4
 
 /* Path selector of patch_gemm_ex. */
-#define PATCH_PATH_AUTO 0    /* M <= PATCH_DECODE_MAX_M: decode, else prefill */
-#define PATCH_PATH_DECODE 1  /* stream-K weight streaming kernel (TMA + tcgen05, N = 16), M in 1..16 */
+#define PATCH_PATH_AUTO 0    /* M <= PATCH_DECODE_MAX_M: decode (CUDA-core when N > 524288), else prefill */
+#define PATCH_PATH_DECODE 1  /* stream-K weight streaming kernel (TMA + tcgen05, N = 16), M in 1..16, N <= 524288 */
 #define PATCH_PATH_PREFILL 2 /* TMA + tcgen05 (dense and 2:4 sparse MMA), any M >= 1 */
 #define PATCH_PATH_DECODE_SIMT 3 /* split-K GEMV on CUDA cores (16-byte loads, fp32 FMA), M in 1..16 */
 /* Test hook, OR-ed into PATCH_PATH_PREFILL: the prefill producer stops after
@@ -276,10 +276,12 @@ PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight
  *   W  packed weight (host struct)
  *   Y  bf16 [M][N] (16-byte aligned)
  *   workspace: patch_gemm_workspace_size bytes (may be NULL when that is 0).
- *     It must be zero-filled before its first use; every successful call
- *     leaves it zero-filled again (the decode path keeps per-row arrival
- *     counters there), so one zero-fill at allocation suffices.  After a call
- *     that reported an error, zero it again.
+ *     Its first 64 KiB hold the decode path's per-row arrival counters: they
+ *     must be zero before the first use, and every successful call leaves
+ *     them zero; the rest is scratch (fp32 partial sums) whose contents do not
+ *     matter.  So one zero-fill at allocation suffices, and one workspace of
+ *     the largest size serves every layer, token count and path, in any
+ *     order.  After a call that reported an error, zero it again.
  * M <= 16 runs the decode path: 1.5 CTAs per SM each stream an equal share
  * of the stored panels through a TMA ring (stream-K), the tensor cores reduce
  * them (N = 16 tokens, zero-padded); a tile row cut between CTAs is finished
@@ -356,7 +358,8 @@ PATCH_API patch_status_t patch_gemm_decode_noalloc(const uint16_t *X, int64_t M,
  * M <= 16: two decode GEMMs write G and U (bf16) into the workspace, then one
  * elementwise launch forms H.
  * workspace: patch_gemm_mlp_workspace_size bytes, zero-filled before its first
- * use and left so by every successful call (as for patch_gemm).
+ * use: a patch_gemm workspace (whose counter region every successful call
+ * leaves zero) followed by G and U.
  * Errors as patch_gemm; PATCH_ERR_SHAPE also when the two weights differ in shape.
  */
 PATCH_API patch_status_t patch_gemm_mlp_workspace_size(int64_t M, const patch_weight *W_gate, const patch_weight *W_up,

@@ -63,6 +63,9 @@ def test_host_checks_reject_before_any_launch(lib):
     assert lib.patch_gemm_ex(fake, 4, ctypes.byref(w), fake, None, 0, fake, None, 7, 0) == 1
     assert lib.patch_gemm_ex(fake, 17, ctypes.byref(w), fake, None, 0, fake, None, 1, 0) == 1
     assert lib.patch_gemm_ex(fake, -1, ctypes.byref(w), fake, None, 0, fake, None, 0, 0) == 1
+    # the tensor-core decode path holds arrival counters for at most 4096 tile rows (N <= 524288)
+    wide = tsg._Weight(128 * 4097, 128, 0, 0x10000, None, 0x10000)
+    assert lib.patch_gemm_ex(fake, 4, ctypes.byref(wide), fake, None, 0, fake, None, 1, 0) == 2
     # the stall test hook is refused outside the prefill path
     assert lib.patch_gemm_ex(fake, 4, ctypes.byref(w), fake, None, 0, fake, None, 0x101, 0) == 1
     # M == 0 is a no-op that needs no device

@@ -488,6 +488,46 @@ def test_decode_workspace_reused_across_calls():
         check_gemm(bits_of(y), ref[: 16 - it], f"call {it}")
 
 
+def test_one_workspace_serves_layers_paths_and_token_counts_in_any_order():
+    """One zero-filled workspace of the largest size, shared by layers whose
+    grids differ (a layer with fewer panels than CTAs, clustered and even
+    ones), both decode paths, the gated MLP and every token count, in an
+    interleaved order.  The tensor-core kernel's arrival counters live in a
+    fixed region at the start that every call leaves zero; scratch written by
+    one call (partial sums of another layout, the other path's split-K
+    partials, the MLP's G and U) never lands there."""
+    specs = [(128, 896, 0.5, "clustered"), (4864, 896, 0.5, "clustered"), (384, 640, 0.5, "exact")]
+    layers = []
+    for i, (N, K, frac, kind) in enumerate(specs):
+        x, w, bm, ids = _layer(N, K, 16, kind, frac, cfg=14, shape_idx=i)
+        layers.append((x, w, bm, ids, pack_on_gpu(w, bm, ids)))
+    gate, up = layers[1][4], _layer(4864, 896, 16, "exact", 0.5, cfg=14, shape_idx=7)
+    up_pw = pack_on_gpu(up[1], up[2], up[3])
+    import ctypes
+    b = ctypes.c_size_t()
+    sg, su = gate.struct(), up_pw.struct()
+    assert tsg.lib().patch_gemm_mlp_workspace_size(16, ctypes.byref(sg), ctypes.byref(su), ctypes.byref(b)) == 0
+    need = max([b.value] + [tsg.patch_gemm_workspace_size(M, L[4]) for L in layers for M in (1, 7, 16)])
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    order = [(0, 16, tsg.PATH_AUTO), (1, 1, tsg.PATH_DECODE_SIMT), (2, 7, tsg.PATH_AUTO), ("mlp", 16, None),
+             (0, 1, tsg.PATH_AUTO), (1, 16, tsg.PATH_AUTO), (2, 16, tsg.PATH_DECODE_SIMT), (1, 7, tsg.PATH_AUTO),
+             (0, 7, tsg.PATH_DECODE_SIMT), (2, 1, tsg.PATH_AUTO)]
+    for li, M, path in order:
+        status = tsg.new_status()
+        if li == "mlp":
+            x = layers[1][0][:M]
+            h = tsg.patch_gemm_mlp(to_dev_bf16(x), gate, up_pw, workspace=ws, status=status)
+            assert tsg.patch_read_status(status)[0] == 0
+            ref = oracle.hybrid_mlp(x, (layers[1][1], layers[1][2], layers[1][3]), up[1:4])
+            check_gemm(bits_of(h), ref, "gated MLP on the shared workspace")
+        else:
+            x, w, bm, ids, pw = layers[li]
+            y = tsg.patch_gemm_ex(to_dev_bf16(x[:M]), pw, workspace=ws, status=status, path=path)
+            assert tsg.patch_read_status(status)[0] == 0
+            check_gemm(bits_of(y), oracle.hybrid_gemm(x[:M], w, bm, ids), f"layer {li} M={M} path {path}")
+        assert int(torch.count_nonzero(ws[:65536]).item()) == 0, f"counter region not left zero after {li} M={M}"
+
+
 def test_gemm_zero_tokens_is_noop():
     x, w, bm, ids = _layer(256, 256, 4, "exact", 0.5)
     pw = pack_on_gpu(w, bm, ids)

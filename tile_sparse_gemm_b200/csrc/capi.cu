@@ -207,8 +207,9 @@ patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight* W, size_
   int sms = 0;
   patch_status_t st = device_sms(&sms);
   if (st != PATCH_OK) return st;
-  // enough for either decode kernel
-  const size_t tc = decode_tc_workspace_bytes(M, *W, sms), simt = decode_plan(M, W->N, W->K, sms).ws_bytes;
+  // enough for either decode kernel: the counter region, then its scratch
+  const size_t tc = W->N / kTile <= kDecodeMaxTileRows ? decode_tc_workspace_bytes(M, *W, sms) : 0;
+  const size_t simt = kDecodeCounterBytes + decode_plan(M, W->N, W->K, sms).ws_bytes;
   *bytes = tc > simt ? tc : simt;
   return PATCH_OK;
 }
@@ -222,10 +223,13 @@ patch_status_t patch_gemm_ex(const uint16_t* X, int64_t M, const patch_weight* W
   if (inject && path != PATCH_PATH_PREFILL) return PATCH_ERR_INVALID_ARG;
   patch_status_t st = check_weight(W);
   if (st != PATCH_OK) return st;
-  if (path == PATCH_PATH_AUTO) path = M <= PATCH_DECODE_MAX_M ? PATCH_PATH_DECODE : PATCH_PATH_PREFILL;
+  if (path == PATCH_PATH_AUTO)  // tensor-core decode up to kDecodeMaxTileRows tile rows, CUDA-core beyond
+    path = M > PATCH_DECODE_MAX_M ? PATCH_PATH_PREFILL
+                                  : (W->N / kTile <= kDecodeMaxTileRows ? PATCH_PATH_DECODE : PATCH_PATH_DECODE_SIMT);
   if (path != PATCH_PATH_DECODE && path != PATCH_PATH_PREFILL && path != PATCH_PATH_DECODE_SIMT)
     return PATCH_ERR_INVALID_ARG;
   if (path != PATCH_PATH_PREFILL && M > PATCH_DECODE_MAX_M) return PATCH_ERR_INVALID_ARG;
+  if (path == PATCH_PATH_DECODE && W->N / kTile > kDecodeMaxTileRows) return PATCH_ERR_SHAPE;
   if (M == 0) return PATCH_OK;
   if (!X || !Y) return PATCH_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Y)) return PATCH_ERR_ALIGN;
@@ -242,9 +246,12 @@ patch_status_t patch_gemm_ex(const uint16_t* X, int64_t M, const patch_weight* W
     e = launch_decode_tc(X, M, *W, Y, workspace, dev_status, sms, limit_ns, s);
   } else if (path == PATCH_PATH_DECODE_SIMT) {
     const DecodePlan p = decode_plan(M, W->N, W->K, sms);
-    if (p.ws_bytes > 0 && (!workspace || workspace_bytes < p.ws_bytes || !aligned16(workspace)))
+    if (p.ws_bytes > 0 &&
+        (!workspace || workspace_bytes < kDecodeCounterBytes + p.ws_bytes || !aligned16(workspace)))
       return PATCH_ERR_WORKSPACE;
-    e = launch_decode(X, M, *W, Y, workspace, sms, s);
+    // its scratch follows the tensor-core kernel's counter region, which it leaves untouched
+    void* scratch = p.ws_bytes > 0 ? static_cast<uint8_t*>(workspace) + kDecodeCounterBytes : nullptr;
+    e = launch_decode(X, M, *W, Y, scratch, sms, s);
   } else {
     e = launch_prefill(X, M, *W, Y, dev_status, sms, limit_ns, inject, s);
   }

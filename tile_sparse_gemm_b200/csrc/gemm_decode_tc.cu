@@ -87,7 +87,7 @@ struct Args {
   const patch_tile_desc* desc;
   const uint8_t* meta;
   uint16_t* Y;
-  float* ws;           // [G][2][128][16] fp32 partials
+  float* ws;           // [G][2][128][16] fp32 partials (contents between calls do not matter)
   uint32_t* counters;  // [Tn][4] arrivals per tile row and TMEM lane quarter (zero between calls)
   int M, N, Tk, Tn;
   int64_t P;  // panels in the values blob
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 
 struct Plan {
   int64_t Tn, Tk, P, G;
-  size_t ws_floats_bytes, counter_bytes;
+  size_t ws_floats_bytes;
 };
 
 static Plan plan(const patch_weight& W, int num_sms) {
@@ -550,7 +550,6 @@ static Plan plan(const patch_weight& W, int num_sms) {
   const int64_t g = int64_t(num_sms) * 3 / 2;
   p.G = p.P < g ? p.P : g;
   p.ws_floats_bytes = size_t(p.G) * WS_FLOATS_PER_CTA * sizeof(float);
-  p.counter_bytes = (size_t(p.Tn) * 4 * sizeof(uint32_t) + 255) & ~size_t(255);
   return p;
 }
 
@@ -559,13 +558,14 @@ static Plan plan(const patch_weight& W, int num_sms) {
 size_t decode_tc_workspace_bytes(int64_t M, const patch_weight& W, int num_sms) {
   (void)M;
   const decode_tc::Plan p = decode_tc::plan(W, num_sms);
-  return p.ws_floats_bytes + p.counter_bytes;
+  return kDecodeCounterBytes + p.ws_floats_bytes;
 }
 
 cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
                              int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream) {
   using namespace decode_tc;
   const Plan pl = plan(W, num_sms);
+  if (pl.Tn > kDecodeMaxTileRows) return cudaErrorInvalidValue;
   CUtensorMap tmap_x, tmap_w;
   // X boxes carry exactly the M token rows: the MMA still reads 16 rows (N = 16),
   // but accumulator columns >= M are never stored, so rows >= M may hold anything
@@ -576,8 +576,8 @@ cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W
   a.desc = W.desc;
   a.meta = static_cast<const uint8_t*>(W.meta);
   a.Y = Y;
-  a.ws = static_cast<float*>(workspace);
-  a.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.ws_floats_bytes);
+  a.counters = static_cast<uint32_t*>(workspace);
+  a.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kDecodeCounterBytes);
   a.M = int(M);
   a.N = int(W.N);
   a.Tk = int(pl.Tk);

@@ -56,7 +56,16 @@ cudaError_t launch_hard_mask_tiles(const uint16_t* W, int64_t N, int64_t K, int6
 cudaError_t launch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, uint8_t* exec,
                               int64_t* n_sparse, int num_sms, cudaStream_t stream);
 
-// Tensor-core decode (stream-K over panels, M <= 16).
+// Workspace layout of the decode paths (patch_gemm_workspace_size covers
+// both): the tensor-core kernel's arrival counters (one u32 per tile-row
+// quarter) sit in a fixed region at the start, which every call leaves zero,
+// and each path's scratch (fp32 partial sums) follows it.  Since no call puts
+// anything else in that region, one workspace serves every layer, token count
+// and decode path in any order.
+constexpr size_t kDecodeCounterBytes = 65536;
+constexpr int64_t kDecodeMaxTileRows = int64_t(kDecodeCounterBytes / 16);  // tensor-core decode: N <= 524288
+
+// Tensor-core decode (stream-K over panels, M <= 16, N / 128 <= kDecodeMaxTileRows).
 size_t decode_tc_workspace_bytes(int64_t M, const patch_weight& W, int num_sms);
 cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
                              int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream);
