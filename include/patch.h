@@ -236,7 +236,8 @@ PATCH_API patch_status_t patch_exec_tiles(const uint8_t *bitmap, int64_t N, int6
  *               the same decision patch_hard_mask takes;
  *   n_sparse    one int64 on the DEVICE out: the number of sparse tiles (the
  *               caller reads it to size the packed blobs with patch_pack_sizes).
- * One launch, no other memory touched.  Errors: PATCH_ERR_INVALID_ARG (NULL),
+ * The count is zeroed on the stream, then one launch fills both; no other
+ * memory is touched.  Errors: PATCH_ERR_INVALID_ARG (NULL),
  * PATCH_ERR_SHAPE, PATCH_ERR_ALIGN (tile_logits or n_sparse not 8-byte aligned),
  * PATCH_ERR_DEVICE.
  */

@@ -177,30 +177,36 @@ cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* 
   return cudaGetLastError();
 }
 
-// Tile kinds from the tile logits (argmax of 2, ties -> dense) and their count.
-__global__ void __launch_bounds__(kScanThreads) tile_kinds_kernel(const float2* __restrict__ tile_logits, int64_t T,
-                                                                  uint8_t* __restrict__ bitmap,
-                                                                  int64_t* __restrict__ n_sparse) {
-  __shared__ int64_t total;
-  if (threadIdx.x == 0) total = 0;
+// Tile kinds from the tile logits (argmax of 2, ties -> dense) and their count:
+// one thread per tile over a grid of 256-thread blocks, the count summed per
+// warp (shuffle), per block (shared memory) and then once per block into the
+// device count, which is zeroed on the stream before the launch.
+__global__ void __launch_bounds__(256) tile_kinds_kernel(const float2* __restrict__ tile_logits, int64_t T,
+                                                         uint8_t* __restrict__ bitmap,
+                                                         unsigned long long* __restrict__ n_sparse) {
+  __shared__ unsigned int block_total;
+  if (threadIdx.x == 0) block_total = 0;
   __syncthreads();
-  int64_t mine = 0;
-  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
-    const float2 l = tile_logits[t];
-    const uint8_t sparse = l.y > l.x ? 1 : 0;
-    bitmap[t] = sparse;
-    mine += sparse;
+  const int64_t t = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  unsigned int sparse = 0;
+  if (t < T) {
+    const float2 l = __ldg(tile_logits + t);
+    sparse = l.y > l.x ? 1u : 0u;
+    bitmap[t] = uint8_t(sparse);
   }
-  atomicAdd(reinterpret_cast<unsigned long long*>(&total), static_cast<unsigned long long>(mine));
+  const unsigned int warp_total = __reduce_add_sync(0xFFFFFFFFu, sparse);
+  if ((threadIdx.x & 31) == 0) atomicAdd(&block_total, warp_total);
   __syncthreads();
-  if (threadIdx.x == 0) *n_sparse = total;
+  if (threadIdx.x == 0 && block_total) atomicAdd(n_sparse, static_cast<unsigned long long>(block_total));
 }
 
 cudaError_t launch_tile_kinds(const float* tile_logits, int64_t N, int64_t K, uint8_t* bitmap, int64_t* n_sparse,
                               cudaStream_t stream) {
   const int64_t T = (N / kTile) * (K / kTile);
-  tile_kinds_kernel<<<1, kScanThreads, 0, stream>>>(reinterpret_cast<const float2*>(tile_logits), T, bitmap,
-                                                    n_sparse);
+  cudaError_t e = cudaMemsetAsync(n_sparse, 0, sizeof(int64_t), stream);
+  if (e != cudaSuccess) return e;
+  tile_kinds_kernel<<<int((T + 255) / 256), 256, 0, stream>>>(reinterpret_cast<const float2*>(tile_logits), T,
+                                                              bitmap, reinterpret_cast<unsigned long long*>(n_sparse));
   return cudaGetLastError();
 }
 
