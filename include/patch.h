@@ -264,8 +264,9 @@ PATCH_API patch_status_t patch_pack_from_logits(const uint16_t *W, int64_t N, in
 
 /*
  * patch_gemm_workspace_size: device scratch bytes patch_gemm needs for M rows
- * of X and this weight (0 when none is needed; for M <= 16 enough for either
- * decode kernel).  Host only, but queries the current device's SM count.
+ * of X and this weight, enough for every path M can take (0 when none is
+ * needed: the prefill path at an M that fills the GPU).  Host only, but
+ * queries the current device's SM count.
  */
 PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight *W, size_t *bytes);
 
@@ -290,7 +291,11 @@ PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight
  * workspace in CTA order (deterministic).
  * Larger M runs the prefill path (TMA-fed tcgen05 kernel: each CTA takes two
  * tile rows x up to 240 tokens at a time, dense and sparse MMAs into one TMEM
- * fp32 accumulator per tile row).
+ * fp32 accumulator per tile row).  When those units would leave SMs idle
+ * (few tile rows and few tokens) and the workspace holds the fp32 partials,
+ * K is split across CTAs and the last part of each output block to finish
+ * adds the parts in K order (deterministic); with a smaller or NULL
+ * workspace the whole-K units run instead.
  * The kernels are launched with programmatic dependent launch: they read W,
  * its metadata and descriptors before the previous kernel in the stream has
  * completed, and X only after.  X may therefore be that kernel's output; the

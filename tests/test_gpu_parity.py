@@ -374,6 +374,46 @@ def test_prefill_path_small_m_matches_decode(M):
     check_gemm(ys, ref, "decode simt")
 
 
+@pytest.mark.parametrize("N,K,M", [(384, 1280, 17), (384, 1280, 100), (384, 1280, 300), (4096, 1024, 64),
+                                   (1024, 4096, 200)])
+def test_prefill_split_k_matches_oracle_and_whole_k(N, K, M):
+    """Few units for the SMs: K is split across CTAs (3 tile rows: a pair with
+    one row; ragged token tails) and the last part of each block adds the
+    parts.  A workspace too small for the partials runs whole-K units
+    instead; both match the oracle."""
+    x, w, bm, ids = _layer(N, K, M, "exact", 0.5, cfg=16, shape_idx=M % 7)
+    pw = pack_on_gpu(w, bm, ids)
+    ref = oracle.hybrid_gemm(x, w, bm, ids)
+    need = tsg.patch_gemm_workspace_size(M, pw)
+    assert need > 65536  # the split plan needs room for its partials
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for it in range(2):
+        status = tsg.new_status()
+        y = tsg.patch_gemm_ex(to_dev_bf16(x), pw, workspace=ws, status=status, path=tsg.PATH_PREFILL)
+        assert tsg.patch_read_status(status)[0] == 0
+        check_gemm(bits_of(y), ref, f"split-K prefill {N}x{K} M={M} call {it}")
+        assert int(torch.count_nonzero(ws[:65536]).item()) == 0
+    status = tsg.new_status()
+    y = tsg.patch_gemm_ex(to_dev_bf16(x), pw, workspace=torch.zeros(16, dtype=torch.uint8, device="cuda"),
+                          status=status, path=tsg.PATH_PREFILL)
+    assert tsg.patch_read_status(status)[0] == 0
+    check_gemm(bits_of(y), ref, f"whole-K prefill {N}x{K} M={M}")
+
+
+def test_split_k_prefill_and_decode_share_one_workspace():
+    N, K = 4096, 1024
+    x, w, bm, ids = _layer(N, K, 96, "exact", 0.5, cfg=17)
+    pw = pack_on_gpu(w, bm, ids)
+    ws = torch.zeros(max(tsg.patch_gemm_workspace_size(M, pw) for M in (1, 16, 40, 96)), dtype=torch.uint8,
+                     device="cuda")
+    for M in (96, 16, 40, 1, 96, 7):
+        status = tsg.new_status()
+        y = tsg.patch_gemm(to_dev_bf16(x[:M]), pw, workspace=ws, status=status)
+        assert tsg.patch_read_status(status)[0] == 0
+        check_gemm(bits_of(y), oracle.hybrid_gemm(x[:M], w, bm, ids), f"M={M}")
+        assert int(torch.count_nonzero(ws[:65536]).item()) == 0
+
+
 def test_prefill_many_output_tiles():
     """More work units (row pairs x token blocks) than SMs: the persistent schedule wraps around."""
     N, K, M = 128 * 80, 256, 1100
@@ -540,9 +580,10 @@ def test_decode_workspace_too_small_is_rejected():
     x, w, bm, ids = _layer(4096, 4096, 4, "exact", 0.5)
     pw = pack_on_gpu(w, bm, ids)
     need = tsg.patch_gemm_workspace_size(4, pw)
-    assert need > 0
+    assert need > 65536
+    # the counter region alone: no room for the decode kernel's partial rows
     with pytest.raises(tsg.PatchError) as e:
-        tsg.patch_gemm(to_dev_bf16(x), pw, workspace=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
+        tsg.patch_gemm(to_dev_bf16(x), pw, workspace=torch.zeros(65536, dtype=torch.uint8, device="cuda"))
     assert e.value.code == 8
 
 

@@ -287,7 +287,7 @@ def patch_gemm_ex(X: torch.Tensor, weight: PackedWeight, Y: torch.Tensor | None 
     status = new_status(dev) if status is None else status
     st = weight.struct()
     if workspace is None:
-        need = patch_gemm_workspace_size(M, weight) if (path & 0xFF) != PATH_PREFILL else 0
+        need = patch_gemm_workspace_size(M, weight)  # covers every path M can take
         workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)  # must start zero-filled
     _check(lib().patch_gemm_ex(_dev(X, "X"), M, ctypes.byref(st), _dev(Y, "Y"), _dev(workspace, "workspace"),
                                workspace.numel(), _dev(status, "status"), _stream(stream), path, wait_limit_us),

@@ -203,14 +203,20 @@ patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight* W, size_
   const int64_t T = (W->N / kTile) * (W->K / kTile);
   if (W->n_sparse < 0 || W->n_sparse > T) return PATCH_ERR_INVALID_ARG;
   *bytes = 0;
-  if (M == 0 || M > PATCH_DECODE_MAX_M) return PATCH_OK;
+  if (M == 0) return PATCH_OK;
   int sms = 0;
   patch_status_t st = device_sms(&sms);
   if (st != PATCH_OK) return st;
-  // enough for either decode kernel: the counter region, then its scratch
+  // enough for every path M can take: the counter region, then that path's scratch
+  const size_t pf = prefill_workspace_bytes(M, *W, sms);
+  if (M > PATCH_DECODE_MAX_M) {
+    *bytes = pf;
+    return PATCH_OK;
+  }
   const size_t tc = W->N / kTile <= kDecodeMaxTileRows ? decode_tc_workspace_bytes(M, *W, sms) : 0;
   const size_t simt = kDecodeCounterBytes + decode_plan(M, W->N, W->K, sms).ws_bytes;
-  *bytes = tc > simt ? tc : simt;
+  size_t b = tc > simt ? tc : simt;
+  *bytes = b > pf ? b : pf;
   return PATCH_OK;
 }
 
@@ -253,7 +259,8 @@ patch_status_t patch_gemm_ex(const uint16_t* X, int64_t M, const patch_weight* W
     void* scratch = p.ws_bytes > 0 ? static_cast<uint8_t*>(workspace) + kDecodeCounterBytes : nullptr;
     e = launch_decode(X, M, *W, Y, scratch, sms, s);
   } else {
-    e = launch_prefill(X, M, *W, Y, dev_status, sms, limit_ns, inject, s);
+    if (workspace && !aligned16(workspace)) return PATCH_ERR_ALIGN;
+    e = launch_prefill(X, M, *W, Y, workspace, workspace ? workspace_bytes : 0, dev_status, sms, limit_ns, inject, s);
   }
   return e == cudaSuccess ? PATCH_OK : PATCH_ERR_CUDA;
 }

@@ -100,7 +100,10 @@ struct Args {
   const patch_tile_desc* desc[ROWS];
   int mlp;                            // 1: row 0 = gate, row 1 = up tile row rp; Y = silu(gate) * up
   uint16_t* Y;
-  int M, N, Tn, Tk, n_pairs, n_tb, n_items;  // units: row pair rp = item / n_tb, token block tb = item % n_tb
+  int M, N, Tn, Tk, n_pairs, n_tb, n_items;  // units: see unit_of()
+  int ks;                      // K parts per output block (split K; 1 = whole K per unit)
+  float* part;                 // ks > 1: fp32 partials [block][ks][ROWS][bt][128]
+  uint32_t* counters;          // ks > 1: arrivals [block][ROWS][4] (zero between calls)
   int bt;                      // tokens per unit: a multiple of 16, at most BT
   uint32_t idesc_dense, idesc_sparse;
   uint64_t limit_ns;
@@ -129,6 +132,24 @@ __device__ __forceinline__ int tile_row(const Args& p, int rp, int r) { return p
 // moment; only the order of the fp32 sum changes.
 __device__ __forceinline__ int k_rotation(int rp, int tb, int Tk) { return (rp + 7 * tb) % Tk; }
 
+// Work unit `item`: output block blk = (row pair rp, token block tb) and its K
+// part kp, which covers K-tiles [k0, k0 + len).  With ks = 1 a unit is a whole
+// output block (item = blk).  The K loop starts at a rotated tile of the part.
+struct Unit {
+  int blk, kp, rp, tb, k0, len, rot;
+};
+__device__ __forceinline__ Unit unit_of(const Args& p, int item) {
+  Unit u;
+  u.blk = item / p.ks;
+  u.kp = item - u.blk * p.ks;
+  u.rp = u.blk / p.n_tb;
+  u.tb = u.blk - u.rp * p.n_tb;
+  u.k0 = int(int64_t(u.kp) * p.Tk / p.ks);
+  u.len = int(int64_t(u.kp + 1) * p.Tk / p.ks) - u.k0;
+  u.rot = k_rotation(u.rp, u.tb, u.len);
+  return u;
+}
+
 // ---------------------------------------------------------------- roles
 
 // W producer of row r: the row's descriptors, metadata and W panels.  It never
@@ -144,7 +165,7 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
   bool ok = true;
   // stage (or, for a pair without row r, complete with no bytes) the descriptor row of an item
   auto stage_row = [&](int item, int buf) {
-    const int rp = item / p.n_tb;
+    const int rp = unit_of(p, item).rp;
     const bool has = r < rows_of(p, rp);
     mbar_expect_tx(&s.pdesc_full[r][buf], has ? row_bytes : 0u);
     if (has) bulk_load(s.pdesc[r][buf], desc + int64_t(tile_row(p, rp, r)) * p.Tk, row_bytes, &s.pdesc_full[r][buf]);
@@ -153,7 +174,8 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
   if (staged && int(blockIdx.x) < p.n_items) stage_row(blockIdx.x, 0);
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const int rp = item / p.n_tb, tb = item % p.n_tb, tn = tile_row(p, rp, r);
+    const Unit u = unit_of(p, item);
+    const int rp = u.rp, tn = tile_row(p, rp, r);
     const int buf = it & 1;
     if (staged) {
       if (!(ok = wait_bounded(&s.pdesc_full[r][buf], (it >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
@@ -162,8 +184,8 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
       if (item + int(gridDim.x) < p.n_items) stage_row(item + gridDim.x, buf ^ 1);
     }
     if (r >= rows_of(p, rp)) continue;
-    int kt = k_rotation(rp, tb, p.Tk);
-    for (int j = 0; ok && j < p.Tk; ++j, kt = (kt + 1 == p.Tk ? 0 : kt + 1)) {
+    int kt = u.k0 + u.rot;
+    for (int j = 0; ok && j < u.len; ++j, kt = (kt + 1 == u.k0 + u.len ? u.k0 : kt + 1)) {
       if (p.inject && r == 0 && (item != int(blockIdx.x) || j > 0)) {
         ok = false;
         break;
@@ -206,9 +228,10 @@ __device__ void producer_x(Shared& s, const CUtensorMap* tmap_x, const Args& p) 
   // X may be the previous kernel's output: wait for it before the first X load
   pdl_wait_previous();
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-    const int rp = item / p.n_tb, tb = item % p.n_tb;
-    int kt = k_rotation(rp, tb, p.Tk);
-    for (int j = 0; ok && j < p.Tk; ++j, kt = (kt + 1 == p.Tk ? 0 : kt + 1)) {
+    const Unit u = unit_of(p, item);
+    const int tb = u.tb;
+    int kt = u.k0 + u.rot;
+    for (int j = 0; ok && j < u.len; ++j, kt = (kt + 1 == u.k0 + u.len ? u.k0 : kt + 1)) {
       for (int h = 0; ok && h < 2; ++h) {
         const uint32_t bs = b_i % NB;
         if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
@@ -233,11 +256,12 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
   bool ok = true;
   int it = 0;
   for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const bool active = r < rows_of(p, item / p.n_tb);
+    const Unit u = unit_of(p, item);
+    const bool active = r < rows_of(p, u.rp);
     if (!(ok = wait_bounded(&s.acc_empty[r], (it & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
     tc_fence_after();
     uint32_t accumulate = 0;
-    for (int kt = 0; ok && kt < p.Tk; ++kt) {
+    for (int kt = 0; ok && kt < u.len; ++kt) {
       uint32_t kind = 0, as = 0, es = 0;
       for (int h = 0; h < 2; ++h) {
         // the tile's kind arrives with its first panel; a sparse tile's one
@@ -311,6 +335,66 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
 // after the store that read it has finished reading.  Group g drains row g of
 // the pair; for the gated MLP both groups read both rows (gate and up of the
 // same 128 features) and take every other chunk: Y = silu(gate) * up.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v) : "memory");
+  return old;
+}
+
+// Split K (ks > 1): the unit's fp32 accumulator of row g goes to its slot of
+// the workspace, token-major ([bt][128]: a warp's 32 rows of one token are
+// 128 contiguous bytes, for its stores and for the reduction's loads), the
+// accumulator is released, and the last of the block's ks units to arrive
+// (counted per row and TMEM lane quarter, acquire-release) adds the ks
+// partials in K-part order (deterministic), stores Y and resets the counter.
+__device__ void epilogue_split(Shared& s, uint32_t tmem, const Args& p, const Unit& u, int g, int q, int lane) {
+  const bool has = g < rows_of(p, u.rp);
+  const int row = 32 * q + lane;
+  const int64_t n = int64_t(tile_row(p, u.rp, g)) * BM + row;
+  const int m0 = u.tb * p.bt;
+  const int valid = p.M - m0 < p.bt ? p.M - m0 : p.bt;  // tokens of this block inside X
+  const int64_t slot_floats = int64_t(BM) * p.bt;        // one row g of one unit
+  const int64_t blk_base = int64_t(u.blk) * p.ks * ROWS;
+  if (has) {
+    float* mine = p.part + ((blk_base + int64_t(u.kp) * ROWS + g) * slot_floats) + row;
+    const uint32_t lanes = tmem + (uint32_t(32 * q) << 16) + ACC_STRIDE * g;
+    for (int c = 0; c * YT < valid; ++c) {
+      uint32_t v[YT];
+      tmem_ld_16cols(lanes + uint32_t(YT * c), v);
+#pragma unroll
+      for (int j = 0; j < YT; ++j) __stcg(mine + int64_t(YT * c + j) * BM, __uint_as_float(v[j]));
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&s.acc_empty[g]);
+  if (!has) return;
+  // the warp's partial stores are ordered before lane 0's release-acquire increment
+  uint32_t* counter = p.counters + (int64_t(u.blk) * ROWS + g) * 4 + q;
+  uint32_t old = 0;
+  if (lane == 0) old = atom_add_acq_rel_gpu(counter, 1u);
+  old = __shfl_sync(0xFFFFFFFFu, old, 0);
+  if (old != uint32_t(p.ks - 1)) return;
+  __syncwarp();  // orders lane 0's acquire before every lane's loads
+  for (int c = 0; c * YT < valid; ++c) {
+    float sum[YT];
+#pragma unroll
+    for (int j = 0; j < YT; ++j) sum[j] = 0.0f;
+    for (int kp = 0; kp < p.ks; ++kp) {
+      const float* src = p.part + ((blk_base + int64_t(kp) * ROWS + g) * slot_floats) + int64_t(YT * c) * BM + row;
+      float part[YT];
+#pragma unroll
+      for (int j = 0; j < YT; ++j) part[j] = __ldcg(src + int64_t(j) * BM);
+#pragma unroll
+      for (int j = 0; j < YT; ++j) sum[j] += part[j];
+    }
+#pragma unroll
+    for (int j = 0; j < YT; ++j)
+      if (YT * c + j < valid) p.Y[int64_t(m0 + YT * c + j) * p.N + n] = f32_to_bf16_rne(sum[j]);
+  }
+  if (lane == 0) *counter = 0;  // ready for the next call
+}
+
 __device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, const Args& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3;                  // the TMEM lane quarter this warp may access
@@ -320,12 +404,17 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, co
   uint32_t chunk = 0;                      // chunks stored by this group so far (buffer = chunk & 1)
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
-    const int rp = item / p.n_tb, tb = item % p.n_tb;
+    const Unit u = unit_of(p, item);
+    const int rp = u.rp, tb = u.tb;
     // the four warps of a group take the same decision, so none is left at a barrier
     bool ok = wait_bounded(&s.acc_full[g], it & 1, &s.abort_flag, p.limit_ns, p.status, false);
     if (p.mlp) ok = ok && wait_bounded(&s.acc_full[g ^ 1], it & 1, &s.abort_flag, p.limit_ns, p.status, false);
     if (!named_bar_and(bar_id, 128, ok)) break;
     tc_fence_after();
+    if (p.ks > 1) {  // split K (never with the gated MLP)
+      epilogue_split(s, tmem, p, u, g, q, lane);
+      continue;
+    }
     if (p.mlp || g < rows_of(p, rp)) {
       const int n0 = tile_row(p, rp, g) * BM, m0 = tb * p.bt;
       const int valid = p.M - m0 < p.bt ? p.M - m0 : p.bt;  // tokens of this unit inside X
@@ -498,31 +587,62 @@ static bool make_map_y(CUtensorMap* map, void* Y, uint64_t N, uint64_t M) {
 // 128 K at 8192 FLOP per cycle) and the cycles to bring its 64 KiB of W plus
 // 256 bt bytes of X from L2 at about 64 B per cycle; a unit adds ~4000 cycles
 // of pipeline fill and epilogue.  Ties go to the larger bt.
-static int pick_bt(int64_t M, int64_t n_pairs, int64_t Tk, int num_sms) {
+// Launch plan: tokens per unit (bt) and K parts per output block (ks).  Cost
+// model in SM cycles: waves x per-unit time, a unit's K-tile costing the larger
+// of its MMAs (8 bt) and its weight feed (1024 + 4 bt), plus a fixed 4000; a
+// split unit also stores its fp32 partial and one of the ks reads all of them
+// back (32 bt cycles per partial, and 8000 for the hand-over), constants fitted
+// to LLaMA-2-7B q, gate and down timings at M = 17 ... 512.  K is split only
+// to fill one wave of otherwise idle SMs, with at least 4 K-tiles per part.
+struct PrefillPlan {
+  int bt, ks;
+  int64_t n_pairs, n_tb;
+  size_t part_bytes;  // split-K partials (0 when ks == 1)
+};
+
+static PrefillPlan prefill_plan(int64_t M, int64_t n_pairs, int64_t Tk, int num_sms, bool allow_split) {
   using prefill::BT;
-  int best = BT;
+  PrefillPlan best{BT, 1, n_pairs, 0, 0};
   int64_t best_cost = -1;
   for (int bt = BT; bt >= 64; bt -= 16) {
     const int64_t units = n_pairs * ((M + bt - 1) / bt);
-    const int64_t mma = 8 * bt, feed = 1024 + 4 * bt;
-    const int64_t cost = (units + num_sms - 1) / num_sms * (Tk * (mma > feed ? mma : feed) + 4000);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = bt;
+    const int64_t mma = 8 * bt, feed = 1024 + 4 * bt, per_tile = mma > feed ? mma : feed;
+    for (int ks = 1; ks <= (allow_split ? 4 : 1); ++ks) {
+      if (ks > 1 && (units * ks > num_sms || Tk / ks < 4)) break;
+      const int64_t waves = (units * ks + num_sms - 1) / num_sms;
+      const int64_t cost = waves * ((Tk + ks - 1) / ks * per_tile + 4000 + (ks > 1 ? (ks + 1) * 32 * bt + 8000 : 0));
+      if (best_cost < 0 || cost < best_cost) {
+        best_cost = cost;
+        best.bt = bt;
+        best.ks = ks;
+      }
     }
   }
+  best.n_tb = (M + best.bt - 1) / best.bt;
+  best.part_bytes = best.ks > 1 ? size_t(n_pairs * best.n_tb * best.ks) * prefill::ROWS * prefill::BM * best.bt * 4 : 0;
   return best;
+}
+
+size_t prefill_workspace_bytes(int64_t M, const patch_weight& W, int num_sms) {
+  const PrefillPlan pl = prefill_plan(M, (W.N / prefill::BM + prefill::ROWS - 1) / prefill::ROWS, W.K / kTile,
+                                      num_sms, true);
+  return pl.ks > 1 ? kDecodeCounterBytes + pl.part_bytes : 0;
 }
 
 // Shared by the plain GEMM (w1 == w0, units of two consecutive tile rows) and
 // the gated MLP (w0 = gate, w1 = up, units of one tile row of each).
 static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch_weight& W0, const patch_weight& W1,
-                                       bool mlp, uint16_t* Y, int32_t* status, int num_sms, uint64_t limit_ns,
-                                       int inject, cudaStream_t stream) {
+                                       bool mlp, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                                       int32_t* status, int num_sms, uint64_t limit_ns, int inject,
+                                       cudaStream_t stream) {
   using namespace prefill;
   const int64_t Tn = W0.N / BM, Tk = W0.K / kTile;
   const int64_t n_pairs = mlp ? Tn : (Tn + ROWS - 1) / ROWS;
-  const int bt = pick_bt(M, n_pairs, Tk, num_sms);
+  // split K only when the caller's workspace holds the partials (and never for the gated MLP)
+  PrefillPlan plan = prefill_plan(M, n_pairs, Tk, num_sms, !mlp);
+  if (plan.ks > 1 && (!workspace || workspace_bytes < kDecodeCounterBytes + plan.part_bytes))
+    plan = prefill_plan(M, n_pairs, Tk, num_sms, false);
+  const int bt = plan.bt;
   CUtensorMap tmap_x, tmap_w0, tmap_w1, tmap_y;
   if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W0.K), uint64_t(M), uint64_t(W0.K) * 2, 64, uint32_t(bt)))
     return cudaErrorUnknown;
@@ -546,9 +666,12 @@ static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch
   p.Tn = int(Tn);
   p.Tk = int(Tk);
   p.n_pairs = int(n_pairs);
-  p.n_tb = int((M + bt - 1) / bt);
-  p.n_items = int(n_pairs) * p.n_tb;
+  p.n_tb = int(plan.n_tb);
+  p.ks = plan.ks;
+  p.n_items = int(n_pairs) * p.n_tb * p.ks;
   p.bt = bt;
+  p.counters = static_cast<uint32_t*>(workspace);  // the fixed counter region at the start (used when ks > 1)
+  p.part = plan.ks > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kDecodeCounterBytes) : nullptr;
   p.idesc_dense = tc::idesc_bf16(BM, bt, false);
   p.idesc_sparse = tc::idesc_bf16(BM, bt, true);
   p.limit_ns = limit_ns;
@@ -561,15 +684,16 @@ static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch
                     tmap_y, p);
 }
 
-cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
-                           int32_t* status, int num_sms, uint64_t limit_ns, int inject,
+cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
+                           size_t workspace_bytes, int32_t* status, int num_sms, uint64_t limit_ns, int inject,
                            cudaStream_t stream) {
-  return launch_prefill_impl(X, M, W, W, false, Y, status, num_sms, limit_ns, inject, stream);
+  return launch_prefill_impl(X, M, W, W, false, Y, workspace, workspace_bytes, status, num_sms, limit_ns, inject,
+                             stream);
 }
 
 cudaError_t launch_prefill_mlp(const uint16_t* X, int64_t M, const patch_weight& W_gate, const patch_weight& W_up,
                                uint16_t* H, int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream) {
-  return launch_prefill_impl(X, M, W_gate, W_up, true, H, status, num_sms, limit_ns, 0, stream);
+  return launch_prefill_impl(X, M, W_gate, W_up, true, H, nullptr, 0, status, num_sms, limit_ns, 0, stream);
 }
 
 }  // namespace patch

@@ -36,9 +36,13 @@ DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_decode(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
                           void* workspace, int num_sms, cudaStream_t stream);
 
-cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
-                           int32_t* status, int num_sms, uint64_t limit_ns, int inject,
+// Prefill (any M): splits K across CTAs when the units would leave SMs idle and
+// the workspace holds the partials (prefill_workspace_bytes; its counters use
+// the decode paths' fixed counter region), else runs whole-K units.
+cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
+                           size_t workspace_bytes, int32_t* status, int num_sms, uint64_t limit_ns, int inject,
                            cudaStream_t stream);
+size_t prefill_workspace_bytes(int64_t M, const patch_weight& W, int num_sms);
 
 // Gated MLP first half, M > 16: H = silu(X W_gate^T) * (X W_up^T) in one prefill launch.
 cudaError_t launch_prefill_mlp(const uint16_t* X, int64_t M, const patch_weight& W_gate, const patch_weight& W_up,
