@@ -374,13 +374,13 @@ def test_prefill_path_small_m_matches_decode(M):
     check_gemm(ys, ref, "decode simt")
 
 
-@pytest.mark.parametrize("N,K,M", [(384, 1280, 17), (384, 1280, 100), (384, 1280, 300), (4096, 1024, 64),
-                                   (1024, 4096, 200)])
+@pytest.mark.parametrize("N,K,M", [(384, 4096, 17), (384, 4096, 100), (384, 4096, 300), (1024, 4096, 200),
+                                   (384, 5376, 50)])
 def test_prefill_split_k_matches_oracle_and_whole_k(N, K, M):
     """Few units for the SMs: K is split across CTAs (3 tile rows: a pair with
-    one row; ragged token tails) and the last part of each block adds the
-    parts.  A workspace too small for the partials runs whole-K units
-    instead; both match the oracle."""
+    one row; ragged token tails; 42 K-tiles in parts of unequal length) and the
+    last part of each block adds the parts.  A workspace too small for the
+    partials runs whole-K units instead; both match the oracle."""
     x, w, bm, ids = _layer(N, K, M, "exact", 0.5, cfg=16, shape_idx=M % 7)
     pw = pack_on_gpu(w, bm, ids)
     ref = oracle.hybrid_gemm(x, w, bm, ids)
@@ -401,7 +401,7 @@ def test_prefill_split_k_matches_oracle_and_whole_k(N, K, M):
 
 
 def test_split_k_prefill_and_decode_share_one_workspace():
-    N, K = 4096, 1024
+    N, K = 1024, 4096
     x, w, bm, ids = _layer(N, K, 96, "exact", 0.5, cfg=17)
     pw = pack_on_gpu(w, bm, ids)
     ws = torch.zeros(max(tsg.patch_gemm_workspace_size(M, pw) for M in (1, 16, 40, 96)), dtype=torch.uint8,
