@@ -278,10 +278,10 @@ PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight
  *   W  packed weight (host struct)
  *   Y  bf16 [M][N] (16-byte aligned)
  *   workspace: patch_gemm_workspace_size bytes (may be NULL when that is 0).
- *     Its first 64 KiB hold the decode path's per-row arrival counters: they
- *     must be zero before the first use, and every successful call leaves
- *     them zero; the rest is scratch (fp32 partial sums) whose contents do not
- *     matter.  So one zero-fill at allocation suffices, and one workspace of
+ *     Its first 64 KiB hold the arrival counters of the decode path and of
+ *     the prefill path's split-K mode: they must be zero before the first
+ *     use, and every successful call leaves them zero; the rest is scratch
+ *     (fp32 partial sums) whose contents do not matter.  So one zero-fill at allocation suffices, and one workspace of
  *     the largest size serves every layer, token count and path, in any
  *     order.  After a call that reported an error, zero it again.
  * M <= 16 runs the decode path: 1.5 CTAs per SM each stream an equal share

@@ -60,12 +60,12 @@ cudaError_t launch_hard_mask_tiles(const uint16_t* W, int64_t N, int64_t K, int6
 cudaError_t launch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, uint8_t* exec,
                               int64_t* n_sparse, int num_sms, cudaStream_t stream);
 
-// Workspace layout of the decode paths (patch_gemm_workspace_size covers
-// both): the tensor-core kernel's arrival counters (one u32 per tile-row
-// quarter) sit in a fixed region at the start, which every call leaves zero,
-// and each path's scratch (fp32 partial sums) follows it.  Since no call puts
-// anything else in that region, one workspace serves every layer, token count
-// and decode path in any order.
+// Workspace layout (patch_gemm_workspace_size covers every path): arrival
+// counters sit in a fixed region at the start (the tensor-core decode kernel's,
+// one u32 per tile-row quarter; the split-K prefill's, one per output block,
+// row and lane quarter), which every call leaves zero, and each path's scratch
+// (fp32 partial sums) follows it.  Since no call puts anything else in that
+// region, one workspace serves every layer, token count and path in any order.
 constexpr size_t kDecodeCounterBytes = 65536;
 constexpr int64_t kDecodeMaxTileRows = int64_t(kDecodeCounterBytes / 16);  // tensor-core decode: N <= 524288
 
