@@ -228,10 +228,11 @@ def call_flops(L, M):
 # ------------------------------------------------------------ CPU oracle
 
 
-def cpu_baseline(workload, budget_s=15.0, min_s=0.0):
+def cpu_baseline(workload, budget_s=15.0, min_s=0.0, one_thread=True):
     """Time the CPU oracle on a bounded sample of the workload (same metric):
     passes over the step's calls until `min_s` seconds are spent, stopping
-    within a pass once `budget_s` is reached."""
+    within a pass once `budget_s` is reached; with `one_thread`, also the same
+    oracle on one thread over the sample's first calls."""
     import oracle
     layers = build_layers(workload)
     done_units, spent, what, passes = 0.0, 0.0, [], 0
@@ -259,8 +260,31 @@ def cpu_baseline(workload, budget_s=15.0, min_s=0.0):
                 break
         if spent >= budget_s or spent >= min_s:
             break
+    # the same oracle on one thread, over the first calls of the sample (about a second)
+    cores = oracle.num_threads()
+    one_units, one_spent = 0.0, 0.0
+    oracle.set_num_threads(1)
+    try:
+        for li, M in (calls_of(layers)[:4] if one_thread else []):
+            L = layers[li]
+            rows = np.arange(0, M, M // 16)[:16] if workload == "prefill" else None
+            t0 = time.perf_counter()
+            oracle.hybrid_gemm(L["xs"][M], L["w"], L["bm"], L["ids"], rows=rows)
+            one_spent += time.perf_counter() - t0
+            one_units += (call_bytes(L, M) / 1e9) if is_decode(workload) else (call_flops(L, 16) / 1e12)
+            if one_spent >= 2.0:
+                break
+    finally:
+        oracle.set_num_threads(cores)
+    cpu_model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            cpu_model = next((ln.split(":", 1)[1].strip() for ln in f if ln.startswith("model name")), None)
+    except OSError:
+        pass
     return {"value": done_units / spent, "unit": "GB/s" if is_decode(workload) else "TFLOP/s",
-            "cores": oracle.num_threads(), "kind": "oracle", "seconds": round(spent, 3), "passes": passes,
+            "cores": cores, "kind": "oracle", "seconds": round(spent, 3), "passes": passes,
+            "one_thread_value": round(one_units / one_spent, 6) if one_spent > 0 else None, "cpu_model": cpu_model,
             "sample": ("decode GEMMs " if is_decode(workload) else "prefill GEMMs, 16 of 2048 token rows each: ")
             + ", ".join(what[:8]) + (" ..." if len(what) > 8 else "") + f" ({len(what)} calls per pass)"}
 
@@ -823,9 +847,9 @@ def main():
         steps = []
         cb = None
         for _ in range(args.warmup):
-            cpu_baseline(args.workload, budget_s=1.0)
+            cpu_baseline(args.workload, budget_s=1.0, one_thread=False)
         for _ in range(args.steps):
-            cb = cpu_baseline(args.workload, budget_s=5.0)
+            cb = cpu_baseline(args.workload, budget_s=5.0, one_thread=False)
             steps.append(cb["value"])
         value = statistics.median(steps)
         cb = dict(cb, value=round(value, 4))

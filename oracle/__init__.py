@@ -56,6 +56,8 @@ def _load():
         lib.oracle_pack_sizes.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_num_threads.restype = None
         _lib = lib
     return _lib
 
@@ -78,6 +80,11 @@ def _check(rc: int, what: str):
 
 def num_threads() -> int:
     return _load().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """OpenMP threads for the following oracle calls (CPU-baseline timing only)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def apply_mask(w: np.ndarray, bitmap: np.ndarray, pat_id: np.ndarray) -> np.ndarray:

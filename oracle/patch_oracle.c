@@ -390,3 +390,14 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Threads for the following calls (the timing of the CPU baseline only). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
