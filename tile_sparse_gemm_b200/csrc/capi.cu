@@ -259,8 +259,9 @@ patch_status_t patch_gemm_ex(const uint16_t* X, int64_t M, const patch_weight* W
     void* scratch = p.ws_bytes > 0 ? static_cast<uint8_t*>(workspace) + kDecodeCounterBytes : nullptr;
     e = launch_decode(X, M, *W, Y, scratch, sms, s);
   } else {
-    if (workspace && !aligned16(workspace)) return PATCH_ERR_ALIGN;
-    e = launch_prefill(X, M, *W, Y, workspace, workspace ? workspace_bytes : 0, dev_status, sms, limit_ns, inject, s);
+    // the split-K mode uses the workspace only when it is there, aligned and big enough
+    void* ws = workspace && aligned16(workspace) ? workspace : nullptr;
+    e = launch_prefill(X, M, *W, Y, ws, ws ? workspace_bytes : 0, dev_status, sms, limit_ns, inject, s);
   }
   return e == cudaSuccess ? PATCH_OK : PATCH_ERR_CUDA;
 }
