@@ -37,7 +37,7 @@ def _rank_main(rank, world, port, out):
 
 def test_job_time_is_max_over_ranks_and_throughput_counts_all_ranks():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of this multi-threaded process
     mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
     for r in range(world):
         ms, e2e, value = out[r]

@@ -84,7 +84,7 @@ def _rank(rank, world, port, out):
 
 def test_two_ranks_concatenate_to_the_whole_layer():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of this multi-threaded process
     mp.start_processes(_rank, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
     N, K, M = 128 * 7, 256, 5
     w, x = si.gen_w(N, K, 15, 0), si.gen_x(M, K, 15, 0)
