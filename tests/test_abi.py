@@ -80,3 +80,30 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(tsg, "_LIB_PATH", tmp_path / "libpatch.so")
     with pytest.raises(ImportError):
         tsg.lib()
+
+
+def test_packed_weight_save_load_round_trip(tmp_path):
+    """save_packed / load_packed keep a packed weight's blobs bit for bit (CPU
+    tensors here; the blobs are the oracle's packing of a mixed layer) and
+    refuse a file whose blob sizes do not fit its shape."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import synth_inputs as si
+    N, K = 256, 384
+    w = si.gen_w(N, K, 18, 0)
+    bm = si.tiles_exact(N, K, 0.5, 18, 0)
+    ids = si.patterns_top2(w)
+    v, m, d = oracle.pack(w, bm, ids)
+    pw = tsg.PackedWeight(N, K, int(bm.sum()), torch.from_numpy(v), torch.from_numpy(m), torch.from_numpy(d))
+    path = tmp_path / "layer.npz"
+    tsg.save_packed(pw, path)
+    back = tsg.load_packed(path, device="cpu")
+    assert (back.N, back.K, back.n_sparse) == (N, K, int(bm.sum()))
+    for a, b in ((back.values, v), (back.meta, m), (back.desc, d)):
+        assert np.array_equal(a.numpy(), b)
+    bad = tsg.PackedWeight(N, K, int(bm.sum()) + 1, pw.values, pw.meta, pw.desc)
+    tsg.save_packed(bad, tmp_path / "bad.npz")
+    with pytest.raises(ValueError):
+        tsg.load_packed(tmp_path / "bad.npz", device="cpu")

@@ -15,6 +15,10 @@ Entry points (same names as the C ABI):
     patch_gemm(X, weight)                     -> Y
     patch_gemm_ex(X, weight, path=..., wait_limit_us=...) -> Y
     patch_read_status(status)                 -> (status code, device bits)
+    patch_gemm_mlp, patch_tile_kinds, patch_pack_from_logits, patch_soft_mask,
+    patch_hard_mask_tiles, patch_exec_tiles, shard_rows / shard_of (see each docstring)
+Helpers of this binding: save_packed(weight, path) / load_packed(path) keep a
+packed weight in one .npz file (shape, sparse-tile count, the three blobs).
 """
 from __future__ import annotations
 
@@ -147,6 +151,35 @@ def patch_pack_sizes(N: int, K: int, n_sparse: int) -> tuple[int, int, int]:
     _check(lib().patch_pack_sizes(N, K, n_sparse, ctypes.byref(v), ctypes.byref(m), ctypes.byref(d)),
            "patch_pack_sizes")
     return v.value, m.value, d.value
+
+
+_PACKED_FORMAT = 1  # version of the saved layout below
+
+
+def save_packed(weight: PackedWeight, path) -> None:
+    """Write a packed weight to one .npz file: its shape, sparse-tile count and
+    the three blobs as bytes (pack once offline, load at serving time)."""
+    import numpy as np
+    np.savez(path, format=_PACKED_FORMAT, N=weight.N, K=weight.K, n_sparse=weight.n_sparse,
+             values=weight.values.cpu().numpy(), meta=weight.meta.cpu().numpy(), desc=weight.desc.cpu().numpy())
+
+
+def load_packed(path, device="cuda") -> PackedWeight:
+    """Read a packed weight written by save_packed onto `device`, checking the
+    blob sizes against patch_pack_sizes for its shape and sparse-tile count."""
+    import numpy as np
+    with np.load(path) as f:
+        if int(f["format"]) != _PACKED_FORMAT:
+            raise ValueError(f"{path}: packed-weight format {int(f['format'])}, expected {_PACKED_FORMAT}")
+        N, K, n_sparse = int(f["N"]), int(f["K"]), int(f["n_sparse"])
+        blobs = {k: np.ascontiguousarray(f[k], dtype=np.uint8) for k in ("values", "meta", "desc")}
+    sizes = dict(zip(("values", "meta", "desc"), patch_pack_sizes(N, K, n_sparse)))
+    for k, b in blobs.items():
+        if b.size != sizes[k]:
+            raise ValueError(f"{path}: {k} blob has {b.size} bytes, a packed {N}x{K} weight with "
+                             f"{n_sparse} sparse tiles has {sizes[k]}")
+    t = {k: torch.from_numpy(b).to(device) for k, b in blobs.items()}
+    return PackedWeight(N, K, n_sparse, t["values"], t["meta"], t["desc"])
 
 
 def patch_hard_mask(W: torch.Tensor | None, tile_logits: torch.Tensor, pattern_logits: torch.Tensor,
