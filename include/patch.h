@@ -281,9 +281,15 @@ PATCH_API patch_status_t patch_gemm_workspace_size(int64_t M, const patch_weight
  *     Its first 64 KiB hold the arrival counters of the decode path and of
  *     the prefill path's split-K mode: they must be zero before the first
  *     use, and every successful call leaves them zero; the rest is scratch
- *     (fp32 partial sums) whose contents do not matter.  So one zero-fill at allocation suffices, and one workspace of
- *     the largest size serves every layer, token count and path, in any
- *     order.  After a call that reported an error, zero it again.
+ *     (fp32 partial sums) whose contents do not matter.  So one zero-fill at
+ *     allocation suffices, and one workspace of the largest size serves every
+ *     layer, token count and path, in any order.  After a call that reported
+ *     an error, zero it again.  The decode path needs it 16-byte aligned
+ *     (PATCH_ERR_WORKSPACE otherwise); the prefill path uses it only when it
+ *     is aligned and large enough for the split-K partials.
+ *     The tensor-core decode path takes layers of up to 4096 tile rows
+ *     (N <= 524288); PATCH_PATH_AUTO sends wider ones to the CUDA-core decode
+ *     path.
  * M <= 16 runs the decode path: 1.5 CTAs per SM each stream an equal share
  * of the stored panels through a TMA ring (stream-K), the tensor cores reduce
  * them (N = 16 tokens, zero-padded); a tile row cut between CTAs is finished
