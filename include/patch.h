@@ -333,22 +333,31 @@ PATCH_API patch_status_t patch_gemm_ex(const uint16_t *X, int64_t M, const patch
  * framework that owns the device memory pool and passes the plugin only its
  * input and output buffers, or a latency-critical loop where a cudaMalloc
  * (which may synchronise the whole device) is not acceptable.  This entry
- * point computes exactly what patch_gemm computes on its decode path, with
- * the same kernels, but keeps the split-K partial sums in a buffer compiled
- * into the library instead of a caller-provided workspace:
+ * point runs the CUDA-core split-K decode path (the one patch_gemm_ex runs
+ * with PATCH_PATH_DECODE_SIMT), not patch_gemm's default tensor-core decode
+ * kernel, and keeps that path's split-K partial sums in a buffer compiled
+ * into the library instead of a caller-provided workspace.  Its output
+ * therefore equals patch_gemm's within the GEMM tolerance (relative
+ * Frobenius error <= 5e-3, |err| <= 1e-2 (1 + |ref|)), not bit for bit: the
+ * two paths add the fp32 products in different orders.
  *   - the buffer is PATCH_NOALLOC_SCRATCH_BYTES of device memory that every
  *     GPU which loads the library holds until the process exits;
  *   - the first call on each device looks the buffer's device address up
  *     (cudaGetSymbolAddress, with that device current), so make that first
  *     call before any stream capture;
  *   - a problem whose partial sums need more than the buffer holds is
- *     rejected with PATCH_ERR_WORKSPACE (no launch);
+ *     rejected with PATCH_ERR_WORKSPACE (no launch); the partials take
+ *     S * M * N * 4 bytes, S being the number of K splits the path chooses
+ *     (1, needing none, when the layer alone has enough row slabs to fill
+ *     the GPU);
  *   - every call shares the one buffer: calls whose kernels may overlap on
  *     the GPU (different streams, or different host threads) race and give
  *     wrong results; serialise them, e.g. on one stream.  Nothing in the
  *     buffer needs to start at zero: each call overwrites what it reads.
- * Arguments are as for patch_gemm (X, Y, the packed weight and dev_status
- * are caller-owned device memory); M must be in 0..16.  The call allocates
+ * X, Y and the packed weight are caller-owned device memory as for
+ * patch_gemm; M must be in 0..16.  This path has no bounded waits and checks
+ * no pattern ids, so it never sets a device status bit: dev_status is
+ * accepted for symmetry with patch_gemm and may be NULL.  The call allocates
  * nothing and never synchronises the stream.
  */
 #define PATCH_NOALLOC_SCRATCH_BYTES (4u << 20) /* 4 MiB */

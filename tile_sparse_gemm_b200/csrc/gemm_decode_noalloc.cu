@@ -5,9 +5,11 @@
 // a host framework that owns the device memory pool and hands the plugin
 // only its input and output buffers, or a latency-critical loop in which a
 // cudaMalloc (which may synchronise the whole device) is not acceptable.
-// This entry point runs the same split-K decode kernels as patch_gemm, but
-// their fp32 partial sums live in a fixed buffer compiled into the library
-// (below) instead of a caller-provided workspace.
+// This entry point runs the CUDA-core split-K decode kernels (the path
+// patch_gemm_ex takes with PATCH_PATH_DECODE_SIMT, not patch_gemm's default
+// tensor-core decode kernel), with their fp32 partial sums in a fixed buffer
+// compiled into the library (below) instead of a caller-provided workspace.
+// That path sets no device status bits, so dev_status may be NULL.
 //
 // The buffer is a file-scope __device__ array: every GPU that loads the
 // library holds PATCH_NOALLOC_SCRATCH_BYTES of it until the process exits.
@@ -47,7 +49,8 @@ using namespace patch;
 
 extern "C" patch_status_t patch_gemm_decode_noalloc(const uint16_t* X, int64_t M, const patch_weight* W,
                                                    uint16_t* Y, int32_t* dev_status, void* stream) {
-  if (M < 0 || M > PATCH_DECODE_MAX_M || !dev_status || !W) return PATCH_ERR_INVALID_ARG;
+  (void)dev_status;  // nothing on this path reports through the status word
+  if (M < 0 || M > PATCH_DECODE_MAX_M || !W) return PATCH_ERR_INVALID_ARG;
   if (!W->values || !W->desc || (W->n_sparse > 0 && !W->meta)) return PATCH_ERR_INVALID_ARG;
   if (W->N <= 0 || W->K <= 0 || W->N % kTile || W->K % kTile) return PATCH_ERR_SHAPE;
   const int64_t T = (W->N / kTile) * (W->K / kTile);
