@@ -184,6 +184,61 @@ def test_descriptor_table():
     assert offs.tolist() == list(np.concatenate([[0], np.cumsum(sizes)[:-1]]))
 
 
+def spec_values_blob(w, bm, ids, desc_offsets):
+    """The values blob restated from the packed format's text (a panel is 128
+    rows x 64 bf16 with 128-byte rows; a dense tile is 2 panels, k 0..63 then
+    k 64..127; a sparse tile is 1 panel whose row r holds group g's two kept
+    values in ascending k at positions 2g, 2g + 1), placed at each tile's
+    val_offset.  Written with numpy slicing, independently of the C oracle."""
+    N, K = w.shape
+    Tn, Tk = N // TILE, K // TILE
+    size = int(sum(16384 if bm[tn, tk] else 32768 for tn in range(Tn) for tk in range(Tk)))
+    blob = np.zeros(size // 2, np.uint16)
+    for tn in range(Tn):
+        for tk in range(Tk):
+            o = int(desc_offsets[tn * Tk + tk]) // 2
+            tile = w[tn * TILE:(tn + 1) * TILE, tk * TILE:(tk + 1) * TILE]
+            if not bm[tn, tk]:
+                for h in range(2):
+                    panel = tile[:, 64 * h:64 * (h + 1)]                    # 128 rows x 64 values
+                    blob[o + 8192 * h:o + 8192 * (h + 1)] = panel.reshape(-1)  # row-major, 128-byte rows
+            else:
+                groups = tile.reshape(TILE, 32, 4)
+                pid = ids[tn * TILE:(tn + 1) * TILE, tk * 32:(tk + 1) * 32]
+                first = np.array([PAIRS[i][0] for i in pid.ravel()]).reshape(TILE, 32)
+                second = np.array([PAIRS[i][1] for i in pid.ravel()]).reshape(TILE, 32)
+                kept = np.stack([np.take_along_axis(groups, first[..., None], 2)[..., 0],
+                                 np.take_along_axis(groups, second[..., None], 2)[..., 0]], axis=2)
+                blob[o:o + 8192] = kept.reshape(-1)                         # row r: g0a g0b g1a g1b ...
+    return blob.view(np.uint8)
+
+
+def test_values_blob_layout_against_the_format_text():
+    # every weight a distinct bf16 bit pattern, so a byte in the wrong place
+    # (panel order, row stride, kept-value order) cannot match by accident
+    N, K = 2 * TILE, 2 * TILE
+    w = np.arange(N * K, dtype=np.uint32).astype(np.uint16).reshape(N, K)
+    assert len(np.unique(w)) == N * K
+    rng = np.random.default_rng(7)
+    ids = rng.integers(0, 6, size=(N, K // 4)).astype(np.uint8)
+    for bm in (np.array([[0, 1], [1, 0]], np.uint8), np.array([[1, 1], [0, 0]], np.uint8),
+               np.zeros((2, 2), np.uint8), np.ones((2, 2), np.uint8)):
+        values, _, desc = oracle.pack(w, bm, ids)
+        offs = desc.reshape(-1, 16)[:, 8:16].copy().view("<u8").ravel()
+        expect = spec_values_blob(w, bm, ids, offs)
+        assert values.size == expect.size
+        assert np.array_equal(values, expect), bm.tolist()
+    # a few bytes spelled out: dense tile (0, 0), panel 1, row 3, value 5 is W[3][64 + 5]
+    bm = np.array([[0, 1], [1, 0]], np.uint8)
+    values, _, desc = oracle.pack(w, bm, ids)
+    v16 = values.view(np.uint16)
+    assert v16[(16384 + 3 * 128 + 5 * 2) // 2] == w[3, 69]
+    # sparse tile (0, 1) starts after the 32 KiB dense tile; its row 7, group 9 keeps PAIRS[id]
+    a, b = PAIRS[ids[7, 32 + 9]]
+    assert v16[(32768 + 7 * 128 + 9 * 4) // 2] == w[7, 128 + 36 + a]
+    assert v16[(32768 + 7 * 128 + 9 * 4 + 2) // 2] == w[7, 128 + 36 + b]
+
+
 def test_pattern_codes_against_golden():
     codes = golden_codes()
     assert [(a, b) for _, a, b, _ in codes] == PAIRS
