@@ -134,6 +134,34 @@ def patterns_top2(w_bits: np.ndarray) -> np.ndarray:
     return table[lo, hi]
 
 
+def gen_w_device(N: int, K: int, config: int, shape_idx: int, device, std: float = 0.02):
+    """Weights W [N][K] as a bf16 torch tensor drawn on `device` with torch's
+    generator seeded like gen_w: the same distribution, N(0, std) rounded to
+    bf16 to nearest even, but not the same numbers (a different generator).
+    For workloads too large to draw on the host (the 32-layer stack)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(BASE_SEED + 1000 * config + 10 * shape_idx + STREAM_W)
+    w = torch.randn((N, K), generator=g, device=device, dtype=torch.float32) * std
+    return w.to(torch.bfloat16)  # round to nearest even
+
+
+def patterns_top2_torch(w):
+    """patterns_top2 of a bf16 torch tensor, on its device: keep the two largest
+    |w| of each group of 4 (ties -> lower index), lexicographic pair id."""
+    import torch
+    N, K = w.shape
+    mag = (w.view(torch.int16).to(torch.int32) & 0x7FFF).view(N, K // 4, 4)  # |w| order on the bit pattern
+    # rank key: larger magnitude first, then lower index
+    key = mag * 4 + (3 - torch.arange(4, device=w.device, dtype=torch.int32))
+    top = torch.topk(key, 2, dim=2).indices
+    lo, hi = torch.minimum(top[..., 0], top[..., 1]), torch.maximum(top[..., 0], top[..., 1])
+    table = torch.full((4, 4), 255, dtype=torch.uint8, device=w.device)
+    for (a, b), pid in _PAIR_ID.items():
+        table[a, b] = pid
+    return table[lo, hi]
+
+
 def gen_tile_logits(N: int, K: int, config: int = 0, shape_idx: int = 0, tile: int = TILE) -> np.ndarray:
     r = rng(config, shape_idx, STREAM_TILE_LOGITS)
     return r.standard_normal((N // tile, K // tile, 2), dtype=np.float32)

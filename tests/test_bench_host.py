@@ -1,0 +1,112 @@
+"""Host-side arithmetic of bench.py (no GPU): workload tables, call order, the
+roofline and throughput formulas, and the fraction-sweep summary, on fake
+timings whose answers are known in closed form."""
+import argparse
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth_inputs as si  # noqa: E402
+
+PK = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1200.0, "source": "test"}
+
+
+def _args(steps=4):
+    return argparse.Namespace(steps=steps, warmup=3)
+
+
+def _fake_t(ms_total, seg_ms=None, launches=1):
+    return {"ms": ms_total, "e2e_ms": 2 * ms_total, "seg_ms": seg_ms, "clocks": {}, "h2d": 10, "d2h": 20,
+            "launches": launches}
+
+
+def test_stack_layers_order_and_fractions():
+    layers = bench.build_layers("stack", only=["q", "down"])
+    assert len(layers) == 2 * bench.STACK_LAYERS
+    calls = bench.calls_of(layers)
+    # every layer at M = 1 in order, then every layer at M = 8
+    assert calls[:len(layers)] == [(i, 1) for i in range(len(layers))]
+    assert calls[len(layers):] == [(i, 8) for i in range(len(layers))]
+    fr = {L["name"]: L["frac"] for L in layers}
+    assert fr["L0.q"] == 0.1 and fr["L0.down"] == 0.2 and fr["L16.q"] == 0.7 and np.isclose(fr["L16.down"], 0.8)
+    assert fr["L31.q"] == 0.1
+    for L in layers:  # exact sparse-tile counts, weights drawn on the device later
+        T = (L["N"] // 128) * (L["K"] // 128)
+        assert int(L["bm"].sum()) == si.exact_sparse_count(T, L["frac"]) and "gen" in L and "w" not in L
+    # distinct seeds per layer
+    assert len({L["gen"] for L in layers}) == len(layers)
+
+
+def test_llama3_qwen_layers_are_clustered_half_sparse():
+    layers = bench.build_layers("llama3_qwen", only=["k", "v"])
+    assert [L["name"] for L in layers] == ["llama3.k", "llama3.v", "qwen.k", "qwen.v"]
+    for L in layers:
+        T = (L["N"] // 128) * (L["K"] // 128)
+        flat = L["bm"].ravel()
+        on = np.flatnonzero(flat)
+        assert len(on) == si.exact_sparse_count(T, 0.5) and on[-1] - on[0] + 1 == len(on)  # one contiguous run
+        assert sorted(L["xs"]) == [1, 512]
+
+
+def test_roofline_time_closed_forms():
+    N, K, M = 256, 384, 100
+    T = (N // 128) * (K // 128)
+    dense = {"N": N, "K": K, "bm": np.zeros((2, 3), np.uint8)}
+    sparse = {"N": N, "K": K, "bm": np.ones((2, 3), np.uint8)}
+    assert np.isclose(bench.roof_seconds(dense, M, 1000.0, 2.0), 2 * M * N * K / 1e15)
+    assert np.isclose(bench.roof_seconds(sparse, M, 1000.0, 2.0), 2 * M * N * K / 2e15)
+    assert np.isclose(bench.roof_seconds(sparse, M, 1000.0, 1.5), 2 * M * N * K / 1.5e15)
+    assert bench.stored_bytes(N, K, 0) == T * (32768 + 16)
+    assert bench.stored_bytes(N, K, T) == T * (18432 + 16)
+
+
+def test_bytes_block_throughput_and_segments():
+    layers = [{"name": "a", "N": 128, "K": 128, "bm": np.zeros((1, 1), np.uint8), "frac": 0.0},
+              {"name": "b", "N": 256, "K": 128, "bm": np.ones((2, 1), np.uint8), "frac": 1.0}]
+    calls = [(0, 1), (1, 1), (0, 8), (1, 8)]
+    by = [bench.call_bytes(layers[li], M) for li, M in calls]
+    steps = 4
+    t = _fake_t(ms_total=steps * 0.010)  # 10 us per step, no event split: proportional to bytes
+    out = bench.bytes_block(_args(steps), "x", layers, calls, t, PK, 1, segments=[(0, 2), (2, 4)],
+                            seg_names=["p1", "p8"])
+    gbs = sum(by) / 1e9 / 10e-6
+    assert np.isclose(out["value"], gbs, rtol=1e-3) and np.isclose(out["roofline"]["achieved"], gbs, rtol=1e-3)
+    assert np.isclose(out["roofline"]["frac"], gbs / 6000.0, atol=1e-4)
+    assert np.isclose(out["e2e"]["value"], gbs / 2, rtol=1e-3)
+    assert set(out["per_segment"]) == {"p1", "p8"}
+    # with an event split, segments take the measured shares of the event-free step time
+    seg = np.tile([0.002, 0.006], (steps, 1))  # ms, scaled up to the 0.010 ms step
+    out = bench.bytes_block(_args(steps), "x", layers, calls, _fake_t(steps * 0.010, seg), PK, 1,
+                            segments=[(0, 2), (2, 4)], seg_names=["p1", "p8"])
+    assert np.isclose(out["per_segment"]["p1"]["us"], 2.5) and np.isclose(out["per_segment"]["p8"]["us"], 7.5)
+
+
+def test_flops_block_and_monotonic_sweep():
+    layers = [{"name": "q", "N": 256, "K": 256, "bm": bm, "frac": f}
+              for f, bm in ((0.0, np.zeros((2, 2), np.uint8)), (0.5, np.array([[1, 0], [0, 1]], np.uint8)),
+                            (1.0, np.ones((2, 2), np.uint8)))]
+    calls = [(0, 65536), (1, 65536), (2, 65536)]
+    steps = 2
+    seg = np.tile([0.004, 0.003, 0.002], (steps, 1))
+    out, split = bench.flops_block(_args(steps), "p", layers, calls, _fake_t(steps * 0.009, seg), PK, 1,
+                                   sparse_ratio=1.7)
+    fl = 2 * 65536 * 256 * 256
+    assert np.isclose(out["value"], 3 * fl / 1e12 / 9e-6, rtol=1e-3)
+    r2 = sum(bench.roof_seconds(L, 65536, 1500.0, 2.0) for L in layers)
+    assert np.isclose(out["roofline"]["frac"], r2 / 9e-6, atol=1e-4)
+    rm = sum(bench.roof_seconds(L, 65536, 1500.0, 1.7) for L in layers)
+    assert np.isclose(out["roofline"]["frac_measured_sparse_peak"], rm / 9e-6, atol=1e-4)
+    sweep, mono = bench.sweep_summary(layers, calls, split)
+    assert mono and sweep["q"]["speedup_vs_all_dense"] == [1.0, round(4 / 3, 3), 2.0]
+    # a slower middle fraction breaks monotonicity
+    sweep, mono = bench.sweep_summary(layers, calls, np.array([0.004, 0.005, 0.002]))
+    assert not mono and not sweep["q"]["monotonic"]
+
+
+def test_job_throughput_counts_every_rank():
+    assert bench.job_throughput(2.0, 5, 4, 1000.0) == 2.0 * 5 * 4

@@ -68,3 +68,22 @@ def test_workload_shapes_are_tile_multiples():
     assert dict((n, (N, K)) for n, N, K in si.LLAMA2_7B) == {
         "q": (4096, 4096), "k": (4096, 4096), "v": (4096, 4096), "o": (4096, 4096),
         "gate": (11008, 4096), "up": (11008, 4096), "down": (4096, 11008)}
+
+
+def test_device_generators_match_the_host_recipe():
+    """The torch form of the magnitude top-2 choice (used for workloads drawn on
+    the device) equals the numpy form, ties and signed zeros included; the torch
+    weight draw is seeded (repeatable) with the recipe's distribution."""
+    import torch
+    rng = np.random.default_rng(5)
+    w = si.f32_to_bf16_bits(rng.standard_normal((64, 256)).astype(np.float32) * 0.02)
+    w[0, :8] = [0x3F80, 0xBF80, 0x3F80, 0x0000, 0x8000, 0x0000, 0x8000, 0x0000]  # ties, +0 / -0
+    w[1, :4] = 0x3F80
+    wt = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16)
+    assert np.array_equal(si.patterns_top2_torch(wt).numpy(), si.patterns_top2(w))
+    a = si.gen_w_device(256, 512, 4, 3, "cpu")
+    b = si.gen_w_device(256, 512, 4, 3, "cpu")
+    assert a.dtype == torch.bfloat16 and torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert not torch.equal(a.view(torch.int16), si.gen_w_device(256, 512, 4, 4, "cpu").view(torch.int16))
+    std = float(a.float().std())
+    assert 0.019 < std < 0.021 and abs(float(a.float().mean())) < 1e-3
