@@ -194,6 +194,26 @@ def hybrid_gemm(x: np.ndarray, w: np.ndarray, bitmap: np.ndarray, pat_id: np.nda
     return y
 
 
+def chain(x0: np.ndarray, layers) -> list:
+    """Hybrid layers run back to back ("Experimental Results" -> "Speedup &
+    Efficiency": the model's linear layers executed in sequence): layer i
+    multiplies the previous layer's output, rounded once to bf16 (nearest
+    even) as a bf16 activation is, by its hybrid weight.  layers: list of
+    (w, bitmap, pat_id); x0 bf16 bits [M][K0].  Returns every layer's output:
+    fp64, unrounded (for comparison), and the bf16 bits fed to the next."""
+    outs, x = [], np.ascontiguousarray(x0, np.uint16)
+    for w, bm, ids in layers:
+        y = hybrid_gemm(x, w, bm, ids)
+        outs.append(y)
+        x = _f64_to_bf16_rne(y)
+    return outs
+
+
+def bf16_rne(x: np.ndarray) -> np.ndarray:
+    """fp64 -> bf16 bits, round to nearest even (the rounding of every output)."""
+    return _f64_to_bf16_rne(x)
+
+
 def silu(z):
     """SiLU, z * sigmoid(z), in fp64: the gate activation of LLaMA's gated MLP
     (the linears of the pages' LLaMA-2 7B end-to-end runs, "Experimental

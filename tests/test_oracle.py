@@ -372,6 +372,45 @@ def test_bf16_rounding_is_rne():
     assert abs(si.bf16_bits_to_f32(b)[4] - 3.0e-3) < 3.0e-3 * 2 ** -8
 
 
+def test_bf16_rne_from_fp64_ties_and_double_rounding():
+    one = 1.0
+    ulp = 2.0 ** -7  # bf16 spacing at 1
+    # exact ties go to even; just above / below a tie go up / down
+    x = np.array([one + ulp / 2, one + 3 * ulp / 2, one + ulp / 2 + 2 ** -40, one + ulp / 2 - 2 ** -40, -2.5, 0.0])
+    assert oracle.bf16_rne(x).tolist() == [0x3F80, 0x3F82, 0x3F81, 0x3F80, 0xC020, 0x0000]
+    # a value whose fp32 rounding lands exactly on a bf16 midpoint (double rounding) still rounds by the fp64 value
+    x = np.array([one + ulp / 2 + 2 ** -30])  # fp32 rounds it to the midpoint 1 + ulp/2
+    assert np.float32(x[0]) == np.float32(one + ulp / 2)
+    assert oracle.bf16_rne(x).tolist() == [0x3F81]
+
+
+def _identity_layer(n):
+    w = np.zeros((n, n), np.uint16)
+    w[np.arange(n), np.arange(n)] = ONE
+    return w, np.zeros((n // TILE, n // TILE), np.uint8), np.zeros((n, n // 4), np.uint8)
+
+
+def test_chain_composes_layers_in_order_with_bf16_between():
+    M, K = 3, TILE
+    x0 = si.gen_x(M, K, 9, 0)
+    w1 = si.gen_w(K, K, 9, 1)
+    bm1 = np.ones((1, 1), np.uint8)
+    ids1 = si.patterns_top2(w1)
+    # one layer: the hybrid GEMM itself
+    (y,) = oracle.chain(x0, [(w1, bm1, ids1)])
+    assert np.array_equal(y, oracle.hybrid_gemm(x0, w1, bm1, ids1))
+    # identity after it: the first output rounded once to bf16, exactly
+    y1, y2 = oracle.chain(x0, [(w1, bm1, ids1), _identity_layer(K)])
+    assert np.array_equal(y2, f64(oracle.bf16_rne(y1)))
+    # a permutation before it: the same as permuting X's columns
+    perm = np.random.default_rng(3).permutation(K)
+    wp = np.zeros((K, K), np.uint16)
+    wp[np.arange(K), perm] = ONE  # (X Wp^T)[m][n] = X[m][perm[n]]
+    zero_bm, zero_ids = np.zeros((1, 1), np.uint8), np.zeros((K, K // 4), np.uint8)
+    _, y = oracle.chain(x0, [(wp, zero_bm, zero_ids), (w1, bm1, ids1)])
+    assert np.array_equal(y, oracle.hybrid_gemm(x0[:, perm], w1, bm1, ids1))
+
+
 # ---------------------------------------------------------------- gated MLP
 
 
