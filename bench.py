@@ -594,6 +594,38 @@ def tile_ablation(args):
             "rows": rows}
 
 
+def mma_rates(dev, iters=20000, rounds=3):
+    """Tensor-core MMA rate probe (patch_mma_probe): dense and 2:4-sparse
+    rounds of M = 128, N = 240 MMAs on shared-memory operands, one CTA per SM,
+    alternated `rounds` times; the best of each, in dense-equivalent TFLOP/s,
+    and their ratio (the sparse half of the prefill path's mixed roofline)."""
+    import torch
+
+    import tile_sparse_gemm_b200 as tsg
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    status = tsg.new_status(dev)
+    best = {False: 0.0, True: 0.0}
+    for sparse in (False, True):  # warm-up (clocks up, code loaded)
+        tsg.patch_mma_probe(sparse, iters // 4, status)
+    torch.cuda.synchronize()
+    for _ in range(rounds):
+        for sparse in (False, True):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            tsg.patch_mma_probe(sparse, iters, status)
+            e1.record()
+            torch.cuda.synchronize()
+            flops = sms * iters * 4 * 2 * 128 * 240 * (32 if sparse else 16)
+            best[sparse] = max(best[sparse], flops / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+    code, bits = tsg.patch_read_status(status)
+    if code != 0:
+        raise RuntimeError(f"mma probe: device status {code} bits {bits}")
+    return {"dense_tflops": round(best[False], 1), "sparse_tflops": round(best[True], 1),
+            "sparse_over_dense": round(best[True] / best[False], 3),
+            "how": f"patch_mma_probe: {sms} CTAs, {iters} rounds of four M=128 N=240 MMAs each (dense K=16, "
+                   "sparse K=32 dense-equivalent) on shared-memory operands, best of %d alternating runs" % rounds}
+
+
 def job_times(ms, e2e_ms, world, dev=None):
     """Timed-region and end-to-end times (ms) of the whole job: the maximum over
     ranks, since the job ends when its slowest rank does."""
@@ -637,7 +669,7 @@ def pack_layers(layers, dev, status):
     return packed
 
 
-def time_calls(args, layers, packed, calls, dev, world, status, segments=None):
+def time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False):
     """Device time of K steps of `calls` (each a patch_gemm), and the same steps
     end to end with host buffers.
 
@@ -647,6 +679,9 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None):
     same steps with an (external) event pair around each segment of the step
     (every call, or the ranges in `segments`) gives the split of the step;
     event nodes add a few microseconds each, so it is not used for totals.
+    With `chain`, a step is one patch_gemm_chain over the same calls, each
+    waiting for the previous one (the ordering of separate calls on one
+    stream), and the split has one segment.
     Returns ms (timed region), e2e_ms, seg_ms [K][segments], clocks, bytes moved
     by the end-to-end copies, and the launch count."""
     import torch
@@ -654,7 +689,7 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None):
 
     import tile_sparse_gemm_b200 as tsg
     if segments is None:
-        segments = [(j, j + 1) for j in range(len(calls))]
+        segments = [(0, len(calls))] if chain else [(j, j + 1) for j in range(len(calls))]
     # every call's X (and Y) is a view into one device buffer, so that the
     # end-to-end run moves a step's inputs and results with one copy each way
     x_sizes = [M * layers[li]["K"] for li, M in calls]
@@ -674,10 +709,24 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None):
     for j, (li, M) in enumerate(calls):
         views[0][0][j].copy_(torch.from_numpy(layers[li]["xs"][M].view(np.int16)).view(torch.bfloat16))
     ws_bytes = max(tsg.patch_gemm_workspace_size(M, packed[li]) for li, M in calls)
+    chains = None
+    if chain:  # per buffer set, one chain per segment; every call waits for the previous one
+        chains = [{(lo, hi): tsg.Chain([(views[b][0][j], packed[calls[j][0]], views[b][1][j], True)
+                                        for j in range(lo, hi)]) for lo, hi in segments} for b in range(2)]
+        ws_bytes = max([ws_bytes] + [ch.workspace_bytes for ch in chains[0].values()])
     ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)  # zero-filled once, left zeroed by each call
+    if chain:
+        for per_set in chains:
+            for ch in per_set.values():
+                ch.workspace, ch.status = ws, status
     stream = torch.cuda.current_stream()
 
     def run_calls(bset, lo=0, hi=None):
+        if chain:
+            for (a, b), ch in chains[bset].items():
+                if a >= lo and (hi is None or b <= hi):
+                    ch.run()
+            return
         xv, yv = views[bset]
         for j in range(lo, len(calls) if hi is None else hi):
             li, M = calls[j]
@@ -804,8 +853,11 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None):
     del stage_graphs
     e2e_ms = e0.elapsed_time(e1)
     ms, e2e_ms = job_times(ms, e2e_ms, world, dev)
+    # kernels per step: one per patch_gemm call, or a plan kernel and a chain kernel per chain launch
+    per_step = sum(2 * ((hi - lo + tsg.CHAIN_MAX_CALLS - 1) // tsg.CHAIN_MAX_CALLS) for lo, hi in segments) \
+        if chain else len(calls)
     return {"ms": ms, "e2e_ms": e2e_ms, "seg_ms": seg_ms, "clocks": clocks.summary(), "h2d": h2d, "d2h": d2h,
-            "launches": len(calls) * args.steps}
+            "launches": per_step * args.steps}
 
 
 def split_of(t, units, steps):
@@ -825,12 +877,14 @@ def block_common(args, t, per_step, unit, world):
             "gpu_launches": t["launches"], "clocks": t["clocks"]}
 
 
-def bytes_block(args, name, layers, calls, t, pk, world, segments=None, seg_names=None, traffic_kind=None):
+def bytes_block(args, name, layers, calls, t, pk, world, segments=None, seg_names=None, traffic_kind=None,
+                chain=False):
     """A GB/s block (decode-sized calls): HBM bytes the calls must move."""
     alg = np.array([call_bytes(layers[li], M) for li, M in calls], dtype=np.float64)
     if segments is None:
         segments = [(j, j + 1) for j in range(len(calls))]
         seg_names = [f"{layers[li]['name']}@M={M}" for li, M in calls]
+    kernel = "chain_kernel (patch_gemm_chain)" if chain else "decode_tc_kernel"
     seg_bytes = np.array([alg[lo:hi].sum() for lo, hi in segments])
     split = split_of(t, seg_bytes, args.steps)
     achieved = float(alg.sum() / 1e9 / (split.sum() / 1e3))
@@ -842,7 +896,7 @@ def bytes_block(args, name, layers, calls, t, pk, world, segments=None, seg_name
                        "traffic": None if traffic is None else round(traffic),
                        "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
                        "algorithmic_bytes_per_launch": round(float(alg.mean())),
-                       "kernel": "decode_tc_kernel", "peak_source": pk["source"]}
+                       "kernel": kernel, "peak_source": pk["source"]}
     out["per_segment" if len(segments) != len(calls) else "per_call"] = {
         n: {"us": round(1e3 * split[s], 2), "GB/s": round(seg_bytes[s] / 1e9 / (split[s] / 1e3), 1)}
         for s, n in enumerate(seg_names)}
@@ -870,6 +924,7 @@ def flops_block(args, name, layers, calls, t, pk, world, sparse_ratio=None, traf
             "kernel": "prefill_kernel (tcgen05)", "peak_source": pk["source"],
             "note": "frac = mixed roofline time (dense tiles at the dense peak, sparse tiles at 2x it) / measured"}
     if sparse_ratio:
+        # the same roofline with sparse tiles at the measured sparse/dense MMA rate ratio
         tm = np.array([roof_seconds(layers[li], M, P, sparse_ratio) for li, M in calls])
         roof["sparse_ratio_measured"] = round(sparse_ratio, 3)
         roof["frac_measured_sparse_peak"] = round(float(tm.sum() / (split.sum() / 1e3)), 4)
@@ -911,10 +966,19 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
     full = not (args.layers or args.fracs or args.tokens)
     if workload in ("decode", "decode_fused"):
         calls = calls_of(layers)
+        # the step as separate patch_gemm calls, then as one patch_gemm_chain
+        # whose calls each wait for the previous one (the same ordering)
         t = time_calls(args, layers, packed, calls, dev, world, status)
-        out = bytes_block(args, workload, layers, calls, t, pk, world, traffic_kind="decode")
+        sep = bytes_block(args, workload, layers, calls, t, pk, world, traffic_kind="decode")
+        t = time_calls(args, layers, packed, calls, dev, world, status, chain=True)
+        out = bytes_block(args, workload, layers, calls, t, pk, world, segments=[(0, len(calls))],
+                          seg_names=["step"], traffic_kind="decode_chain", chain=True)
         out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (decode" + (
             ", fused q|k|v and gate|up projections)" if workload == "decode_fused" else ")")
+        out["step"] = ("one patch_gemm_chain launch over the step's calls, each waiting for the previous "
+                       "one's completion before reading its X")
+        out["separate_calls"] = dict(sep, step="one patch_gemm call per GEMM, on one stream (programmatic "
+                                               "dependent launch), captured in one CUDA graph")
         out["config"] = {"workload": f"LLaMA-2-7B linear layers ({workload})",
                          "shapes": [f"{L['name']}:{L['N']}x{L['K']}" for L in layers],
                          "tokens": sorted({M for _, M in calls}),
@@ -947,8 +1011,14 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
             names.append(f"pass@M={M}")
             lo += n
         t = time_calls(args, layers, packed, calls, dev, world, status, segments=segments)
-        out = bytes_block(args, workload, layers, calls, t, pk, world, segments, names)
+        sep = bytes_block(args, workload, layers, calls, t, pk, world, segments, names)
+        t = time_calls(args, layers, packed, calls, dev, world, status, segments=segments, chain=True)
+        out = bytes_block(args, workload, layers, calls, t, pk, world, segments, names, chain=True)
         out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (32-layer stack, sequential)"
+        out["step"] = ("per pass (M = 1, then M = 8) patch_gemm_chain over the 224 layers in order, each call "
+                       "waiting for the previous one (64 calls per launch)")
+        out["separate_calls"] = dict(sep, step="one patch_gemm call per layer, captured in one CUDA graph")
+        out["separate_calls"]["ms_per_pass"] = {n: v["us"] / 1e3 for n, v in sep["per_segment"].items()}
         out["ms_per_pass"] = {n: v["us"] / 1e3 for n, v in out["per_segment"].items()}
         out["stored_gb_per_pass"] = round(sum(p.stored_bytes for p in packed) / 1e9, 3)
         out["config"] = {"workload": "32-layer LLaMA-2-7B linear stack, 7 projections per layer, run in order",
@@ -990,15 +1060,19 @@ def run_ours(args, rank, world):
     pk = peaks()
     status = tsg.new_status(dev)
     blocks = BLOCKS if args.workload == "all" else (args.workload,)
+    probe = mma_rates(dev) if any(b in ("prefill", "llama3_qwen") for b in blocks) else None
+    ratio = probe["sparse_over_dense"] if probe else None
     results = {}
     for b in blocks:
-        results[b] = run_block(args, b, rank, world, dev, pk, status)
+        results[b] = run_block(args, b, rank, world, dev, pk, status, sparse_ratio=ratio)
     head = results[blocks[0]]
     out = {"metric": head.pop("metric"), "value": head.pop("value"), "unit": head.pop("unit"), "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head.pop("ms_per_step"),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic"}
     out.update(head)
+    if probe:
+        out["mma_probe"] = probe
     if args.workload == "all":
         out["config"]["blocks"] = list(BLOCKS)
         for b in blocks[1:]:

@@ -325,6 +325,69 @@ PATCH_API patch_status_t patch_gemm_ex(const uint16_t *X, int64_t M, const patch
                              void *stream, int path, uint64_t wait_limit_us);
 
 /*
+ * patch_gemm_chain_workspace_size / patch_gemm_chain: a sequence of decode
+ * GEMMs (each M <= 16 tokens), Y_j = X_j * W_j_eff^T, run by one persistent
+ * launch per up to PATCH_CHAIN_MAX_CALLS calls ("Inference & Deployment":
+ * the same hybrid execution as patch_gemm's decode path; running a model's
+ * layers back to back is how the pages measure LLaMA-2 7B end to end,
+ * "Experimental Results" -> "Speedup & Efficiency").
+ *
+ * A decode GEMM is bound by the bytes of its packed weight, but a separate
+ * launch per layer also pays, per layer, the drain of the previous kernel,
+ * the start of its own CTAs, the X load once its input is ready and the
+ * finish of tile rows cut between CTAs, while the memory idles.  In a chain
+ * every CTA (one per SM, all resident: cooperative launch) streams the
+ * weight panels of call j+1 into its shared-memory ring while call j ends;
+ * only X waits for the previous call.
+ *
+ *   calls[j].X  bf16 [M][K] device, 16-byte aligned
+ *   calls[j].Y  bf16 [M][N] device, 16-byte aligned
+ *   calls[j].W  packed weight (by value; its blobs are caller-owned device memory)
+ *   calls[j].M  0..16 (0: the call is skipped)
+ *   calls[j].after_previous
+ *       nonzero: X_j may be written by earlier calls of the chain, so call j
+ *       reads X_j only after every earlier call has completed (Y written and
+ *       visible) -- the ordering of separate patch_gemm calls on one stream;
+ *       0: X_j is ready when the chain starts, and call j may overlap earlier
+ *       calls.  A call with after_previous == 0 must not write memory that an
+ *       earlier call reads or writes.  The first call of a chain never waits.
+ * Results equal patch_gemm's decode path (same tile kernels, same fp32 sum
+ * order within a tile row; cut rows are added in CTA order): within the GEMM
+ * tolerance of each other, deterministic run to run.
+ * workspace: patch_gemm_chain_workspace_size bytes, 16-byte aligned, zero
+ * before the first use.  Its first 64 KiB are the counter region of
+ * patch_gemm's workspace (completion counters of the calls, then arrival
+ * counters of their cut tile rows), which every successful call leaves
+ * zero; so one zero-filled workspace of the largest size serves patch_gemm
+ * and patch_gemm_chain in any order.  After an error, zero it again.  The
+ * rest is scratch: fp32 partial sums and, per panel of every call, the tile
+ * it belongs to (written by a small kernel launched first).
+ * Calls are split into launches of at most PATCH_CHAIN_MAX_CALLS calls whose
+ * tile rows fit the counter region (4 counters per tile row); each launch
+ * starts after the previous one in the stream has completed.
+ * Limits: N <= 524160 per call (4095 tile rows).  Every wait (on a ring
+ * slot or on another CTA's completion counter) is bounded by wait_limit_us
+ * (0 = 2 s); on expiry PATCH_DEV_TIMEOUT is set and Y is undefined.
+ * Errors: PATCH_ERR_INVALID_ARG (NULL, M outside 0..16, n_calls < 0),
+ * PATCH_ERR_SHAPE, PATCH_ERR_ALIGN, PATCH_ERR_WORKSPACE, PATCH_ERR_DEVICE,
+ * PATCH_ERR_CUDA (including a GPU that cannot keep one CTA per SM resident).
+ */
+#define PATCH_CHAIN_MAX_CALLS 64
+typedef struct {
+    const uint16_t *X;
+    uint16_t *Y;
+    patch_weight W;
+    int64_t M;
+    int32_t after_previous;
+    int32_t reserved; /* set to 0 */
+} patch_chain_call;
+PATCH_API patch_status_t patch_gemm_chain_workspace_size(const patch_chain_call *calls, int64_t n_calls,
+                                                         size_t *bytes);
+PATCH_API patch_status_t patch_gemm_chain(const patch_chain_call *calls, int64_t n_calls, void *workspace,
+                                          size_t workspace_bytes, int32_t *dev_status, void *stream,
+                                          uint64_t wait_limit_us);
+
+/*
  * patch_gemm_decode_noalloc: the decode GEMM (M <= 16) for callers that
  * cannot allocate device memory.  The paper has no counterpart; this is a
  * deployment convenience of this library.
@@ -407,6 +470,24 @@ PATCH_API patch_status_t patch_gemm_mlp(const uint16_t *X, int64_t M, const patc
  */
 PATCH_API patch_status_t patch_shard_rows(const uint8_t *bitmap, int64_t Tn, int64_t Tk, int64_t n_shards,
                                           int64_t *row_begin);
+
+/*
+ * patch_mma_probe: a measurement of this GPU's tensor-core MMA rate for the
+ * two instruction forms of the hybrid GEMM ("Inference & Deployment": dense
+ * tiles on the dense tensor-core MMA, sparse tiles on the 2:4 sparse one),
+ * free of memory traffic: one CTA per SM issues `iters` rounds of four
+ * M = 128, N = 240 MMAs (the prefill kernel's shape) on pseudo-random bf16
+ * operands in shared memory.  A dense round is four K = 16 MMAs, a sparse
+ * round four K = 32 (logical) .sp MMAs with valid metadata, so a round does
+ * 4 x 2 x 128 x 240 x 16 (dense) or x 32 (sparse, dense-equivalent) FLOPs on
+ * each SM.  The caller times the launch on `stream` (the call itself never
+ * synchronises); the ratio of the two rates is the sparse/dense speed ratio
+ * that the prefill path's mixed roofline needs.  dev_status gets
+ * PATCH_DEV_TIMEOUT if the final wait for the MMAs runs out (2 s).
+ * Errors: PATCH_ERR_INVALID_ARG (iters < 1, NULL dev_status), PATCH_ERR_DEVICE,
+ * PATCH_ERR_CUDA.
+ */
+PATCH_API patch_status_t patch_mma_probe(int sparse, int64_t iters, int32_t *dev_status, void *stream);
 
 /*
  * patch_read_status: synchronise `stream`, copy *dev_status to *host_bits and

@@ -16,7 +16,8 @@ Entry points (same names as the C ABI):
     patch_gemm_ex(X, weight, path=..., wait_limit_us=...) -> Y
     patch_read_status(status)                 -> (status code, device bits)
     patch_gemm_mlp, patch_tile_kinds, patch_pack_from_logits, patch_soft_mask,
-    patch_hard_mask_tiles, patch_exec_tiles, shard_rows / shard_of (see each docstring)
+    patch_hard_mask_tiles, patch_exec_tiles, shard_rows / shard_of,
+    patch_gemm_chain / Chain (a sequence of decode GEMMs in one launch; see each docstring)
 Helpers of this binding: save_packed(weight, path) / load_packed(path) keep a
 packed weight in one .npz file (shape, sparse-tile count, the three blobs).
 """
@@ -54,6 +55,14 @@ class _Weight(ctypes.Structure):
                 ("values", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("desc", ctypes.c_void_p)]
 
 
+class _ChainCall(ctypes.Structure):
+    _fields_ = [("X", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("W", _Weight), ("M", ctypes.c_int64),
+                ("after_previous", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+CHAIN_MAX_CALLS = 64  # calls per launch of patch_gemm_chain (longer chains take several launches)
+
+
 _lib = None
 
 
@@ -82,6 +91,9 @@ def lib() -> ctypes.CDLL:
             "patch_read_status": [P, P, ctypes.POINTER(ctypes.c_int32)],
             "patch_gemm_mlp_workspace_size": [I64, WP, WP, ctypes.POINTER(SZ)],
             "patch_gemm_mlp": [P, I64, WP, WP, P, P, SZ, P, P],
+            "patch_gemm_chain_workspace_size": [P, I64, ctypes.POINTER(SZ)],
+            "patch_gemm_chain": [P, I64, P, SZ, P, P, ctypes.c_uint64],
+            "patch_mma_probe": [I32, I64, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -338,6 +350,60 @@ def patch_gemm(X: torch.Tensor, weight: PackedWeight, Y: torch.Tensor | None = N
     return patch_gemm_ex(X, weight, Y, workspace, status, PATH_AUTO, 0, stream)
 
 
+class Chain:
+    """A fixed sequence of decode GEMMs (M <= 16 each) for patch_gemm_chain.
+
+    calls: list of (X, weight, Y, after_previous) with X bf16 [M][K], Y bf16
+    [M][N] (device tensors; Y None allocates it) and after_previous True when
+    X is written by an earlier call of the chain (the call then reads X only
+    after every earlier call has completed).  The ctypes array of calls and a
+    zero-filled workspace are built once; run() launches the chain on the
+    current stream (capturable in a CUDA graph after one eager run)."""
+
+    def __init__(self, calls, workspace: torch.Tensor | None = None, status: torch.Tensor | None = None):
+        self.Y = []
+        arr = (_ChainCall * len(calls))()
+        self._keep = []
+        for j, (X, weight, Y, after) in enumerate(calls):
+            M, K = X.shape
+            if K != weight.K:
+                raise ValueError(f"call {j}: X has K={K}, weight has K={weight.K}")
+            if Y is None:
+                Y = torch.empty((M, weight.N), dtype=torch.bfloat16, device=X.device)
+            arr[j] = _ChainCall(_dev(X, "X") if M else None, _dev(Y, "Y") if M else None, weight.struct(), M,
+                                1 if after else 0, 0)
+            self.Y.append(Y)
+            self._keep += [X, Y, weight]
+        self.calls = arr
+        self.n = len(calls)
+        b = ctypes.c_size_t()
+        _check(lib().patch_gemm_chain_workspace_size(ctypes.cast(arr, ctypes.c_void_p), self.n, ctypes.byref(b)),
+               "patch_gemm_chain_workspace_size")
+        dev = calls[0][0].device if calls else None
+        if workspace is None:
+            workspace = torch.zeros(max(b.value, 16), dtype=torch.uint8, device=dev)  # must start zero-filled
+        elif workspace.numel() < b.value:
+            raise ValueError(f"workspace of {workspace.numel()} bytes < {b.value} needed")
+        self.workspace = workspace
+        self.status = new_status(dev) if status is None else status
+
+    @property
+    def workspace_bytes(self) -> int:
+        return self.workspace.numel()
+
+    def run(self, wait_limit_us: int = 0, stream=None):
+        _check(lib().patch_gemm_chain(ctypes.cast(self.calls, ctypes.c_void_p), self.n, _dev(self.workspace, "workspace"),
+                                      self.workspace.numel(), _dev(self.status, "status"), _stream(stream),
+                                      wait_limit_us), "patch_gemm_chain")
+        return self.Y
+
+
+def patch_gemm_chain(calls, workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                     wait_limit_us: int = 0, stream=None) -> list[torch.Tensor]:
+    """One launch (per 64 calls) of a sequence of decode GEMMs: see Chain."""
+    return Chain(calls, workspace, status).run(wait_limit_us, stream)
+
+
 def patch_gemm_mlp(X: torch.Tensor, gate: PackedWeight, up: PackedWeight, H: torch.Tensor | None = None,
                    workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
                    stream=None) -> torch.Tensor:
@@ -377,6 +443,16 @@ def shard_of(W: torch.Tensor, bitmap: torch.Tensor, pat_id: torch.Tensor, rows: 
     """Views of one shard's W rows, bitmap rows and pattern-id rows (no copy)."""
     b, e = rows
     return W[b * 128:e * 128], bitmap[b:e], pat_id[b * 128:e * 128]
+
+
+def patch_mma_probe(sparse: bool, iters: int, status: torch.Tensor | None = None, stream=None) -> None:
+    """Launch the tensor-core MMA rate probe (dense or 2:4 sparse rounds of four
+    M = 128, N = 240 MMAs per SM on shared-memory operands); time it with CUDA
+    events on the stream.  FLOPs per launch: SMs x iters x 4 x 2 x 128 x 240 x
+    (32 if sparse else 16), dense-equivalent."""
+    status = new_status() if status is None else status
+    _check(lib().patch_mma_probe(1 if sparse else 0, iters, _dev(status, "status"), _stream(stream)),
+           "patch_mma_probe")
 
 
 def patch_read_status(status: torch.Tensor, stream=None) -> tuple[int, int]:

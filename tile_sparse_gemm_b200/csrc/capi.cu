@@ -2,6 +2,8 @@
 // Every entry point is declared and documented in include/patch.h.
 #include <cuda_runtime.h>
 
+#include <vector>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -271,6 +273,68 @@ patch_status_t patch_gemm(const uint16_t* X, int64_t M, const patch_weight* W, u
   return patch_gemm_ex(X, M, W, Y, workspace, workspace_bytes, dev_status, stream, PATCH_PATH_AUTO, 0);
 }
 
+// Checks of one chain call; M == 0 calls are valid and skipped.
+static patch_status_t check_chain_call(const patch_chain_call& c) {
+  if (c.M < 0 || c.M > PATCH_DECODE_MAX_M) return PATCH_ERR_INVALID_ARG;
+  patch_status_t st = check_weight(&c.W);
+  if (st != PATCH_OK) return st;
+  if (c.W.N / kTile > kChainMaxTileRows) return PATCH_ERR_SHAPE;
+  if (c.M == 0) return PATCH_OK;
+  if (!c.X || !c.Y) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(c.X) || !aligned16(c.Y)) return PATCH_ERR_ALIGN;
+  return PATCH_OK;
+}
+
+// The calls that do work (M > 0), in order.
+static patch_status_t chain_calls(const patch_chain_call* calls, int64_t n, std::vector<patch_chain_call>& out) {
+  if (n < 0 || (n > 0 && !calls)) return PATCH_ERR_INVALID_ARG;
+  out.clear();
+  for (int64_t j = 0; j < n; ++j) {
+    patch_status_t st = check_chain_call(calls[j]);
+    if (st != PATCH_OK) return st;
+    if (calls[j].M > 0) out.push_back(calls[j]);
+  }
+  return PATCH_OK;
+}
+
+patch_status_t patch_gemm_chain_workspace_size(const patch_chain_call* calls, int64_t n_calls, size_t* bytes) {
+  if (!bytes) return PATCH_ERR_INVALID_ARG;
+  std::vector<patch_chain_call> cs;
+  patch_status_t st = chain_calls(calls, n_calls, cs);
+  if (st != PATCH_OK) return st;
+  *bytes = 0;
+  if (cs.empty()) return PATCH_OK;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  *bytes = chain_workspace_bytes(cs.data(), int64_t(cs.size()), sms);
+  return PATCH_OK;
+}
+
+patch_status_t patch_gemm_chain(const patch_chain_call* calls, int64_t n_calls, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, void* stream, uint64_t wait_limit_us) {
+  if (!dev_status) return PATCH_ERR_INVALID_ARG;
+  std::vector<patch_chain_call> cs;
+  patch_status_t st = chain_calls(calls, n_calls, cs);
+  if (st != PATCH_OK) return st;
+  if (cs.empty()) return PATCH_OK;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  const int64_t n = int64_t(cs.size());
+  if (!workspace || !aligned16(workspace) || workspace_bytes < chain_workspace_bytes(cs.data(), n, sms))
+    return PATCH_ERR_WORKSPACE;
+  const uint64_t limit_ns = (wait_limit_us ? wait_limit_us : 2000000ull) * 1000ull;
+  for (int64_t j0 = 0; j0 < n;) {
+    const int64_t j1 = chain_launch_end(cs.data(), j0, n);
+    if (launch_chain(cs.data(), j0, j1, workspace, dev_status, sms, limit_ns, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+      return PATCH_ERR_CUDA;
+    j0 = j1;
+  }
+  return PATCH_OK;
+}
+
 // decode scratch for the gated MLP: [decode GEMM workspace][G][U], 256-byte aligned parts
 static size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
 
@@ -361,6 +425,17 @@ patch_status_t patch_shard_rows(const uint8_t* bitmap, int64_t Tn, int64_t Tk, i
   }
   row_begin[n_shards] = Tn;
   return PATCH_OK;
+}
+
+patch_status_t patch_mma_probe(int sparse, int64_t iters, int32_t* dev_status, void* stream) {
+  if (iters < 1 || !dev_status) return PATCH_ERR_INVALID_ARG;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  return launch_mma_probe(sparse ? 1 : 0, iters, sms, 2000000000ull, dev_status, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? PATCH_OK
+             : PATCH_ERR_CUDA;
 }
 
 patch_status_t patch_read_status(const int32_t* dev_status, void* stream, int32_t* host_bits) {

@@ -74,6 +74,19 @@ size_t decode_tc_workspace_bytes(int64_t M, const patch_weight& W, int num_sms);
 cudaError_t launch_decode_tc(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
                              int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream);
 
+// Chained decode GEMMs (patch_gemm_chain).  chain_launch_end: end of the
+// launch that starts at call j0 (calls fit PATCH_CHAIN_MAX_CALLS and the
+// counter region); chain_workspace_bytes: workspace for all launches.
+int64_t chain_launch_end(const patch_chain_call* calls, int64_t j0, int64_t n);
+size_t chain_workspace_bytes(const patch_chain_call* calls, int64_t n, int num_sms);
+cudaError_t launch_chain(const patch_chain_call* calls, int64_t j0, int64_t j1, void* workspace, int32_t* status,
+                         int num_sms, uint64_t limit_ns, cudaStream_t stream);
+constexpr int64_t kChainMaxTileRows = int64_t(kDecodeCounterBytes / 16) - 1;  // 4 counters per row + 2 words
+
+// Tensor-core MMA rate probe (patch_mma_probe).
+cudaError_t launch_mma_probe(int sparse, int64_t iters, int num_sms, uint64_t limit_ns, int32_t* status,
+                             cudaStream_t stream);
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel in the stream is finishing; it must call
 // griddepcontrol.wait before touching anything that kernel may write.
