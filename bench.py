@@ -669,7 +669,7 @@ def pack_layers(layers, dev, status):
     return packed
 
 
-def time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False):
+def time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False, after=True):
     """Device time of K steps of `calls` (each a patch_gemm), and the same steps
     end to end with host buffers.
 
@@ -679,9 +679,11 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
     same steps with an (external) event pair around each segment of the step
     (every call, or the ranges in `segments`) gives the split of the step;
     event nodes add a few microseconds each, so it is not used for totals.
-    With `chain`, a step is one patch_gemm_chain over the same calls, each
-    waiting for the previous one (the ordering of separate calls on one
-    stream), and the split has one segment.
+    With `chain`, a step is one patch_gemm_chain per segment over the same
+    calls; with `after` every call waits for the previous one's completion
+    before reading its X (the ordering of separate calls on one stream),
+    without it the calls run as the independent GEMMs they are (each X is an
+    input of the step, not an earlier call's output).
     Returns ms (timed region), e2e_ms, seg_ms [K][segments], clocks, bytes moved
     by the end-to-end copies, and the launch count."""
     import torch
@@ -711,7 +713,7 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
     ws_bytes = max(tsg.patch_gemm_workspace_size(M, packed[li]) for li, M in calls)
     chains = None
     if chain:  # per buffer set, one chain per segment; every call waits for the previous one
-        chains = [{(lo, hi): tsg.Chain([(views[b][0][j], packed[calls[j][0]], views[b][1][j], True)
+        chains = [{(lo, hi): tsg.Chain([(views[b][0][j], packed[calls[j][0]], views[b][1][j], after)
                                         for j in range(lo, hi)]) for lo, hi in segments} for b in range(2)]
         ws_bytes = max([ws_bytes] + [ch.workspace_bytes for ch in chains[0].values()])
     ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)  # zero-filled once, left zeroed by each call
@@ -966,19 +968,23 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
     full = not (args.layers or args.fracs or args.tokens)
     if workload in ("decode", "decode_fused"):
         calls = calls_of(layers)
-        # the step as separate patch_gemm calls, then as one patch_gemm_chain
-        # whose calls each wait for the previous one (the same ordering)
+        # the step as separate patch_gemm calls (the headline), then as one
+        # patch_gemm_chain whose calls each wait for the previous one (the same
+        # ordering), and as one chain of the independent GEMMs they are
         t = time_calls(args, layers, packed, calls, dev, world, status)
-        sep = bytes_block(args, workload, layers, calls, t, pk, world, traffic_kind="decode")
-        t = time_calls(args, layers, packed, calls, dev, world, status, chain=True)
-        out = bytes_block(args, workload, layers, calls, t, pk, world, segments=[(0, len(calls))],
-                          seg_names=["step"], traffic_kind="decode_chain", chain=True)
+        out = bytes_block(args, workload, layers, calls, t, pk, world, traffic_kind="decode")
         out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (decode" + (
             ", fused q|k|v and gate|up projections)" if workload == "decode_fused" else ")")
-        out["step"] = ("one patch_gemm_chain launch over the step's calls, each waiting for the previous "
-                       "one's completion before reading its X")
-        out["separate_calls"] = dict(sep, step="one patch_gemm call per GEMM, on one stream (programmatic "
-                                               "dependent launch), captured in one CUDA graph")
+        out["step"] = ("one patch_gemm call per GEMM on one stream (programmatic dependent launch: each "
+                       "waits for the previous one before reading its X), captured in one CUDA graph")
+        for key, after, what in (("chain", True, "each waiting for the previous one's completion before reading "
+                                                 "its X"),
+                                 ("chain_independent", False, "the step's GEMMs are independent (every X is an "
+                                                              "input of the step), so none waits")):
+            t = time_calls(args, layers, packed, calls, dev, world, status, chain=True, after=after)
+            out[key] = bytes_block(args, workload, layers, calls, t, pk, world, segments=[(0, len(calls))],
+                                   seg_names=["step"], chain=True)
+            out[key]["step"] = "one patch_gemm_chain launch over the step's calls, " + what
         out["config"] = {"workload": f"LLaMA-2-7B linear layers ({workload})",
                          "shapes": [f"{L['name']}:{L['N']}x{L['K']}" for L in layers],
                          "tokens": sorted({M for _, M in calls}),
@@ -1011,14 +1017,14 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
             names.append(f"pass@M={M}")
             lo += n
         t = time_calls(args, layers, packed, calls, dev, world, status, segments=segments)
-        sep = bytes_block(args, workload, layers, calls, t, pk, world, segments, names)
-        t = time_calls(args, layers, packed, calls, dev, world, status, segments=segments, chain=True)
-        out = bytes_block(args, workload, layers, calls, t, pk, world, segments, names, chain=True)
+        out = bytes_block(args, workload, layers, calls, t, pk, world, segments, names)
         out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (32-layer stack, sequential)"
-        out["step"] = ("per pass (M = 1, then M = 8) patch_gemm_chain over the 224 layers in order, each call "
-                       "waiting for the previous one (64 calls per launch)")
-        out["separate_calls"] = dict(sep, step="one patch_gemm call per layer, captured in one CUDA graph")
-        out["separate_calls"]["ms_per_pass"] = {n: v["us"] / 1e3 for n, v in sep["per_segment"].items()}
+        out["step"] = "one patch_gemm call per layer, in order, captured in one CUDA graph"
+        t = time_calls(args, layers, packed, calls, dev, world, status, segments=segments, chain=True)
+        ch = bytes_block(args, workload, layers, calls, t, pk, world, segments, names, chain=True)
+        out["chain"] = dict(ch, step="per pass (M = 1, then M = 8) patch_gemm_chain over the 224 layers in order, "
+                                     "each call waiting for the previous one (64 calls per launch)")
+        out["chain"]["ms_per_pass"] = {n: v["us"] / 1e3 for n, v in ch["per_segment"].items()}
         out["ms_per_pass"] = {n: v["us"] / 1e3 for n, v in out["per_segment"].items()}
         out["stored_gb_per_pass"] = round(sum(p.stored_bytes for p in packed) / 1e9, 3)
         out["config"] = {"workload": "32-layer LLaMA-2-7B linear stack, 7 projections per layer, run in order",
