@@ -267,6 +267,37 @@ def calls_of(layers, ms=None):
     return [(li, M) for M in all_ms if ms is None or M in ms for li, L in enumerate(layers) if M in L["xs"]]
 
 
+def shard_layers(layers, rank, world, shard_rows):
+    """Column-parallel shard of every layer for `rank` of `world` ranks: its
+    contiguous tile rows (shard_rows(bitmap, world): balanced by stored bytes)
+    of W, the bitmap and the pattern ids.  Each shard keeps the layer's X; its
+    Y is the layer's Y columns [128 b, 128 e)."""
+    out = []
+    for L in layers:
+        b, e = shard_rows(L["bm"], world)[rank]
+        S = dict(L, N=(e - b) * 128, bm=L["bm"][b:e], full_N=L["N"], rows=(b, e))
+        if "w" in L:
+            S.update(w=L["w"][b * 128:e * 128], ids=L["ids"][b * 128:e * 128])
+        out.append(S)
+    return out
+
+
+def gather_layout(layers, calls, world, shard_rows):
+    """Where each rank's Y shards sit in the buffer that one all-gather moves:
+    rank r's Y of call j (M_j x 128 (e - b) bf16) at offset[r][j] elements of
+    its segment; every rank's segment is padded to the largest, `seg`."""
+    sizes = [[0] * len(calls) for _ in range(world)]
+    offset = [[0] * len(calls) for _ in range(world)]
+    for r in range(world):
+        o = 0
+        for j, (li, M) in enumerate(calls):
+            b, e = shard_rows(layers[li]["bm"], world)[r]
+            offset[r][j], sizes[r][j] = o, M * (e - b) * 128
+            o += sizes[r][j]
+    seg = max(sum(s_) for s_ in sizes)
+    return offset, sizes, seg
+
+
 def call_bytes(L, M):
     return stored_bytes(L["N"], L["K"], int(L["bm"].sum())) + 2 * M * L["K"] + 2 * M * L["N"]
 
@@ -669,7 +700,8 @@ def pack_layers(layers, dev, status):
     return packed
 
 
-def time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False, after=True):
+def time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False, after=True,
+               gather=None):
     """Device time of K steps of `calls` (each a patch_gemm), and the same steps
     end to end with host buffers.
 
@@ -684,6 +716,9 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
     before reading its X (the ordering of separate calls on one stream),
     without it the calls run as the independent GEMMs they are (each X is an
     input of the step, not an earlier call's output).
+    With `gather` (column-parallel shards, one per rank), every step ends with
+    one NCCL all-gather of all ranks' Y shards (padded to `gather` elements
+    each), and the steps run eagerly (no graph).
     Returns ms (timed region), e2e_ms, seg_ms [K][segments], clocks, bytes moved
     by the end-to-end copies, and the launch count."""
     import torch
@@ -697,7 +732,8 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
     x_sizes = [M * layers[li]["K"] for li, M in calls]
     y_sizes = [M * layers[li]["N"] for li, M in calls]
     x_all = torch.empty(sum(x_sizes), dtype=torch.bfloat16, device=dev)
-    y_all = torch.empty(sum(y_sizes), dtype=torch.bfloat16, device=dev)
+    y_all = torch.empty(max(sum(y_sizes), gather or 0), dtype=torch.bfloat16, device=dev)
+    gathered = torch.empty(world * gather, dtype=torch.bfloat16, device=dev) if gather else None
     x_sets, y_sets = [x_all, torch.empty_like(x_all)], [y_all, torch.empty_like(y_all)]
     views = []
     for bset in range(2):
@@ -724,6 +760,10 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
     stream = torch.cuda.current_stream()
 
     def run_calls(bset, lo=0, hi=None):
+        if gather and hi is None and lo == 0:
+            run_calls(bset, 0, len(calls))
+            dist.all_gather_into_tensor(gathered, y_sets[bset][:gather])
+            return
         if chain:
             for (a, b), ch in chains[bset].items():
                 if a >= lo and (hi is None or b <= hi):
@@ -764,7 +804,7 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
         torch.cuda.synchronize()
         return g, evs
 
-    graph = None if args.no_graph else capture(False)[0]
+    graph = None if (args.no_graph or gather) else capture(False)[0]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clocks:
         clocks.wait_first_sample()
@@ -784,7 +824,7 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
     ms = t_start.elapsed_time(t_end)
     del graph
     seg_ms = None
-    if not args.no_graph:
+    if not (args.no_graph or gather):
         g_ev, ev = capture(True)
         g_ev.replay()
         torch.cuda.synchronize()
@@ -826,7 +866,7 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
         cur.wait_stream(s_out)
 
     stage_graphs = None
-    if not args.no_graph:
+    if not (args.no_graph or gather):
         stage_graphs = []
         for p in range(2):
             g = torch.cuda.CUDAGraph()
@@ -963,6 +1003,11 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
     """One workload's timed block (see the module docstring)."""
     import torch
     layers = build_layers(workload, args.layers, args.fracs, args.tokens)
+    full_layers = layers
+    shard = getattr(args, "shard", False) and world > 1 and workload == "decode"
+    if shard:
+        import tile_sparse_gemm_b200 as tsg
+        layers = shard_layers(full_layers, rank, world, tsg.shard_rows)
     packed = pack_layers(layers, dev, status)
     resident = sum(p.stored_bytes for p in packed)
     full = not (args.layers or args.fracs or args.tokens)
@@ -971,6 +1016,20 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
         # the step as separate patch_gemm calls (the headline), then as one
         # patch_gemm_chain whose calls each wait for the previous one (the same
         # ordering), and as one chain of the independent GEMMs they are
+        if shard:  # one column-parallel shard per rank, the step's Y shards all-gathered once per step
+            import tile_sparse_gemm_b200 as tsg
+            _, _, seg = gather_layout(full_layers, calls, world, tsg.shard_rows)
+            t = time_calls(args, layers, packed, calls, dev, world, status, gather=seg)
+            out = bytes_block(args, workload, full_layers, calls, t, pk, 1)
+            out["scaling"] = "strong"
+            out["step"] = (f"column-parallel: each of {world} ranks multiplies its tile rows of every layer "
+                           "(balanced by stored bytes), then one NCCL all-gather of the step's Y shards")
+            out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (decode, sharded)"
+            out["config"] = {"workload": "LLaMA-2-7B linear layers (decode), column-parallel shards",
+                             "parallelism": f"column-parallel x{world}"}
+            del packed
+            torch.cuda.synchronize()
+            return out
         t = time_calls(args, layers, packed, calls, dev, world, status)
         out = bytes_block(args, workload, layers, calls, t, pk, world, traffic_kind="decode")
         out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (decode" + (
@@ -1074,7 +1133,7 @@ def run_ours(args, rank, world):
     head = results[blocks[0]]
     out = {"metric": head.pop("metric"), "value": head.pop("value"), "unit": head.pop("unit"), "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head.pop("ms_per_step"),
-           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "higher_is_better": True, "scaling": head.pop("scaling", "weak"), "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic"}
     out.update(head)
     if probe:
@@ -1099,6 +1158,9 @@ def main():
     ap.add_argument("--layers", nargs="*", help="profiling: only these projections (q k v o gate up down)")
     ap.add_argument("--fracs", nargs="*", type=float, help="profiling: only these sparse-tile fractions")
     ap.add_argument("--tokens", nargs="*", type=int, help="profiling: only these token counts M")
+    ap.add_argument("--shard", action="store_true",
+                    help="decode under torchrun: each rank multiplies a column-parallel shard of every layer, "
+                         "then one all-gather of Y per step (strong scaling) instead of independent replicas")
     args = ap.parse_args()
     if args.impl == "ours" and args.warmup < 3:
         ap.error("--warmup must be at least 3 (timing rule)")

@@ -91,3 +91,58 @@ def test_two_ranks_concatenate_to_the_whole_layer():
     ref = oracle.hybrid_gemm(x, w, si.tiles_clustered(N, K, 0.5, 15, 0), si.patterns_top2(w))
     for r in range(world):
         assert np.array_equal(out[r], ref)
+
+
+def _bench_rank(rank, world, port, out):
+    """bench.py's sharded decode step on CPU: its shard plan, its gather layout and
+    one all-gather (gloo), with the oracle standing in for each rank's GEMMs."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        import oracle as orc
+        import synth_inputs as s
+        import tile_sparse_gemm_b200 as t
+        layers = []
+        for i, (N, K) in enumerate([(128 * 7, 256), (128 * 3, 384), (128 * 10, 128)]):
+            w = s.gen_w(N, K, 18, i)
+            layers.append(dict(name=f"l{i}", N=N, K=K, w=w, bm=s.tiles_clustered(N, K, 0.5, 18, i),
+                               ids=s.patterns_top2(w), xs={M: s.gen_x(M, K, 18, 10 * i + M) for M in (1, 5)}))
+        calls = bench.calls_of(layers)
+        mine = bench.shard_layers(layers, rank, world, t.shard_rows)
+        offset, sizes, seg = bench.gather_layout(layers, calls, world, t.shard_rows)
+        buf = torch.zeros(seg, dtype=torch.float64)
+        for j, (li, M) in enumerate(calls):
+            L = mine[li]
+            y = orc.hybrid_gemm(L["xs"][M], L["w"], L["bm"], L["ids"])  # this rank's columns
+            assert y.size == sizes[rank][j]
+            buf[offset[rank][j]:offset[rank][j] + y.size] = torch.from_numpy(y.ravel())
+        got = [torch.zeros(seg, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(got, buf)
+        full = []
+        for j, (li, M) in enumerate(calls):
+            parts = [got[r][offset[r][j]:offset[r][j] + sizes[r][j]].numpy().reshape(M, -1) for r in range(world)]
+            full.append(np.concatenate(parts, axis=1))
+        out[rank] = full
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_shard_plan_and_gather_reassemble_every_call():
+    world = 2
+    out = mp.get_context("spawn").Manager().dict()
+    mp.start_processes(_bench_rank, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+    for i, (N, K) in enumerate([(128 * 7, 256), (128 * 3, 384), (128 * 10, 128)]):
+        w = si.gen_w(N, K, 18, i)
+        bm, ids = si.tiles_clustered(N, K, 0.5, 18, i), si.patterns_top2(w)
+        for M in (1, 5):
+            ref = oracle.hybrid_gemm(si.gen_x(M, K, 18, 10 * i + M), w, bm, ids)
+            j = (0 if M == 1 else 3) + i  # calls: every layer at M = 1, then every layer at M = 5
+            for r in range(world):
+                assert np.array_equal(out[r][j], ref)
