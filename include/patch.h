@@ -87,13 +87,15 @@ typedef enum {
     PATCH_ERR_BAD_PATTERN = 6, /* device: pattern id > 5 inside a sparse tile */
     PATCH_ERR_TIMEOUT = 7,     /* device: a bounded wait in a kernel ran out */
     PATCH_ERR_WORKSPACE = 8,   /* workspace pointer null or too small */
-    PATCH_ERR_COUNT = 9        /* device: bitmap's sparse-tile count != n_sparse */
+    PATCH_ERR_COUNT = 9,       /* device: bitmap's sparse-tile count != n_sparse */
+    PATCH_ERR_BOUNDS = 10      /* device: a packed weight breaks the format (patch_check_weight) */
 } patch_status_t;
 
 /* Bits OR-ed into *dev_status by the kernels. */
 #define PATCH_DEV_BAD_PATTERN 0x1
 #define PATCH_DEV_TIMEOUT 0x2
 #define PATCH_DEV_COUNT 0x4
+#define PATCH_DEV_BOUNDS 0x8
 
 /* Path selector of patch_gemm_ex. */
 #define PATCH_PATH_AUTO 0    /* M <= PATCH_DECODE_MAX_M: decode (CUDA-core when N > 524288), else prefill */
@@ -490,9 +492,36 @@ PATCH_API patch_status_t patch_shard_rows(const uint8_t *bitmap, int64_t Tn, int
 PATCH_API patch_status_t patch_mma_probe(int sparse, int64_t iters, int32_t *dev_status, void *stream);
 
 /*
+ * patch_check_weight: check a packed weight's descriptor table against the
+ * packed format on the device ("Core Mechanism": dense tiles whole, 2:4 tiles
+ * as their kept half): every tile's kind is 0 or 1, a sparse tile's ordinal
+ * counts the sparse tiles before it (a dense tile's is 0xFFFFFFFF), every
+ * values offset is the sum of the sizes of the tiles before it, and the table
+ * holds exactly n_sparse sparse tiles.  A weight that passes only indexes
+ * memory inside its blobs in every GEMM path.  A violation ORs
+ * PATCH_DEV_BOUNDS into *dev_status (read it with patch_read_status).  One
+ * launch of one CTA on `stream`; reads only the Tn*Tk descriptors.  Use it on
+ * weights that did not come from patch_pack in this process (loaded from a
+ * file, received from elsewhere).
+ *
+ * Debug build.  The library can also be built with PATCH_DEBUG defined
+ * (libpatch_debug.so: `python -m tile_sparse_gemm_b200.build --debug`).  There
+ * every GEMM entry point (patch_gemm, patch_gemm_ex, patch_gemm_mlp,
+ * patch_gemm_chain, patch_gemm_decode_noalloc) first runs this check on each
+ * weight it is given, synchronises the stream, and returns PATCH_ERR_BOUNDS
+ * without launching the GEMM when a weight fails; the GEMM kernels then only
+ * see indices inside the weight's blobs.  The debug build therefore
+ * synchronises in those calls (it cannot be captured in a CUDA graph), and
+ * patch_gemm_decode_noalloc needs a non-NULL dev_status there.
+ * Errors: PATCH_ERR_INVALID_ARG (NULL), PATCH_ERR_SHAPE, PATCH_ERR_ALIGN,
+ * PATCH_ERR_DEVICE, PATCH_ERR_CUDA.
+ */
+PATCH_API patch_status_t patch_check_weight(const patch_weight *W, int32_t *dev_status, void *stream);
+
+/*
  * patch_read_status: synchronise `stream`, copy *dev_status to *host_bits and
- * return the first error it encodes (PATCH_ERR_TIMEOUT, then BAD_PATTERN,
- * then COUNT) or PATCH_OK.  host_bits may be NULL.
+ * return the first error it encodes (PATCH_ERR_TIMEOUT, then BOUNDS, then
+ * BAD_PATTERN, then COUNT) or PATCH_OK.  host_bits may be NULL.
  */
 PATCH_API patch_status_t patch_read_status(const int32_t *dev_status, void *stream, int32_t *host_bits);
 

@@ -30,9 +30,18 @@ def test_every_declared_symbol_is_exported(lib):
         assert hasattr(lib, n), f"{n} declared in patch.h but not exported"
 
 
+def test_debug_build_exports_the_same_symbols():
+    path = tsg_build.build(debug=True)
+    dbg = ctypes.CDLL(str(path))
+    for n in declared_symbols():
+        assert hasattr(dbg, n), f"{n} declared in patch.h but not exported by the debug build"
+    dbg.patch_version.restype = ctypes.c_char_p
+    assert b"debug" in dbg.patch_version()
+
+
 def test_version_and_strerror(lib):
     assert b"sm_100a" in lib.patch_version()
-    for code in range(10):
+    for code in range(11):
         assert lib.patch_strerror(code)
     assert lib.patch_strerror(99) == b"unknown status"
 

@@ -24,12 +24,15 @@ packed weight in one .npz file (shape, sparse-tile count, the three blobs).
 from __future__ import annotations
 
 import ctypes
+import os
 from dataclasses import dataclass
 from pathlib import Path
 
 import torch
 
-_LIB_PATH = Path(__file__).resolve().parent / "libpatch.so"
+# TSG_DEBUG=1 loads the debug build (every GEMM entry point checks its weights first)
+_LIB_PATH = Path(__file__).resolve().parent / ("libpatch_debug.so" if os.environ.get("TSG_DEBUG") == "1"
+                                               else "libpatch.so")
 
 TILE = 128
 PANEL_BYTES = 16384
@@ -39,8 +42,8 @@ MASK_TILES = (4, 8, 16, 32, 64, 128)  # mask tile sizes patch_hard_mask_tiles ta
 PATCH_OK = 0
 STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_INVALID_ARG", 2: "PATCH_ERR_SHAPE", 3: "PATCH_ERR_ALIGN",
                 4: "PATCH_ERR_DEVICE", 5: "PATCH_ERR_CUDA", 6: "PATCH_ERR_BAD_PATTERN",
-                7: "PATCH_ERR_TIMEOUT", 8: "PATCH_ERR_WORKSPACE", 9: "PATCH_ERR_COUNT"}
-DEV_BAD_PATTERN, DEV_TIMEOUT, DEV_COUNT = 0x1, 0x2, 0x4
+                7: "PATCH_ERR_TIMEOUT", 8: "PATCH_ERR_WORKSPACE", 9: "PATCH_ERR_COUNT", 10: "PATCH_ERR_BOUNDS"}
+DEV_BAD_PATTERN, DEV_TIMEOUT, DEV_COUNT, DEV_BOUNDS = 0x1, 0x2, 0x4, 0x8
 PATH_AUTO, PATH_DECODE, PATH_PREFILL, PATH_DECODE_SIMT, PATH_TEST_STALL = 0, 1, 2, 3, 0x100
 
 
@@ -94,6 +97,7 @@ def lib() -> ctypes.CDLL:
             "patch_gemm_chain_workspace_size": [P, I64, ctypes.POINTER(SZ)],
             "patch_gemm_chain": [P, I64, P, SZ, P, P, ctypes.c_uint64],
             "patch_mma_probe": [I32, I64, P, P],
+            "patch_check_weight": [WP, P, P],
         }
         for name, args in sigs.items():
             f = getattr(L, name)
@@ -176,9 +180,10 @@ def save_packed(weight: PackedWeight, path) -> None:
              values=weight.values.cpu().numpy(), meta=weight.meta.cpu().numpy(), desc=weight.desc.cpu().numpy())
 
 
-def load_packed(path, device="cuda") -> PackedWeight:
+def load_packed(path, device="cuda", check: bool = True) -> PackedWeight:
     """Read a packed weight written by save_packed onto `device`, checking the
-    blob sizes against patch_pack_sizes for its shape and sparse-tile count."""
+    blob sizes against patch_pack_sizes for its shape and sparse-tile count and,
+    with `check` on a CUDA device, its descriptor table (patch_check_weight)."""
     import numpy as np
     with np.load(path) as f:
         if int(f["format"]) != _PACKED_FORMAT:
@@ -191,7 +196,12 @@ def load_packed(path, device="cuda") -> PackedWeight:
             raise ValueError(f"{path}: {k} blob has {b.size} bytes, a packed {N}x{K} weight with "
                              f"{n_sparse} sparse tiles has {sizes[k]}")
     t = {k: torch.from_numpy(b).to(device) for k, b in blobs.items()}
-    return PackedWeight(N, K, n_sparse, t["values"], t["meta"], t["desc"])
+    w = PackedWeight(N, K, n_sparse, t["values"], t["meta"], t["desc"])
+    if check and torch.device(device).type == "cuda":
+        code, bits = patch_read_status(patch_check_weight(w))
+        if code != PATCH_OK:
+            raise PatchError(code, f"{path}: descriptor table")
+    return w
 
 
 def patch_hard_mask(W: torch.Tensor | None, tile_logits: torch.Tensor, pattern_logits: torch.Tensor,
@@ -453,6 +463,16 @@ def patch_mma_probe(sparse: bool, iters: int, status: torch.Tensor | None = None
     status = new_status() if status is None else status
     _check(lib().patch_mma_probe(1 if sparse else 0, iters, _dev(status, "status"), _stream(stream)),
            "patch_mma_probe")
+
+
+def patch_check_weight(weight: PackedWeight, status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Check a packed weight's descriptor table on the device (tile kinds, sparse
+    ordinals, values offsets, sparse-tile count); a violation sets DEV_BOUNDS in
+    the returned status word (read it with patch_read_status)."""
+    status = new_status(weight.desc.device) if status is None else status
+    st = weight.struct()
+    _check(lib().patch_check_weight(ctypes.byref(st), _dev(status, "status"), _stream(stream)), "patch_check_weight")
+    return status
 
 
 def patch_read_status(status: torch.Tensor, stream=None) -> tuple[int, int]:

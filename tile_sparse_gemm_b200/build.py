@@ -2,12 +2,15 @@
 
     python -m tile_sparse_gemm_b200.build          # compile if sources changed
     python -m tile_sparse_gemm_b200.build --force  # always recompile
+    python -m tile_sparse_gemm_b200.build --debug  # libpatch_debug.so: every GEMM entry point
+                                                   # first checks its weights on the device
 """
 from __future__ import annotations
 
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 from pathlib import Path
 
 PKG = Path(__file__).resolve().parent
@@ -15,8 +18,9 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 INCLUDE = ROOT / "include"
 LIB = PKG / "libpatch.so"
+LIB_DEBUG = PKG / "libpatch_debug.so"
 SOURCES = ["capi.cu", "hard_mask.cu", "pack.cu", "gemm_decode.cu", "gemm_decode_tc.cu", "gemm_prefill.cu",
-           "gemm_decode_noalloc.cu", "gated_mlp.cu", "gemm_decode_chain.cu", "mma_probe.cu"]
+           "gemm_decode_noalloc.cu", "gated_mlp.cu", "gemm_decode_chain.cu", "mma_probe.cu", "validate.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]
 
@@ -26,35 +30,39 @@ def _nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def _stale() -> bool:
-    if not LIB.exists():
+def _stale(lib: Path) -> bool:
+    if not lib.exists():
         return True
-    t = LIB.stat().st_mtime
+    t = lib.stat().st_mtime
     deps = [CSRC / s for s in SOURCES] + list(CSRC.glob("*.cuh")) + [INCLUDE / "patch.h"]
     return any(d.stat().st_mtime > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> Path:
-    if not force and not _stale():
-        return LIB
-    objs = []
-    build_dir = PKG / "_build"
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> Path:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not _stale(lib):
+        return lib
+    build_dir = PKG / ("_build_debug" if debug else "_build")
     build_dir.mkdir(exist_ok=True)
-    for src in SOURCES:
+    extra = ["-DPATCH_DEBUG"] if debug else []
+
+    def compile_one(src):
         obj = build_dir / (src + ".o")
-        cmd = [_nvcc(), *NVCC_FLAGS, "-I", str(INCLUDE), "-c", str(CSRC / src), "-o", str(obj)]
+        cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", str(INCLUDE), "-c", str(CSRC / src), "-o", str(obj)]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-        objs.append(str(obj))
-    tmp = LIB.with_suffix(f".so.{os.getpid()}.tmp")
+        return str(obj)
+
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, SOURCES))
+    tmp = lib.with_suffix(f".so.{os.getpid()}.tmp")
     subprocess.run([_nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", str(tmp), *objs,
                     "-lcudart"], check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -37,13 +37,40 @@ static patch_status_t check_weight(const patch_weight* W) {
   return PATCH_OK;
 }
 
+#ifdef PATCH_DEBUG
+// Debug build: check a weight on the device before a GEMM indexes memory with
+// it; synchronises the stream and refuses the call when the check fails.
+static patch_status_t debug_check(const patch_weight* W, int32_t* status, void* stream) {
+  if (!status) return PATCH_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_check_weight(*W, status, s) != cudaSuccess) return PATCH_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PATCH_ERR_CUDA;
+  int32_t bits = 0;
+  if (cudaMemcpy(&bits, status, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess) return PATCH_ERR_CUDA;
+  return (bits & PATCH_DEV_BOUNDS) ? PATCH_ERR_BOUNDS : PATCH_OK;
+}
+#define PATCH_DEBUG_CHECK(W, status, stream)           \
+  do {                                                 \
+    patch_status_t dbg_ = debug_check(W, status, stream); \
+    if (dbg_ != PATCH_OK) return dbg_;                 \
+  } while (0)
+#else
+#define PATCH_DEBUG_CHECK(W, status, stream) \
+  do {                                       \
+  } while (0)
+#endif
+
 }  // namespace patch
 
 using namespace patch;
 
 extern "C" {
 
-const char* patch_version(void) { return "patch-b200 0.1 (sm_100a)"; }
+#ifdef PATCH_DEBUG
+const char* patch_version(void) { return "patch-b200 0.2 (sm_100a, debug: weights checked before every GEMM)"; }
+#else
+const char* patch_version(void) { return "patch-b200 0.2 (sm_100a)"; }
+#endif
 
 const char* patch_strerror(patch_status_t s) {
   switch (s) {
@@ -57,6 +84,7 @@ const char* patch_strerror(patch_status_t s) {
     case PATCH_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
     case PATCH_ERR_WORKSPACE: return "workspace missing or too small";
     case PATCH_ERR_COUNT: return "bitmap's sparse-tile count differs from n_sparse";
+    case PATCH_ERR_BOUNDS: return "packed weight breaks the format (descriptor table)";
   }
   return "unknown status";
 }
@@ -245,6 +273,7 @@ patch_status_t patch_gemm_ex(const uint16_t* X, int64_t M, const patch_weight* W
   int sms = 0;
   st = device_sms(&sms);
   if (st != PATCH_OK) return st;
+  PATCH_DEBUG_CHECK(W, dev_status, stream);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint64_t limit_ns = (wait_limit_us ? wait_limit_us : 2000000ull) * 1000ull;
   cudaError_t e;
@@ -324,6 +353,7 @@ patch_status_t patch_gemm_chain(const patch_chain_call* calls, int64_t n_calls, 
   const int64_t n = int64_t(cs.size());
   if (!workspace || !aligned16(workspace) || workspace_bytes < chain_workspace_bytes(cs.data(), n, sms))
     return PATCH_ERR_WORKSPACE;
+  for (int64_t j = 0; j < n; ++j) PATCH_DEBUG_CHECK(&cs[j].W, dev_status, stream);
   const uint64_t limit_ns = (wait_limit_us ? wait_limit_us : 2000000ull) * 1000ull;
   for (int64_t j0 = 0; j0 < n;) {
     const int64_t j1 = chain_launch_end(cs.data(), j0, n);
@@ -368,6 +398,8 @@ patch_status_t patch_gemm_mlp(const uint16_t* X, int64_t M, const patch_weight* 
   int sms = 0;
   st = device_sms(&sms);
   if (st != PATCH_OK) return st;
+  PATCH_DEBUG_CHECK(W_gate, dev_status, stream);
+  PATCH_DEBUG_CHECK(W_up, dev_status, stream);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint64_t limit_ns = 2000000ull * 1000ull;
   if (M > PATCH_DECODE_MAX_M) {
@@ -438,6 +470,17 @@ patch_status_t patch_mma_probe(int sparse, int64_t iters, int32_t* dev_status, v
              : PATCH_ERR_CUDA;
 }
 
+patch_status_t patch_check_weight(const patch_weight* W, int32_t* dev_status, void* stream) {
+  if (!dev_status) return PATCH_ERR_INVALID_ARG;
+  patch_status_t st = check_weight(W);
+  if (st != PATCH_OK) return st;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  return launch_check_weight(*W, dev_status, static_cast<cudaStream_t>(stream)) == cudaSuccess ? PATCH_OK
+                                                                                                : PATCH_ERR_CUDA;
+}
+
 patch_status_t patch_read_status(const int32_t* dev_status, void* stream, int32_t* host_bits) {
   if (!dev_status) return PATCH_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -446,6 +489,7 @@ patch_status_t patch_read_status(const int32_t* dev_status, void* stream, int32_
   if (cudaMemcpy(&bits, dev_status, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess) return PATCH_ERR_CUDA;
   if (host_bits) *host_bits = bits;
   if (bits & PATCH_DEV_TIMEOUT) return PATCH_ERR_TIMEOUT;
+  if (bits & PATCH_DEV_BOUNDS) return PATCH_ERR_BOUNDS;
   if (bits & PATCH_DEV_BAD_PATTERN) return PATCH_ERR_BAD_PATTERN;
   if (bits & PATCH_DEV_COUNT) return PATCH_ERR_COUNT;
   return PATCH_OK;

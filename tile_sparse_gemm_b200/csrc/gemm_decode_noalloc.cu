@@ -49,7 +49,7 @@ using namespace patch;
 
 extern "C" patch_status_t patch_gemm_decode_noalloc(const uint16_t* X, int64_t M, const patch_weight* W,
                                                    uint16_t* Y, int32_t* dev_status, void* stream) {
-  (void)dev_status;  // nothing on this path reports through the status word
+  (void)dev_status;  // nothing on this path's kernels reports through the status word
   if (M < 0 || M > PATCH_DECODE_MAX_M || !W) return PATCH_ERR_INVALID_ARG;
   if (!W->values || !W->desc || (W->n_sparse > 0 && !W->meta)) return PATCH_ERR_INVALID_ARG;
   if (W->N <= 0 || W->K <= 0 || W->N % kTile || W->K % kTile) return PATCH_ERR_SHAPE;
@@ -69,6 +69,18 @@ extern "C" patch_status_t patch_gemm_decode_noalloc(const uint16_t* X, int64_t M
   if (major != 10) return PATCH_ERR_DEVICE;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return PATCH_ERR_CUDA;
 
+#ifdef PATCH_DEBUG
+  // debug build: the weight is checked on the device (needs the status word) before use
+  if (!dev_status) return PATCH_ERR_INVALID_ARG;
+  {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_check_weight(*W, dev_status, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+      return PATCH_ERR_CUDA;
+    int32_t bits = 0;
+    if (cudaMemcpy(&bits, dev_status, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess) return PATCH_ERR_CUDA;
+    if (bits & PATCH_DEV_BOUNDS) return PATCH_ERR_BOUNDS;
+  }
+#endif
   // the built-in buffer must hold the split-K partials of this problem
   const DecodePlan plan = decode_plan(M, W->N, W->K, sms);
   if (plan.ws_bytes > PATCH_NOALLOC_SCRATCH_BYTES) return PATCH_ERR_WORKSPACE;

@@ -83,6 +83,9 @@ cudaError_t launch_chain(const patch_chain_call* calls, int64_t j0, int64_t j1, 
                          int num_sms, uint64_t limit_ns, cudaStream_t stream);
 constexpr int64_t kChainMaxTileRows = int64_t(kDecodeCounterBytes / 16) - 1;  // 4 counters per row + 2 words
 
+// Device check of a packed weight's descriptor table (patch_check_weight).
+cudaError_t launch_check_weight(const patch_weight& W, int32_t* status, cudaStream_t stream);
+
 // Tensor-core MMA rate probe (patch_mma_probe).
 cudaError_t launch_mma_probe(int sparse, int64_t iters, int num_sms, uint64_t limit_ns, int32_t* status,
                              cudaStream_t stream);
