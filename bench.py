@@ -930,8 +930,11 @@ def bytes_block(args, name, layers, calls, t, pk, world, segments=None, seg_name
     seg_bytes = np.array([alg[lo:hi].sum() for lo, hi in segments])
     split = split_of(t, seg_bytes, args.steps)
     achieved = float(alg.sum() / 1e9 / (split.sum() / 1e3))
-    traffic = measured_traffic(traffic_kind, [f"{layers[li]['name']}@M={M}" for li, M in calls]) \
-        if traffic_kind else None
+    traffic = None
+    if traffic_kind == "chain":  # one launch per step: its DRAM bytes, if captured for this workload
+        traffic = measured_traffic("chain", ["+".join(f"{layers[li]['name']}@M={M}" for li, M in calls)])
+    elif traffic_kind:
+        traffic = measured_traffic(traffic_kind, [f"{layers[li]['name']}@M={M}" for li, M in calls])
     out = block_common(args, t, alg.sum() / 1e9, "GB/s", world)
     out["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                        "frac": round(achieved / pk["hbm_gbs"], 4),
@@ -1013,44 +1016,28 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
     full = not (args.layers or args.fracs or args.tokens)
     if workload in ("decode", "decode_fused"):
         calls = calls_of(layers)
-        # the step as separate patch_gemm calls (the headline), then as one
-        # patch_gemm_chain whose calls each wait for the previous one (the same
-        # ordering), and as one chain of the independent GEMMs they are
-        if shard:  # one column-parallel shard per rank, the step's Y shards all-gathered once per step
-            import tile_sparse_gemm_b200 as tsg
-            _, _, seg = gather_layout(full_layers, calls, world, tsg.shard_rows)
-            t = time_calls(args, layers, packed, calls, dev, world, status, gather=seg)
-            out = bytes_block(args, workload, full_layers, calls, t, pk, 1)
-            out["scaling"] = "strong"
-            out["step"] = (f"column-parallel: each of {world} ranks multiplies its tile rows of every layer "
-                           "(balanced by stored bytes), then one NCCL all-gather of the step's Y shards")
-            out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (decode, sharded)"
-            out["config"] = {"workload": "LLaMA-2-7B linear layers (decode), column-parallel shards",
-                             "parallelism": f"column-parallel x{world}"}
-            del packed
-            torch.cuda.synchronize()
-            return out
-        t = time_calls(args, layers, packed, calls, dev, world, status)
-        out = bytes_block(args, workload, layers, calls, t, pk, world, traffic_kind="decode")
+        # the step's 21 GEMMs are independent (every X is an input of the step):
+        # the headline runs them as one patch_gemm_chain in which none waits for
+        # another, so the CTAs split the whole step's panel sequence; beside it the
+        # same GEMMs as separate patch_gemm calls (each kernel waits for the one
+        # before it) and as a chain whose calls wait for each other
+        t = time_calls(args, layers, packed, calls, dev, world, status, chain=True, after=False)
+        out = bytes_block(args, workload, layers, calls, t, pk, world, segments=[(0, len(calls))],
+                          seg_names=["step"], traffic_kind="chain", chain=True)
         out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (decode" + (
             ", fused q|k|v and gate|up projections)" if workload == "decode_fused" else ")")
-        out["step"] = ("one patch_gemm call per GEMM on one stream (programmatic dependent launch: each "
-                       "waits for the previous one before reading its X), captured in one CUDA graph")
-        for key, after, what in (("chain", True, "each waiting for the previous one's completion before reading "
-                                                 "its X"),
-                                 ("chain_independent", False, "the step's GEMMs are independent (every X is an "
-                                                              "input of the step), so none waits")):
-            t = time_calls(args, layers, packed, calls, dev, world, status, chain=True, after=after)
-            out[key] = bytes_block(args, workload, layers, calls, t, pk, world, segments=[(0, len(calls))],
-                                   seg_names=["step"], chain=True)
-            out[key]["step"] = "one patch_gemm_chain launch over the step's calls, " + what
-        out["config"] = {"workload": f"LLaMA-2-7B linear layers ({workload})",
-                         "shapes": [f"{L['name']}:{L['N']}x{L['K']}" for L in layers],
-                         "tokens": sorted({M for _, M in calls}),
-                         "sparse_tile_fraction": sorted({L["frac"] for L in layers}),
-                         "resident_weight_bytes": resident,
-                         "l2": f"inputs larger than L2: {resident / 2**20:.0f} MiB of packed weights read in rotation",
-                         "parallelism": f"replicas x{world}"}
+        out["step"] = ("the step's GEMMs (independent: every X is an input of the step) as one patch_gemm_chain "
+                       "launch in which no call waits for another: the CTAs split the step's whole panel sequence")
+        t = time_calls(args, layers, packed, calls, dev, world, status)
+        out["separate_calls"] = bytes_block(args, workload, layers, calls, t, pk, world, traffic_kind="decode")
+        out["separate_calls"]["step"] = ("one patch_gemm call per GEMM on one stream (programmatic dependent "
+                                         "launch: each waits for the previous one before reading its X), "
+                                         "captured in one CUDA graph")
+        t = time_calls(args, layers, packed, calls, dev, world, status, chain=True, after=True)
+        out["chain_dependent"] = bytes_block(args, workload, layers, calls, t, pk, world,
+                                             segments=[(0, len(calls))], seg_names=["step"], chain=True)
+        out["chain_dependent"]["step"] = ("one patch_gemm_chain launch whose calls each wait for the previous "
+                                          "one's completion before reading their X")
         if workload == "decode" and full:
             out["offline"] = offline_steps(layers, dev, pk)
     elif workload == "prefill":
@@ -1084,6 +1071,12 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
         out["chain"] = dict(ch, step="per pass (M = 1, then M = 8) patch_gemm_chain over the 224 layers in order, "
                                      "each call waiting for the previous one (64 calls per launch)")
         out["chain"]["ms_per_pass"] = {n: v["us"] / 1e3 for n, v in ch["per_segment"].items()}
+        t = time_calls(args, layers, packed, calls, dev, world, status, segments=segments, chain=True, after=False)
+        ch = bytes_block(args, workload, layers, calls, t, pk, world, segments, names, chain=True)
+        out["chain_independent"] = dict(ch, step="per pass patch_gemm_chain over the 224 layers' GEMMs as the "
+                                                 "independent GEMMs they are here (no call waits; each launch's "
+                                                 "CTAs split its whole panel sequence)")
+        out["chain_independent"]["ms_per_pass"] = {n: v["us"] / 1e3 for n, v in ch["per_segment"].items()}
         out["ms_per_pass"] = {n: v["us"] / 1e3 for n, v in out["per_segment"].items()}
         out["stored_gb_per_pass"] = round(sum(p.stored_bytes for p in packed) / 1e9, 3)
         out["config"] = {"workload": "32-layer LLaMA-2-7B linear stack, 7 projections per layer, run in order",

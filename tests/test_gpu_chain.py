@@ -62,6 +62,32 @@ def test_independent_calls_mixed_shapes_and_tokens():
         assert np.array_equal(a, bits_of(b))
 
 
+def test_calls_that_wait_for_none_split_the_whole_launch():
+    """With no call waiting for another the CTAs split the launch's whole panel
+    sequence (runs cross call boundaries; small calls fall inside one CTA's run;
+    only the rows at the ends of each run are cut)."""
+    specs = [(128, 896, 0.5, 3), (4096, 4096, 0.5, 16), (256, 128, 1.0, 1), (11008, 512, 0.5, 5),
+             (128, 128, 0.0, 2), (1024, 2048, 0.75, 8), (896, 4864, 0.5, 16), (128, 256, 0.5, 1)]
+    calls, refs = [], []
+    for idx, (N, K, f, M) in enumerate(specs):
+        w, bm, ids, pw = layer(N, K, f, 80 + idx, clustered=(idx % 3 == 0))
+        x = si.gen_x(M, K, CFG, 800 + idx)
+        calls.append((to_dev_bf16(x), pw, None, False))
+        refs.append(oracle.hybrid_gemm(x, w, bm, ids))
+    ch = tsg.Chain(calls)
+    first = None
+    for _ in range(2):
+        ys = ch.run()
+        assert tsg.patch_read_status(ch.status)[0] == 0
+        got = [bits_of(y) for y in ys]
+        for (N, K, f, M), y, ref in zip(specs, got, refs):
+            check_gemm(y, ref, f"global split {N}x{K} f={f} M={M}")
+        if first is not None:
+            for a_, b_ in zip(first, got):
+                assert np.array_equal(a_, b_)
+        first = got
+
+
 def test_dependent_calls_read_the_previous_output():
     # x0 -> L0 (4096 x 2048) -> L1 (1024 x 4096) -> L2 (4096 x 1024) -> L3 (2048 x 4096)
     shapes = [(4096, 2048, 0.5), (1024, 4096, 0.25), (4096, 1024, 0.75), (2048, 4096, 0.5)]
@@ -133,9 +159,11 @@ def test_workspace_shared_with_patch_gemm_and_zero_token_calls():
     assert tsg.patch_read_status(status)[0] == 0
 
 
-def test_llama2_decode_step_as_one_chain():
-    """The benchmark's decode step: 7 LLaMA-2-7B layers x M = 1, 4, 16, each call
-    waiting for the previous one; every output checked."""
+@pytest.mark.parametrize("after", [True, False])
+def test_llama2_decode_step_as_one_chain(after):
+    """The benchmark's decode step: 7 LLaMA-2-7B layers x M = 1, 4, 16 as one chain,
+    each call waiting for the previous one, or none waiting (the split of the
+    whole step's panel sequence the benchmark's headline runs); every output checked."""
     calls, refs = [], []
     packs = {}
     for idx, (name, N, K) in enumerate(si.LLAMA2_7B):
@@ -147,7 +175,7 @@ def test_llama2_decode_step_as_one_chain():
         for idx, (name, N, K) in enumerate(si.LLAMA2_7B):
             w, bm, ids, pw = packs[idx]
             x = si.gen_x(M, K, 2, idx)
-            calls.append((to_dev_bf16(x), pw, None, True))
+            calls.append((to_dev_bf16(x), pw, None, after))
             refs.append((f"{name}@M={M}", x, w, bm, ids))
     ch = tsg.Chain(calls)
     ys = ch.run()

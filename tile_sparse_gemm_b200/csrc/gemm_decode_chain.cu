@@ -102,6 +102,7 @@ struct Call {
   int M, N, Tk, Tn;
   uint32_t ctr_base;  // this call's row counters: counters[ctr_base + 4 tn + q]
   int after;          // read X only after every earlier call of the launch has completed
+  int64_t off;        // first panel of the call in the launch's panel sequence (global split)
 };
 
 struct Args {
@@ -111,6 +112,8 @@ struct Args {
   float* part;         // [PART_RING][G][2][128][16] fp32 partials
   uint64_t limit_ns;
   int32_t* status;
+  int global;    // 1: no call waits for another; CTAs split the launch's whole panel sequence
+  int64_t Ptot;  // panels of all calls
 };
 
 struct Maps {
@@ -131,6 +134,23 @@ __device__ __forceinline__ void cta_range(int64_t c, int64_t P, int64_t G, int64
   const int64_t Ga = active_ctas(P, G);
   p0 = c < Ga ? range_begin(c, P, Ga) : P;
   p1 = c < Ga ? range_begin(c + 1, P, Ga) : P;
+}
+// Panel range [p0, p1) of CTA c in call j: its share of the call (per-call
+// split), or, when no call waits for another, the part of call j inside the
+// CTA's share of the whole launch's panel sequence (global split: a CTA then
+// streams one contiguous run of panels across call boundaries, and only the
+// rows at the two ends of its run are cut).  Empty ranges are [P, P).
+__device__ __forceinline__ void call_range(const Args& a, int j, int64_t c, int64_t G, int64_t& p0, int64_t& p1) {
+  const Call& cl = a.call[j];
+  if (!a.global) {
+    cta_range(c, cl.P, G, p0, p1);
+    return;
+  }
+  int64_t g0, g1;
+  cta_range(c, a.Ptot, G, g0, g1);
+  const int64_t lo = g0 > cl.off ? g0 : cl.off, hi = g1 < cl.off + cl.P ? g1 : cl.off + cl.P;
+  p0 = lo < hi ? lo - cl.off : cl.P;
+  p1 = lo < hi ? hi - cl.off : cl.P;
 }
 __device__ __forceinline__ int64_t panel_of(const patch_tile_desc& d) {
   return int64_t(d.val_offset / PATCH_PANEL_BYTES);
@@ -221,7 +241,7 @@ __device__ void producer_w(Shared& s, const Maps& maps, const Args& a) {
   for (int j = 0; ok && j < a.J; ++j) {
     const Call& cl = a.call[j];
     int64_t p0, p1;
-    cta_range(c, cl.P, G, p0, p1);
+    call_range(a, j, c, G, p0, p1);
     for (int64_t p = p0; p < p1; ++p, ++i) {
       const uint32_t st = i % NS;
       if (!(ok = wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false)))
@@ -246,24 +266,45 @@ __device__ __forceinline__ void load_x(Stage& g, uint64_t* full, const CUtensorM
   }
 }
 
-// Stage the panel records [p0, p1) of call j in shared memory buffer j & 1
-// (when they fit; otherwise the producer reads them from global memory).  The
-// bulk copy starts at the even record q0 <= p0 and covers whole 16-byte units
-// (a call's records are padded to an even count), so record p sits at p - q0.
-__device__ __forceinline__ void stage_records(Shared& s, const Args& a, int j) {
+// The X producer's panel records, staged in shared memory in chunks of at
+// most RECBUF records (a run of one call's panels), one chunk ahead, in two
+// buffers.  A chunk's bulk copy starts at the even record q0 <= its first
+// panel and covers whole 16-byte units (a call's records are padded to an
+// even count), so record p sits at p - q0 of its buffer.
+struct ChunkIter {
+  int j;          // call (a.J: past the end)
+  int64_t p, p1;  // the chunk's first panel; end of the CTA's range in call j
+};
+
+__device__ __forceinline__ void chunk_first(const Args& a, ChunkIter& it) {
   const int64_t G = gridDim.x, c = blockIdx.x;
-  const Call& cl = a.call[j];
-  int64_t p0, p1;
-  cta_range(c, cl.P, G, p0, p1);
-  uint64_t* bar = &s.rec_full[j & 1];
-  if (p1 > p0 && p1 - p0 <= RECBUF) {
-    const int64_t q0 = p0 & ~int64_t(1);
-    const uint32_t bytes = uint32_t(((p1 - q0) * 8 + 15) & ~int64_t(15));  // <= (RECBUF + 2) * 8
-    mbar_expect_tx(bar, bytes);
-    bulk_load(s.rec[j & 1], cl.rec + q0, bytes, bar);
-  } else {
-    mbar_arrive(bar);
+  for (it.j = 0; it.j < a.J; ++it.j) {
+    int64_t p0;
+    call_range(a, it.j, c, G, p0, it.p1);
+    it.p = p0;
+    if (p0 < it.p1) return;
   }
+}
+
+__device__ __forceinline__ void chunk_next(const Args& a, ChunkIter& it) {
+  const int64_t G = gridDim.x, c = blockIdx.x;
+  it.p += RECBUF;
+  if (it.p < it.p1) return;
+  for (++it.j; it.j < a.J; ++it.j) {
+    int64_t p0;
+    call_range(a, it.j, c, G, p0, it.p1);
+    it.p = p0;
+    if (p0 < it.p1) return;
+  }
+}
+
+__device__ __forceinline__ void stage_chunk(Shared& s, const Args& a, const ChunkIter& it, uint32_t k) {
+  const Call& cl = a.call[it.j];
+  const int64_t e = it.p + RECBUF < it.p1 ? it.p + RECBUF : it.p1;
+  const int64_t q0 = it.p & ~int64_t(1);
+  const uint32_t bytes = uint32_t(((e - q0) * 8 + 15) & ~int64_t(15));  // <= (RECBUF + 2) * 8
+  mbar_expect_tx(&s.rec_full[k & 1], bytes);
+  bulk_load(s.rec[k & 1], cl.rec + q0, bytes, &s.rec_full[k & 1]);
 }
 
 // X producer: per panel its record (tile, half, kind), the stage's info word,
@@ -274,25 +315,32 @@ __device__ void producer_x(Shared& s, const Maps& maps, const Args& a) {
   const int64_t G = gridDim.x, c = blockIdx.x;
   uint32_t i = 0;
   bool ok = true;
-  int staged_calls = 0, waited_calls = 0;  // record copies issued / waited for
-  if (a.J > 0) stage_records(s, a, staged_calls++);
-  for (int j = 0; ok && j < a.J; ++j) {
+  uint32_t staged = 0, waited = 0;  // record chunks copied / waited for; chunk n uses buffer n & 1
+  ChunkIter cur;
+  chunk_first(a, cur);
+  if (cur.j < a.J) stage_chunk(s, a, cur, staged++);
+  while (ok && cur.j < a.J) {
+    // stage the chunk after this one into the other buffer (it held the chunk before, which is done)
+    ChunkIter nxt = cur;
+    chunk_next(a, nxt);
+    if (nxt.j < a.J) stage_chunk(s, a, nxt, staged++);
+    if (!(ok = wait_bounded(&s.rec_full[waited & 1], (waited >> 1) & 1, &s.abort_flag, a.limit_ns, a.status, false)))
+      break;
+    const uint2* recs = s.rec[waited & 1];
+    ++waited;
+    const int j = cur.j;
     const Call& cl = a.call[j];
-    int64_t p0, p1;
-    cta_range(c, cl.P, G, p0, p1);
-    if (j + 1 < a.J) stage_records(s, a, staged_calls++);  // buffer (j+1)&1 held call j-1's, which is done
-    // the records' bulk copy completes a phase even when nothing is staged
-    if (!(ok = wait_bounded(&s.rec_full[j & 1], (j >> 1) & 1, &s.abort_flag, a.limit_ns, a.status, false))) break;
-    ++waited_calls;
-    const bool staged = p1 - p0 <= RECBUF;
-    const int64_t q0 = p0 & ~int64_t(1);  // first staged record
+    int64_t p0, p1;  // the CTA's whole range in call j (segment boundaries); the chunk is [cb, ce)
+    call_range(a, j, c, G, p0, p1);
+    const int64_t cb = cur.p, ce = cur.p + RECBUF < cur.p1 ? cur.p + RECBUF : cur.p1;
+    const int64_t q0 = cb & ~int64_t(1);
     const uint32_t xb = uint32_t(cl.M) * 128;  // an X slice holds M token rows
-    bool dep_ok = !cl.after || j == 0;
-    for (int64_t p = p0; p < p1; ++p, ++i) {
+    bool dep_ok = !cl.after || j == 0 || cb > p0;  // waited for at the call's first chunk
+    for (int64_t p = cb; p < ce; ++p, ++i) {
       const uint32_t st = i % NS;
       if (!(ok = wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false)))
         break;
-      const uint2 r = staged ? s.rec[j & 1][p - q0] : cl.rec[p];
+      const uint2 r = recs[p - q0];
       const int t = int(r.x), kt = t % cl.Tk, h = int(r.y & 1u);
       const bool sparse = (r.y >> 1) & 1u;
       uint32_t info = sparse ? INFO_SPARSE : 0u;
@@ -315,9 +363,10 @@ __device__ void producer_x(Shared& s, const Maps& maps, const Args& a) {
       if (sparse) bulk_load(s.st[st].e, cl.meta + uint64_t(r.y >> 2) * E_BYTES, E_BYTES, &s.full[st]);
       load_x(s.st[st], &s.full[st], &maps.x[j], kt, h, sparse);
     }
+    cur = nxt;
   }
   // every copy issued must have landed before the CTA may exit
-  for (int k = waited_calls; k < staged_calls; ++k)
+  for (uint32_t k = waited; k < staged; ++k)
     wait_bounded(&s.rec_full[k & 1], (k >> 1) & 1, &s.abort_flag, drain_limit(a), a.status, true);
   for (uint32_t k = (i > NS ? i - NS : 0); k < i; ++k)
     wait_bounded(&s.full[k % NS], (k / NS) & 1, &s.abort_flag, drain_limit(a), a.status, true);
@@ -335,7 +384,7 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& a, int u) {
   for (int j = 0; ok && j < a.J; ++j) {
     const Call& cl = a.call[j];
     int64_t p0, p1;
-    cta_range(c, cl.P, G, p0, p1);
+    call_range(a, j, c, G, p0, p1);
     for (int64_t p = p0; p < p1; ++p, ++i) {
       const uint32_t st = i % NS;
       if (!(ok = wait_bounded(&s.full[st], (i / NS) & 1, &s.abort_flag, a.limit_ns, a.status, false))) break;
@@ -422,11 +471,13 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a) {
   const int64_t G = gridDim.x, c = blockIdx.x;
   const bool leader = warp == 2 && lane == 0;
   uint32_t seg = 0;
-  bool ok = true;
+  bool ok = true, seen = false;
   for (int j = 0; j < a.J; ++j) {
     const Call& cl = a.call[j];
     int64_t p0, p1;
-    cta_range(c, cl.P, G, p0, p1);
+    call_range(a, j, c, G, p0, p1);
+    const bool first_call = p1 > p0 && !seen;  // the call holding the CTA's first segment
+    seen = seen || p1 > p0;
     if (ok && p1 > p0) {
       // the CTA's first and last panel records and the boundaries of the rows they lie in
       const uint2 r0 = __ldcg(cl.rec + p0), r1 = __ldcg(cl.rec + p1 - 1);
@@ -446,8 +497,10 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a) {
         row_hi[0] = row_start(tn_last);
         row_hi[1] = row_start(tn_last + 1);
       }
-      float* ring = a.part + int64_t(j % PART_RING) * G * WS_FLOATS_PER_CTA;
-      bool guard_done = j < PART_RING;  // partial buffer j % 4 last served call j - 4
+      // per-call split: partial buffer j % 4, which last served call j - 4; global
+      // split: one buffer (a CTA cuts only its first and last segment of the launch)
+      float* ring = a.part + (a.global ? 0 : int64_t(j % PART_RING) * G * WS_FLOATS_PER_CTA);
+      bool guard_done = a.global || j < PART_RING;
       for (int tn = tn_first; tn <= tn_last; ++tn, ++seg) {
         const uint32_t buf = seg % NACC;
         if (!(ok = wait_bounded(&s.acc_full[buf], (seg / NACC) & 1, &s.abort_flag, a.limit_ns, a.status, false)))
@@ -472,17 +525,19 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a) {
           if (!(ok = wait_calls_done(a, s, j - PART_RING, uint32_t(G)))) break;
           guard_done = true;
         }
-        float4* mine = reinterpret_cast<float4*>(ring + c * WS_FLOATS_PER_CTA + (tn == tn_first ? 0 : BT * BM) +
-                                                 r * BT);
+        const bool first_seg = tn == tn_first && (!a.global || first_call);
+        float4* mine = reinterpret_cast<float4*>(ring + c * WS_FLOATS_PER_CTA + (first_seg ? 0 : BT * BM) + r * BT);
 #pragma unroll
         for (int k = 0; k < BT / 4; ++k)
           if (4 * k < cl.M)
             mine[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
                                   __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
-        const int64_t rb = tn == tn_first ? row_lo[0] : row_hi[0];
-        const int64_t re = tn == tn_first ? row_lo[1] : row_hi[1];
-        const int64_t Ga = active_ctas(cl.P, G);
-        const int64_t c_lo = cta_of_panel(rb, cl.P, Ga), c_hi = cta_of_panel(re - 1, cl.P, Ga);
+        // the row's panels in the split's index space (the call's, or the launch's)
+        const int64_t base = a.global ? cl.off : 0, Pspace = a.global ? a.Ptot : cl.P;
+        const int64_t rb = base + (tn == tn_first ? row_lo[0] : row_hi[0]);
+        const int64_t re = base + (tn == tn_first ? row_lo[1] : row_hi[1]);
+        const int64_t Ga = active_ctas(Pspace, G);
+        const int64_t c_lo = cta_of_panel(rb, Pspace, Ga), c_hi = cta_of_panel(re - 1, Pspace, Ga);
         uint32_t* counter = a.counters + cl.ctr_base + 4 * tn + q;
         __syncwarp();
         uint32_t old = 0;
@@ -490,7 +545,7 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a) {
         old = __shfl_sync(0xFFFFFFFFu, old, 0);
         if (old != uint32_t(c_hi - c_lo)) continue;
         __syncwarp();
-        const int slot_lo = range_begin(c_lo, cl.P, Ga) < rb ? 1 : 0;
+        const int slot_lo = range_begin(c_lo, Pspace, Ga) < rb ? 1 : 0;
         const int nv = (cl.M + 3) / 4;
         float sum[BT];
         if (nv <= 2)
@@ -635,6 +690,8 @@ cudaError_t launch_chain(const patch_chain_call* calls, int64_t j0, int64_t j1, 
   Args args;
   PlanArgs pa;
   uint32_t ctr = uint32_t(J + 1);
+  int64_t rec_off_panels = 0;  // the calls' panels, one after another
+  bool any_after = false;
   int64_t tiles = 0, rec_off = 0;
   for (int j = 0; j < J; ++j) {
     const patch_chain_call& cl = calls[j0 + j];
@@ -654,7 +711,10 @@ cudaError_t launch_chain(const patch_chain_call* calls, int64_t j0, int64_t j1, 
     c.Tk = int(g.Tk);
     c.Tn = int(g.Tn);
     c.ctr_base = ctr;
-    c.after = cl.after_previous ? 1 : 0;
+    c.after = cl.after_previous && j > 0 ? 1 : 0;  // the launch's first call never waits
+    c.off = rec_off_panels;
+    rec_off_panels += g.P;
+    any_after = any_after || c.after;
     ctr += uint32_t(4 * g.Tn);
     pa.desc[j] = cl.W.desc;
     pa.rec[j] = rec + rec_off;
@@ -667,6 +727,9 @@ cudaError_t launch_chain(const patch_chain_call* calls, int64_t j0, int64_t j1, 
   args.part = reinterpret_cast<float*>(ws + kDecodeCounterBytes);
   args.limit_ns = limit_ns;
   args.status = status;
+  // when no call waits for another, the CTAs split the whole panel sequence
+  args.global = any_after ? 0 : 1;
+  args.Ptot = rec_off_panels;
   pa.J = J;
 
   int plan_blocks = int((tiles + 255) / 256);
