@@ -1038,6 +1038,13 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
                                              segments=[(0, len(calls))], seg_names=["step"], chain=True)
         out["chain_dependent"]["step"] = ("one patch_gemm_chain launch whose calls each wait for the previous "
                                           "one's completion before reading their X")
+        out["config"] = {"workload": f"LLaMA-2-7B linear layers ({workload})",
+                         "shapes": [f"{L['name']}:{L['N']}x{L['K']}" for L in layers],
+                         "tokens": sorted({M for _, M in calls}),
+                         "sparse_tile_fraction": sorted({L["frac"] for L in layers}),
+                         "resident_weight_bytes": resident,
+                         "l2": f"inputs larger than L2: {resident / 2**20:.0f} MiB of packed weights read in rotation",
+                         "parallelism": f"replicas x{world}"}
         if workload == "decode" and full:
             out["offline"] = offline_steps(layers, dev, pk)
     elif workload == "prefill":

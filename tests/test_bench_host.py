@@ -110,3 +110,68 @@ def test_flops_block_and_monotonic_sweep():
 
 def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(2.0, 5, 4, 1000.0) == 2.0 * 5 * 4
+
+
+def test_run_ours_assembles_every_block_on_fake_timings(monkeypatch):
+    """The default run's JSON assembly (every block and mode) on CPU: GPU work is
+    replaced by fakes that return fixed timings, so a missing or misnamed key in
+    any block fails here rather than on the GPU machine."""
+    import types
+
+    import torch
+
+    class FakePacked:
+        def __init__(self, L):
+            self.stored_bytes = bench.stored_bytes(L["N"], L["K"], int(L["bm"].sum()))
+
+    def fake_time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False, after=True,
+                        gather=None):
+        segs = segments or ([(0, len(calls))] if chain else [(j, j + 1) for j in range(len(calls))])
+        return {"ms": 1.0 * args.steps, "e2e_ms": 2.0 * args.steps, "seg_ms": None, "clocks": {"sm_mhz": 1965.0},
+                "h2d": 1, "d2h": 1, "launches": len(segs)}
+
+    monkeypatch.setattr(bench, "pack_layers", lambda layers, dev, status: [FakePacked(L) for L in layers])
+    monkeypatch.setattr(bench, "time_calls", fake_time_calls)
+    monkeypatch.setattr(bench, "offline_steps", lambda layers, dev, pk: {})
+    monkeypatch.setattr(bench, "mlp_steps", lambda dev, pk: {})
+    monkeypatch.setattr(bench, "mma_rates", lambda dev: {"sparse_over_dense": 1.5})
+    monkeypatch.setattr(bench, "build_layers", lambda w, *a: bench_small_layers(w))
+    monkeypatch.setattr(torch.cuda, "set_device", lambda d: None)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    monkeypatch.setattr(torch.cuda, "empty_cache", lambda: None)
+    import tile_sparse_gemm_b200 as tsg
+    monkeypatch.setattr(tsg, "new_status", lambda dev=None: None)
+    args = types.SimpleNamespace(steps=4, warmup=3, no_graph=False, layers=None, fracs=None, tokens=None,
+                                 shard=False, workload="all")
+    out = bench.run_ours(args, 0, 1)
+    for key in ("metric", "value", "unit", "ms_per_step", "roofline", "e2e", "clocks", "config", "gpu_launches",
+                "separate_calls", "chain_dependent", "prefill", "stack", "llama3_qwen", "mma_probe"):
+        assert key in out, key
+    assert out["config"]["blocks"] == list(bench.BLOCKS)
+    assert out["prefill"]["roofline"]["frac_measured_sparse_peak"] > 0 and "sweep" in out["prefill"]
+    for key in ("chain", "chain_independent"):
+        assert "ms_per_pass" in out["stack"][key]
+    assert set(out["llama3_qwen"]) >= {"M=1", "M=512"}
+    import json
+    json.dumps(out)  # serialisable
+
+
+def bench_small_layers(workload):
+    """Small stand-ins for each workload's layers (shapes, bitmaps and X only)."""
+    rng = np.random.default_rng(0)
+
+    def L(name, N, K, frac, ms, **kw):
+        T = (N // 128) * (K // 128)
+        bm = np.zeros(T, np.uint8)
+        bm[:si.exact_sparse_count(T, frac)] = 1
+        return dict(name=name, N=N, K=K, bm=bm.reshape(N // 128, K // 128), frac=frac,
+                    xs={M: np.zeros((M, K), np.uint16) for M in ms}, **kw)
+    if workload in ("decode", "decode_fused"):
+        return [L(n, 256, 256, 0.5, (1, 4, 16)) for n in ("q", "gate")]
+    if workload == "prefill":
+        return [L(n, 256, 256, f, (2048,)) for n in ("q", "down") for f in bench.FRACS]
+    if workload == "stack":
+        return [L(f"L{i}.{n}", 256, 256, 0.1, (1, 8), proj=n) for i in range(2) for n in ("q", "down")]
+    if workload == "llama3_qwen":
+        return [L(n, 256, 128, 0.5, (1, 512)) for n in ("llama3.q", "qwen.k")]
+    raise ValueError(workload)
