@@ -936,11 +936,13 @@ def bytes_block(args, name, layers, calls, t, pk, world, segments=None, seg_name
     elif traffic_kind:
         traffic = measured_traffic(traffic_kind, [f"{layers[li]['name']}@M={M}" for li, M in calls])
     out = block_common(args, t, alg.sum() / 1e9, "GB/s", world)
+    # a chain launch covers up to 64 calls of a segment, a separate call one
+    launches = sum((hi - lo + 63) // 64 for lo, hi in segments) if chain else len(calls)
     out["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                        "frac": round(achieved / pk["hbm_gbs"], 4),
                        "traffic": None if traffic is None else round(traffic),
                        "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
-                       "algorithmic_bytes_per_launch": round(float(alg.mean())),
+                       "algorithmic_bytes_per_launch": round(float(alg.sum()) / launches),
                        "kernel": kernel, "peak_source": pk["source"]}
     out["per_segment" if len(segments) != len(calls) else "per_call"] = {
         n: {"us": round(1e3 * split[s], 2), "GB/s": round(seg_bytes[s] / 1e9 / (split[s] / 1e3), 1)}
