@@ -48,12 +48,18 @@ def _load():
             "oracle_unpack": [P, P, P, I64, I64, P],
             "oracle_gemm_rows": [P, I64, P, I64, P, I64, I64, P],
             "oracle_hybrid_gemm": [P, I64, P, I64, P, I64, I64, P, P, P],
+            "oracle_apply_mask_tiles": [P, I64, I64, I64, P, P, P],
+            "oracle_exec_tiles_e": [P, I64, I64, I64, I64, P, P],
+            "oracle_pack64": [P, I64, I64, P, P, I64, P, P, P],
+            "oracle_unpack64": [P, P, P, I64, I64, P],
         }.items():
             f = getattr(lib, name)
             f.argtypes = args
             f.restype = ctypes.c_int
         lib.oracle_pack_sizes.argtypes = [I64, I64, I64, P, P, P]
         lib.oracle_pack_sizes.restype = None
+        lib.oracle_pack64_sizes.argtypes = [I64, I64, I64, P, P, P]
+        lib.oracle_pack64_sizes.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
@@ -160,6 +166,63 @@ def unpack(values: np.ndarray, meta: np.ndarray, desc: np.ndarray, N: int, K: in
     meta = np.ascontiguousarray(meta, np.uint8) if meta.size else np.zeros(1, np.uint8)
     _check(_load().oracle_unpack(_ptr(np.ascontiguousarray(values, np.uint8)), _ptr(meta),
                                  _ptr(np.ascontiguousarray(desc, np.uint8)), N, K, _ptr(out)), "unpack")
+    return out
+
+
+# ---- 64 x 64 execution tiles ("Ablation Studies", tile size)
+
+TILE64 = 64
+
+
+def apply_mask_tiles(w: np.ndarray, bitmap: np.ndarray, pat_id: np.ndarray, mask_tile: int) -> np.ndarray:
+    """The hybrid mask with b x b tiles (bitmap [N/b][K/b]) applied to W."""
+    w = np.ascontiguousarray(w, np.uint16)
+    N, K = w.shape
+    out = np.empty_like(w)
+    _check(_load().oracle_apply_mask_tiles(_ptr(w), N, K, int(mask_tile),
+                                           _ptr(np.ascontiguousarray(bitmap, np.uint8)),
+                                           _ptr(np.ascontiguousarray(pat_id, np.uint8)), _ptr(out)),
+           "apply_mask_tiles")
+    return out
+
+
+def exec_tiles_e(bitmap: np.ndarray, N: int, K: int, mask_tile: int, exec_tile: int):
+    """E x E execution tiles (E = 64 or 128) of a b x b mask bitmap: (exec [N/E][K/E] u8, n_sparse)."""
+    bitmap = np.ascontiguousarray(bitmap, np.uint8)
+    E = int(exec_tile)
+    ex = np.empty((N // E, K // E), np.uint8)
+    n = ctypes.c_int64()
+    _check(_load().oracle_exec_tiles_e(_ptr(bitmap), N, K, int(mask_tile), E, _ptr(ex), ctypes.byref(n)),
+           "exec_tiles_e")
+    return ex, n.value
+
+
+def pack64_sizes(N: int, K: int, n_sparse: int):
+    v, m, d = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    _load().oracle_pack64_sizes(N, K, n_sparse, ctypes.byref(v), ctypes.byref(m), ctypes.byref(d))
+    return v.value, m.value, d.value
+
+
+def pack64(w: np.ndarray, bitmap: np.ndarray, pat_id: np.ndarray):
+    """Blobs (values, meta, desc) of the 64 x 64 execution-tile format; bitmap [N/64][K/64]."""
+    w = np.ascontiguousarray(w, np.uint16)
+    N, K = w.shape
+    bitmap = np.ascontiguousarray(bitmap, np.uint8)
+    ns = int(np.count_nonzero(bitmap))
+    vb, mb, db = pack64_sizes(N, K, ns)
+    values = np.zeros(vb, np.uint8)
+    meta = np.zeros(max(mb, 1), np.uint8)
+    desc = np.zeros(db, np.uint8)
+    _check(_load().oracle_pack64(_ptr(w), N, K, _ptr(bitmap), _ptr(np.ascontiguousarray(pat_id, np.uint8)),
+                                 ns, _ptr(values), _ptr(meta), _ptr(desc)), "pack64")
+    return values, meta[:mb], desc
+
+
+def unpack64(values: np.ndarray, meta: np.ndarray, desc: np.ndarray, N: int, K: int) -> np.ndarray:
+    out = np.empty((N, K), np.uint16)
+    meta = np.ascontiguousarray(meta, np.uint8) if meta.size else np.zeros(1, np.uint8)
+    _check(_load().oracle_unpack64(_ptr(np.ascontiguousarray(values, np.uint8)), _ptr(meta),
+                                   _ptr(np.ascontiguousarray(desc, np.uint8)), N, K, _ptr(out)), "unpack64")
     return out
 
 

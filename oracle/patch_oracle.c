@@ -48,6 +48,9 @@
  * that the execution tile stays 128 x 128 and runs sparse only when all its
  * mask tiles are sparse.
  *
+ * The 64 x 64 execution-tile format (oracle_*64, oracle_exec_tiles_e,
+ * oracle_apply_mask_tiles) is described above its functions near the end.
+ *
  * Parity pins (tests/test_oracle.py): brute force over the 6 patterns with
  * one-hot logits, argmax ties, the exactly-2-of-4 invariant, global sparsity
  * = 0.5 x sparse-tile fraction, all-dense == numpy dense matmul, all-sparse
@@ -379,6 +382,186 @@ int oracle_hybrid_gemm(const uint16_t *X, int64_t M, const int64_t *rows, int64_
         rc = oracle_gemm_rows(X, M, rows, n_rows, W_eff, N, K, Y);
     free(W_eff);
     return rc;
+}
+
+/*
+ * 64 x 64 execution tiles ("Ablation Studies", tile size: smaller tiles give
+ * finer control over where the 2:4 pattern applies; larger ones run more
+ * efficiently on the hardware).  The library's second packed format runs the
+ * same hybrid layer on 64 x 64 execution tiles:
+ *   - Tiles 64 x 64 in row-major tile order t = tn*(K/64) + tk; N and K are
+ *     multiples of 64.  Descriptors as in the 128 x 128 format.
+ *   - Values blob: "panels" of 64 rows x 32 bf16 stored row major (64-byte
+ *     rows, 4096 bytes).  A dense tile occupies 2 panels (k 0..31, then
+ *     k 32..63); a sparse tile 1 panel in which row r holds, for each group
+ *     g = 0..15, its two kept values in ascending k at positions 2g, 2g+1.
+ *   - Metadata blob: 512 bytes per sparse tile at ordinal*512; the 4-bit
+ *     code of group g of tile row r sits in nibble (g & 1) of byte
+ *        ((g>>1)&1) | ((r>>3)&1)<<1 | (g>>3)<<2 | (r&7)<<3
+ *        | ((g>>2)&1)<<6 | (r>>4)<<7 .
+ * Mask tiles b x b with b <= E (E = 64 or 128) map to execution tiles by the
+ * same rule as for 128: an execution tile is sparse only when every mask
+ * tile inside it is sparse.
+ */
+#define TILE64 64
+
+static int shape64_ok(int64_t N, int64_t K)
+{
+    return N > 0 && K > 0 && N % TILE64 == 0 && K % TILE64 == 0;
+}
+
+/* The hybrid mask with b x b tiles applied to W (b = 4..128, N and K multiples of b). */
+int oracle_apply_mask_tiles(const uint16_t *W, int64_t N, int64_t K, int64_t b, const uint8_t *bitmap,
+                            const uint8_t *pat_id, uint16_t *W_eff)
+{
+    if (!mask_tile_ok(b) || N <= 0 || K <= 0 || N % b != 0 || K % b != 0)
+        return ERR_SHAPE;
+    int64_t Tkb = K / b;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            int keep = 1;
+            if (bitmap[(n / b) * Tkb + k / b]) {
+                int id = pat_id[n * (K / 4) + k / 4];
+                if (id > 5)
+                    return ERR_BAD_PATTERN;
+                int pos = (int)(k % 4);
+                keep = pos == KEEP[id][0] || pos == KEEP[id][1];
+            }
+            W_eff[n * K + k] = keep ? W[n * K + k] : (uint16_t)0x0000;
+        }
+    }
+    return OK;
+}
+
+/* Execution tiles of size E (64 or 128) of a b x b mask bitmap (b <= E):
+ * exec [N/E][K/E], sparse only when all its mask tiles are sparse. */
+int oracle_exec_tiles_e(const uint8_t *bitmap, int64_t N, int64_t K, int64_t b, int64_t E, uint8_t *exec,
+                        int64_t *n_sparse)
+{
+    if ((E != 64 && E != 128) || !mask_tile_ok(b) || b > E || N <= 0 || K <= 0 || N % E != 0 ||
+        K % E != 0)
+        return ERR_SHAPE;
+    int64_t Tn = N / E, Tk = K / E, Tkb = K / b, r = E / b;
+    int64_t count = 0;
+    for (int64_t tn = 0; tn < Tn; ++tn) {
+        for (int64_t tk = 0; tk < Tk; ++tk) {
+            int all_sparse = 1;
+            for (int64_t i = 0; i < r; ++i)
+                for (int64_t j = 0; j < r; ++j)
+                    if (!bitmap[(tn * r + i) * Tkb + tk * r + j])
+                        all_sparse = 0;
+            exec[tn * Tk + tk] = (uint8_t)all_sparse;
+            count += all_sparse;
+        }
+    }
+    *n_sparse = count;
+    return OK;
+}
+
+/* Byte of a 64 x 64 tile's 512-byte metadata block that holds group g (0..15) of row r (0..63). */
+static int64_t meta64_byte(int r, int g)
+{
+    return (int64_t)(((g >> 1) & 1) | (((r >> 3) & 1) << 1) | ((g >> 3) << 2) | ((r & 7) << 3) |
+                     (((g >> 2) & 1) << 6) | ((r >> 4) << 7));
+}
+
+void oracle_pack64_sizes(int64_t N, int64_t K, int64_t n_sparse, int64_t *values_bytes, int64_t *meta_bytes,
+                         int64_t *desc_bytes)
+{
+    int64_t T = (N / TILE64) * (K / TILE64);
+    *values_bytes = (T - n_sparse) * 8192 + n_sparse * 4096;
+    *meta_bytes = n_sparse * 512;
+    *desc_bytes = T * 16;
+}
+
+/* Pack W into the 64 x 64 format under an execution bitmap [N/64][K/64] and pattern ids. */
+int oracle_pack64(const uint16_t *W, int64_t N, int64_t K, const uint8_t *bitmap, const uint8_t *pat_id,
+                  int64_t n_sparse, uint8_t *values, uint8_t *meta, uint8_t *desc)
+{
+    if (!shape64_ok(N, K))
+        return ERR_SHAPE;
+    int64_t Tn = N / TILE64, Tk = K / TILE64;
+    int64_t counted = 0;
+    for (int64_t t = 0; t < Tn * Tk; ++t)
+        counted += bitmap[t] != 0;
+    if (counted != n_sparse)
+        return ERR_COUNT;
+    memset(meta, 0, (size_t)(n_sparse * 512));
+
+    uint64_t offset = 0;
+    uint32_t ordinal = 0;
+    for (int64_t tn = 0; tn < Tn; ++tn) {
+        for (int64_t tk = 0; tk < Tk; ++tk) {
+            uint8_t *d = desc + 16 * (tn * Tk + tk);
+            uint16_t *panel = (uint16_t *)(values + offset);
+            int sparse = bitmap[tn * Tk + tk] != 0;
+            put_u32(d, (uint32_t)sparse);
+            put_u32(d + 4, sparse ? ordinal : 0xFFFFFFFFu);
+            put_u64(d + 8, offset);
+            if (!sparse) {
+                for (int h = 0; h < 2; ++h)
+                    for (int r = 0; r < TILE64; ++r)
+                        for (int c = 0; c < 32; ++c)
+                            panel[h * TILE64 * 32 + r * 32 + c] =
+                                W[(tn * TILE64 + r) * K + tk * TILE64 + h * 32 + c];
+                offset += 8192;
+            } else {
+                uint8_t *mb = meta + (int64_t)ordinal * 512;
+                for (int r = 0; r < TILE64; ++r) {
+                    int64_t n = tn * TILE64 + r;
+                    for (int g = 0; g < 16; ++g) {
+                        int64_t k0 = tk * TILE64 + 4 * g;
+                        int id = pat_id[n * (K / 4) + k0 / 4];
+                        if (id > 5)
+                            return ERR_BAD_PATTERN;
+                        int i0 = KEEP[id][0], i1 = KEEP[id][1];
+                        panel[r * 32 + 2 * g] = W[n * K + k0 + i0];
+                        panel[r * 32 + 2 * g + 1] = W[n * K + k0 + i1];
+                        uint8_t code = (uint8_t)(i0 | (i1 << 2));
+                        mb[meta64_byte(r, g)] |= (uint8_t)(code << (4 * (g & 1)));
+                    }
+                }
+                offset += 4096;
+                ordinal += 1;
+            }
+        }
+    }
+    return OK;
+}
+
+/* Rebuild the effective W from a 64 x 64 packed blob, by its own decoding. */
+int oracle_unpack64(const uint8_t *values, const uint8_t *meta, const uint8_t *desc, int64_t N, int64_t K,
+                    uint16_t *W_eff)
+{
+    if (!shape64_ok(N, K))
+        return ERR_SHAPE;
+    int64_t Tn = N / TILE64, Tk = K / TILE64;
+    for (int64_t tn = 0; tn < Tn; ++tn) {
+        for (int64_t tk = 0; tk < Tk; ++tk) {
+            const uint8_t *d = desc + 16 * (tn * Tk + tk);
+            uint32_t kind = get_u32(d), ordinal = get_u32(d + 4);
+            const uint16_t *panel = (const uint16_t *)(values + get_u64(d + 8));
+            for (int r = 0; r < TILE64; ++r) {
+                int64_t n = tn * TILE64 + r;
+                uint16_t *row = W_eff + n * K + tk * TILE64;
+                if (kind == 0) {
+                    for (int c = 0; c < TILE64; ++c)
+                        row[c] = panel[(c / 32) * TILE64 * 32 + r * 32 + (c % 32)];
+                } else {
+                    const uint8_t *mb = meta + (int64_t)ordinal * 512;
+                    for (int g = 0; g < 16; ++g) {
+                        int code = (mb[meta64_byte(r, g)] >> (4 * (g & 1))) & 0xF;
+                        int i0 = code & 3, i1 = code >> 2;
+                        for (int i = 0; i < 4; ++i)
+                            row[4 * g + i] = 0;
+                        row[4 * g + i0] = panel[r * 32 + 2 * g];
+                        row[4 * g + i1] = panel[r * 32 + 2 * g + 1];
+                    }
+                }
+            }
+        }
+    }
+    return OK;
 }
 
 int oracle_num_threads(void)

@@ -626,3 +626,216 @@ def test_fine_mask_packs_and_multiplies_as_the_masked_weight(b):
     x = si.gen_x(M, K, 7, b)
     y = oracle.gemm(x, oracle.unpack(v, m, d, N, K))
     assert np.allclose(y, f64(x) @ f64(wm).T, rtol=1e-12, atol=1e-12)
+
+
+# ---- 64 x 64 execution tiles ("Ablation Studies", tile size): the second packed format
+
+T64 = 64
+
+
+def spec_values_blob64(w, bm, ids, offs):
+    """The 64 x 64 values blob, restated from the format text: a dense tile is
+    2 panels (k 0..31, then 32..63) of 64 rows x 32 values with 64-byte rows;
+    a sparse tile one panel whose row r holds group g's kept pair at 2g, 2g+1."""
+    N, K = w.shape
+    Tn, Tk = N // T64, K // T64
+    size = sum(8192 if not bm[t // Tk, t % Tk] else 4096 for t in range(Tn * Tk))
+    blob = np.zeros(size // 2, np.uint16)
+    for tn in range(Tn):
+        for tk in range(Tk):
+            o = int(offs[tn * Tk + tk]) // 2
+            tile = w[tn * T64:(tn + 1) * T64, tk * T64:(tk + 1) * T64]
+            if not bm[tn, tk]:
+                for h in range(2):
+                    blob[o + 2048 * h:o + 2048 * (h + 1)] = tile[:, 32 * h:32 * (h + 1)].reshape(-1)
+            else:
+                for r in range(T64):
+                    for g in range(16):
+                        a, b = PAIRS[ids[tn * T64 + r, tk * 16 + g]]
+                        blob[o + r * 32 + 2 * g] = tile[r, 4 * g + a]
+                        blob[o + r * 32 + 2 * g + 1] = tile[r, 4 * g + b]
+    return blob.view(np.uint8)
+
+
+def test_pack64_values_blob_against_the_format_text():
+    N, K = 2 * T64, 3 * T64
+    w = np.arange(N * K, dtype=np.uint32).astype(np.uint16).reshape(N, K)  # distinct bit patterns
+    assert len(np.unique(w)) == N * K
+    ids = np.random.default_rng(17).integers(0, 6, size=(N, K // 4)).astype(np.uint8)
+    for bm in (np.array([[0, 1, 0], [1, 0, 1]], np.uint8), np.array([[1, 1, 0], [0, 0, 1]], np.uint8),
+               np.zeros((2, 3), np.uint8), np.ones((2, 3), np.uint8)):
+        values, meta, desc = oracle.pack64(w, bm, ids)
+        d = desc.reshape(-1, 16)
+        kinds = d[:, 0:4].copy().view("<u4").ravel()
+        ords = d[:, 4:8].copy().view("<u4").ravel()
+        offs = d[:, 8:16].copy().view("<u8").ravel()
+        assert np.array_equal(kinds, bm.ravel())
+        sizes = np.where(bm.ravel() == 1, 4096, 8192)
+        assert np.array_equal(offs, np.concatenate([[0], np.cumsum(sizes)[:-1]]))
+        assert np.array_equal(ords[bm.ravel() == 1], np.arange(int(bm.sum())))
+        assert np.all(ords[bm.ravel() == 0] == 0xFFFFFFFF)
+        assert values.size == int(sizes.sum()) and meta.size == 512 * int(bm.sum())
+        assert np.array_equal(values, spec_values_blob64(w, bm, ids, offs)), bm.tolist()
+    # bytes spelled out for bm [[0,1,0],[1,0,1]]: dense tile (0,0), panel 1, row 3, value 5 is W[3][32+5]
+    bm = np.array([[0, 1, 0], [1, 0, 1]], np.uint8)
+    values, _, _ = oracle.pack64(w, bm, ids)
+    v16 = values.view(np.uint16)
+    assert v16[(4096 + 3 * 64 + 5 * 2) // 2] == w[3, 37]
+    # sparse tile (0,1) starts after the 8 KiB dense tile; row 7, group 9 keeps PAIRS[id]
+    a, b = PAIRS[ids[7, 16 + 9]]
+    assert v16[(8192 + 7 * 64 + 9 * 4) // 2] == w[7, 64 + 36 + a]
+    assert v16[(8192 + 7 * 64 + 9 * 4 + 2) // 2] == w[7, 64 + 36 + b]
+
+
+def hw_meta64_position(r, g):
+    """Byte and nibble of group g of row r in a 64 x 64 tile's metadata block,
+    restated from where the 16-bit sparse MMA with M = 64 reads it in tensor
+    memory: lane = r%8 + 8*((k//16)%2) + 32*(r//16) (the first 16 lanes of each
+    32-lane subpartition), 32-bit column = k//32, byte in column =
+    (k%16)//8 + 2*((r//8)%2), nibble = (k//4)%2, with k = 4g; the block stores
+    the two columns of lane L at bytes 128*(L//32) + 8*(L%32) .. +7 (a 32-lane,
+    2-column store per subpartition moves it without reshuffling)."""
+    k = 4 * g
+    lane = r % 8 + 8 * ((k // 16) % 2) + 32 * (r // 16)
+    col = k // 32
+    byte = (k % 16) // 8 + 2 * ((r // 8) % 2)
+    return 128 * (lane // 32) + 8 * (lane % 32) + 4 * col + byte, (k // 4) % 2
+
+
+def test_metadata64_layout_positions():
+    w = np.full((T64, T64), ONE, np.uint16)
+    bm = np.ones((1, 1), np.uint8)
+    seen = set()
+    for r in range(T64):
+        for g in range(16):
+            ids = np.zeros((T64, T64 // 4), np.uint8)  # code 0x4 everywhere
+            ids[r, g] = 5                               # code 0xE at one group
+            _, meta, _ = oracle.pack64(w, bm, ids)
+            byte, nib = hw_meta64_position(r, g)
+            assert (meta[byte] >> (4 * nib)) & 0xF == 0xE
+            others = meta.copy()
+            others[byte] &= ~np.uint8(0xF << (4 * nib))
+            others[byte] |= np.uint8(0x4 << (4 * nib))
+            assert np.all(others == 0x44)
+            seen.add((byte, nib))
+    assert len(seen) == 1024  # a bijection onto the 512 bytes x 2 nibbles
+
+
+def test_pattern_codes64_against_golden():
+    w = np.full((T64, T64), ONE, np.uint16)
+    bm = np.ones((1, 1), np.uint8)
+    for pid, a, b, code in golden_codes():
+        _, meta, _ = oracle.pack64(w, bm, np.full((T64, T64 // 4), pid, np.uint8))
+        assert meta.size == 512 and np.all(meta == (code | (code << 4)))
+
+
+def test_pack64_sizes_follow_the_blobs():
+    for N, K, ns in ((64, 64, 0), (64, 64, 1), (192, 320, 7), (4096, 4096, 2048)):
+        v, m, d = oracle.pack64_sizes(N, K, ns)
+        T = (N // 64) * (K // 64)
+        assert (v, m, d) == ((T - ns) * 2 * 4096 + ns * 4096, ns * 512, 16 * T)
+
+
+@pytest.mark.parametrize("frac", [0.0, 0.3, 1.0])
+def test_pack64_unpack64_round_trip(frac):
+    N, K = 3 * T64, 5 * T64
+    w = si.gen_w(N, K, 3, int(frac * 10))
+    rng = np.random.default_rng(int(frac * 10))
+    bm = (rng.random((N // T64, K // T64)) < frac).astype(np.uint8)
+    ids = rng.integers(0, 6, (N, K // 4)).astype(np.uint8)
+    v, m, d = oracle.pack64(w, bm, ids)
+    wm = oracle.apply_mask_tiles(w, bm, ids, 64)
+    assert np.array_equal(oracle.unpack64(v, m, d, N, K), wm)
+    # packing the already-masked weight gives the same blobs (pruned values are never stored)
+    v2, m2, d2 = oracle.pack64(wm, bm, ids)
+    assert np.array_equal(v, v2) and np.array_equal(m, m2) and np.array_equal(d, d2)
+
+
+def test_apply_mask_tiles_at_128_is_apply_mask_and_agrees_with_hard_mask_tiles():
+    N, K = 2 * TILE, 2 * TILE
+    w = si.gen_w(N, K, 4, 2)
+    rng = np.random.default_rng(21)
+    ids = rng.integers(0, 6, (N, K // 4)).astype(np.uint8)
+    bm = rng.integers(0, 2, (N // TILE, K // TILE)).astype(np.uint8)
+    assert np.array_equal(oracle.apply_mask_tiles(w, bm, ids, 128), oracle.apply_mask(w, bm, ids))
+    for b in (4, 16, 64):
+        tl = rng.standard_normal((N // b, K // b, 2)).astype(np.float32)
+        pl = rng.standard_normal((N, K // 4, 6)).astype(np.float32)
+        wm, bmb, pid = oracle.hard_mask_tiles(w, tl, pl, b)
+        assert np.array_equal(oracle.apply_mask_tiles(w, bmb, pid, b), wm)
+
+
+def test_exec_tiles_e_at_128_is_exec_tiles():
+    rng = np.random.default_rng(5)
+    for b in MASK_TILES:
+        bm = (rng.random((2 * TILE // b, 3 * TILE // b)) < 0.9).astype(np.uint8)
+        ex, n = oracle.exec_tiles_e(bm, 2 * TILE, 3 * TILE, b, 128)
+        ex0, n0 = oracle.exec_tiles(bm, 2 * TILE, 3 * TILE, b)
+        assert np.array_equal(ex, ex0) and n == n0
+
+
+@pytest.mark.parametrize("b", [4, 8, 16, 32, 64])
+def test_exec_tiles64_is_all_of_its_mask_tiles(b):
+    """Brute force with numpy: the 64 x 64 execution tile is sparse iff all of
+    its (64/b)^2 mask tiles are; at b = 64 it is the bitmap itself."""
+    N, K = 3 * T64, 2 * T64
+    rng = np.random.default_rng(40 + b)
+    bm = (rng.random((N // b, K // b)) < 0.85).astype(np.uint8)
+    r = T64 // b
+    want = bm.reshape(N // T64, r, K // T64, r).all(axis=(1, 3)).astype(np.uint8)
+    ex, n = oracle.exec_tiles_e(bm, N, K, b, 64)
+    assert np.array_equal(ex, want) and n == int(want.sum())
+    if b == 64:
+        assert np.array_equal(ex, bm)
+
+
+def test_exec_tiles64_with_one_dense_4x4_tile():
+    N = K = 2 * T64
+    r = T64 // 4
+    for (i, j) in [(0, 0), (r - 1, r), (2 * r - 1, 2 * r - 1)]:
+        bm = np.ones((N // 4, K // 4), np.uint8)
+        bm[i, j] = 0
+        ex, n = oracle.exec_tiles_e(bm, N, K, 4, 64)
+        want = np.ones((2, 2), np.uint8)
+        want[i // r, j // r] = 0
+        assert np.array_equal(ex, want) and n == 3
+
+
+def test_gemm64_all_dense_and_all_sparse_are_numpy_matmuls():
+    """All-dense 64-tiles multiply as numpy's dense matmul; all-sparse ones as
+    numpy's matmul of W with the 2:4 keep-mask built from the itertools pairs."""
+    N, K, M = 2 * T64, 3 * T64, 5
+    w = si.gen_w(N, K, 6, 0)
+    x = si.gen_x(M, K, 6, 0)
+    ids = np.random.default_rng(9).integers(0, 6, (N, K // 4)).astype(np.uint8)
+    v, m, d = oracle.pack64(w, np.zeros((N // T64, K // T64), np.uint8), ids)
+    assert np.allclose(oracle.gemm(x, oracle.unpack64(v, m, d, N, K)), f64(x) @ f64(w).T, rtol=1e-12, atol=1e-12)
+    v, m, d = oracle.pack64(w, np.ones((N // T64, K // T64), np.uint8), ids)
+    pos = np.arange(K) % 4
+    a = np.array([[PAIRS[i][0] for i in row] for row in ids]).repeat(4, axis=1)
+    b = np.array([[PAIRS[i][1] for i in row] for row in ids]).repeat(4, axis=1)
+    keep = (pos[None, :] == a) | (pos[None, :] == b)
+    w24 = np.where(keep, f64(w), 0.0)
+    y = oracle.gemm(x, oracle.unpack64(v, m, d, N, K))
+    assert np.allclose(y, f64(x) @ w24.T, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("b", [4, 32, 64])
+def test_fine_mask_packs64_as_the_masked_weight(b):
+    """At b <= 64 the 64 x 64 format keeps every all-sparse 64-tile sparse
+    (at b = 64, every sparse mask tile) and still unpacks to W_masked."""
+    N, K = 2 * TILE, 2 * TILE
+    w = si.gen_w(N, K, 8, b)
+    rng = np.random.default_rng(60 + b)
+    tl = np.zeros((N // b, K // b, 2), np.float32)
+    tl[..., 1] = 1.0
+    tl[: N // (2 * b), : K // (2 * b), 1] = rng.choice([1.0, -1.0], (N // (2 * b), K // (2 * b)))
+    pl = rng.standard_normal((N, K // 4, 6)).astype(np.float32)
+    wm, bm, pid = oracle.hard_mask_tiles(w, tl, pl, b)
+    ex, ns = oracle.exec_tiles_e(bm, N, K, b, 64)
+    ex128, ns128 = oracle.exec_tiles(bm, N, K, b)
+    assert ns >= 4 * ns128  # a sparse 128-tile is four sparse 64-tiles
+    if b == 64:
+        assert ns == int(bm.sum())
+    v, m, d = oracle.pack64(wm, ex, pid)
+    assert np.array_equal(oracle.unpack64(v, m, d, N, K), wm)
