@@ -519,6 +519,131 @@ PATCH_API patch_status_t patch_mma_probe(int sparse, int64_t iters, int32_t *dev
 PATCH_API patch_status_t patch_check_weight(const patch_weight *W, int32_t *dev_status, void *stream);
 
 /*
+ * ---- 64 x 64 execution tiles ("Experimental Results", "Ablation Studies",
+ * tile size: finer tiles give more control over where the 2:4 pattern
+ * applies, and with 128 x 128 masks every tile still runs on the hardware's
+ * efficient path).  A second packed format that executes 64 x 64 tiles, with
+ * its own calls, so that a mask of 64 x 64 tiles (or finer) keeps every
+ * sparse 64-tile sparse instead of only the 128-tiles whose four quarters
+ * are all sparse.  The hybrid layer it computes is the same; the GEMM runs
+ * M = 64 tensor-core MMAs (dense kind::f16 K = 16, and the 2:4 sparse form
+ * K = 32), which this GPU executes at half the FLOP rate of the M = 128
+ * forms for dense tiles (patch_mma_probe_m measures both).
+ *
+ * Format (this library's specification):
+ *   - Tiles of 64 x 64 in row-major tile order t = tn*(K/64) + tk; N and K
+ *     multiples of 64.  Descriptors as for the 128 x 128 format
+ *     (patch_tile_desc: kind, sparse ordinal, byte offset of the first panel).
+ *   - Values blob: panels of 64 rows x 32 bf16, row major with 64-byte rows
+ *     (4096 bytes).  A dense tile occupies 2 panels (the tile's k 0..31, then
+ *     k 32..63); a sparse tile 1 panel in which row r holds, for each group
+ *     g = 0..15, its two kept values in ascending k at positions 2g, 2g+1.
+ *   - Metadata blob: 512 bytes per sparse tile at sparse_ordinal*512.  Group
+ *     g of row r has the 4-bit code i0 | (i1 << 2) in the low nibble of its
+ *     byte when g is even, the high nibble when g is odd; the byte is
+ *         ((g>>1)&1) | ((r>>3)&1)<<1 | (g>>3)<<2 | (r&7)<<3
+ *         | ((g>>2)&1)<<6 | (r>>4)<<7.
+ *     This is the tensor-memory placement the 16-bit sparse MMA with M = 64
+ *     reads (rows 16q..16q+15 in the first 16 lanes of lane quarter q, one
+ *     32-bit column per K = 32 step), stored 8 bytes per lane so that each
+ *     quarter's 128 bytes move with one 32-lane, 2-column tensor-memory store.
+ *   - All blobs 16-byte aligned.
+ */
+#define PATCH_TILE64 64
+#define PATCH_PANEL64_BYTES 4096
+#define PATCH_DENSE_TILE64_BYTES 8192
+#define PATCH_SPARSE_TILE64_BYTES 4096
+#define PATCH_META_TILE64_BYTES 512
+
+/* A weight packed in the 64 x 64 format (host struct of device pointers, owned by the caller). */
+typedef struct {
+    int64_t N, K;                /* logical shape of W (multiples of 64) */
+    int64_t n_sparse;            /* number of sparse 64 x 64 tiles */
+    const void *values;          /* values blob, patch_pack64_sizes bytes */
+    const void *meta;            /* metadata blob (may be NULL when n_sparse == 0) */
+    const patch_tile_desc *desc; /* (N/64)*(K/64) descriptors */
+} patch_weight64;
+
+/*
+ * patch_pack64_sizes: blob sizes of the 64 x 64 format (host only):
+ *   values = (T - n_sparse)*8192 + n_sparse*4096, meta = n_sparse*512,
+ *   desc = 16*T with T = (N/64)*(K/64).
+ * Errors: PATCH_ERR_SHAPE (N, K not positive multiples of 64, or > 2^31);
+ * PATCH_ERR_INVALID_ARG (n_sparse outside [0, T], NULL output).
+ */
+PATCH_API patch_status_t patch_pack64_sizes(int64_t N, int64_t K, int64_t n_sparse, size_t *values_bytes,
+                                            size_t *meta_bytes, size_t *desc_bytes);
+
+/*
+ * patch_exec_tiles64: the 64 x 64 execution tiles of a b x b mask (b =
+ * mask_tile in {4, 8, 16, 32, 64}): exec[tn][tk] = 1 only when all (64/b)^2
+ * mask tiles inside it are sparse (at b = 64 the bitmap itself).
+ *   bitmap u8 [N/b][K/b]; exec u8 [N/64][K/64] out; n_sparse one int64 on the
+ *   DEVICE out (8-byte aligned), zeroed on the stream and then counted.
+ * Errors: PATCH_ERR_INVALID_ARG (NULL, mask_tile), PATCH_ERR_SHAPE,
+ * PATCH_ERR_ALIGN, PATCH_ERR_DEVICE, PATCH_ERR_CUDA.
+ */
+PATCH_API patch_status_t patch_exec_tiles64(const uint8_t *bitmap, int64_t N, int64_t K, int64_t mask_tile,
+                                            uint8_t *exec, int64_t *n_sparse, void *stream);
+
+/*
+ * patch_pack64: build the 64 x 64 format from W, an execution bitmap
+ * [N/64][K/64] (nonzero = sparse) and pattern ids u8 [N][K/4] (read only in
+ * sparse tiles).  As for patch_pack: only kept positions of sparse tiles are
+ * read (W masked or not gives the same blobs); n_sparse must equal the
+ * bitmap's count (PATCH_DEV_COUNT otherwise, nothing written past the blob
+ * sizes); an id > 5 sets PATCH_DEV_BAD_PATTERN and is packed as id 0.
+ * values/meta/desc sized by patch_pack64_sizes.  Two launches (scan, tiles).
+ * Errors: PATCH_ERR_INVALID_ARG, PATCH_ERR_SHAPE, PATCH_ERR_ALIGN (W, blobs
+ * 16-byte aligned), PATCH_ERR_DEVICE, PATCH_ERR_CUDA.
+ */
+PATCH_API patch_status_t patch_pack64(const uint16_t *W, int64_t N, int64_t K, const uint8_t *bitmap,
+                                      const uint8_t *pat_id, int64_t n_sparse, void *values, void *meta,
+                                      patch_tile_desc *desc, int32_t *dev_status, void *stream);
+
+/*
+ * patch_gemm64_workspace_size: device scratch bytes patch_gemm64 needs for M
+ * rows of X and this weight (host only; queries the SM count).
+ */
+PATCH_API patch_status_t patch_gemm64_workspace_size(int64_t M, const patch_weight64 *W, size_t *bytes);
+
+/*
+ * patch_gemm64: Y = X * W_eff^T for a weight in the 64 x 64 format, fp32
+ * accumulation in tensor memory and one round to bf16 (nearest even).
+ *   X bf16 [M][K] (16-byte aligned, M >= 0; M == 0 is a no-op);
+ *   Y bf16 [M][N];
+ *   workspace: patch_gemm64_workspace_size bytes, 16-byte aligned.  Its
+ *     first part holds arrival counters that must be zero before the first
+ *     use and that every successful call leaves zero (zero it again after a
+ *     call that reported an error); the rest is scratch.
+ * One kernel: the tokens are cut into blocks of 16 (M <= 16; two CTAs per
+ * SM) or 256 tokens (one CTA per SM), and the CTAs split the sequence of
+ * (token block, tile) pairs into shares of equal stored bytes (stream-K).  A
+ * CTA accumulates each tile row's tiles in tensor memory (M = 64 MMAs, N =
+ * the token block); a tile row cut between CTAs is finished by the last
+ * covering CTA, which adds the fp32 partials in CTA order (deterministic).
+ * Sparse tiles' metadata goes from shared to tensor memory through
+ * registers.  Launched with
+ * programmatic dependent launch as patch_gemm (X may be the previous
+ * kernel's output).  A bounded wait that runs out (wait_limit_us, 0 = 2 s)
+ * sets PATCH_DEV_TIMEOUT.
+ * Errors: PATCH_ERR_INVALID_ARG, PATCH_ERR_SHAPE, PATCH_ERR_ALIGN,
+ * PATCH_ERR_WORKSPACE (too small or unaligned), PATCH_ERR_DEVICE,
+ * PATCH_ERR_CUDA.
+ */
+PATCH_API patch_status_t patch_gemm64(const uint16_t *X, int64_t M, const patch_weight64 *W, uint16_t *Y,
+                                      void *workspace, size_t workspace_bytes, int32_t *dev_status, void *stream,
+                                      uint64_t wait_limit_us);
+
+/*
+ * patch_mma_probe_m: patch_mma_probe for MMA shape M = 64 or 128 (A of M
+ * rows; same N = 240, K and rounds).  A round does 4 x 2 x M x 240 x 16
+ * (dense) or x 32 (sparse) FLOPs per SM.  Errors as patch_mma_probe, and
+ * PATCH_ERR_INVALID_ARG for another M.
+ */
+PATCH_API patch_status_t patch_mma_probe_m(int m, int sparse, int64_t iters, int32_t *dev_status, void *stream);
+
+/*
  * patch_read_status: synchronise `stream`, copy *dev_status to *host_bits and
  * return the first error it encodes (PATCH_ERR_TIMEOUT, then BOUNDS, then
  * BAD_PATTERN, then COUNT) or PATCH_OK.  host_bits may be NULL.

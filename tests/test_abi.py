@@ -84,6 +84,46 @@ def test_host_checks_reject_before_any_launch(lib):
     assert lib.patch_gemm(fake, 4, ctypes.byref(wbad), fake, None, 0, fake, None) == 2
 
 
+def test_64_tile_format_host_checks(lib):
+    """The 64 x 64 execution-tile calls: closed-form sizes, and host checks that
+    refuse before any device query or launch."""
+    assert tsg.patch_pack64_sizes(192, 320, 7) == ((15 - 7) * 8192 + 7 * 4096, 7 * 512, 16 * 15)
+    assert tsg.patch_pack64_sizes(64, 64, 0) == (8192, 0, 16)
+    with pytest.raises(tsg.PatchError) as e:
+        tsg.patch_pack64_sizes(96, 64, 0)
+    assert e.value.code == 2
+    with pytest.raises(tsg.PatchError) as e:
+        tsg.patch_pack64_sizes(64, 64, 2)
+    assert e.value.code == 1
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    SZ = ctypes.c_size_t
+    w = tsg._Weight(192, 320, 0, 0x10000, None, 0x10000)
+    # M == 0: no-op, zero workspace, no device needed
+    b = SZ(123)
+    assert lib.patch_gemm64_workspace_size(0, ctypes.byref(w), ctypes.byref(b)) == 0 and b.value == 0
+    assert lib.patch_gemm64(None, 0, ctypes.byref(w), None, None, 0, fake, None, 0) == 0
+    # bad shape, n_sparse out of range, missing metadata, misaligned blob, negative M, NULL status
+    assert lib.patch_gemm64(fake, 4, ctypes.byref(tsg._Weight(192, 96 + 1, 0, 0x10000, None, 0x10000)),
+                            fake, None, 0, fake, None, 0) == 2
+    assert lib.patch_gemm64(fake, 4, ctypes.byref(tsg._Weight(64, 64, 2, 0x10000, 0x10000, 0x10000)),
+                            fake, None, 0, fake, None, 0) == 1
+    assert lib.patch_gemm64(fake, 4, ctypes.byref(tsg._Weight(64, 64, 1, 0x10000, None, 0x10000)),
+                            fake, None, 0, fake, None, 0) == 1
+    assert lib.patch_gemm64(fake, 4, ctypes.byref(tsg._Weight(64, 64, 0, 0x10008, None, 0x10000)),
+                            fake, None, 0, fake, None, 0) == 3
+    assert lib.patch_gemm64(fake, -1, ctypes.byref(w), fake, None, 0, fake, None, 0) == 1
+    assert lib.patch_gemm64(fake, 4, ctypes.byref(w), fake, None, 0, None, None, 0) == 1
+    # pack64: shape, n_sparse range, alignment; exec tiles: mask tile above 64
+    assert lib.patch_pack64(fake, 96, 64, fake, fake, 0, fake, None, fake, fake, None) == 2
+    assert lib.patch_pack64(fake, 64, 64, fake, fake, 2, fake, fake, fake, fake, None) == 1
+    assert lib.patch_pack64(P(0x10002), 64, 64, fake, fake, 0, fake, None, fake, fake, None) == 3
+    assert lib.patch_exec_tiles64(fake, 128, 128, 128, fake, fake, None) == 1
+    assert lib.patch_exec_tiles64(fake, 96, 128, 32, fake, fake, None) == 2
+    # the MMA probe takes M = 64 or 128 only
+    assert lib.patch_mma_probe_m(96, 0, 10, fake, None) == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(tsg, "_lib", None)
     monkeypatch.setattr(tsg, "_LIB_PATH", tmp_path / "libpatch.so")

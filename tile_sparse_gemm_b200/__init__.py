@@ -18,6 +18,8 @@ Entry points (same names as the C ABI):
     patch_gemm_mlp, patch_tile_kinds, patch_pack_from_logits, patch_soft_mask,
     patch_hard_mask_tiles, patch_exec_tiles, shard_rows / shard_of,
     patch_gemm_chain / Chain (a sequence of decode GEMMs in one launch; see each docstring)
+    64 x 64 execution tiles: patch_pack64_sizes, patch_exec_tiles64, patch_pack64 -> PackedWeight64,
+    patch_gemm64_workspace_size, patch_gemm64; patch_mma_probe_m (M = 64 or 128 MMA rate)
 Helpers of this binding: save_packed(weight, path) / load_packed(path) keep a
 packed weight in one .npz file (shape, sparse-tile count, the three blobs).
 """
@@ -97,6 +99,12 @@ def lib() -> ctypes.CDLL:
             "patch_gemm_chain_workspace_size": [P, I64, ctypes.POINTER(SZ)],
             "patch_gemm_chain": [P, I64, P, SZ, P, P, ctypes.c_uint64],
             "patch_mma_probe": [I32, I64, P, P],
+            "patch_mma_probe_m": [I32, I32, I64, P, P],
+            "patch_pack64_sizes": [I64, I64, I64, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)],
+            "patch_exec_tiles64": [P, I64, I64, I64, P, P, P],
+            "patch_pack64": [P, I64, I64, P, P, I64, P, P, P, P, P],
+            "patch_gemm64_workspace_size": [I64, WP, ctypes.POINTER(SZ)],
+            "patch_gemm64": [P, I64, WP, P, P, SZ, P, P, ctypes.c_uint64],
             "patch_check_weight": [WP, P, P],
         }
         for name, args in sigs.items():
@@ -484,3 +492,101 @@ def patch_read_status(status: torch.Tensor, stream=None) -> tuple[int, int]:
 
 def version() -> str:
     return lib().patch_version().decode()
+
+
+# ---- 64 x 64 execution tiles ("Ablation Studies", tile size)
+
+TILE64 = 64
+
+
+@dataclass
+class PackedWeight64:
+    """A weight packed in the 64 x 64 execution-tile format (patch_pack64)."""
+    N: int
+    K: int
+    n_sparse: int
+    values: torch.Tensor  # uint8, patch_pack64_sizes bytes
+    meta: torch.Tensor    # uint8 (may be empty)
+    desc: torch.Tensor    # uint8, 16 bytes per 64 x 64 tile
+
+    def struct(self) -> _Weight:  # patch_weight64 has patch_weight's layout
+        return _Weight(self.N, self.K, self.n_sparse, self.values.data_ptr(),
+                       self.meta.data_ptr() if self.meta.numel() else None, self.desc.data_ptr())
+
+    @property
+    def stored_bytes(self) -> int:
+        return self.values.numel() + self.meta.numel() + self.desc.numel()
+
+
+def patch_pack64_sizes(N: int, K: int, n_sparse: int) -> tuple[int, int, int]:
+    v, m, d = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().patch_pack64_sizes(N, K, n_sparse, ctypes.byref(v), ctypes.byref(m), ctypes.byref(d)),
+           "patch_pack64_sizes")
+    return v.value, m.value, d.value
+
+
+def patch_exec_tiles64(bitmap: torch.Tensor, N: int, K: int, mask_tile: int,
+                       stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """64 x 64 execution tiles of a b x b mask bitmap (b <= 64): (exec u8 [N/64][K/64],
+    n_sparse int64 [1]), on the device."""
+    dev = bitmap.device
+    ex = torch.empty((N // TILE64, K // TILE64), dtype=torch.uint8, device=dev)
+    n_sparse = torch.empty(1, dtype=torch.int64, device=dev)
+    _check(lib().patch_exec_tiles64(_dev(bitmap, "bitmap"), N, K, int(mask_tile), _dev(ex, "exec"),
+                                    _dev(n_sparse, "n_sparse"), _stream(stream)), "patch_exec_tiles64")
+    return ex, n_sparse
+
+
+def patch_pack64(W: torch.Tensor, bitmap: torch.Tensor, pat_id: torch.Tensor, n_sparse: int | None = None,
+                 status: torch.Tensor | None = None, stream=None) -> PackedWeight64:
+    """Pack W (bf16 [N][K]) under a 64 x 64 execution bitmap and pattern ids."""
+    N, K = W.shape
+    if n_sparse is None:
+        n_sparse = int(torch.count_nonzero(bitmap).item())
+    vb, mb, db = patch_pack64_sizes(N, K, n_sparse)
+    dev = W.device
+    status = new_status(dev) if status is None else status
+    values = torch.empty(vb, dtype=torch.uint8, device=dev)
+    meta = torch.empty(mb, dtype=torch.uint8, device=dev)
+    desc = torch.empty(db, dtype=torch.uint8, device=dev)
+    _check(lib().patch_pack64(_dev(W, "W"), N, K, _dev(bitmap, "bitmap"), _dev(pat_id, "pat_id"), n_sparse,
+                              _dev(values, "values"), _dev(meta, "meta") if mb else None, _dev(desc, "desc"),
+                              _dev(status, "status"), _stream(stream)), "patch_pack64")
+    return PackedWeight64(N, K, n_sparse, values, meta, desc)
+
+
+def patch_gemm64_workspace_size(M: int, weight: PackedWeight64) -> int:
+    b = ctypes.c_size_t()
+    st = weight.struct()
+    _check(lib().patch_gemm64_workspace_size(M, ctypes.byref(st), ctypes.byref(b)), "patch_gemm64_workspace_size")
+    return b.value
+
+
+def patch_gemm64(X: torch.Tensor, weight: PackedWeight64, Y: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                 wait_limit_us: int = 0, stream=None) -> torch.Tensor:
+    """Y = X * W_eff^T for a 64 x 64 packed weight (bf16 out, fp32 accumulate), any M."""
+    if not isinstance(weight, PackedWeight64):
+        raise TypeError("patch_gemm64 takes a PackedWeight64 (patch_pack64)")
+    M, K = X.shape
+    if K != weight.K:
+        raise ValueError(f"X has K={K}, weight has K={weight.K}")
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, weight.N), dtype=torch.bfloat16, device=dev)
+    status = new_status(dev) if status is None else status
+    st = weight.struct()
+    if workspace is None:
+        workspace = torch.zeros(max(patch_gemm64_workspace_size(M, weight), 16), dtype=torch.uint8, device=dev)
+    _check(lib().patch_gemm64(_dev(X, "X"), M, ctypes.byref(st), _dev(Y, "Y"), _dev(workspace, "workspace"),
+                              workspace.numel(), _dev(status, "status"), _stream(stream), wait_limit_us),
+           "patch_gemm64")
+    return Y
+
+
+def patch_mma_probe_m(m: int, sparse: bool, iters: int, status: torch.Tensor | None = None, stream=None) -> None:
+    """patch_mma_probe for MMA shape M = 64 or 128: FLOPs per launch SMs x iters x 4 x 2 x m x 240 x
+    (32 if sparse else 16), dense-equivalent."""
+    status = new_status() if status is None else status
+    _check(lib().patch_mma_probe_m(int(m), 1 if sparse else 0, iters, _dev(status, "status"), _stream(stream)),
+           "patch_mma_probe_m")

@@ -20,7 +20,8 @@ INCLUDE = ROOT / "include"
 LIB = PKG / "libpatch.so"
 LIB_DEBUG = PKG / "libpatch_debug.so"
 SOURCES = ["capi.cu", "hard_mask.cu", "pack.cu", "gemm_decode.cu", "gemm_decode_tc.cu", "gemm_prefill.cu",
-           "gemm_decode_noalloc.cu", "gated_mlp.cu", "gemm_decode_chain.cu", "mma_probe.cu", "validate.cu"]
+           "gemm_decode_noalloc.cu", "gated_mlp.cu", "gemm_decode_chain.cu", "mma_probe.cu", "validate.cu",
+           "gemm64.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]
 

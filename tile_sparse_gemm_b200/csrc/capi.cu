@@ -149,7 +149,7 @@ patch_status_t patch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int
   int sms = 0;
   patch_status_t st = device_sms(&sms);
   if (st != PATCH_OK) return st;
-  if (launch_exec_tiles(bitmap, N, K, mask_tile, exec, n_sparse, sms, static_cast<cudaStream_t>(stream)) !=
+  if (launch_exec_tiles(bitmap, N, K, mask_tile, kTile, exec, n_sparse, sms, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return PATCH_ERR_CUDA;
   return PATCH_OK;
@@ -459,12 +459,114 @@ patch_status_t patch_shard_rows(const uint8_t* bitmap, int64_t Tn, int64_t Tk, i
   return PATCH_OK;
 }
 
-patch_status_t patch_mma_probe(int sparse, int64_t iters, int32_t* dev_status, void* stream) {
-  if (iters < 1 || !dev_status) return PATCH_ERR_INVALID_ARG;
+patch_status_t patch_mma_probe_m(int m, int sparse, int64_t iters, int32_t* dev_status, void* stream) {
+  if (iters < 1 || !dev_status || (m != 64 && m != 128)) return PATCH_ERR_INVALID_ARG;
   int sms = 0;
   patch_status_t st = device_sms(&sms);
   if (st != PATCH_OK) return st;
-  return launch_mma_probe(sparse ? 1 : 0, iters, sms, 2000000000ull, dev_status, static_cast<cudaStream_t>(stream)) ==
+  return launch_mma_probe(m, sparse ? 1 : 0, iters, sms, 2000000000ull, dev_status,
+                          static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PATCH_OK
+             : PATCH_ERR_CUDA;
+}
+
+patch_status_t patch_mma_probe(int sparse, int64_t iters, int32_t* dev_status, void* stream) {
+  return patch_mma_probe_m(128, sparse, iters, dev_status, stream);
+}
+
+// ---- the 64 x 64 execution-tile format
+
+static bool shape64_ok(int64_t N, int64_t K) {
+  return N > 0 && K > 0 && N % 64 == 0 && K % 64 == 0 && N <= (int64_t(1) << 31) && K <= (int64_t(1) << 31);
+}
+
+static patch_status_t check_weight64(const patch_weight64* W) {
+  if (!W || !W->values || !W->desc) return PATCH_ERR_INVALID_ARG;
+  if (!shape64_ok(W->N, W->K)) return PATCH_ERR_SHAPE;
+  const int64_t T = (W->N / 64) * (W->K / 64);
+  if (W->n_sparse < 0 || W->n_sparse > T) return PATCH_ERR_INVALID_ARG;
+  if (W->n_sparse > 0 && !W->meta) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(W->values) || !aligned16(W->desc) || (W->meta && !aligned16(W->meta))) return PATCH_ERR_ALIGN;
+  return PATCH_OK;
+}
+
+patch_status_t patch_pack64_sizes(int64_t N, int64_t K, int64_t n_sparse, size_t* values_bytes, size_t* meta_bytes,
+                                  size_t* desc_bytes) {
+  if (!values_bytes || !meta_bytes || !desc_bytes) return PATCH_ERR_INVALID_ARG;
+  if (!shape64_ok(N, K)) return PATCH_ERR_SHAPE;
+  const int64_t T = (N / 64) * (K / 64);
+  if (n_sparse < 0 || n_sparse > T) return PATCH_ERR_INVALID_ARG;
+  *values_bytes = size_t(T - n_sparse) * PATCH_DENSE_TILE64_BYTES + size_t(n_sparse) * PATCH_SPARSE_TILE64_BYTES;
+  *meta_bytes = size_t(n_sparse) * PATCH_META_TILE64_BYTES;
+  *desc_bytes = size_t(T) * sizeof(patch_tile_desc);
+  return PATCH_OK;
+}
+
+patch_status_t patch_exec_tiles64(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, uint8_t* exec,
+                                  int64_t* n_sparse, void* stream) {
+  if (!bitmap || !exec || !n_sparse) return PATCH_ERR_INVALID_ARG;
+  if (mask_tile != 4 && mask_tile != 8 && mask_tile != 16 && mask_tile != 32 && mask_tile != 64)
+    return PATCH_ERR_INVALID_ARG;
+  if (!shape64_ok(N, K)) return PATCH_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(n_sparse) % 8) return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_exec_tiles(bitmap, N, K, mask_tile, 64, exec, n_sparse, sms, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
+patch_status_t patch_pack64(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap, const uint8_t* pat_id,
+                            int64_t n_sparse, void* values, void* meta, patch_tile_desc* desc, int32_t* dev_status,
+                            void* stream) {
+  if (!W || !bitmap || !pat_id || !values || !desc || !dev_status) return PATCH_ERR_INVALID_ARG;
+  if (!shape64_ok(N, K)) return PATCH_ERR_SHAPE;
+  const int64_t T = (N / 64) * (K / 64);
+  if (n_sparse < 0 || n_sparse > T) return PATCH_ERR_INVALID_ARG;
+  if (n_sparse > 0 && !meta) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(pat_id) || !aligned16(values) || !aligned16(desc) || (meta && !aligned16(meta)))
+    return PATCH_ERR_ALIGN;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  if (launch_pack64(W, N, K, bitmap, pat_id, n_sparse, values, meta, desc, dev_status, sms,
+                    static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PATCH_ERR_CUDA;
+  return PATCH_OK;
+}
+
+patch_status_t patch_gemm64_workspace_size(int64_t M, const patch_weight64* W, size_t* bytes) {
+  if (!bytes || M < 0) return PATCH_ERR_INVALID_ARG;
+  patch_status_t st = check_weight64(W);
+  if (st != PATCH_OK) return st;
+  *bytes = 0;
+  if (M == 0) return PATCH_OK;
+  if (M > (int64_t(1) << 30)) return PATCH_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  *bytes = gemm64_workspace_bytes(M, *W, sms);
+  return PATCH_OK;
+}
+
+patch_status_t patch_gemm64(const uint16_t* X, int64_t M, const patch_weight64* W, uint16_t* Y, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream, uint64_t wait_limit_us) {
+  if (M < 0 || !dev_status) return PATCH_ERR_INVALID_ARG;
+  patch_status_t st = check_weight64(W);
+  if (st != PATCH_OK) return st;
+  if (M == 0) return PATCH_OK;
+  if (!X || !Y) return PATCH_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y)) return PATCH_ERR_ALIGN;
+  if (M > (int64_t(1) << 30)) return PATCH_ERR_INVALID_ARG;
+  int sms = 0;
+  st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  const size_t need = gemm64_workspace_bytes(M, *W, sms);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PATCH_ERR_WORKSPACE;
+  const uint64_t limit_ns = (wait_limit_us ? wait_limit_us : 2000000ull) * 1000ull;
+  return launch_gemm64(X, M, *W, Y, workspace, dev_status, sms, limit_ns, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? PATCH_OK
              : PATCH_ERR_CUDA;

@@ -37,6 +37,14 @@ __host__ __device__ __forceinline__ uint32_t meta_byte_index(uint32_t r, uint32_
          (((g >> 2) & 1u) << 7) | ((r >> 4) << 8);
 }
 
+// Byte of a 64 x 64 sparse tile's 512-byte metadata block holding group g
+// (0..15) of tile row r (0..63): 8 bytes per tensor-memory lane of the M = 64
+// sparse MMA (lane 32*(r>>4) + (r&7) + 8*((g>>2)&1)), column g>>3 in bytes 4*(g>>3)..
+__host__ __device__ __forceinline__ uint32_t meta64_byte_index(uint32_t r, uint32_t g) {
+  return ((g >> 1) & 1u) | (((r >> 3) & 1u) << 1) | ((g >> 3) << 2) | ((r & 7u) << 3) | (((g >> 2) & 1u) << 6) |
+         ((r >> 4) << 7);
+}
+
 // kept pair (i0, i1) of pattern id p, packed as i0 | i1 << 2 (the metadata code)
 __host__ __device__ __forceinline__ uint32_t pattern_code(uint32_t p) {
   // ids 0..5 -> codes 0x4 0x8 0xC 0x9 0xD 0xE, nibble p of this constant

@@ -503,8 +503,10 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a) {
       bool guard_done = a.global || j < PART_RING;
       for (int tn = tn_first; tn <= tn_last; ++tn, ++seg) {
         const uint32_t buf = seg % NACC;
-        if (!(ok = wait_bounded(&s.acc_full[buf], (seg / NACC) & 1, &s.abort_flag, a.limit_ns, a.status, false)))
-          break;
+        // a warp-uniform decision: the tensor-memory loads below are warp-collective
+        ok = __all_sync(0xFFFFFFFFu,
+                        wait_bounded(&s.acc_full[buf], (seg / NACC) & 1, &s.abort_flag, a.limit_ns, a.status, false));
+        if (!ok) break;
         tc_fence_after();
         uint32_t v[16], w[16];
         tmem_ld_16cols(tmem + (uint32_t(32 * q) << 16) + uint32_t(NISS * buf * BT), v);

@@ -398,7 +398,9 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& a, int64_t p0, in
   const bool last_row_whole = s.t_last % a.Tk == a.Tk - 1 && p1 == panel_of(dl) + (dl.kind ? 1 : 2);
   for (int tn = tn_first; tn <= tn_last; ++tn) {
     const int seg = tn - tn_first, buf = seg % NACC;
-    if (!wait_bounded(&s.acc_full[buf], (seg / NACC) & 1, &s.abort_flag, a.limit_ns, a.status, false)) break;
+    // a warp-uniform decision: the tensor-memory load below is warp-collective
+    const bool ok = wait_bounded(&s.acc_full[buf], (seg / NACC) & 1, &s.abort_flag, a.limit_ns, a.status, false);
+    if (!__all_sync(0xFFFFFFFFu, ok)) break;
     tc_fence_after();
     uint32_t v[16];
     tmem_ld_16cols(tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * BT), v);

@@ -207,11 +207,11 @@ __global__ void __launch_bounds__(256) exec_tiles_kernel(const uint8_t* __restri
   }
 }
 
-cudaError_t launch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, uint8_t* exec,
-                              int64_t* n_sparse, int num_sms, cudaStream_t stream) {
+cudaError_t launch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, int64_t exec_tile,
+                              uint8_t* exec, int64_t* n_sparse, int num_sms, cudaStream_t stream) {
   int lr = 0;
-  while ((int64_t(kTile) >> lr) > mask_tile) ++lr;
-  const int64_t Tn = N / kTile, Tk = K / kTile;
+  while ((exec_tile >> lr) > mask_tile) ++lr;
+  const int64_t Tn = N / exec_tile, Tk = K / exec_tile;
   cudaError_t e = cudaMemsetAsync(n_sparse, 0, sizeof(int64_t), stream);
   if (e != cudaSuccess) return e;
   const int threads = 256;

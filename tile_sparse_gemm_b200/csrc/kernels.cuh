@@ -56,9 +56,17 @@ cudaError_t launch_silu_mul(const uint16_t* G, const uint16_t* U, uint16_t* H, i
 cudaError_t launch_hard_mask_tiles(const uint16_t* W, int64_t N, int64_t K, int64_t mask_tile,
                                    const float* tile_logits, const float* pattern_logits, uint16_t* W_masked,
                                    uint8_t* bitmap, uint8_t* pat_id, int num_sms, cudaStream_t stream);
-// 128 x 128 execution tiles of a b x b mask bitmap, and their sparse count (device int64).
-cudaError_t launch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, uint8_t* exec,
-                              int64_t* n_sparse, int num_sms, cudaStream_t stream);
+// exec_tile x exec_tile execution tiles (64 or 128) of a b x b mask bitmap, and their sparse count (device int64).
+cudaError_t launch_exec_tiles(const uint8_t* bitmap, int64_t N, int64_t K, int64_t mask_tile, int64_t exec_tile,
+                              uint8_t* exec, int64_t* n_sparse, int num_sms, cudaStream_t stream);
+
+// The 64 x 64 execution-tile format: pack (scan + tiles) and GEMM.
+cudaError_t launch_pack64(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap, const uint8_t* pat_id,
+                          int64_t n_sparse, void* values, void* meta, patch_tile_desc* desc, int32_t* status,
+                          int num_sms, cudaStream_t stream);
+size_t gemm64_workspace_bytes(int64_t M, const patch_weight64& W, int num_sms);
+cudaError_t launch_gemm64(const uint16_t* X, int64_t M, const patch_weight64& W, uint16_t* Y, void* workspace,
+                          int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream);
 
 // Workspace layout (patch_gemm_workspace_size covers every path): arrival
 // counters sit in a fixed region at the start (the tensor-core decode kernel's,
@@ -86,8 +94,8 @@ constexpr int64_t kChainMaxTileRows = int64_t(kDecodeCounterBytes / 16) - 1;  //
 // Device check of a packed weight's descriptor table (patch_check_weight).
 cudaError_t launch_check_weight(const patch_weight& W, int32_t* status, cudaStream_t stream);
 
-// Tensor-core MMA rate probe (patch_mma_probe).
-cudaError_t launch_mma_probe(int sparse, int64_t iters, int num_sms, uint64_t limit_ns, int32_t* status,
+// Tensor-core MMA rate probe (patch_mma_probe, patch_mma_probe_m): MMA shape m = 64 or 128.
+cudaError_t launch_mma_probe(int m, int sparse, int64_t iters, int num_sms, uint64_t limit_ns, int32_t* status,
                              cudaStream_t stream);
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -112,5 +120,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // 2D bf16 tensor map with 128-byte swizzle (out-of-bounds reads fill zeros).
 bool make_map_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                       uint32_t box_inner, uint32_t box_outer);
+// The same with the 64-byte swizzle (box_inner <= 32 elements).
+bool make_map_2d_bf16_sw64(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                           uint32_t box_inner, uint32_t box_outer);
 
 }  // namespace patch

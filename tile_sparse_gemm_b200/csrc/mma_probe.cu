@@ -8,13 +8,15 @@
 //
 // One CTA per SM; its shared memory holds pseudo-random bf16 operands (so the
 // datapath toggles as it does on real weights) and valid metadata codes.  One
-// thread issues `iters` rounds of four M = 128, N = 240 MMAs (the prefill
-// kernel's shape) into two alternating TMEM accumulators: dense rounds cover K = 64 (four K = 16
-// MMAs over one 128 x 64 panel), sparse rounds K = 128 logical (four K = 32
-// .sp MMAs over a 128 x 64 panel of kept values and its metadata), so a
-// sparse round does twice a dense round's dense-equivalent work.  The caller
-// times the launch; FLOPs = SMs x iters x 4 x 2 x 128 x 240 x (16 dense, 32
-// sparse).
+// thread issues `iters` rounds of four M = 128 (or M = 64: the first 64 rows
+// of the panel, the shape of 64 x 64 execution tiles), N = 240 MMAs (the
+// prefill kernel's token block) into two alternating TMEM accumulators: dense
+// rounds cover K = 64 (four K = 16 MMAs over one panel), sparse rounds K = 128
+// logical (four K = 32 .sp MMAs over a panel of kept values and its
+// metadata), so a sparse round does twice a dense round's dense-equivalent
+// work.  The caller times the launch; FLOPs = SMs x iters x 4 x 2 x M x 240 x
+// (16 dense, 32 sparse).  Every metadata column an MMA may read holds valid
+// codes for both shapes (four columns x 128 lanes are copied).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -54,7 +56,7 @@ __device__ __forceinline__ uint16_t rand_bf16(uint32_t h) {
   return uint16_t(((h >> 31) << 15) | ((119u + (h >> 28 & 7u)) << 7) | (h & 0x7Fu));
 }
 
-__global__ void __launch_bounds__(THREADS, 1) probe_kernel(int sparse, int64_t iters, uint64_t limit_ns,
+__global__ void __launch_bounds__(THREADS, 1) probe_kernel(int m, int sparse, int64_t iters, uint64_t limit_ns,
                                                            int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   Shared& s = *reinterpret_cast<Shared*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(THREADS, 1) probe_kernel(int sparse, int64_t i
   if (threadIdx.x == 0) {
     const uint32_t e_tmem = tmem + META_COL;  // 4 metadata columns after the first accumulator
     const uint64_t a0 = sw128_desc(smem_u32(s.a));
-    const uint32_t id_d = idesc_bf16(128, N, false), id_s = idesc_bf16(128, N, true);
+    const uint32_t id_d = idesc_bf16(m, N, false), id_s = idesc_bf16(m, N, true);
     if (sparse) tmem_cp_128x128b(e_tmem, meta_desc(smem_u32(s.e)));
     for (int64_t it = 0; it < iters; ++it) {
       const uint32_t acc = tmem + uint32_t(it & 1) * ACC1;
@@ -112,12 +114,12 @@ __global__ void __launch_bounds__(THREADS, 1) probe_kernel(int sparse, int64_t i
 
 }  // namespace probe
 
-cudaError_t launch_mma_probe(int sparse, int64_t iters, int num_sms, uint64_t limit_ns, int32_t* status,
+cudaError_t launch_mma_probe(int m, int sparse, int64_t iters, int num_sms, uint64_t limit_ns, int32_t* status,
                              cudaStream_t stream) {
   using namespace probe;
   cudaError_t e = cudaFuncSetAttribute(probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES));
   if (e != cudaSuccess) return e;
-  probe_kernel<<<num_sms, THREADS, SMEM_BYTES, stream>>>(sparse, iters, limit_ns, status);
+  probe_kernel<<<num_sms, THREADS, SMEM_BYTES, stream>>>(m, sparse, iters, limit_ns, status);
   return cudaGetLastError();
 }
 

@@ -20,7 +20,7 @@ namespace patch {
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads) pack_scan_kernel(
-    const uint8_t* __restrict__ bitmap, int64_t T, int64_t n_sparse,
+    const uint8_t* __restrict__ bitmap, int64_t T, int64_t n_sparse, uint64_t panel_bytes,
     patch_tile_desc* __restrict__ desc, int32_t* status) {
   __shared__ uint32_t warp_sums[kScanThreads / 32];
   __shared__ uint64_t carry_s;
@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(kScanThreads) pack_scan_kernel(
       d.kind = kind;
       d.sparse_ordinal = kind ? uint32_t(before) : 0xFFFFFFFFu;
       // dense tiles before t take 2 panels each, sparse ones 1
-      d.val_offset = uint64_t(PATCH_PANEL_BYTES) * (2ull * uint64_t(t) - before);
+      d.val_offset = panel_bytes * (2ull * uint64_t(t) - before);
       desc[t] = d;
     }
     __syncthreads();
@@ -185,7 +185,7 @@ cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* 
   const int64_t T = (N / kTile) * (K / kTile);
   const uint64_t values_bytes =
       uint64_t(T - n_sparse) * PATCH_DENSE_TILE_BYTES + uint64_t(n_sparse) * PATCH_SPARSE_TILE_BYTES;
-  pack_scan_kernel<<<1, kScanThreads, 0, stream>>>(bitmap, T, n_sparse, desc, status);
+  pack_scan_kernel<<<1, kScanThreads, 0, stream>>>(bitmap, T, n_sparse, PATCH_PANEL_BYTES, desc, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   int64_t blocks = T < int64_t(num_sms) * 16 ? T : int64_t(num_sms) * 16;
@@ -197,6 +197,95 @@ cudaError_t launch_pack(const uint16_t* W, int64_t N, int64_t K, const uint8_t* 
     pack_tiles_kernel<false><<<int(blocks), kPackThreads, 0, stream>>>(W, K, pat_id, nullptr, desc, T, n_sparse,
                                                               values_bytes, static_cast<uint8_t*>(values),
                                                               static_cast<uint8_t*>(meta), status);
+  return cudaGetLastError();
+}
+
+// The 64 x 64 execution-tile format: 64 rows x 32 bf16 panels (64-byte rows),
+// a dense tile = 2 panels (k 0..31, 32..63), a sparse tile = 1 panel of kept
+// values plus 512 B of metadata stored 8 bytes per tensor-memory lane of the
+// M = 64 sparse MMA.  One CTA of 128 threads per tile; 4 items of 16 bytes
+// per thread (all loads, then all stores).
+constexpr int kPack64Threads = 128;
+constexpr int kPack64Items = 512 / kPack64Threads;
+
+__global__ void __launch_bounds__(kPack64Threads) pack64_tiles_kernel(
+    const uint16_t* __restrict__ W, int64_t K, const uint8_t* __restrict__ pat_id,
+    const patch_tile_desc* __restrict__ desc, int64_t T, int64_t n_sparse, uint64_t values_bytes,
+    uint8_t* __restrict__ values, uint8_t* __restrict__ meta, int32_t* status) {
+  __shared__ __align__(16) uint8_t meta_s[PATCH_META_TILE64_BYTES];
+  const int64_t Tk = K / 64;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const patch_tile_desc d = desc[t];
+    const int64_t tn = t / Tk, tk = t - tn * Tk;
+    const uint64_t size = d.kind ? PATCH_SPARSE_TILE64_BYTES : PATCH_DENSE_TILE64_BYTES;
+    if (d.val_offset + size > values_bytes || (d.kind && int64_t(d.sparse_ordinal) >= n_sparse))
+      continue;  // PATCH_DEV_COUNT is raised by the scan
+    uint8_t* panel = values + d.val_offset;
+    const uint16_t* wt = W + (tn * 64) * K + tk * 64;
+    uint4 v[kPack64Items];
+    if (d.kind == 0) {
+      // 64 rows x 8 chunks of 8 values: chunk q of row r goes to panel q/4, byte 16*(q%4) of row r
+#pragma unroll
+      for (int j = 0; j < kPack64Items; ++j) {
+        const int c = threadIdx.x + j * kPack64Threads, r = c >> 3, q = c & 7;
+        v[j] = __ldcs(reinterpret_cast<const uint4*>(wt + int64_t(r) * K + q * 8));
+      }
+#pragma unroll
+      for (int j = 0; j < kPack64Items; ++j) {
+        const int c = threadIdx.x + j * kPack64Threads, r = c >> 3, q = c & 7;
+        *reinterpret_cast<uint4*>(panel + (q >> 2) * PATCH_PANEL64_BYTES + r * 64 + (q & 3) * 16) = v[j];
+      }
+    } else {
+      // 64 rows x 8 pairs of groups; item (r, p) reads groups 2p, 2p+1 of row r
+      uint32_t ids[kPack64Items][2];
+#pragma unroll
+      for (int j = 0; j < kPack64Items; ++j) {
+        const int c = threadIdx.x + j * kPack64Threads, r = c >> 3, p = c & 7;
+        v[j] = __ldcs(reinterpret_cast<const uint4*>(wt + int64_t(r) * K + p * 8));
+        const uint16_t ids2 =
+            *reinterpret_cast<const uint16_t*>(pat_id + (tn * 64 + r) * (K / 4) + tk * 16 + 2 * p);
+        ids[j][0] = ids2 & 0xFF;
+        ids[j][1] = ids2 >> 8;
+      }
+#pragma unroll
+      for (int j = 0; j < kPack64Items; ++j) {
+        const int c = threadIdx.x + j * kPack64Threads, r = c >> 3, p = c & 7;
+        uint32_t id0 = ids[j][0], id1 = ids[j][1];
+        if (id0 > 5 || id1 > 5) {
+          set_status(status, PATCH_DEV_BAD_PATTERN);
+          if (id0 > 5) id0 = 0;
+          if (id1 > 5) id1 = 0;
+        }
+        const uint32_t c0 = pattern_code(id0), c1 = pattern_code(id1);
+        const uint64_t g0 = uint64_t(v[j].y) << 32 | v[j].x, g1 = uint64_t(v[j].w) << 32 | v[j].z;
+        uint2 out;
+        out.x = uint32_t((g0 >> (16 * (c0 & 3))) & 0xFFFFu) | uint32_t((g0 >> (16 * (c0 >> 2))) & 0xFFFFu) << 16;
+        out.y = uint32_t((g1 >> (16 * (c1 & 3))) & 0xFFFFu) | uint32_t((g1 >> (16 * (c1 >> 2))) & 0xFFFFu) << 16;
+        *reinterpret_cast<uint2*>(panel + r * 64 + p * 8) = out;
+        meta_s[meta64_byte_index(r, 2 * p)] = uint8_t(c0 | (c1 << 4));
+      }
+      __syncthreads();
+      uint8_t* mt = meta + uint64_t(d.sparse_ordinal) * PATCH_META_TILE64_BYTES;
+      for (int c = threadIdx.x; c < PATCH_META_TILE64_BYTES / 16; c += blockDim.x)
+        reinterpret_cast<uint4*>(mt)[c] = reinterpret_cast<const uint4*>(meta_s)[c];
+      __syncthreads();
+    }
+  }
+}
+
+cudaError_t launch_pack64(const uint16_t* W, int64_t N, int64_t K, const uint8_t* bitmap, const uint8_t* pat_id,
+                          int64_t n_sparse, void* values, void* meta, patch_tile_desc* desc, int32_t* status,
+                          int num_sms, cudaStream_t stream) {
+  const int64_t T = (N / 64) * (K / 64);
+  const uint64_t values_bytes =
+      uint64_t(T - n_sparse) * PATCH_DENSE_TILE64_BYTES + uint64_t(n_sparse) * PATCH_SPARSE_TILE64_BYTES;
+  pack_scan_kernel<<<1, kScanThreads, 0, stream>>>(bitmap, T, n_sparse, PATCH_PANEL64_BYTES, desc, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t blocks = T < int64_t(num_sms) * 16 ? T : int64_t(num_sms) * 16;
+  pack64_tiles_kernel<<<int(blocks), kPack64Threads, 0, stream>>>(W, K, pat_id, desc, T, n_sparse, values_bytes,
+                                                                   static_cast<uint8_t*>(values),
+                                                                   static_cast<uint8_t*>(meta), status);
   return cudaGetLastError();
 }
 

@@ -222,6 +222,21 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
+// Shared-memory matrix descriptor for a K-major operand stored with the
+// 64-byte swizzle (64-byte rows, 8-row atoms 512 B apart): as above with
+// layout type 4 at bits 61-63.
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(512 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(4) << 61);
+}
+
+// Two 32-bit columns of the warp's 32 tensor-memory lanes from registers
+// (thread i -> lane i of the warp's subpartition), and the wait for them.
+__device__ __forceinline__ void tmem_st_32x32b_x2(uint32_t taddr, uint32_t v0, uint32_t v1) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(v0), "r"(v1) : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Descriptor of a 128-row x 16-byte metadata block for tcgen05.cp 128x128b:
 // no swizzle, rows 16 B apart, 8-row core matrices 128 B apart.
 __device__ __forceinline__ uint64_t meta_desc(uint32_t saddr) {
