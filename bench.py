@@ -519,14 +519,17 @@ def mlp_steps(dev, pk, reps=10):
 
 
 def tile_ablation(args):
-    """Mask tile size ablation ("Ablation Studies", tile size: performance holds
+    """Tile-size ablation ("Ablation Studies", tile size: performance holds
     across learned tile sizes down to 4 x 4, while hardware efficiency needs
     128 x 128 execution tiles).  For each mask tile b and layout (b x b tiles
     sparse at seeded random positions, or as one band of tile rows), half of
-    the mask tiles sparse, the product path runs: patch_hard_mask_tiles ->
-    patch_exec_tiles -> patch_pack of W_masked; then patch_gemm is timed at
-    M = 1 (decode) and M = 2048 (prefill) against the same layer packed with
-    an all-dense bitmap.  Weights rotate over copies that exceed L2."""
+    the mask tiles sparse, the product path runs at both execution-tile sizes:
+    patch_hard_mask_tiles -> patch_exec_tiles (128 x 128) -> patch_pack of
+    W_masked -> patch_gemm, and for b <= 64 patch_exec_tiles64 ->
+    patch_pack64 -> patch_gemm64 (64 x 64 execution tiles, M = 64 MMAs).
+    Each is timed at M = 1 (decode) and M = 2048 (prefill) against the same
+    layer packed all-dense in the 128 x 128 format (and, for the 64 x 64 rows,
+    also in its own format).  Weights rotate over copies that exceed L2."""
     import torch
 
     import tile_sparse_gemm_b200 as tsg
@@ -538,22 +541,25 @@ def tile_ablation(args):
     l2_bytes = 126e6
 
     def copies_of(pw):
-        n = max(2, int(np.ceil(3 * l2_bytes / (pw.values.numel() + pw.meta.numel() + pw.desc.numel()))))
-        return [pw] + [tsg.PackedWeight(pw.N, pw.K, pw.n_sparse, pw.values.clone(), pw.meta.clone(),
-                                        pw.desc.clone()) for _ in range(n - 1)]
+        n = max(2, int(np.ceil(3 * l2_bytes / pw.stored_bytes)))
+        return [pw] + [type(pw)(pw.N, pw.K, pw.n_sparse, pw.values.clone(), pw.meta.clone(), pw.desc.clone())
+                       for _ in range(n - 1)]
 
     def time_us(packs, M, reps):
         K, N = packs[0].K, packs[0].N
+        is64 = isinstance(packs[0], tsg.PackedWeight64)
+        gemm = tsg.patch_gemm64 if is64 else tsg.patch_gemm
+        need = (tsg.patch_gemm64_workspace_size if is64 else tsg.patch_gemm_workspace_size)(M, packs[0])
         x = torch.randn(M, K, device=dev).to(torch.bfloat16)
         y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        ws = torch.zeros(max(tsg.patch_gemm_workspace_size(M, packs[0]), 16), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
         for i in range(len(packs)):
-            tsg.patch_gemm(x, packs[i], Y=y, workspace=ws, status=status)
+            gemm(x, packs[i], Y=y, workspace=ws, status=status)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for r in range(reps):
-            tsg.patch_gemm(x, packs[r % len(packs)], Y=y, workspace=ws, status=status)
+            gemm(x, packs[r % len(packs)], Y=y, workspace=ws, status=status)
         e1.record()
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) * 1e3 / reps
@@ -566,6 +572,7 @@ def tile_ablation(args):
             a.append(time_us(packs, M, reps))
         return statistics.median(a), statistics.median(d)
 
+    runs = (("decode", 1, 2000), ("prefill", 2048, 200))
     rows = []
     warm = torch.empty(2**28, dtype=torch.uint8, device=dev)
     t_end = time.time() + 1.0
@@ -581,80 +588,105 @@ def tile_ablation(args):
         w = torch.from_numpy(w_np.view(np.int16)).view(torch.bfloat16).to(dev)
         pl = torch.from_numpy(pl_np).to(dev)
         del pl_np
-        dense = tsg.patch_pack(w, torch.zeros((N // 128, K // 128), dtype=torch.uint8, device=dev),
-                               torch.from_numpy(ids).to(dev), 0, status=status)
+        pid_dev = torch.from_numpy(ids).to(dev)
+        dense = tsg.patch_pack(w, torch.zeros((N // 128, K // 128), dtype=torch.uint8, device=dev), pid_dev, 0,
+                               status=status)
         dense_packs = copies_of(dense)
-        dense_bytes = dense.values.numel() + dense.desc.numel()
+        dense_bytes = dense.stored_bytes
+        dense64_packs = copies_of(tsg.patch_pack64(w, torch.zeros((N // 64, K // 64), dtype=torch.uint8,
+                                                                   device=dev), pid_dev, 0, status=status))
         base_all = {"decode": [], "prefill": []}
+        base64 = {kind: paired(dense64_packs, dense_packs, M, reps)[0] for kind, M, reps in runs}
         for clustered in (False, True):
             for b in sizes:
                 kinds = si.mask_tiles(N, K, b, 0.5, clustered, 2, idx)
                 tl = torch.from_numpy(si.choice_logits(kinds)).to(dev)
                 wm, bm, pid = tsg.patch_hard_mask_tiles(w, tl, pl, b, status=status)
-                ex, n_dev = tsg.patch_exec_tiles(bm, N, K, b)
-                pw = tsg.patch_pack(wm, ex, pid, int(n_dev.item()), status=status)
-                packs = copies_of(pw)
-                stored = pw.values.numel() + pw.meta.numel() + pw.desc.numel()
-                t, base = {}, {}
-                for kind, M, reps in (("decode", 1, 2000), ("prefill", 2048, 200)):
-                    t[kind], base[kind] = paired(packs, dense_packs, M, reps)
-                    base_all[kind].append(base[kind])
-                rows.append({"shape": f"{name} {N}x{K}", "mask_tile": b,
-                             "layout": "band of tile rows" if clustered else "random",
-                             "sparse_mask_tiles": 0.5,
-                             "sparse_exec_tiles": round(pw.n_sparse / ((N // 128) * (K // 128)), 4),
-                             "stored_vs_dense": round(stored / dense_bytes, 4),
-                             "decode_us": round(t["decode"], 2),
-                             "decode_GBps": round(stored / t["decode"] / 1e3, 1),
-                             "decode_speedup": round(base["decode"] / t["decode"], 3),
-                             "prefill_us": round(t["prefill"], 2),
-                             "prefill_speedup": round(base["prefill"] / t["prefill"], 3)})
-                del packs, pw, wm
-        del dense_packs
-        rows.append({"shape": f"{name} {N}x{K}", "mask_tile": None, "layout": "all dense",
+                layouts = [(128, tsg.patch_exec_tiles, tsg.patch_pack)]
+                if b <= 64:
+                    layouts.append((64, tsg.patch_exec_tiles64, tsg.patch_pack64))
+                for E, exec_fn, pack_fn in layouts:
+                    ex, n_dev = exec_fn(bm, N, K, b)
+                    pw = pack_fn(wm, ex, pid, int(n_dev.item()), status=status)
+                    packs = copies_of(pw)
+                    t, base = {}, {}
+                    for kind, M, reps in runs:
+                        t[kind], base[kind] = paired(packs, dense_packs, M, reps)
+                        base_all[kind].append(base[kind])
+                    row = {"shape": f"{name} {N}x{K}", "mask_tile": b, "exec_tile": E,
+                           "layout": "band of tile rows" if clustered else "random",
+                           "sparse_mask_tiles": 0.5,
+                           "sparse_exec_tiles": round(pw.n_sparse / ((N // E) * (K // E)), 4),
+                           "stored_vs_dense": round(pw.stored_bytes / dense_bytes, 4),
+                           "decode_us": round(t["decode"], 2),
+                           "decode_GBps": round(pw.stored_bytes / t["decode"] / 1e3, 1),
+                           "decode_speedup": round(base["decode"] / t["decode"], 3),
+                           "prefill_us": round(t["prefill"], 2),
+                           "prefill_speedup": round(base["prefill"] / t["prefill"], 3)}
+                    if E == 64:  # against the all-dense layer in the 64 x 64 format itself
+                        row["decode_speedup_vs_dense64"] = round(base64["decode"] / t["decode"], 3)
+                        row["prefill_speedup_vs_dense64"] = round(base64["prefill"] / t["prefill"], 3)
+                    rows.append(row)
+                    del packs, pw
+                del wm
+        del dense_packs, dense64_packs
+        rows.append({"shape": f"{name} {N}x{K}", "mask_tile": None, "exec_tile": 128, "layout": "all dense",
                      "decode_us": round(statistics.median(base_all["decode"]), 2),
                      "prefill_us": round(statistics.median(base_all["prefill"]), 2)})
+        rows.append({"shape": f"{name} {N}x{K}", "mask_tile": None, "exec_tile": 64, "layout": "all dense",
+                     "decode_us": round(base64["decode"], 2), "prefill_us": round(base64["prefill"], 2)})
     code, bits = tsg.patch_read_status(status)
     if code != 0:
         raise RuntimeError(f"device status {code} bits {bits}")
-    return {"metric": "mask tile-size ablation: speedup over the all-dense bitmap", "value": None, "unit": "x",
+    return {"metric": "tile-size ablation: speedup over the all-dense bitmap", "value": None, "unit": "x",
             "n_gpus": 1, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "LLaMA-2-7B q and gate, mask tiles 128..4, half of them sparse",
+            "config": {"workload": "LLaMA-2-7B q and gate, mask tiles 128..4, half of them sparse, "
+                                   "128 x 128 and (b <= 64) 64 x 64 execution tiles",
                        "l2": "weights rotate over copies holding 3x L2", "decode_M": 1, "prefill_M": 2048,
-                       "timing": "median of 5 rounds, each timing the all-dense layer then this one"},
+                       "timing": "median of 5 rounds, each timing the all-dense 128 x 128 layer then this one"},
+            "mma_probe": mma_rates(dev),
             "rows": rows}
 
 
 def mma_rates(dev, iters=20000, rounds=3):
-    """Tensor-core MMA rate probe (patch_mma_probe): dense and 2:4-sparse
-    rounds of M = 128, N = 240 MMAs on shared-memory operands, one CTA per SM,
-    alternated `rounds` times; the best of each, in dense-equivalent TFLOP/s,
-    and their ratio (the sparse half of the prefill path's mixed roofline)."""
+    """Tensor-core MMA rate probe (patch_mma_probe_m): dense and 2:4-sparse
+    rounds of M = 128 and M = 64, N = 240 MMAs on shared-memory operands, one
+    CTA per SM, alternated `rounds` times; the best of each, in
+    dense-equivalent TFLOP/s, and their ratios: sparse over dense is the
+    sparse half of the prefill path's mixed roofline, M = 64 over M = 128 the
+    hardware side of the tile-size trade-off (64 x 64 execution tiles run the
+    M = 64 forms)."""
     import torch
 
     import tile_sparse_gemm_b200 as tsg
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     status = tsg.new_status(dev)
-    best = {False: 0.0, True: 0.0}
-    for sparse in (False, True):  # warm-up (clocks up, code loaded)
-        tsg.patch_mma_probe(sparse, iters // 4, status)
+    forms = [(m, sparse) for m in (128, 64) for sparse in (False, True)]
+    best = {f: 0.0 for f in forms}
+    for m, sparse in forms:  # warm-up (clocks up, code loaded)
+        tsg.patch_mma_probe_m(m, sparse, iters // 4, status)
     torch.cuda.synchronize()
     for _ in range(rounds):
-        for sparse in (False, True):
+        for m, sparse in forms:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            tsg.patch_mma_probe(sparse, iters, status)
+            tsg.patch_mma_probe_m(m, sparse, iters, status)
             e1.record()
             torch.cuda.synchronize()
-            flops = sms * iters * 4 * 2 * 128 * 240 * (32 if sparse else 16)
-            best[sparse] = max(best[sparse], flops / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+            flops = sms * iters * 4 * 2 * m * 240 * (32 if sparse else 16)
+            best[(m, sparse)] = max(best[(m, sparse)], flops / (e0.elapsed_time(e1) * 1e-3) / 1e12)
     code, bits = tsg.patch_read_status(status)
     if code != 0:
         raise RuntimeError(f"mma probe: device status {code} bits {bits}")
-    return {"dense_tflops": round(best[False], 1), "sparse_tflops": round(best[True], 1),
-            "sparse_over_dense": round(best[True] / best[False], 3),
-            "how": f"patch_mma_probe: {sms} CTAs, {iters} rounds of four M=128 N=240 MMAs each (dense K=16, "
-                   "sparse K=32 dense-equivalent) on shared-memory operands, best of %d alternating runs" % rounds}
+    d, sp = best[(128, False)], best[(128, True)]
+    d64, sp64 = best[(64, False)], best[(64, True)]
+    return {"dense_tflops": round(d, 1), "sparse_tflops": round(sp, 1),
+            "sparse_over_dense": round(sp / d, 3),
+            "m64": {"dense_tflops": round(d64, 1), "sparse_tflops": round(sp64, 1),
+                    "dense_over_m128": round(d64 / d, 3), "sparse_over_m128": round(sp64 / sp, 3)},
+            "how": f"patch_mma_probe_m: {sms} CTAs, {iters} rounds of four M=128 (or M=64) N=240 MMAs each "
+                   "(dense K=16, sparse K=32 dense-equivalent) on shared-memory operands, best of %d alternating "
+                   "runs" % rounds}
 
 
 def job_times(ms, e2e_ms, world, dev=None):
