@@ -68,7 +68,8 @@ constexpr int A_BYTES = PATCH_PANEL_BYTES;
 constexpr int B_BYTES = BT * 64 * 2;
 constexpr int E_BYTES = PATCH_META_TILE_BYTES;
 constexpr int EPI_WARP0 = 8;             // warps 8-11 drain row 0, 12-15 row 1
-constexpr int YT = 16;                   // tokens per Y chunk the epilogue stores with one TMA store
+constexpr int YT = 16;                   // tokens per chunk of the split-K epilogue
+constexpr int YC = 32;                   // tokens per chunk of the whole-K epilogue (one 32-column TMEM load)
 constexpr int THREADS = 32 * (EPI_WARP0 + 4 * ROWS);
 constexpr int MAXTK = 128;               // descriptors of one tile row staged in shared memory (K <= 16384)
 constexpr uint32_t TMEM_COLS = 512;
@@ -82,7 +83,6 @@ struct Shared {
   alignas(1024) uint8_t a[ROWS][NA][A_BYTES];
   alignas(1024) uint8_t b[NB][B_BYTES];
   alignas(128) uint8_t e[ROWS][NE][E_BYTES];
-  alignas(128) uint16_t y[ROWS][2][YT][BM];  // epilogue: bf16 Y chunks (YT tokens x 128 features) per row, 2 buffers
   uint64_t a_full[ROWS][NA], a_empty[ROWS][NA], e_full[ROWS][NE], e_empty[ROWS][NE];
   uint64_t b_full[NB], b_empty[NB];   // b_empty: one arrival per row's MMA thread
   uint64_t acc_full[ROWS], acc_empty[ROWS], drain[ROWS];
@@ -328,11 +328,10 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
 }
 
 // Epilogue warp groups (4 warps each, one per TMEM lane quarter): per chunk
-// of YT tokens, each warp loads its 32 features x YT tokens from TMEM, rounds
-// to bf16 and writes them into a shared [YT][128] chunk; one thread then
-// stores the chunk to Y with a TMA store (full 256-byte rows of Y instead of
-// 64-byte pieces).  Two chunk buffers per group: a buffer is rewritten only
-// after the store that read it has finished reading.  Group g drains row g of
+// of YC tokens, each warp loads its 32 features x YC tokens from TMEM (one
+// load), rounds to bf16 and stores them to Y from registers: per token, the
+// warp's 32 features are 64 contiguous bytes.  No shared-memory staging, so
+// no barrier or wait on an earlier store per chunk.  Group g drains row g of
 // the pair; for the gated MLP both groups read both rows (gate and up of the
 // same 128 features) and take every other chunk: Y = silu(gate) * up.
 __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* a, uint32_t v) {
@@ -395,13 +394,11 @@ __device__ void epilogue_split(Shared& s, uint32_t tmem, const Args& p, const Un
   if (lane == 0) *counter = 0;  // ready for the next call
 }
 
-__device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, const Args& p) {
+__device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3;                  // the TMEM lane quarter this warp may access
   const int g = (warp - EPI_WARP0) >> 2;   // warp group
   const uint32_t bar_id = 1 + g;           // named barrier of the group's 128 threads
-  const bool leader = warp == EPI_WARP0 + 4 * g && lane == 0;
-  uint32_t chunk = 0;                      // chunks stored by this group so far (buffer = chunk & 1)
   int it = 0;
   for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
     const Unit u = unit_of(p, item);
@@ -420,34 +417,33 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, co
       const int valid = p.M - m0 < p.bt ? p.M - m0 : p.bt;  // tokens of this unit inside X
       const uint32_t lanes = tmem + (uint32_t(32 * q) << 16);
       const int c0 = p.mlp ? g : 0, dc = p.mlp ? 2 : 1;
-      for (int c = c0; c * YT < valid; c += dc, ++chunk) {
-        uint32_t v[YT];
+      // this thread's feature; a warp's 32 stores of one token fill 64 contiguous bytes of Y
+      uint16_t* yp = p.Y + int64_t(m0) * p.N + n0 + 32 * q + lane;
+      for (int c = c0; c * YC < valid; c += dc) {
+        uint32_t v[YC];
         if (p.mlp) {
-          uint32_t u[YT];
-          tmem_ld_16cols(lanes + uint32_t(YT * c), v);               // gate
-          tmem_ld_16cols(lanes + ACC_STRIDE + uint32_t(YT * c), u);  // up
 #pragma unroll
-          for (int j = 0; j < YT; ++j) {
-            // silu(gate) = gate / (1 + e^-gate), with CUDA's fast exponential and
-            // division (relative error ~1e-6, far below the bf16 rounding of H);
-            // a huge denominator gives -0 for a very negative gate
-            const float gate = __uint_as_float(v[j]);
-            v[j] = __float_as_uint(__fdividef(gate, 1.0f + __expf(-gate)) * __uint_as_float(u[j]));
+          for (int hh = 0; hh < YC / 16; ++hh) {  // in 16-column halves (registers)
+            uint32_t gt[16], u[16];
+            tmem_ld_16cols(lanes + uint32_t(YC * c + 16 * hh), gt);               // gate
+            tmem_ld_16cols(lanes + ACC_STRIDE + uint32_t(YC * c + 16 * hh), u);   // up
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              // silu(gate) = gate / (1 + e^-gate), with CUDA's fast exponential and
+              // division (relative error ~1e-6, far below the bf16 rounding of H);
+              // a huge denominator gives -0 for a very negative gate
+              const float gate = __uint_as_float(gt[j]);
+              v[16 * hh + j] = __float_as_uint(__fdividef(gate, 1.0f + __expf(-gate)) * __uint_as_float(u[j]));
+            }
           }
         } else {
-          tmem_ld_16cols(lanes + ACC_STRIDE * g + uint32_t(YT * c), v);
+          tmem_ld_32cols(lanes + ACC_STRIDE * g + uint32_t(YC * c), v);
         }
-        uint16_t(*buf)[BM] = s.y[g][chunk & 1];
+        uint16_t* yr = yp + int64_t(YC * c) * p.N;
+        const int nj = valid - YC * c < YC ? valid - YC * c : YC;
 #pragma unroll
-        for (int j = 0; j < YT; ++j) buf[j][32 * q + lane] = f32_to_bf16_rne(__uint_as_float(v[j]));
-        fence_proxy_async_smem();
-        if (leader) bulk_wait_read_all();  // the previous chunk's store has read the other buffer
-        named_bar_sync(bar_id, 128);
-        // token rows past M are clipped by the store
-        if (leader) {
-          tma_store_2d(tmap_y, buf, n0, m0 + YT * c);
-          bulk_commit_group();
-        }
+        for (int j = 0; j < YC; ++j, yr += p.N)
+          if (j < nj) *yr = f32_to_bf16_rne(__uint_as_float(v[j]));
       }
     }
     tc_fence_before();
@@ -457,12 +453,11 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const CUtensorMap* tmap_y, co
       if (p.mlp) mbar_arrive(&s.acc_empty[g ^ 1]);
     }
   }
-  if (leader) bulk_wait_all();  // Y written before the CTA exits
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w0,
-                   const __grid_constant__ CUtensorMap tmap_w1, const __grid_constant__ CUtensorMap tmap_y,
+                   const __grid_constant__ CUtensorMap tmap_w1,
                    const Args p) {
   extern __shared__ uint8_t smem_raw[];
   Shared& s = *reinterpret_cast<Shared*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -494,7 +489,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     prefetch_tensormap(&tmap_x);
     prefetch_tensormap(&tmap_w0);
     prefetch_tensormap(&tmap_w1);
-    prefetch_tensormap(&tmap_y);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -521,7 +515,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) producer_x(s, &tmap_x, p);
     __syncwarp();
   } else if (warp >= EPI_WARP0) {
-    epilogue(s, tmem, &tmap_y, p);
+    epilogue(s, tmem, p);
   }
 
   tc_fence_before();
@@ -582,18 +576,6 @@ bool make_map_2d_bf16_sw64(CUtensorMap* map, const void* base, uint64_t inner, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Y [M][N] bf16 as a TMA store target: boxes of 16 token rows x 128 features,
-// no swizzle (the epilogue writes the chunk row-major).
-static bool make_map_y(CUtensorMap* map, void* Y, uint64_t N, uint64_t M) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {N, M};
-  const cuuint64_t strides[1] = {N * 2};
-  const cuuint32_t box[2] = {uint32_t(prefill::BM), uint32_t(prefill::YT)};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 // Tokens per unit: the multiple of 16 in [64, BT] that minimises the time of
 // the slowest CTA, modelled as (units per CTA, rounded up) x (unit time).  A
@@ -657,7 +639,7 @@ static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch
   if (plan.ks > 1 && (!workspace || workspace_bytes < kDecodeCounterBytes + plan.part_bytes))
     plan = prefill_plan(M, n_pairs, Tk, num_sms, false);
   const int bt = plan.bt;
-  CUtensorMap tmap_x, tmap_w0, tmap_w1, tmap_y;
+  CUtensorMap tmap_x, tmap_w0, tmap_w1;
   if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W0.K), uint64_t(M), uint64_t(W0.K) * 2, 64, uint32_t(bt)))
     return cudaErrorUnknown;
   const patch_weight* Ws[2] = {&W0, &W1};
@@ -667,7 +649,6 @@ static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch
     const uint64_t n_panels = uint64_t(2 * (T - Ws[r]->n_sparse) + Ws[r]->n_sparse);
     if (!make_map_2d_bf16(maps[r], Ws[r]->values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
   }
-  if (!make_map_y(&tmap_y, Y, uint64_t(Tn * BM), uint64_t(M))) return cudaErrorUnknown;
   Args p;
   for (int r = 0; r < ROWS; ++r) {
     p.meta[r] = static_cast<const uint8_t*>(Ws[r]->meta);
@@ -695,7 +676,7 @@ static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES));
   if (e != cudaSuccess) return e;
   return launch_pdl(prefill_kernel, dim3(unsigned(grid)), dim3(THREADS), SMEM_BYTES, stream, tmap_x, tmap_w0, tmap_w1,
-                    tmap_y, p);
+                    p);
 }
 
 cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,
