@@ -28,12 +28,14 @@
 // Launch: a plan kernel first writes, for every panel of every call, the tile
 // it belongs to (tile index, half, kind, sparse ordinal); then the chain
 // kernel runs cooperatively (all CTAs resident: they wait on each other's
-// completion counters), one CTA per SM.  Roles per CTA (8 warps): warp 0 W
-// producer, warp 6 X producer (panel records, metadata, X slices, the
-// dependency waits), warps 1 and 7 MMA issuers (warp 1 owns TMEM), each
-// issuing half of every panel's MMAs into its own accumulator (one thread
-// issuing all of them caps an SM at ~5.5 TB/s of weight panels, two reach the
-// memory's ~7 TB/s), warps 2-5 epilogue.
+// completion counters), one CTA per SM.  Roles per CTA (9 warps): warp 0 W
+// producer, warps 6 and 8 X producers (panel records, metadata, X slices, the
+// dependency waits; each takes every other panel: one thread's turn per panel,
+// up to three copies and the record bookkeeping, took ~420 ns and set the pace
+// of the whole ring at ~5.5 TB/s), warps 1 and 7 MMA issuers (warp 1 owns
+// TMEM), each issuing half of every panel's MMAs into its own accumulator (one
+// thread issuing all of them caps an SM at ~5.5 TB/s of weight panels, two
+// reach the memory's ~7 TB/s), warps 2-5 epilogue.
 // Every wait, on an mbarrier or on another CTA's counter, is bounded in time.
 #include <cuda.h>
 
@@ -54,7 +56,7 @@ constexpr int A_BYTES = PATCH_PANEL_BYTES;
 constexpr int X_BYTES = BT * 64 * 2;     // one 64-k slice of X (room for 16 token rows)
 constexpr int E_BYTES = PATCH_META_TILE_BYTES;
 constexpr int NISS = 2;                  // MMA-issuing threads, each half of every panel's K
-constexpr int THREADS = 256;             // warps: 0 W producer, 1 and 7 MMA, 2-5 epilogue, 6 X producer
+constexpr int THREADS = 288;             // warps: 0 W producer, 1 and 7 MMA, 2-5 epilogue, 6 and 8 X producers
 constexpr uint32_t TMEM_COLS = 256;
 // accumulator of segment buffer b, issuer u: columns (NISS b + u) BT; issuer u's
 // metadata slot of stage st: META_COL0 + 4 (NS u + st)
@@ -86,6 +88,7 @@ struct Shared {
   alignas(16) uint2 rec[2][RECBUF + 2];  // the X producer's panel records, by call parity
   uint64_t full[NS], empty[NS];
   uint64_t acc_full[NACC], acc_empty[NACC], drain[NISS], rec_full[2];
+  uint64_t rec_empty[2];  // X producer 1 is done with the chunk in buffer b
   uint32_t info[NS];
   uint32_t tmem_base;
   int abort_flag;
@@ -307,23 +310,31 @@ __device__ __forceinline__ void stage_chunk(Shared& s, const Args& a, const Chun
   bulk_load(s.rec[k & 1], cl.rec + q0, bytes, &s.rec_full[k & 1]);
 }
 
-// X producer: per panel its record (tile, half, kind), the stage's info word,
-// a sparse tile's metadata and the panel's X slices.  A call that reads the
-// output of earlier calls loads its first X slice only after they have
-// completed on every CTA.
-__device__ void producer_x(Shared& s, const Maps& maps, const Args& a) {
+// X producer `par` (0 or 1): for the CTA's panels i with i % 2 == par, the
+// panel's record (tile, half, kind), the stage's info word, a sparse tile's
+// metadata and the panel's X slices.  A call that reads the output of earlier
+// calls loads its X slices only after they have completed on every CTA.
+// Producer 0 stages the record chunks, producer 1 tells it (rec_empty) when it
+// is done with a buffer, so the chunk two ahead may overwrite it.
+__device__ void producer_x(Shared& s, const Maps& maps, const Args& a, int par) {
   const int64_t G = gridDim.x, c = blockIdx.x;
   uint32_t i = 0;
   bool ok = true;
   uint32_t staged = 0, waited = 0;  // record chunks copied / waited for; chunk n uses buffer n & 1
   ChunkIter cur;
   chunk_first(a, cur);
-  if (cur.j < a.J) stage_chunk(s, a, cur, staged++);
+  if (par == 0 && cur.j < a.J) stage_chunk(s, a, cur, staged++);
   while (ok && cur.j < a.J) {
-    // stage the chunk after this one into the other buffer (it held the chunk before, which is done)
+    // stage the chunk after this one into the other buffer, once producer 1
+    // is done with the chunk before this one, which that buffer held
     ChunkIter nxt = cur;
     chunk_next(a, nxt);
-    if (nxt.j < a.J) stage_chunk(s, a, nxt, staged++);
+    if (par == 0 && nxt.j < a.J) {
+      if (staged >= 2 && !(ok = wait_bounded(&s.rec_empty[staged & 1], ((staged >> 1) - 1) & 1, &s.abort_flag,
+                                             a.limit_ns, a.status, false)))
+        break;
+      stage_chunk(s, a, nxt, staged++);
+    }
     if (!(ok = wait_bounded(&s.rec_full[waited & 1], (waited >> 1) & 1, &s.abort_flag, a.limit_ns, a.status, false)))
       break;
     const uint2* recs = s.rec[waited & 1];
@@ -337,6 +348,7 @@ __device__ void producer_x(Shared& s, const Maps& maps, const Args& a) {
     const uint32_t xb = uint32_t(cl.M) * 128;  // an X slice holds M token rows
     bool dep_ok = !cl.after || j == 0 || cb > p0;  // waited for at the call's first chunk
     for (int64_t p = cb; p < ce; ++p, ++i) {
+      if ((i & 1u) != uint32_t(par)) continue;  // the other producer's panel
       const uint32_t st = i % NS;
       if (!(ok = wait_bounded(&s.empty[st], ((i / NS) & 1) ^ 1, &s.abort_flag, a.limit_ns, a.status, false)))
         break;
@@ -363,13 +375,15 @@ __device__ void producer_x(Shared& s, const Maps& maps, const Args& a) {
       if (sparse) bulk_load(s.st[st].e, cl.meta + uint64_t(r.y >> 2) * E_BYTES, E_BYTES, &s.full[st]);
       load_x(s.st[st], &s.full[st], &maps.x[j], kt, h, sparse);
     }
+    if (par == 1) mbar_arrive(&s.rec_empty[(waited - 1) & 1]);  // done with this chunk's buffer
     cur = nxt;
   }
   // every copy issued must have landed before the CTA may exit
   for (uint32_t k = waited; k < staged; ++k)
     wait_bounded(&s.rec_full[k & 1], (k >> 1) & 1, &s.abort_flag, drain_limit(a), a.status, true);
   for (uint32_t k = (i > NS ? i - NS : 0); k < i; ++k)
-    wait_bounded(&s.full[k % NS], (k / NS) & 1, &s.abort_flag, drain_limit(a), a.status, true);
+    if ((k & 1u) == uint32_t(par))
+      wait_bounded(&s.full[k % NS], (k / NS) & 1, &s.abort_flag, drain_limit(a), a.status, true);
 }
 
 // MMA issuer u (one thread each, u = 0, 1): every panel's four MMAs are split
@@ -587,6 +601,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&s.drain[1], 1);
     mbar_init(&s.rec_full[0], 1);
     mbar_init(&s.rec_full[1], 1);
+    mbar_init(&s.rec_empty[0], 1);
+    mbar_init(&s.rec_empty[1], 1);
     s.abort_flag = 0;
     fence_barrier_init();
   }
@@ -606,8 +622,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1 || warp == 7) {
     if (lane == 0) mma_issuer(s, tmem, a, warp == 1 ? 0 : 1);
     __syncwarp();
-  } else if (warp == 6) {
-    if (lane == 0) producer_x(s, maps, a);
+  } else if (warp == 6 || warp == 8) {
+    if (lane == 0) producer_x(s, maps, a, warp == 6 ? 0 : 1);
     __syncwarp();
   } else {
     epilogue(s, tmem, a);
