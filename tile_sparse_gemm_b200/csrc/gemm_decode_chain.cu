@@ -50,7 +50,7 @@ using namespace tc;
 
 constexpr int BM = 128;
 constexpr int BT = 16;                   // MMA N (tokens)
-constexpr int NS = 9;                    // pipeline stages per CTA (one CTA per SM)
+constexpr int NS = 10;                   // pipeline stages per CTA (one CTA per SM)
 constexpr int NACC = 2;                  // accumulator buffers
 constexpr int A_BYTES = PATCH_PANEL_BYTES;
 constexpr int X_BYTES = BT * 64 * 2;     // one 64-k slice of X (room for 16 token rows)
