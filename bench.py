@@ -1139,6 +1139,13 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
             t = time_calls(args, layers, packed, calls, dev, world, status)
             if M <= 16:
                 out[f"M={M}"] = bytes_block(args, workload, layers, calls, t, pk, world)
+                # the same GEMMs as the independent GEMMs they are here, in one launch
+                seg = [(0, len(calls))]
+                t = time_calls(args, layers, packed, calls, dev, world, status, segments=seg, chain=True, after=False)
+                ch = bytes_block(args, workload, layers, calls, t, pk, world, seg, [f"M={M}"], chain=True)
+                out[f"M={M}"]["chain_independent"] = dict(
+                    ch, step="one patch_gemm_chain over the 14 GEMMs as the independent GEMMs they are here "
+                             "(no call waits; the CTAs split the launch's whole panel sequence)")
             else:
                 out[f"M={M}"] = flops_block(args, workload, layers, calls, t, pk, world, sparse_ratio)[0]
     else:

@@ -152,6 +152,7 @@ def test_run_ours_assembles_every_block_on_fake_timings(monkeypatch):
     for key in ("chain", "chain_independent"):
         assert "ms_per_pass" in out["stack"][key]
     assert set(out["llama3_qwen"]) >= {"M=1", "M=512"}
+    assert out["llama3_qwen"]["M=1"]["chain_independent"]["value"] > 0
     import json
     json.dumps(out)  # serialisable
 
