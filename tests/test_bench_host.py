@@ -6,6 +6,7 @@ import os
 import sys
 
 import numpy as np
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -112,7 +113,8 @@ def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(2.0, 5, 4, 1000.0) == 2.0 * 5 * 4
 
 
-def test_run_ours_assembles_every_block_on_fake_timings(monkeypatch):
+@pytest.mark.parametrize("workload", ["all", "decode", "decode_fused", "prefill", "stack", "llama3_qwen"])
+def test_run_ours_assembles_every_block_on_fake_timings(monkeypatch, workload):
     """The default run's JSON assembly (every block and mode) on CPU: GPU work is
     replaced by fakes that return fixed timings, so a missing or misnamed key in
     any block fails here rather than on the GPU machine."""
@@ -142,8 +144,13 @@ def test_run_ours_assembles_every_block_on_fake_timings(monkeypatch):
     import tile_sparse_gemm_b200 as tsg
     monkeypatch.setattr(tsg, "new_status", lambda dev=None: None)
     args = types.SimpleNamespace(steps=4, warmup=3, no_graph=False, layers=None, fracs=None, tokens=None,
-                                 shard=False, workload="all")
+                                 shard=False, workload=workload)
     out = bench.run_ours(args, 0, 1)
+    for key in ("metric", "value", "unit", "ms_per_step", "roofline", "e2e", "clocks", "config", "gpu_launches"):
+        assert key in out, key  # every workload alone gives a full line
+    assert out["value"] > 0
+    if workload != "all":
+        return
     for key in ("metric", "value", "unit", "ms_per_step", "roofline", "e2e", "clocks", "config", "gpu_launches",
                 "separate_calls", "chain_dependent", "prefill", "stack", "llama3_qwen", "mma_probe"):
         assert key in out, key
