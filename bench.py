@@ -733,7 +733,7 @@ def pack_layers(layers, dev, status):
 
 
 def time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False, after=True,
-               gather=None):
+               gather=None, group=False):
     """Device time of K steps of `calls` (each a patch_gemm), and the same steps
     end to end with host buffers.
 
@@ -747,7 +747,9 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
     calls; with `after` every call waits for the previous one's completion
     before reading its X (the ordering of separate calls on one stream),
     without it the calls run as the independent GEMMs they are (each X is an
-    input of the step, not an earlier call's output).
+    input of the step, not an earlier call's output).  With `group` (and
+    `chain`), a step is one patch_gemm_group per segment instead: the
+    independent GEMMs in one launch of the prefill kernel.
     With `gather` (column-parallel shards, one per rank), every step ends with
     one NCCL all-gather of all ranks' Y shards (padded to `gather` elements
     each), and the steps run eagerly (no graph).
@@ -780,12 +782,15 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
         views[0][0][j].copy_(torch.from_numpy(layers[li]["xs"][M].view(np.int16)).view(torch.bfloat16))
     ws_bytes = max(tsg.patch_gemm_workspace_size(M, packed[li]) for li, M in calls)
     chains = None
-    if chain:  # per buffer set, one chain per segment; every call waits for the previous one
+    if chain and group:  # per buffer set, one group launch per segment
+        chains = [{(lo, hi): tsg.Group([(views[b][0][j], packed[calls[j][0]], views[b][1][j])
+                                        for j in range(lo, hi)], status) for lo, hi in segments} for b in range(2)]
+    elif chain:  # per buffer set, one chain per segment; every call waits for the previous one
         chains = [{(lo, hi): tsg.Chain([(views[b][0][j], packed[calls[j][0]], views[b][1][j], after)
                                         for j in range(lo, hi)]) for lo, hi in segments} for b in range(2)]
         ws_bytes = max([ws_bytes] + [ch.workspace_bytes for ch in chains[0].values()])
     ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)  # zero-filled once, left zeroed by each call
-    if chain:
+    if chain and not group:
         for per_set in chains:
             for ch in per_set.values():
                 ch.workspace, ch.status = ws, status
@@ -927,9 +932,14 @@ def time_calls(args, layers, packed, calls, dev, world, status, segments=None, c
     del stage_graphs
     e2e_ms = e0.elapsed_time(e1)
     ms, e2e_ms = job_times(ms, e2e_ms, world, dev)
-    # kernels per step: one per patch_gemm call, or a plan kernel and a chain kernel per chain launch
-    per_step = sum(2 * ((hi - lo + tsg.CHAIN_MAX_CALLS - 1) // tsg.CHAIN_MAX_CALLS) for lo, hi in segments) \
-        if chain else len(calls)
+    # kernels per step: one per patch_gemm call, a plan kernel and a chain kernel per chain launch,
+    # or one prefill kernel per group launch
+    if chain and group:
+        per_step = sum((hi - lo + tsg.GROUP_MAX_CALLS - 1) // tsg.GROUP_MAX_CALLS for lo, hi in segments)
+    elif chain:
+        per_step = sum(2 * ((hi - lo + tsg.CHAIN_MAX_CALLS - 1) // tsg.CHAIN_MAX_CALLS) for lo, hi in segments)
+    else:
+        per_step = len(calls)
     return {"ms": ms, "e2e_ms": e2e_ms, "seg_ms": seg_ms, "clocks": clocks.summary(), "h2d": h2d, "d2h": d2h,
             "launches": per_step * args.steps}
 
@@ -1015,6 +1025,33 @@ def flops_block(args, name, layers, calls, t, pk, world, sparse_ratio=None, traf
     return out, split
 
 
+def group_flops_block(args, layers, calls, t, pk, world, segments, seg_names, sparse_ratio=None):
+    """A TFLOP/s block for calls timed as patch_gemm_group launches (one per
+    segment): the dense-equivalent FLOPs and mixed roofline of flops_block,
+    over the whole step and per segment."""
+    P = pk["bf16_tflops"]
+    alg = np.array([call_flops(layers[li], M) for li, M in calls], dtype=np.float64)
+    t2 = np.array([roof_seconds(layers[li], M, P, 2.0) for li, M in calls])
+    seg_fl = np.array([alg[lo:hi].sum() for lo, hi in segments])
+    split = split_of(t, seg_fl, args.steps)
+    out = block_common(args, t, alg.sum() / 1e12, "TFLOP/s", world)
+    roof = {"bound": "tensor", "achieved": round(float(alg.sum() / 1e12 / (split.sum() / 1e3)), 1), "peak": P,
+            "unit": "TFLOP/s", "frac": round(float(t2.sum() / (split.sum() / 1e3)), 4), "traffic": None,
+            "kernel": "prefill_kernel (patch_gemm_group)", "peak_source": pk["source"],
+            "note": "frac = mixed roofline time (dense tiles at the dense peak, sparse tiles at 2x it) / measured"}
+    if sparse_ratio:
+        tm = np.array([roof_seconds(layers[li], M, P, sparse_ratio) for li, M in calls])
+        roof["sparse_ratio_measured"] = round(sparse_ratio, 3)
+        roof["frac_measured_sparse_peak"] = round(float(tm.sum() / (split.sum() / 1e3)), 4)
+    out["roofline"] = roof
+    if len(segments) > 1:
+        out["per_segment"] = {n: {"us": round(1e3 * split[s], 1),
+                                  "TFLOP/s": round(seg_fl[s] / 1e12 / (split[s] / 1e3), 1),
+                                  "roofline_frac": round(float(t2[lo:hi].sum()) / (split[s] / 1e3), 3)}
+                              for s, (n, (lo, hi)) in enumerate(zip(seg_names, segments))}
+    return out
+
+
 def sweep_summary(layers, calls, split):
     """Per shape: TFLOP/s at each sparse-tile fraction, speedup over the same
     shape packed all-dense (f = 0, same kernel), and whether time falls (so
@@ -1093,6 +1130,16 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
                          "sparse_tile_fraction": sorted({L["frac"] for L in layers}),
                          "resident_weight_bytes": resident,
                          "l2": "inputs larger than L2 (X 16-45 MB and W 26-90 MB per call, 35 calls in rotation)"}
+        # the same 35 GEMMs, those of one sparse-tile fraction (the 7 shapes) per patch_gemm_group launch
+        calls_g = sorted(calls, key=lambda c: layers[c[0]]["frac"])
+        fr = [layers[li]["frac"] for li, _ in calls_g]
+        seg = [(fr.index(f), len(fr) - fr[::-1].index(f)) for f in sorted(set(fr))]
+        tg = time_calls(args, layers, packed, calls_g, dev, world, status, segments=seg, chain=True, group=True)
+        out["group"] = dict(
+            group_flops_block(args, layers, calls_g, tg, pk, world, seg, [f"f={f}" for f in sorted(set(fr))],
+                              sparse_ratio),
+            step="the same 35 GEMMs as 5 patch_gemm_group launches, one per sparse-tile fraction over the 7 "
+                 "shapes (independent GEMMs whose units share one grid)")
         if full:
             out["gated_mlp"] = mlp_steps(dev, pk)
     elif workload == "stack":
@@ -1148,6 +1195,14 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
                              "(no call waits; the CTAs split the launch's whole panel sequence)")
             else:
                 out[f"M={M}"] = flops_block(args, workload, layers, calls, t, pk, world, sparse_ratio)[0]
+                # the same independent GEMMs in one patch_gemm_group launch
+                seg = [(0, len(calls))]
+                t = time_calls(args, layers, packed, calls, dev, world, status, segments=seg, chain=True,
+                               group=True)
+                out[f"M={M}"]["group"] = dict(
+                    group_flops_block(args, layers, calls, t, pk, world, seg, [f"M={M}"], sparse_ratio),
+                    step=f"one patch_gemm_group over the {len(calls)} GEMMs as the independent GEMMs they are "
+                         "(their units share one grid of the prefill kernel)")
     else:
         raise ValueError(workload)
     del packed

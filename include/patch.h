@@ -390,6 +390,41 @@ PATCH_API patch_status_t patch_gemm_chain(const patch_chain_call *calls, int64_t
                                           uint64_t wait_limit_us);
 
 /*
+ * patch_gemm_group: independent GEMMs Y_j = X_j * W_j_eff^T, each with any
+ * token count, run by one persistent launch of the prefill kernel per up to
+ * PATCH_GROUP_MAX_CALLS calls ("Inference & Deployment": the same hybrid
+ * execution as patch_gemm's prefill path: dense tiles on the dense
+ * tensor-core MMA, sparse tiles on the 2:4 sparse one, fp32 accumulation in
+ * tensor memory, one rounding to bf16).
+ *
+ * A prefill GEMM of few tile rows or few tokens (the projections of a small
+ * model, or k and v beside q) has fewer units (2 tile rows x up to 240
+ * tokens) than the GPU has SMs, and as its own kernel it also pays its
+ * set-up, first loads and last partial wave.  Here the units of all the
+ * calls share one grid: the CTAs take them in turn, those of the calls with
+ * the costliest units first.  Token blocks are the fewest of at most 240
+ * tokens, evened out (M = 512: three of 176).
+ *
+ *   calls[j].X, .Y, .W, .M as for patch_gemm_chain, but M may be any value
+ *       0 .. 2^30 (0: the call is skipped; M <= 16 runs in 16-token units on
+ *       the tensor-core prefill kernel, where patch_gemm_chain is faster)
+ *   calls[j].after_previous must be 0: the calls are independent, and no
+ *       call may write memory that another call of the group reads or writes
+ *   calls[j].reserved: ignored
+ * No workspace: K is never split.  Results: within the GEMM tolerance of
+ * patch_gemm's (the token blocking, and so the order in which each output's
+ * fp32 partial sums add up, may differ), deterministic run to run.  Every
+ * wait is bounded by wait_limit_us (0 = 2 s); on expiry PATCH_DEV_TIMEOUT is
+ * set in *dev_status and the Y_j are undefined.
+ * Errors: PATCH_ERR_INVALID_ARG (NULL, M outside 0..2^30, after_previous set,
+ * n_calls < 0), PATCH_ERR_SHAPE, PATCH_ERR_ALIGN, PATCH_ERR_DEVICE,
+ * PATCH_ERR_CUDA.
+ */
+#define PATCH_GROUP_MAX_CALLS 32
+PATCH_API patch_status_t patch_gemm_group(const patch_chain_call *calls, int64_t n_calls, int32_t *dev_status,
+                                          void *stream, uint64_t wait_limit_us);
+
+/*
  * patch_gemm_decode_noalloc: the decode GEMM (M <= 16) for callers that
  * cannot allocate device memory.  The paper has no counterpart; this is a
  * deployment convenience of this library.

@@ -124,6 +124,30 @@ def test_64_tile_format_host_checks(lib):
     assert lib.patch_mma_probe_m(96, 0, 10, fake, None) == 1
 
 
+def test_group_host_checks(lib):
+    """patch_gemm_group refuses bad calls before any device query or launch, and
+    a group of empty calls is a no-op."""
+    P = ctypes.c_void_p
+    fake = 0x10000
+    w = tsg._Weight(256, 256, 0, fake, None, fake)
+
+    def group(*calls, status=P(fake)):
+        arr = (tsg._ChainCall * len(calls))(*calls)
+        return lib.patch_gemm_group(ctypes.cast(arr, P), len(calls), status, None, 0)
+
+    assert group(tsg._ChainCall(None, None, w, 0, 0, 0)) == 0                         # empty call: no-op
+    assert lib.patch_gemm_group(None, 0, P(fake), None, 0) == 0                       # no calls
+    assert lib.patch_gemm_group(None, 1, P(fake), None, 0) == 1                       # NULL calls
+    assert group(tsg._ChainCall(fake, fake, w, 4, 0, 0), status=None) == 1            # NULL status
+    assert group(tsg._ChainCall(fake, fake, w, -1, 0, 0)) == 1                        # negative M
+    assert group(tsg._ChainCall(fake, fake, w, 4, 1, 0)) == 1                         # after_previous set
+    assert group(tsg._ChainCall(fake, None, w, 4, 0, 0)) == 1                         # NULL Y
+    assert group(tsg._ChainCall(fake + 2, fake, w, 4, 0, 0)) == 3                     # misaligned X
+    assert group(tsg._ChainCall(fake, fake, tsg._Weight(256, 200, 0, fake, None, fake), 4, 0, 0)) == 2
+    # the first bad call decides, even after good ones
+    assert group(tsg._ChainCall(None, None, w, 0, 0, 0), tsg._ChainCall(fake, fake, w, 4, 1, 0)) == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(tsg, "_lib", None)
     monkeypatch.setattr(tsg, "_LIB_PATH", tmp_path / "libpatch.so")

@@ -127,7 +127,7 @@ def test_run_ours_assembles_every_block_on_fake_timings(monkeypatch, workload):
             self.stored_bytes = bench.stored_bytes(L["N"], L["K"], int(L["bm"].sum()))
 
     def fake_time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False, after=True,
-                        gather=None):
+                        gather=None, group=False):
         segs = segments or ([(0, len(calls))] if chain else [(j, j + 1) for j in range(len(calls))])
         return {"ms": 1.0 * args.steps, "e2e_ms": 2.0 * args.steps, "seg_ms": None, "clocks": {"sm_mhz": 1965.0},
                 "h2d": 1, "d2h": 1, "launches": len(segs)}
@@ -160,6 +160,8 @@ def test_run_ours_assembles_every_block_on_fake_timings(monkeypatch, workload):
         assert "ms_per_pass" in out["stack"][key]
     assert set(out["llama3_qwen"]) >= {"M=1", "M=512"}
     assert out["llama3_qwen"]["M=1"]["chain_independent"]["value"] > 0
+    assert out["llama3_qwen"]["M=512"]["group"]["value"] > 0 and "frac" in out["llama3_qwen"]["M=512"]["group"]["roofline"]
+    assert set(out["prefill"]["group"]["per_segment"]) == {f"f={f}" for f in bench.FRACS}
     import json
     json.dumps(out)  # serialisable
 

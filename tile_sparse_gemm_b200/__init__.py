@@ -18,6 +18,7 @@ Entry points (same names as the C ABI):
     patch_gemm_mlp, patch_tile_kinds, patch_pack_from_logits, patch_soft_mask,
     patch_hard_mask_tiles, patch_exec_tiles, shard_rows / shard_of,
     patch_gemm_chain / Chain (a sequence of decode GEMMs in one launch; see each docstring)
+    patch_gemm_group / Group (independent GEMMs of any token count in one prefill launch)
     64 x 64 execution tiles: patch_pack64_sizes, patch_exec_tiles64, patch_pack64 -> PackedWeight64,
     patch_gemm64_workspace_size, patch_gemm64; patch_mma_probe_m (M = 64 or 128 MMA rate)
 Helpers of this binding: save_packed(weight, path) / load_packed(path) keep a
@@ -66,6 +67,7 @@ class _ChainCall(ctypes.Structure):
 
 
 CHAIN_MAX_CALLS = 64  # calls per launch of patch_gemm_chain (longer chains take several launches)
+GROUP_MAX_CALLS = 32  # calls per launch of patch_gemm_group
 
 
 _lib = None
@@ -98,6 +100,7 @@ def lib() -> ctypes.CDLL:
             "patch_gemm_mlp": [P, I64, WP, WP, P, P, SZ, P, P],
             "patch_gemm_chain_workspace_size": [P, I64, ctypes.POINTER(SZ)],
             "patch_gemm_chain": [P, I64, P, SZ, P, P, ctypes.c_uint64],
+            "patch_gemm_group": [P, I64, P, P, ctypes.c_uint64],
             "patch_mma_probe": [I32, I64, P, P],
             "patch_mma_probe_m": [I32, I32, I64, P, P],
             "patch_pack64_sizes": [I64, I64, I64, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)],
@@ -420,6 +423,44 @@ def patch_gemm_chain(calls, workspace: torch.Tensor | None = None, status: torch
                      wait_limit_us: int = 0, stream=None) -> list[torch.Tensor]:
     """One launch (per 64 calls) of a sequence of decode GEMMs: see Chain."""
     return Chain(calls, workspace, status).run(wait_limit_us, stream)
+
+
+class Group:
+    """A fixed set of independent GEMMs (any token counts) for patch_gemm_group.
+
+    calls: list of (X, weight, Y) with X bf16 [M][K] and Y bf16 [M][N] device
+    tensors (Y None allocates it); no call may write memory another call reads
+    or writes.  The ctypes array of calls is built once; run() launches the
+    group on the current stream (capturable in a CUDA graph after one eager run)."""
+
+    def __init__(self, calls, status: torch.Tensor | None = None):
+        self.Y = []
+        arr = (_ChainCall * len(calls))()
+        self._keep = []
+        for j, (X, weight, Y) in enumerate(calls):
+            M, K = X.shape
+            if K != weight.K:
+                raise ValueError(f"call {j}: X has K={K}, weight has K={weight.K}")
+            if Y is None:
+                Y = torch.empty((M, weight.N), dtype=torch.bfloat16, device=X.device)
+            arr[j] = _ChainCall(_dev(X, "X") if M else None, _dev(Y, "Y") if M else None, weight.struct(), M, 0, 0)
+            self.Y.append(Y)
+            self._keep += [X, Y, weight]
+        self.calls = arr
+        self.n = len(calls)
+        dev = calls[0][0].device if calls else None
+        self.status = new_status(dev) if status is None else status
+
+    def run(self, wait_limit_us: int = 0, stream=None):
+        _check(lib().patch_gemm_group(ctypes.cast(self.calls, ctypes.c_void_p), self.n, _dev(self.status, "status"),
+                                      _stream(stream), wait_limit_us), "patch_gemm_group")
+        return self.Y
+
+
+def patch_gemm_group(calls, status: torch.Tensor | None = None, wait_limit_us: int = 0,
+                     stream=None) -> list[torch.Tensor]:
+    """One prefill launch (per 32 calls) of independent GEMMs: see Group."""
+    return Group(calls, status).run(wait_limit_us, stream)
 
 
 def patch_gemm_mlp(X: torch.Tensor, gate: PackedWeight, up: PackedWeight, H: torch.Tensor | None = None,

@@ -365,6 +365,36 @@ patch_status_t patch_gemm_chain(const patch_chain_call* calls, int64_t n_calls, 
   return PATCH_OK;
 }
 
+patch_status_t patch_gemm_group(const patch_chain_call* calls, int64_t n_calls, int32_t* dev_status, void* stream,
+                                uint64_t wait_limit_us) {
+  if (!dev_status || n_calls < 0 || (n_calls > 0 && !calls)) return PATCH_ERR_INVALID_ARG;
+  std::vector<PrefillGroupCall> cs;
+  for (int64_t j = 0; j < n_calls; ++j) {
+    const patch_chain_call& c = calls[j];
+    if (c.M < 0 || c.M > (int64_t(1) << 30) || c.after_previous != 0) return PATCH_ERR_INVALID_ARG;
+    patch_status_t st = check_weight(&c.W);
+    if (st != PATCH_OK) return st;
+    if (c.M == 0) continue;
+    if (!c.X || !c.Y) return PATCH_ERR_INVALID_ARG;
+    if (!aligned16(c.X) || !aligned16(c.Y)) return PATCH_ERR_ALIGN;
+    cs.push_back(PrefillGroupCall{c.X, c.M, c.W, c.Y});
+  }
+  if (cs.empty()) return PATCH_OK;
+  int sms = 0;
+  patch_status_t st = device_sms(&sms);
+  if (st != PATCH_OK) return st;
+  for (const PrefillGroupCall& c : cs) PATCH_DEBUG_CHECK(&c.W, dev_status, stream);
+  const uint64_t limit_ns = (wait_limit_us ? wait_limit_us : 2000000ull) * 1000ull;
+  const int n = int(cs.size());
+  for (int j0 = 0; j0 < n; j0 += kPrefillGroupMax) {
+    const int cnt = n - j0 < kPrefillGroupMax ? n - j0 : kPrefillGroupMax;
+    if (launch_prefill_group(cs.data() + j0, cnt, dev_status, sms, limit_ns, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+      return PATCH_ERR_CUDA;
+  }
+  return PATCH_OK;
+}
+
 // decode scratch for the gated MLP: [decode GEMM workspace][G][U], 256-byte aligned parts
 static size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
 

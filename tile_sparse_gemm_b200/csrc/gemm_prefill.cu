@@ -49,6 +49,10 @@
 // freed before the CTA exits.  No cluster multicast is used anywhere.
 #include <cuda.h>
 
+#include <algorithm>
+#include <memory>
+#include <vector>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc_ptx.cuh"
@@ -95,21 +99,66 @@ struct Shared {
 constexpr size_t SMEM_BYTES = sizeof(Shared) + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
-struct Args {
-  const uint8_t* meta[ROWS];          // row r of a unit reads weight r (the same weight unless mlp)
-  const patch_tile_desc* desc[ROWS];
-  int mlp;                            // 1: row 0 = gate, row 1 = up tile row rp; Y = silu(gate) * up
+// One GEMM of a launch.  A launch runs one GEMM (patch_gemm, the gated MLP)
+// or a group of independent ones (patch_gemm_group) whose units share the
+// CTAs: items [item0, next GEMM's item0) are this GEMM's units.
+struct Gemm {
+  const uint8_t* meta;
+  const patch_tile_desc* desc;
   uint16_t* Y;
-  int M, N, Tn, Tk, n_pairs, n_tb, n_items;  // units: see unit_of()
-  int ks;                      // K parts per output block (split K; 1 = whole K per unit)
+  int M, N, Tn, Tk, n_pairs, n_tb;  // units: see unit_of()
+  int bt;                      // tokens per unit: a multiple of 16, at most BT
+  int item0;
+  uint32_t idesc_dense, idesc_sparse;
+};
+
+// Positions of a group launch's units: CTA c runs the items at positions c,
+// c + grid, c + 2 grid, ... in turn, up to the first kNoItem.
+constexpr int kOrderCap = 8192;
+constexpr uint16_t kNoItem = 0xFFFF;
+
+template <int G>
+struct Params {
+  CUtensorMap x[G];            // X of GEMM g: boxes of 64 k x bt tokens
+  CUtensorMap w[G];            // W of GEMM g: 16 KiB panels
+  CUtensorMap w_up;            // gated MLP: the up weight, read by row 1
+  Gemm g[G];
+  int n_gemm, n_items;
+  int n_pos;                   // positions: n_items for one GEMM (item = position), else order[] entries
+  uint16_t order[G > 1 ? kOrderCap : 1];  // groups: the item at each position (host-balanced, see below)
+  int mlp;                     // 1 (one GEMM): row 0 = gate, row 1 = up tile row rp; Y = silu(gate) * up
+  const uint8_t* meta_up;
+  const patch_tile_desc* desc_up;
+  int ks;                      // K parts per output block (split K, one GEMM; 1 = whole K per unit)
   float* part;                 // ks > 1: fp32 partials [block][ks][ROWS][bt][128]
   uint32_t* counters;          // ks > 1: arrivals [block][ROWS][4] (zero between calls)
-  int bt;                      // tokens per unit: a multiple of 16, at most BT
-  uint32_t idesc_dense, idesc_sparse;
+  int staged;                  // 1: every GEMM's descriptor rows fit in shared memory (Tk <= MAXTK)
   uint64_t limit_ns;
   int32_t* status;
   int inject;  // 1: row 0's producer stops after the first K-tile (exercises the timeout path)
 };
+
+// The item at position pos, or -1 past the end of this CTA's list.
+template <int G>
+__device__ __forceinline__ int item_at(const Params<G>& P, int pos) {
+  if (pos >= P.n_pos) return -1;
+  if constexpr (G == 1) {
+    return pos;
+  } else {
+    return P.order[pos] == kNoItem ? -1 : int(P.order[pos]);
+  }
+}
+
+// The GEMM of `item`: the last one whose first item is <= item.
+template <int G>
+__device__ __forceinline__ int gemm_of(const Params<G>& P, int item) {
+  int lo = 0, hi = P.n_gemm - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (P.g[mid].item0 <= item) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
 
 // Row pair rp holds tile rows rp and rp + n_pairs (n_pairs = ceil(Tn / 2);
 // the last pair of an odd Tn has one row).  A unit costs the sum of its two
@@ -118,11 +167,13 @@ struct Args {
 // the rows puts exactly one row of every pair inside it), where neighbouring
 // rows would pair dense with dense and sparse with sparse and a one-wave grid
 // would wait for the dense pairs.  A gated-MLP unit is gate and up tile row rp.
-__device__ __forceinline__ int rows_of(const Args& p, int rp) {
-  return p.mlp ? ROWS : (rp + p.n_pairs < p.Tn ? ROWS : 1);
+__device__ __forceinline__ int rows_of(const Gemm& gm, int mlp, int rp) {
+  return mlp ? ROWS : (rp + gm.n_pairs < gm.Tn ? ROWS : 1);
 }
 // the tile row of its weight that row r of unit row pair rp reads
-__device__ __forceinline__ int tile_row(const Args& p, int rp, int r) { return p.mlp ? rp : rp + r * p.n_pairs; }
+__device__ __forceinline__ int tile_row(const Gemm& gm, int mlp, int rp, int r) {
+  return mlp ? rp : rp + r * gm.n_pairs;
+}
 
 // Units run row pair by row pair (all token blocks of a pair are consecutive
 // items), so the CTAs of one wave read a few row pairs' W, which stays in L2
@@ -132,20 +183,21 @@ __device__ __forceinline__ int tile_row(const Args& p, int rp, int r) { return p
 // moment; only the order of the fp32 sum changes.
 __device__ __forceinline__ int k_rotation(int rp, int tb, int Tk) { return (rp + 7 * tb) % Tk; }
 
-// Work unit `item`: output block blk = (row pair rp, token block tb) and its K
-// part kp, which covers K-tiles [k0, k0 + len).  With ks = 1 a unit is a whole
-// output block (item = blk).  The K loop starts at a rotated tile of the part.
+// Work unit: output block blk = (row pair rp, token block tb) of its GEMM and
+// its K part kp, which covers K-tiles [k0, k0 + len).  With ks = 1 a unit is a
+// whole output block.  The K loop starts at a rotated tile of the part.
 struct Unit {
   int blk, kp, rp, tb, k0, len, rot;
 };
-__device__ __forceinline__ Unit unit_of(const Args& p, int item) {
+__device__ __forceinline__ Unit unit_of(const Gemm& gm, int ks, int item) {
   Unit u;
-  u.blk = item / p.ks;
-  u.kp = item - u.blk * p.ks;
-  u.rp = u.blk / p.n_tb;
-  u.tb = u.blk - u.rp * p.n_tb;
-  u.k0 = int(int64_t(u.kp) * p.Tk / p.ks);
-  u.len = int(int64_t(u.kp + 1) * p.Tk / p.ks) - u.k0;
+  const int local = item - gm.item0;
+  u.blk = local / ks;
+  u.kp = local - u.blk * ks;
+  u.rp = u.blk / gm.n_tb;
+  u.tb = u.blk - u.rp * gm.n_tb;
+  u.k0 = int(int64_t(u.kp) * gm.Tk / ks);
+  u.len = int(int64_t(u.kp + 1) * gm.Tk / ks) - u.k0;
   u.rot = k_rotation(u.rp, u.tb, u.len);
   return u;
 }
@@ -156,44 +208,55 @@ __device__ __forceinline__ Unit unit_of(const Args& p, int item) {
 // touches X, so it may run ahead of the previous kernel in the stream (W, the
 // metadata and the descriptors are inputs that no kernel triggering an early
 // launch writes).
-__device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, int r) {
-  const patch_tile_desc* desc = r ? p.desc[1] : p.desc[0];
-  const uint8_t* meta = r ? p.meta[1] : p.meta[0];
-  const bool staged = p.Tk <= MAXTK;
-  const uint32_t row_bytes = uint32_t(p.Tk * sizeof(patch_tile_desc));
+template <int G>
+__device__ void producer_w(Shared& s, const Params<G>& P, int r) {
+  const bool up = P.mlp && r;  // the gated MLP's row 1 reads the up weight
+  const bool staged = P.staged;
   uint32_t a_i = 0, e_i = 0, d_i = 0;  // loads issued per ring / descriptor rows staged
   bool ok = true;
   // stage (or, for a pair without row r, complete with no bytes) the descriptor row of an item
   auto stage_row = [&](int item, int buf) {
-    const int rp = unit_of(p, item).rp;
-    const bool has = r < rows_of(p, rp);
+    const Gemm& gm = P.g[gemm_of(P, item)];
+    const int rp = unit_of(gm, P.ks, item).rp;
+    const bool has = r < rows_of(gm, P.mlp, rp);
+    const uint32_t row_bytes = uint32_t(gm.Tk * sizeof(patch_tile_desc));
     mbar_expect_tx(&s.pdesc_full[r][buf], has ? row_bytes : 0u);
-    if (has) bulk_load(s.pdesc[r][buf], desc + int64_t(tile_row(p, rp, r)) * p.Tk, row_bytes, &s.pdesc_full[r][buf]);
+    if (has)
+      bulk_load(s.pdesc[r][buf], (up ? P.desc_up : gm.desc) + int64_t(tile_row(gm, P.mlp, rp, r)) * gm.Tk, row_bytes,
+                &s.pdesc_full[r][buf]);
     ++d_i;
   };
-  if (staged && int(blockIdx.x) < p.n_items) stage_row(blockIdx.x, 0);
+  if (staged && item_at(P, blockIdx.x) >= 0) stage_row(item_at(P, blockIdx.x), 0);
   int it = 0;
-  for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const Unit u = unit_of(p, item);
-    const int rp = u.rp, tn = tile_row(p, rp, r);
+  for (int pos = blockIdx.x; ok; pos += gridDim.x, ++it) {
+    const int item = item_at(P, pos);
+    if (item < 0) break;
+    const int g = gemm_of(P, item);
+    const Gemm& gm = P.g[g];
+    const patch_tile_desc* desc = up ? P.desc_up : gm.desc;
+    const uint8_t* meta = up ? P.meta_up : gm.meta;
+    const CUtensorMap* tmap_w = up ? &P.w_up : &P.w[g];
+    const Unit u = unit_of(gm, P.ks, item);
+    const int rp = u.rp, tn = tile_row(gm, P.mlp, rp, r);
     const int buf = it & 1;
     if (staged) {
-      if (!(ok = wait_bounded(&s.pdesc_full[r][buf], (it >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
+      if (!(ok = wait_bounded(&s.pdesc_full[r][buf], (it >> 1) & 1, &s.abort_flag, P.limit_ns, P.status, false)))
         break;
       // prefetch the next unit's row into the other buffer (its previous row is done)
-      if (item + int(gridDim.x) < p.n_items) stage_row(item + gridDim.x, buf ^ 1);
+      const int next = item_at(P, pos + int(gridDim.x));
+      if (next >= 0) stage_row(next, buf ^ 1);
     }
-    if (r >= rows_of(p, rp)) continue;
+    if (r >= rows_of(gm, P.mlp, rp)) continue;
     int kt = u.k0 + u.rot;
     for (int j = 0; ok && j < u.len; ++j, kt = (kt + 1 == u.k0 + u.len ? u.k0 : kt + 1)) {
-      if (p.inject && r == 0 && (item != int(blockIdx.x) || j > 0)) {
+      if (P.inject && r == 0 && (item != int(blockIdx.x) || j > 0)) {
         ok = false;
         break;
       }
-      const patch_tile_desc d = staged ? s.pdesc[r][buf][kt] : desc[int64_t(tn) * p.Tk + kt];
+      const patch_tile_desc d = staged ? s.pdesc[r][buf][kt] : desc[int64_t(tn) * gm.Tk + kt];
       if (d.kind) {
         const uint32_t es = e_i % NE;
-        if (!(ok = wait_bounded(&s.e_empty[r][es], ((e_i / NE) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
+        if (!(ok = wait_bounded(&s.e_empty[r][es], ((e_i / NE) & 1) ^ 1, &s.abort_flag, P.limit_ns, P.status, false)))
           break;
         mbar_expect_tx(&s.e_full[r][es], E_BYTES);
         bulk_load(s.e[r][es], meta + uint64_t(d.sparse_ordinal) * E_BYTES, E_BYTES, &s.e_full[r][es]);
@@ -203,7 +266,7 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
       const int panel = int(d.val_offset / A_BYTES);
       for (int h = 0; h < (d.kind ? 1 : 2); ++h) {
         const uint32_t as = a_i % NA;
-        if (!(ok = wait_bounded(&s.a_empty[r][as], ((a_i / NA) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
+        if (!(ok = wait_bounded(&s.a_empty[r][as], ((a_i / NA) & 1) ^ 1, &s.abort_flag, P.limit_ns, P.status, false)))
           break;
         s.a_kind[r][as] = d.kind;  // published to the MMA thread by the barrier's release
         mbar_expect_tx(&s.a_full[r][as], A_BYTES);
@@ -214,51 +277,60 @@ __device__ void producer_w(Shared& s, const CUtensorMap* tmap_w, const Args& p, 
   }
   // every copy issued must have landed before the CTA may exit
   for (uint32_t i = (a_i > NA ? a_i - NA : 0); i < a_i; ++i)
-    wait_bounded(&s.a_full[r][i % NA], (i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+    wait_bounded(&s.a_full[r][i % NA], (i / NA) & 1, &s.abort_flag, P.limit_ns, P.status, true);
   for (uint32_t i = (e_i > NE ? e_i - NE : 0); i < e_i; ++i)
-    wait_bounded(&s.e_full[r][i % NE], (i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+    wait_bounded(&s.e_full[r][i % NE], (i / NE) & 1, &s.abort_flag, P.limit_ns, P.status, true);
   for (uint32_t i = (d_i > 2 ? d_i - 2 : 0); i < d_i; ++i)
-    wait_bounded(&s.pdesc_full[r][i & 1], (i >> 1) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+    wait_bounded(&s.pdesc_full[r][i & 1], (i >> 1) & 1, &s.abort_flag, P.limit_ns, P.status, true);
 }
 
 // X producer: the two 64-k panels of X per K-tile, in the same rotated K order.
-__device__ void producer_x(Shared& s, const CUtensorMap* tmap_x, const Args& p) {
+template <int G>
+__device__ void producer_x(Shared& s, const Params<G>& P) {
   uint32_t b_i = 0;
   bool ok = true;
   // X may be the previous kernel's output: wait for it before the first X load
   pdl_wait_previous();
-  for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-    const Unit u = unit_of(p, item);
-    const int tb = u.tb;
+  for (int pos = blockIdx.x; ok; pos += gridDim.x) {
+    const int item = item_at(P, pos);
+    if (item < 0) break;
+    const int g = gemm_of(P, item);
+    const Gemm& gm = P.g[g];
+    const Unit u = unit_of(gm, P.ks, item);
     int kt = u.k0 + u.rot;
     for (int j = 0; ok && j < u.len; ++j, kt = (kt + 1 == u.k0 + u.len ? u.k0 : kt + 1)) {
       for (int h = 0; ok && h < 2; ++h) {
         const uint32_t bs = b_i % NB;
-        if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false)))
+        if (!(ok = wait_bounded(&s.b_empty[bs], ((b_i / NB) & 1) ^ 1, &s.abort_flag, P.limit_ns, P.status, false)))
           break;
-        mbar_expect_tx(&s.b_full[bs], uint32_t(p.bt) * 128u);
-        tma_load_2d(s.b[bs], tmap_x, &s.b_full[bs], kt * kTile + 64 * h, tb * p.bt);
+        mbar_expect_tx(&s.b_full[bs], uint32_t(gm.bt) * 128u);
+        tma_load_2d(s.b[bs], &P.x[g], &s.b_full[bs], kt * kTile + 64 * h, u.tb * gm.bt);
         ++b_i;
       }
     }
   }
   for (uint32_t i = (b_i > NB ? b_i - NB : 0); i < b_i; ++i)
-    wait_bounded(&s.b_full[i % NB], (i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, true);
+    wait_bounded(&s.b_full[i % NB], (i / NB) & 1, &s.abort_flag, P.limit_ns, P.status, true);
 }
 
 // MMA issuer of row r (one thread): each row has its own issuing thread, so
 // the two chains' barrier waits, commits and bookkeeping overlap and the
 // tensor core, shared by both, stays fed.  Both consume the same X slots; a
 // slot is free once both rows' MMAs on it are complete (two commits).
-__device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
+template <int G>
+__device__ void mma_issuer(Shared& s, uint32_t tmem, const Params<G>& P, int r) {
   const uint32_t acc = tmem + ACC_STRIDE * r;
   uint32_t a_i = 0, b_i = 0, e_i = 0;
   bool ok = true;
   int it = 0;
-  for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++it) {
-    const Unit u = unit_of(p, item);
-    const bool active = r < rows_of(p, u.rp);
-    if (!(ok = wait_bounded(&s.acc_empty[r], (it & 1) ^ 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+  for (int pos = blockIdx.x; ok; pos += gridDim.x, ++it) {
+    const int item = item_at(P, pos);
+    if (item < 0) break;
+    const Gemm& gm = P.g[gemm_of(P, item)];
+    const uint32_t idesc_dense = gm.idesc_dense, idesc_sparse = gm.idesc_sparse;
+    const Unit u = unit_of(gm, P.ks, item);
+    const bool active = r < rows_of(gm, P.mlp, u.rp);
+    if (!(ok = wait_bounded(&s.acc_empty[r], (it & 1) ^ 1, &s.abort_flag, P.limit_ns, P.status, false))) break;
     tc_fence_after();
     uint32_t accumulate = 0;
     for (int kt = 0; ok && kt < u.len; ++kt) {
@@ -268,13 +340,13 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
         // panel serves both halves and its metadata goes to TMEM first
         if (active && (h == 0 || !kind)) {
           as = a_i % NA;
-          if (!(ok = wait_bounded(&s.a_full[r][as], (a_i / NA) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
+          if (!(ok = wait_bounded(&s.a_full[r][as], (a_i / NA) & 1, &s.abort_flag, P.limit_ns, P.status, false)))
             break;
           ++a_i;
           if (h == 0) kind = *reinterpret_cast<volatile uint32_t*>(&s.a_kind[r][as]);
           if (h == 0 && kind) {
             es = e_i % NE;
-            if (!(ok = wait_bounded(&s.e_full[r][es], (e_i / NE) & 1, &s.abort_flag, p.limit_ns, p.status, false)))
+            if (!(ok = wait_bounded(&s.e_full[r][es], (e_i / NE) & 1, &s.abort_flag, P.limit_ns, P.status, false)))
               break;
             ++e_i;
             tc_fence_after();
@@ -282,7 +354,7 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
           }
         }
         const uint32_t bs = b_i % NB;
-        if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, &s.abort_flag, p.limit_ns, p.status, false))) break;
+        if (!(ok = wait_bounded(&s.b_full[bs], (b_i / NB) & 1, &s.abort_flag, P.limit_ns, P.status, false))) break;
         ++b_i;
         if (!active) {  // the pair's missing row only paces the X ring
           mbar_arrive(&s.b_empty[bs]);
@@ -296,13 +368,13 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
           for (int j = 0; j < 2; ++j) {
             const uint32_t kb = 2 * h + j;  // 32-k block of the tile: 16 kept values = 32 B of A
             mma_sparse(acc, a0 + (kb * 32 >> 4), b0 + (j * 64 >> 4), acc + META_COL0 + 4 * es + (kb & 2u),
-                       p.idesc_sparse | (kb & 1u), accumulate);
+                       idesc_sparse | (kb & 1u), accumulate);
             accumulate = 1;
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {  // K = 16 per MMA = 32 B along the swizzled row
-            mma_dense(acc, a0 + (j * 32 >> 4), b0 + (j * 32 >> 4), p.idesc_dense, accumulate);
+            mma_dense(acc, a0 + (j * 32 >> 4), b0 + (j * 32 >> 4), idesc_dense, accumulate);
             accumulate = 1;
           }
         }
@@ -324,7 +396,7 @@ __device__ void mma_issuer(Shared& s, uint32_t tmem, const Args& p, int r) {
   }
   // all MMAs and copies issued must be complete before TMEM is freed
   tc_commit(&s.drain[r]);
-  wait_bounded(&s.drain[r], 0, &s.abort_flag, p.limit_ns, p.status, true);
+  wait_bounded(&s.drain[r], 0, &s.abort_flag, P.limit_ns, P.status, true);
 }
 
 // Epilogue warp groups (4 warps each, one per TMEM lane quarter): per chunk
@@ -346,16 +418,18 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* a, uint32_t v
 // accumulator is released, and the last of the block's ks units to arrive
 // (counted per row and TMEM lane quarter, acquire-release) adds the ks
 // partials in K-part order (deterministic), stores Y and resets the counter.
-__device__ void epilogue_split(Shared& s, uint32_t tmem, const Args& p, const Unit& u, int g, int q, int lane) {
-  const bool has = g < rows_of(p, u.rp);
+template <int G>
+__device__ void epilogue_split(Shared& s, uint32_t tmem, const Params<G>& P, const Gemm& gm, const Unit& u, int g,
+                               int q, int lane) {
+  const bool has = g < rows_of(gm, P.mlp, u.rp);
   const int row = 32 * q + lane;
-  const int64_t n = int64_t(tile_row(p, u.rp, g)) * BM + row;
-  const int m0 = u.tb * p.bt;
-  const int valid = p.M - m0 < p.bt ? p.M - m0 : p.bt;  // tokens of this block inside X
-  const int64_t slot_floats = int64_t(BM) * p.bt;        // one row g of one unit
-  const int64_t blk_base = int64_t(u.blk) * p.ks * ROWS;
+  const int64_t n = int64_t(tile_row(gm, P.mlp, u.rp, g)) * BM + row;
+  const int m0 = u.tb * gm.bt;
+  const int valid = gm.M - m0 < gm.bt ? gm.M - m0 : gm.bt;  // tokens of this block inside X
+  const int64_t slot_floats = int64_t(BM) * gm.bt;           // one row g of one unit
+  const int64_t blk_base = int64_t(u.blk) * P.ks * ROWS;
   if (has) {
-    float* mine = p.part + ((blk_base + int64_t(u.kp) * ROWS + g) * slot_floats) + row;
+    float* mine = P.part + ((blk_base + int64_t(u.kp) * ROWS + g) * slot_floats) + row;
     const uint32_t lanes = tmem + (uint32_t(32 * q) << 16) + ACC_STRIDE * g;
     for (int c = 0; c * YT < valid; ++c) {
       uint32_t v[YT];
@@ -369,18 +443,18 @@ __device__ void epilogue_split(Shared& s, uint32_t tmem, const Args& p, const Un
   if (lane == 0) mbar_arrive(&s.acc_empty[g]);
   if (!has) return;
   // the warp's partial stores are ordered before lane 0's release-acquire increment
-  uint32_t* counter = p.counters + (int64_t(u.blk) * ROWS + g) * 4 + q;
+  uint32_t* counter = P.counters + (int64_t(u.blk) * ROWS + g) * 4 + q;
   uint32_t old = 0;
   if (lane == 0) old = atom_add_acq_rel_gpu(counter, 1u);
   old = __shfl_sync(0xFFFFFFFFu, old, 0);
-  if (old != uint32_t(p.ks - 1)) return;
+  if (old != uint32_t(P.ks - 1)) return;
   __syncwarp();  // orders lane 0's acquire before every lane's loads
   for (int c = 0; c * YT < valid; ++c) {
     float sum[YT];
 #pragma unroll
     for (int j = 0; j < YT; ++j) sum[j] = 0.0f;
-    for (int kp = 0; kp < p.ks; ++kp) {
-      const float* src = p.part + ((blk_base + int64_t(kp) * ROWS + g) * slot_floats) + int64_t(YT * c) * BM + row;
+    for (int kp = 0; kp < P.ks; ++kp) {
+      const float* src = P.part + ((blk_base + int64_t(kp) * ROWS + g) * slot_floats) + int64_t(YT * c) * BM + row;
       float part[YT];
 #pragma unroll
       for (int j = 0; j < YT; ++j) part[j] = __ldcg(src + int64_t(j) * BM);
@@ -389,39 +463,45 @@ __device__ void epilogue_split(Shared& s, uint32_t tmem, const Args& p, const Un
     }
 #pragma unroll
     for (int j = 0; j < YT; ++j)
-      if (YT * c + j < valid) p.Y[int64_t(m0 + YT * c + j) * p.N + n] = f32_to_bf16_rne(sum[j]);
+      if (YT * c + j < valid) gm.Y[int64_t(m0 + YT * c + j) * gm.N + n] = f32_to_bf16_rne(sum[j]);
   }
   if (lane == 0) *counter = 0;  // ready for the next call
 }
 
-__device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
+template <int G>
+__device__ void epilogue(Shared& s, uint32_t tmem, const Params<G>& P) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3;                  // the TMEM lane quarter this warp may access
   const int g = (warp - EPI_WARP0) >> 2;   // warp group
   const uint32_t bar_id = 1 + g;           // named barrier of the group's 128 threads
+  const bool mlp = P.mlp;
   int it = 0;
-  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++it) {
-    const Unit u = unit_of(p, item);
+  for (int pos = blockIdx.x;; pos += gridDim.x, ++it) {
+    const int item = item_at(P, pos);
+    if (item < 0) break;
+    const Gemm& gm = P.g[gemm_of(P, item)];
+    const Unit u = unit_of(gm, P.ks, item);
     const int rp = u.rp, tb = u.tb;
     // the four warps of a group take the same decision, so none is left at a barrier
-    bool ok = wait_bounded(&s.acc_full[g], it & 1, &s.abort_flag, p.limit_ns, p.status, false);
-    if (p.mlp) ok = ok && wait_bounded(&s.acc_full[g ^ 1], it & 1, &s.abort_flag, p.limit_ns, p.status, false);
+    bool ok = wait_bounded(&s.acc_full[g], it & 1, &s.abort_flag, P.limit_ns, P.status, false);
+    if (mlp) ok = ok && wait_bounded(&s.acc_full[g ^ 1], it & 1, &s.abort_flag, P.limit_ns, P.status, false);
     if (!named_bar_and(bar_id, 128, ok)) break;
     tc_fence_after();
-    if (p.ks > 1) {  // split K (never with the gated MLP)
-      epilogue_split(s, tmem, p, u, g, q, lane);
+    if (P.ks > 1) {  // split K (never with the gated MLP)
+      epilogue_split(s, tmem, P, gm, u, g, q, lane);
       continue;
     }
-    if (p.mlp || g < rows_of(p, rp)) {
-      const int n0 = tile_row(p, rp, g) * BM, m0 = tb * p.bt;
-      const int valid = p.M - m0 < p.bt ? p.M - m0 : p.bt;  // tokens of this unit inside X
+    if (mlp || g < rows_of(gm, mlp, rp)) {
+      const int n0 = tile_row(gm, mlp, rp, g) * BM, m0 = tb * gm.bt;
+      const int valid = gm.M - m0 < gm.bt ? gm.M - m0 : gm.bt;  // tokens of this unit inside X
       const uint32_t lanes = tmem + (uint32_t(32 * q) << 16);
-      const int c0 = p.mlp ? g : 0, dc = p.mlp ? 2 : 1;
+      const int c0 = mlp ? g : 0, dc = mlp ? 2 : 1;
+      const int64_t ldy = gm.N;
       // this thread's feature; a warp's 32 stores of one token fill 64 contiguous bytes of Y
-      uint16_t* yp = p.Y + int64_t(m0) * p.N + n0 + 32 * q + lane;
+      uint16_t* yp = gm.Y + int64_t(m0) * ldy + n0 + 32 * q + lane;
       for (int c = c0; c * YC < valid; c += dc) {
         uint32_t v[YC];
-        if (p.mlp) {
+        if (mlp) {
 #pragma unroll
           for (int hh = 0; hh < YC / 16; ++hh) {  // in 16-column halves (registers)
             uint32_t gt[16], u[16];
@@ -439,10 +519,10 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
         } else {
           tmem_ld_32cols(lanes + ACC_STRIDE * g + uint32_t(YC * c), v);
         }
-        uint16_t* yr = yp + int64_t(YC * c) * p.N;
+        uint16_t* yr = yp + int64_t(YC * c) * ldy;
         const int nj = valid - YC * c < YC ? valid - YC * c : YC;
 #pragma unroll
-        for (int j = 0; j < YC; ++j, yr += p.N)
+        for (int j = 0; j < YC; ++j, yr += ldy)
           if (j < nj) *yr = f32_to_bf16_rne(__uint_as_float(v[j]));
       }
     }
@@ -450,15 +530,13 @@ __device__ void epilogue(Shared& s, uint32_t tmem, const Args& p) {
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(&s.acc_empty[g]);
-      if (p.mlp) mbar_arrive(&s.acc_empty[g ^ 1]);
+      if (mlp) mbar_arrive(&s.acc_empty[g ^ 1]);
     }
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w0,
-                   const __grid_constant__ CUtensorMap tmap_w1,
-                   const Args p) {
+template <int G>
+__global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_constant__ Params<G> P) {
   extern __shared__ uint8_t smem_raw[];
   Shared& s = *reinterpret_cast<Shared*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -475,7 +553,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(&s.e_empty[r][i], 1);
       }
       mbar_init(&s.acc_full[r], 1);
-      mbar_init(&s.acc_empty[r], p.mlp ? 8 : 4);  // the gated MLP's groups both read both rows
+      mbar_init(&s.acc_empty[r], P.mlp ? 8 : 4);  // the gated MLP's groups both read both rows
       mbar_init(&s.drain[r], 1);
       mbar_init(&s.pdesc_full[r][0], 1);
       mbar_init(&s.pdesc_full[r][1], 1);
@@ -486,9 +564,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     s.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    prefetch_tensormap(&tmap_x);
-    prefetch_tensormap(&tmap_w0);
-    prefetch_tensormap(&tmap_w1);
+    for (int i = 0; i < P.n_gemm; ++i) {
+      prefetch_tensormap(&P.x[i]);
+      prefetch_tensormap(&P.w[i]);
+    }
+    if (P.mlp) prefetch_tensormap(&P.w_up);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -506,16 +586,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp < 4) {
     if (lane == 0) {
       if (warp & 1)
-        mma_issuer(s, tmem, p, warp >> 1);
+        mma_issuer(s, tmem, P, warp >> 1);
       else
-        producer_w(s, (warp >> 1) ? &tmap_w1 : &tmap_w0, p, warp >> 1);
+        producer_w(s, P, warp >> 1);
     }
     __syncwarp();
   } else if (warp == 4) {
-    if (lane == 0) producer_x(s, &tmap_x, p);
+    if (lane == 0) producer_x(s, P);
     __syncwarp();
   } else if (warp >= EPI_WARP0) {
-    epilogue(s, tmem, p);
+    epilogue(s, tmem, P);
   }
 
   tc_fence_before();
@@ -625,8 +705,71 @@ size_t prefill_workspace_bytes(int64_t M, const patch_weight& W, int num_sms) {
   return pl.ks > 1 ? kDecodeCounterBytes + pl.part_bytes : 0;
 }
 
-// Shared by the plain GEMM (w1 == w0, units of two consecutive tile rows) and
-// the gated MLP (w0 = gate, w1 = up, units of one tile row of each).
+// The values blob of W as a tensor map of 16 KiB panels (rows of 128 B).
+static bool make_map_w(CUtensorMap* map, const patch_weight& W) {
+  const int64_t T = (W.N / prefill::BM) * (W.K / kTile);
+  const uint64_t n_panels = uint64_t(2 * (T - W.n_sparse) + W.n_sparse);
+  return make_map_2d_bf16(map, W.values, 64, n_panels * 128, 128, 64, 128);
+}
+
+// GEMM i of a launch: Y = X W^T in units of n_pairs row pairs x n_tb token
+// blocks of bt tokens x ks K parts, its items starting at item0.
+template <int G>
+static bool set_gemm(prefill::Params<G>& P, int i, const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y,
+                     int64_t n_pairs, int bt, int ks, int item0) {
+  using namespace prefill;
+  Gemm& gm = P.g[i];
+  gm.meta = static_cast<const uint8_t*>(W.meta);
+  gm.desc = W.desc;
+  gm.Y = Y;
+  gm.M = int(M);
+  gm.N = int(W.N);
+  gm.Tn = int(W.N / BM);
+  gm.Tk = int(W.K / kTile);
+  gm.n_pairs = int(n_pairs);
+  gm.n_tb = int((M + bt - 1) / bt);
+  gm.bt = bt;
+  gm.item0 = item0;
+  gm.idesc_dense = tc::idesc_bf16(BM, bt, false);
+  gm.idesc_sparse = tc::idesc_bf16(BM, bt, true);
+  (void)ks;
+  return make_map_2d_bf16(&P.x[i], X, uint64_t(W.K), uint64_t(M), uint64_t(W.K) * 2, 64, uint32_t(bt)) &&
+         make_map_w(&P.w[i], W);
+}
+
+template <int G>
+static void set_launch(prefill::Params<G>& P, int n_gemm, int n_items, int32_t* status, uint64_t limit_ns) {
+  P.n_gemm = n_gemm;
+  P.n_items = n_items;
+  P.n_pos = n_items;
+  P.mlp = 0;
+  P.meta_up = nullptr;
+  P.desc_up = nullptr;
+  P.ks = 1;
+  P.part = nullptr;
+  P.counters = nullptr;
+  P.staged = 1;
+  for (int i = 0; i < n_gemm; ++i)
+    if (P.g[i].Tk > prefill::MAXTK) P.staged = 0;
+  P.limit_ns = limit_ns;
+  P.status = status;
+  P.inject = 0;
+}
+
+static_assert(sizeof(prefill::Params<kPrefillGroupMax>) <= 32764, "kernel parameter space");
+
+template <int G>
+static cudaError_t launch_params(const prefill::Params<G>& P, int num_sms, cudaStream_t stream) {
+  using namespace prefill;
+  const int grid = P.n_items < num_sms ? P.n_items : num_sms;
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(SMEM_BYTES));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(prefill_kernel<G>, dim3(unsigned(grid)), dim3(THREADS), SMEM_BYTES, stream, P);
+}
+
+// Shared by the plain GEMM (units of tile rows rp and rp + n_pairs of W) and
+// the gated MLP (W0 = gate, W1 = up, units of tile row rp of each).
 static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch_weight& W0, const patch_weight& W1,
                                        bool mlp, uint16_t* Y, void* workspace, size_t workspace_bytes,
                                        int32_t* status, int num_sms, uint64_t limit_ns, int inject,
@@ -638,45 +781,105 @@ static cudaError_t launch_prefill_impl(const uint16_t* X, int64_t M, const patch
   PrefillPlan plan = prefill_plan(M, n_pairs, Tk, num_sms, !mlp);
   if (plan.ks > 1 && (!workspace || workspace_bytes < kDecodeCounterBytes + plan.part_bytes))
     plan = prefill_plan(M, n_pairs, Tk, num_sms, false);
-  const int bt = plan.bt;
-  CUtensorMap tmap_x, tmap_w0, tmap_w1;
-  if (!make_map_2d_bf16(&tmap_x, X, uint64_t(W0.K), uint64_t(M), uint64_t(W0.K) * 2, 64, uint32_t(bt)))
-    return cudaErrorUnknown;
-  const patch_weight* Ws[2] = {&W0, &W1};
-  CUtensorMap* maps[2] = {&tmap_w0, &tmap_w1};
-  for (int r = 0; r < 2; ++r) {
-    const int64_t T = (Ws[r]->N / BM) * Tk;
-    const uint64_t n_panels = uint64_t(2 * (T - Ws[r]->n_sparse) + Ws[r]->n_sparse);
-    if (!make_map_2d_bf16(maps[r], Ws[r]->values, 64, n_panels * 128, 128, 64, 128)) return cudaErrorUnknown;
+  Params<1> P;
+  if (!set_gemm(P, 0, X, M, W0, Y, n_pairs, plan.bt, plan.ks, 0)) return cudaErrorUnknown;
+  set_launch(P, 1, int(n_pairs * plan.n_tb * plan.ks), status, limit_ns);
+  P.mlp = mlp ? 1 : 0;
+  if (mlp) {
+    if (!make_map_w(&P.w_up, W1)) return cudaErrorUnknown;
+    P.meta_up = static_cast<const uint8_t*>(W1.meta);
+    P.desc_up = W1.desc;
   }
-  Args p;
-  for (int r = 0; r < ROWS; ++r) {
-    p.meta[r] = static_cast<const uint8_t*>(Ws[r]->meta);
-    p.desc[r] = Ws[r]->desc;
+  P.ks = plan.ks;
+  P.counters = static_cast<uint32_t*>(workspace);  // the fixed counter region at the start (used when ks > 1)
+  P.part = plan.ks > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kDecodeCounterBytes) : nullptr;
+  P.inject = inject;
+  return launch_params(P, num_sms, stream);
+}
+
+// Units to CTAs for a group: longest first, each to the CTA with the least
+// work so far (ties to the lower index), a unit's work modelled as its
+// K-tiles x tokens x tile rows.  Units of one GEMM cost the same, so those of
+// the costliest GEMM go out first, round the CTAs, then the next GEMM's fill
+// in behind the shortest lists.  CTA c's j-th unit sits at position c + j grid.
+// Returns false when the positions do not fit the table.
+template <int G>
+static bool balance_units(prefill::Params<G>& P, const int64_t* unit_cost, int grid) {
+  using namespace prefill;
+  std::vector<std::vector<uint16_t>> lists(grid);
+  std::vector<std::pair<int64_t, int>> heap;  // (work, cta), a min-heap
+  for (int c = 0; c < grid; ++c) heap.push_back({0, c});
+  auto later = [](const std::pair<int64_t, int>& a, const std::pair<int64_t, int>& b) { return a > b; };
+  for (int i = 0; i < P.n_gemm; ++i) {  // GEMMs are in descending unit cost
+    const int n_units = P.g[i].n_pairs * P.g[i].n_tb;
+    for (int k = 0; k < n_units; ++k) {
+      std::pop_heap(heap.begin(), heap.end(), later);
+      lists[heap.back().second].push_back(uint16_t(P.g[i].item0 + k));
+      heap.back().first += unit_cost[i];
+      std::push_heap(heap.begin(), heap.end(), later);
+    }
   }
-  p.mlp = mlp ? 1 : 0;
-  p.Y = Y;
-  p.M = int(M);
-  p.N = int(Tn * BM);
-  p.Tn = int(Tn);
-  p.Tk = int(Tk);
-  p.n_pairs = int(n_pairs);
-  p.n_tb = int(plan.n_tb);
-  p.ks = plan.ks;
-  p.n_items = int(n_pairs) * p.n_tb * p.ks;
-  p.bt = bt;
-  p.counters = static_cast<uint32_t*>(workspace);  // the fixed counter region at the start (used when ks > 1)
-  p.part = plan.ks > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kDecodeCounterBytes) : nullptr;
-  p.idesc_dense = tc::idesc_bf16(BM, bt, false);
-  p.idesc_sparse = tc::idesc_bf16(BM, bt, true);
-  p.limit_ns = limit_ns;
-  p.status = status;
-  p.inject = inject;
-  const int grid = p.n_items < num_sms ? p.n_items : num_sms;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(SMEM_BYTES));
-  if (e != cudaSuccess) return e;
-  return launch_pdl(prefill_kernel, dim3(unsigned(grid)), dim3(THREADS), SMEM_BYTES, stream, tmap_x, tmap_w0, tmap_w1,
-                    p);
+  size_t rounds = 0;
+  for (const auto& l : lists) rounds = l.size() > rounds ? l.size() : rounds;
+  if (rounds * size_t(grid) > size_t(kOrderCap)) return false;
+  P.n_pos = int(rounds) * grid;
+  for (int pos = 0; pos < P.n_pos; ++pos) {
+    const auto& l = lists[pos % grid];
+    const size_t j = size_t(pos / grid);
+    P.order[pos] = j < l.size() ? l[j] : kNoItem;
+  }
+  return true;
+}
+
+// A group of independent GEMMs in one launch (at most kPrefillGroupMax).
+// Tokens per unit: the fewest 240-token blocks that hold M, evened out
+// (M = 512: 3 blocks of 176, not 240 + 240 + 32), so no block streams its
+// weights for a sliver of tokens; the units of all the GEMMs then share the
+// CTAs as balance_units assigns them.
+cudaError_t launch_prefill_group(const PrefillGroupCall* calls, int n, int32_t* status, int num_sms,
+                                 uint64_t limit_ns, cudaStream_t stream) {
+  using namespace prefill;
+  if (n <= 0) return cudaSuccess;
+  if (n > kPrefillGroupMax) return cudaErrorInvalidValue;
+  int order[kPrefillGroupMax], bts[kPrefillGroupMax];
+  int64_t cost[kPrefillGroupMax];
+  for (int i = 0; i < n; ++i) {
+    const int64_t M = calls[i].M, Tn = calls[i].W.N / BM, Tk = calls[i].W.K / kTile;
+    const int64_t blocks = (M + BT - 1) / BT;
+    const int64_t per = (M + blocks - 1) / blocks;
+    bts[i] = int((per + 15) / 16 * 16);
+    cost[i] = Tk * bts[i] * (Tn > 1 ? ROWS : 1);
+    order[i] = i;
+  }
+  for (int i = 1; i < n; ++i)  // stable insertion sort, costliest units first
+    for (int j = i; j > 0 && cost[order[j]] > cost[order[j - 1]]; --j) {
+      const int t = order[j];
+      order[j] = order[j - 1];
+      order[j - 1] = t;
+    }
+  std::unique_ptr<Params<kPrefillGroupMax>> hold(new Params<kPrefillGroupMax>());  // ~27 KB, copied at launch
+  Params<kPrefillGroupMax>& P = *hold;
+  int items = 0;
+  int64_t unit_cost[kPrefillGroupMax];
+  for (int k = 0; k < n; ++k) {
+    const PrefillGroupCall& c = calls[order[k]];
+    const int64_t n_pairs = (c.W.N / BM + ROWS - 1) / ROWS;
+    if (!set_gemm(P, k, c.X, c.M, c.W, c.Y, n_pairs, bts[order[k]], 1, items)) return cudaErrorUnknown;
+    items += P.g[k].n_pairs * P.g[k].n_tb;
+    unit_cost[k] = cost[order[k]];
+  }
+  set_launch(P, n, items, status, limit_ns);
+  const int grid = items < num_sms ? items : num_sms;
+  if (items > kOrderCap || !balance_units(P, unit_cost, grid)) {
+    // too many units for the table: the first half of the calls, then the rest;
+    // a call alone runs as patch_gemm's prefill path does (no split K)
+    if (n < 2)
+      return launch_prefill(calls[0].X, calls[0].M, calls[0].W, calls[0].Y, nullptr, 0, status, num_sms, limit_ns, 0,
+                            stream);
+    const cudaError_t e = launch_prefill_group(calls, n / 2, status, num_sms, limit_ns, stream);
+    return e != cudaSuccess ? e : launch_prefill_group(calls + n / 2, n - n / 2, status, num_sms, limit_ns, stream);
+  }
+  return launch_params(P, num_sms, stream);
 }
 
 cudaError_t launch_prefill(const uint16_t* X, int64_t M, const patch_weight& W, uint16_t* Y, void* workspace,

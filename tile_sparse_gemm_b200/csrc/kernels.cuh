@@ -48,6 +48,18 @@ size_t prefill_workspace_bytes(int64_t M, const patch_weight& W, int num_sms);
 cudaError_t launch_prefill_mlp(const uint16_t* X, int64_t M, const patch_weight& W_gate, const patch_weight& W_up,
                                uint16_t* H, int32_t* status, int num_sms, uint64_t limit_ns, cudaStream_t stream);
 
+// Independent prefill GEMMs Y_i = X_i W_i^T (M_i >= 1 each) in one launch of
+// the prefill kernel; at most kPrefillGroupMax per launch.
+constexpr int kPrefillGroupMax = 32;
+struct PrefillGroupCall {
+  const uint16_t* X;
+  int64_t M;
+  patch_weight W;
+  uint16_t* Y;
+};
+cudaError_t launch_prefill_group(const PrefillGroupCall* calls, int n, int32_t* status, int num_sms,
+                                 uint64_t limit_ns, cudaStream_t stream);
+
 // H = silu(G) * U elementwise (bf16; count a multiple of 8).
 cudaError_t launch_silu_mul(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t count, int num_sms,
                             cudaStream_t stream);
