@@ -1,7 +1,10 @@
-// Prefill path of patch_gemm (M > 16): a persistent, warp-specialised
-// TMA + tcgen05 kernel for sm_100a in which dense tiles run on the dense
-// tensor-core MMA and 2:4 sparse tiles on the structured-sparse MMA, both
-// accumulating into fp32 tiles in tensor memory.
+// Prefill path of patch_gemm (M > 16), patch_gemm_mlp and patch_gemm_group:
+// a persistent, warp-specialised TMA + tcgen05 kernel for sm_100a in which
+// dense tiles run on the dense tensor-core MMA and 2:4 sparse tiles on the
+// structured-sparse MMA, both accumulating into fp32 tiles in tensor memory.
+// One launch runs the units of one GEMM, or of a group of independent GEMMs
+// (a table of them in the kernel parameters, with a host-balanced list of
+// units per CTA).
 //
 // "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs", section 2
 // "Methodology: PATCH", "Inference & Deployment": hybrid execution over
