@@ -9,23 +9,29 @@ whose blocks time every configuration of the layer this library targets:
 * decode (the headline `value`): the 7 LLaMA-2-7B linear layers (q/k/v/o
   4096x4096, gate/up 11008x4096, down 4096x11008), 50% of the 128x128 tiles
   2:4 sparse (exact count, seeded positions), magnitude-top-2 patterns, at
-  M = 1, 4 and 16 tokens.  One step = the 21 patch_gemm calls over packed
-  weights resident in HBM; the metric is HBM GB/s counting only the bytes the
-  layer must move: stored weight bytes (dense tiles 32 KiB, sparse tiles
-  16 KiB values + 2 KiB metadata, 16 B descriptor per tile) + X + Y.
+  M = 1, 4 and 16 tokens.  One step = the 21 independent GEMMs over packed
+  weights resident in HBM, as one patch_gemm_chain launch (the value; the
+  block also times them as 21 separate patch_gemm calls and as a chain of
+  calls that wait for each other); the metric is HBM GB/s counting only the
+  bytes the layer must move: stored weight bytes (dense tiles 32 KiB, sparse
+  tiles 16 KiB values + 2 KiB metadata, 16 B descriptor per tile) + X + Y.
 * "prefill": the same 7 shapes at M = 2048, sparse-tile fraction swept over
   {0, 0.25, 0.5, 0.75, 1}; dense-equivalent TFLOP/s (2*M*N*K / time), the
   mixed roofline (dense tiles at the dense peak, sparse tiles at r times it),
   the speedup of every fraction over the same shape packed all-dense, and
-  whether throughput rises monotonically with the fraction.
+  whether throughput rises monotonically with the fraction; the same 35 GEMMs
+  also as 5 patch_gemm_group launches (one per fraction).
 * "stack": the 32-layer LLaMA-2-7B linear stack (7 projections per layer, 224
   distinct weights, ~9 GB), run sequentially at M = 1 and at M = 8, with the
   non-uniform per-layer sparse-tile fractions (0.1 / 0.7, +0.1 for the MLP);
   GB/s over stored bytes and milliseconds per pass over the stack.
 * "llama3_qwen": LLaMA-3-8B and Qwen-2.5-0.5B linears with spatially
-  clustered sparse tiles (50%), at M = 1 (GB/s) and M = 512 (TFLOP/s).
+  clustered sparse tiles (50%), at M = 1 (GB/s; also as one patch_gemm_chain)
+  and M = 512 (TFLOP/s; also as one patch_gemm_group).
+* "mma_probe": the dense and 2:4-sparse tensor-core MMA rates (M = 128, 64).
 Other workloads: decode_fused (q|k|v and gate|up as one GEMM each),
-tile_ablation (mask tile sizes 4..128), mma_peak (tensor-core MMA rate probe).
+tile_ablation (mask tile sizes 4..128).  A workload run alone (--workload)
+prints its own line; one timed per token count reports its smallest.
 
 Prints one JSON line (rank 0).  --impl reference times the CPU oracle (plain
 C, fp64) on a bounded sample of the decode workload on the host cores.
