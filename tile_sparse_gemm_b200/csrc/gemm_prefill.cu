@@ -183,8 +183,17 @@ __device__ __forceinline__ int tile_row(const Gemm& gm, int mlp, int rp, int r) 
 // while every token block uses it, instead of every wave reading all of W.
 // Units that share an X block (same tb) or W rows (same rp) start their K loop
 // at different tiles, so they do not all hit the same L2 lines at the same
-// moment; only the order of the fp32 sum changes.
-__device__ __forceinline__ int k_rotation(int rp, int tb, int Tk) { return (rp + 7 * tb) % Tk; }
+// moment; only the order of the fp32 sum changes.  The token blocks of a row
+// pair start one K-tile apart, so each W panel's readers follow each other
+// within a few steps and W streams through L2 once; the row pairs spread
+// evenly over K, so an X block's readers span the whole loop and X stays
+// resident (down at M = 2048 holds 45 MB of X but 90 MB of W: with the row
+// pairs one tile apart and the token blocks spread, its W panels were
+// evicted between readers, 1.5x the layer's bytes from DRAM).
+__device__ __forceinline__ int k_rotation(int rp, int tb, int Tk, int n_pairs) {
+  const int stride = Tk > n_pairs ? Tk / n_pairs : 1;
+  return (rp * stride + tb) % Tk;
+}
 
 // Work unit: output block blk = (row pair rp, token block tb) of its GEMM and
 // its K part kp, which covers K-tiles [k0, k0 + len).  With ks = 1 a unit is a
@@ -201,7 +210,7 @@ __device__ __forceinline__ Unit unit_of(const Gemm& gm, int ks, int item) {
   u.tb = u.blk - u.rp * gm.n_tb;
   u.k0 = int(int64_t(u.kp) * gm.Tk / ks);
   u.len = int(int64_t(u.kp + 1) * gm.Tk / ks) - u.k0;
-  u.rot = k_rotation(u.rp, u.tb, u.len);
+  u.rot = k_rotation(u.rp, u.tb, u.len, gm.n_pairs);
   return u;
 }
 
