@@ -401,9 +401,10 @@ PATCH_API patch_status_t patch_gemm_chain(const patch_chain_call *calls, int64_t
  * model, or k and v beside q) has fewer units (2 tile rows x up to 240
  * tokens) than the GPU has SMs, and as its own kernel it also pays its
  * set-up, first loads and last partial wave.  Here the units of all the
- * calls share one grid: the CTAs take them in turn, those of the calls with
- * the costliest units first.  Token blocks are the fewest of at most 240
- * tokens, evened out (M = 512: three of 176).
+ * calls share one grid: the host deals them out to the CTAs longest first
+ * (work modelled as K-tiles x tokens x tile rows), each to the CTA with the
+ * least work so far.  Token blocks are the fewest of at most 240 tokens,
+ * evened out (M = 512: three of 176).
  *
  *   calls[j].X, .Y, .W, .M as for patch_gemm_chain, but M may be any value
  *       0 .. 2^30 (0: the call is skipped; M <= 16 runs in 16-token units on
