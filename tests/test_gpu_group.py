@@ -8,6 +8,8 @@ checked against the oracle's fp64 product within the layer's tolerance
 (relative Frobenius error <= 5e-3, |err| <= 1e-2 (1 + |ref|)).  The groups mix
 shapes, token counts (1 ... 1000, ragged token blocks) and sparse fractions,
 so the CTAs' waves interleave units of different GEMMs."""
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -109,6 +111,36 @@ def test_group_full_size_llama3_qwen_m512_sampled():
     for y, (name, x, w, bm, ids) in zip(ys, refs):
         ref = oracle.gemm(x, oracle.apply_mask(w, bm, ids), rows=rows)
         check_gemm(bits_of(y)[rows], ref, f"{name} M=512")
+
+
+@functools.lru_cache(maxsize=8)
+def llama2_weight(idx):
+    name, N, K = si.LLAMA2_7B[idx]
+    w = si.gen_w(N, K, 3, idx)
+    return w, si.patterns_top2(w)
+
+
+@pytest.mark.parametrize("frac", [0.0, 1.0])
+def test_group_full_size_llama2_prefill_sampled(frac):
+    """The 7 LLaMA-2-7B linears at M = 2048 and one sparse-tile fraction as one
+    group (the bench's grouped prefill launch), on sampled token rows at the
+    240-token block edges."""
+    calls, refs = [], []
+    status = tsg.new_status()
+    for idx, (name, N, K) in enumerate(si.LLAMA2_7B):
+        w, ids = llama2_weight(idx)
+        bm = si.tiles_exact(N, K, frac, 3, idx)
+        pw = tsg.patch_pack(to_dev_bf16(w), to_dev(bm), to_dev(ids), int(bm.sum()), status=status)
+        x = si.gen_x(2048, K, 3, idx)
+        calls.append((to_dev_bf16(x), pw, None))
+        refs.append((name, x, w, bm, ids))
+    ys = tsg.patch_gemm_group(calls, status=status)
+    code, bits = tsg.patch_read_status(status)
+    assert code == 0, (code, bits)
+    rows = np.array([0, 1, 239, 240, 1023, 1500, 2046, 2047])
+    for y, (name, x, w, bm, ids) in zip(ys, refs):
+        ref = oracle.hybrid_gemm(x, w, bm, ids, rows=rows)
+        check_gemm(bits_of(y)[rows], ref, f"{name} f={frac}")
 
 
 def test_group_skips_empty_calls_and_checks_arguments():
