@@ -109,6 +109,31 @@ def test_flops_block_and_monotonic_sweep():
     assert not mono and not sweep["q"]["monotonic"]
 
 
+def test_group_flops_block_over_segments():
+    """Calls timed as group launches: the step's TFLOP/s and mixed-roofline
+    fraction over all calls, and per segment (one launch) its own share."""
+    layers = [{"name": "q", "N": 256, "K": 256, "bm": bm, "frac": f}
+              for f, bm in ((0.0, np.zeros((2, 2), np.uint8)), (1.0, np.ones((2, 2), np.uint8)))]
+    calls = [(0, 65536), (1, 65536), (0, 512), (1, 512)]
+    steps = 2
+    segs = [(0, 2), (2, 4)]
+    seg = np.tile([0.006, 0.002], (steps, 1))  # ms per launch, the step 0.008 ms
+    out = bench.group_flops_block(_args(steps), layers, calls, _fake_t(steps * 0.008, seg), PK, 1, segs,
+                                  ["big", "small"], sparse_ratio=1.7)
+    fl = np.array([2 * M * 256 * 256 for _, M in calls], dtype=np.float64)
+    assert np.isclose(out["value"], fl.sum() / 1e12 / 8e-6, rtol=1e-3)
+    r2 = [bench.roof_seconds(layers[li], M, 1500.0, 2.0) for li, M in calls]
+    assert np.isclose(out["roofline"]["frac"], sum(r2) / 8e-6, atol=1e-4)
+    rm = sum(bench.roof_seconds(layers[li], M, 1500.0, 1.7) for li, M in calls)
+    assert np.isclose(out["roofline"]["frac_measured_sparse_peak"], rm / 8e-6, atol=1e-4)
+    assert np.isclose(out["per_segment"]["big"]["us"], 6.0) and np.isclose(out["per_segment"]["small"]["us"], 2.0)
+    assert np.isclose(out["per_segment"]["small"]["TFLOP/s"], fl[2:].sum() / 1e12 / 2e-6, rtol=1e-2)
+    assert np.isclose(out["per_segment"]["big"]["roofline_frac"], (r2[0] + r2[1]) / 6e-6, atol=2e-3)
+    # one segment: no per-segment split
+    one = bench.group_flops_block(_args(steps), layers, calls, _fake_t(steps * 0.008, None), PK, 1, [(0, 4)], ["all"])
+    assert "per_segment" not in one and np.isclose(one["value"], out["value"], rtol=1e-6)
+
+
 def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(2.0, 5, 4, 1000.0) == 2.0 * 5 * 4
 
