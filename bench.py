@@ -312,6 +312,14 @@ def call_flops(L, M):
     return 2.0 * M * L["N"] * L["K"]
 
 
+def call_alg_flops(L, M):
+    """FLOPs the tensor cores do: a dense tile 2*M*128*128, a sparse tile half
+    of it (its MMAs multiply only the kept half of W)."""
+    T = (L["N"] // 128) * (L["K"] // 128)
+    ns = int(L["bm"].sum())
+    return 2.0 * M * 128 * (128 * (T - ns) + 64 * ns)
+
+
 def roof_seconds(L, M, P_tflops, ratio):
     """Mixed roofline time of one prefill GEMM: dense tiles at the dense peak P,
     sparse tiles (half the MMA work) at ratio x P."""
@@ -1011,13 +1019,17 @@ def flops_block(args, name, layers, calls, t, pk, world, sparse_ratio=None, traf
     traffic = measured_traffic(traffic_kind, [f"{layers[li]['name']}/f={layers[li]['frac']}" for li, M in calls]) \
         if traffic_kind else None
     out = block_common(args, t, alg.sum() / 1e12, "TFLOP/s", world)
+    done = np.array([call_alg_flops(layers[li], M) for li, M in calls], dtype=np.float64)
     roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": P, "unit": "TFLOP/s",
+            "algorithmic_tflops": round(float(done.sum() / 1e12 / (split.sum() / 1e3)), 1),
             "frac": round(frac, 4), "traffic": None if traffic is None else round(traffic),
             "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
             "frac_of_sustained": round(frac * P / pk["bf16_tflops_sustained"], 4)
             if pk.get("bf16_tflops_sustained") else None,
             "kernel": "prefill_kernel (tcgen05)", "peak_source": pk["source"],
-            "note": "frac = mixed roofline time (dense tiles at the dense peak, sparse tiles at 2x it) / measured"}
+            "note": "frac = mixed roofline time (dense tiles at the dense peak, sparse tiles at 2x it) / measured; "
+                    "achieved counts dense-equivalent FLOPs (2 M N K), algorithmic_tflops the FLOPs the tensor "
+                    "cores do (a sparse tile half of a dense one)"}
     if sparse_ratio:
         # the same roofline with sparse tiles at the measured sparse/dense MMA rate ratio
         tm = np.array([roof_seconds(layers[li], M, P, sparse_ratio) for li, M in calls])
@@ -1026,6 +1038,7 @@ def flops_block(args, name, layers, calls, t, pk, world, sparse_ratio=None, traf
     out["roofline"] = roof
     out["per_call"] = {f"{layers[li]['name']}/f={layers[li]['frac']}@M={M}":
                        {"us": round(1e3 * split[j], 1), "TFLOP/s": round(alg[j] / 1e12 / (split[j] / 1e3), 1),
+                        "algorithmic_TFLOP/s": round(done[j] / 1e12 / (split[j] / 1e3), 1),
                         "roofline_frac": round(t2[j] / (split[j] / 1e3), 3)}
                        for j, (li, M) in enumerate(calls)}
     return out, split
@@ -1041,7 +1054,9 @@ def group_flops_block(args, layers, calls, t, pk, world, segments, seg_names, sp
     seg_fl = np.array([alg[lo:hi].sum() for lo, hi in segments])
     split = split_of(t, seg_fl, args.steps)
     out = block_common(args, t, alg.sum() / 1e12, "TFLOP/s", world)
+    done = sum(call_alg_flops(layers[li], M) for li, M in calls)
     roof = {"bound": "tensor", "achieved": round(float(alg.sum() / 1e12 / (split.sum() / 1e3)), 1), "peak": P,
+            "algorithmic_tflops": round(float(done / 1e12 / (split.sum() / 1e3)), 1),
             "unit": "TFLOP/s", "frac": round(float(t2.sum() / (split.sum() / 1e3)), 4), "traffic": None,
             "kernel": "prefill_kernel (patch_gemm_group)", "peak_source": pk["source"],
             "note": "frac = mixed roofline time (dense tiles at the dense peak, sparse tiles at 2x it) / measured"}

@@ -102,6 +102,10 @@ def test_flops_block_and_monotonic_sweep():
     assert np.isclose(out["roofline"]["frac"], r2 / 9e-6, atol=1e-4)
     rm = sum(bench.roof_seconds(L, 65536, 1500.0, 1.7) for L in layers)
     assert np.isclose(out["roofline"]["frac_measured_sparse_peak"], rm / 9e-6, atol=1e-4)
+    # the tensor cores' own work: all-dense 4 tiles, half-sparse 3 tile-equivalents, all-sparse 2
+    tile = 2 * 65536 * 128 * 128
+    assert np.isclose(out["roofline"]["algorithmic_tflops"], (4 + 3 + 2) * tile / 1e12 / 9e-6, rtol=1e-3)
+    assert np.isclose(out["per_call"]["q/f=1.0@M=65536"]["algorithmic_TFLOP/s"], 2 * tile / 1e12 / 2e-6, rtol=1e-2)
     sweep, mono = bench.sweep_summary(layers, calls, split)
     assert mono and sweep["q"]["speedup_vs_all_dense"] == [1.0, round(4 / 3, 3), 2.0]
     # a slower middle fraction breaks monotonicity
