@@ -510,6 +510,23 @@ PATCH_API patch_status_t patch_shard_rows(const uint8_t *bitmap, int64_t Tn, int
                                           int64_t *row_begin);
 
 /*
+ * patch_shard_rows_by: patch_shard_rows with a choice of what the shards
+ * balance (the same prefix rule and the same non-empty adjustment):
+ *   by = PATCH_SHARD_BY_BYTES: the stored bytes above (decode, M <= 16, streams
+ *        them: patch_shard_rows itself);
+ *   by = PATCH_SHARD_BY_FLOPS: the tensor cores' work, 2 per dense tile and 1
+ *        per sparse tile (prefill: a sparse tile's MMAs multiply half of W,
+ *        "Inference & Deployment"), so that each GPU's prefill GEMM takes the
+ *        same time rather than moving the same bytes.
+ * Host only.  Errors as patch_shard_rows, and PATCH_ERR_INVALID_ARG for any
+ * other value of by.
+ */
+#define PATCH_SHARD_BY_BYTES 0
+#define PATCH_SHARD_BY_FLOPS 1
+PATCH_API patch_status_t patch_shard_rows_by(const uint8_t *bitmap, int64_t Tn, int64_t Tk, int64_t n_shards,
+                                             int64_t by, int64_t *row_begin);
+
+/*
  * patch_mma_probe: a measurement of this GPU's tensor-core MMA rate for the
  * two instruction forms of the hybrid GEMM ("Inference & Deployment": dense
  * tiles on the dense tensor-core MMA, sparse tiles on the 2:4 sparse one),

@@ -148,6 +148,18 @@ def test_group_host_checks(lib):
     assert group(tsg._ChainCall(None, None, w, 0, 0, 0), tsg._ChainCall(fake, fake, w, 4, 1, 0)) == 1
 
 
+def test_shard_rows_by_refuses_an_unknown_balance(lib):
+    import numpy as np
+    bm = np.zeros((4, 2), np.uint8)
+    out = np.zeros(3, np.int64)
+    P = ctypes.c_void_p
+    args = (bm.ctypes.data_as(P), 4, 2, 2)
+    assert lib.patch_shard_rows_by(*args, 0, out.ctypes.data_as(P)) == 0 and list(out) == [0, 2, 4]
+    assert lib.patch_shard_rows_by(*args, 1, out.ctypes.data_as(P)) == 0 and list(out) == [0, 2, 4]
+    assert lib.patch_shard_rows_by(*args, 2, out.ctypes.data_as(P)) == 1
+    assert lib.patch_shard_rows_by(*args, -1, out.ctypes.data_as(P)) == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(tsg, "_lib", None)
     monkeypatch.setattr(tsg, "_LIB_PATH", tmp_path / "libpatch.so")

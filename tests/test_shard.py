@@ -1,5 +1,5 @@
 """Column-parallel sharding of a layer over several GPUs (host logic, CPU):
-the tile-row split balanced by stored bytes, and -- with two gloo ranks --
+the tile-row split balanced by stored bytes or by MMA work, and -- with two gloo ranks --
 that the shards' outputs concatenate to the whole layer's output."""
 import os
 import socket
@@ -41,6 +41,38 @@ def test_shard_rows_definition_and_balance(n, kind):
     # balance: no shard exceeds its fair share by more than one row
     worst = max(prefix[e] - prefix[b] for b, e in rows)
     assert worst <= total / n + rb.max()
+
+
+@pytest.mark.parametrize("n", [2, 3, 8])
+def test_shard_rows_by_flops_balances_the_mma_work(n):
+    """by="flops": each tile row weighs 2 per dense tile and 1 per sparse tile
+    (a sparse tile's MMAs multiply half of W); the same prefix rule as by bytes."""
+    N, K = 128 * 43, 128 * 8
+    bm = si.tiles_clustered(N, K, 0.5, 3, 7 + n)
+    rows = tsg.shard_rows(bm, n, by="flops")
+    rw = np.where(bm != 0, 1, 2).sum(axis=1)
+    prefix = np.concatenate([[0], np.cumsum(rw)])
+    total = prefix[-1]
+    assert rows[0][0] == 0 and rows[-1][1] == bm.shape[0]
+    for i, (b, e) in enumerate(rows):
+        assert e > b
+        if i > 0:
+            assert prefix[b] * n >= i * total and prefix[b - 1] * n < i * total
+    assert max(prefix[e] - prefix[b] for b, e in rows) <= total / n + rw.max()
+
+
+def test_shard_balance_by_bytes_and_by_flops_differ_where_they_should():
+    """A sparse row weighs ~0.56 of a dense one in bytes (18448 vs 32784 with
+    its descriptor) but 0.5 in MMA work: 3 dense rows then 6 sparse ones split
+    4 + 5 by bytes (the 3 dense rows hold 98352 B of 209040, under half, so
+    the second shard starts after row 4) and 3 + 6 by work (6 of 12)."""
+    bm = np.zeros((9, 1), np.uint8)
+    bm[3:] = 1
+    assert tsg.shard_rows(bm, 2, by="flops") == [(0, 3), (3, 9)]
+    assert tsg.shard_rows(bm, 2, by="bytes") == [(0, 4), (4, 9)]
+    assert tsg.shard_rows(bm, 2) == tsg.shard_rows(bm, 2, by="bytes")
+    with pytest.raises(KeyError):
+        tsg.shard_rows(bm, 2, by="rows")
 
 
 def test_shard_rows_keeps_every_shard_non_empty():

@@ -91,6 +91,7 @@ def lib() -> ctypes.CDLL:
             "patch_exec_tiles": [P, I64, I64, I64, P, P, P],
             "patch_soft_mask": [P, I64, I64, P, P, P, P, ctypes.c_float, P, P, P],
             "patch_shard_rows": [P, I64, I64, I64, P],
+            "patch_shard_rows_by": [P, I64, I64, I64, I64, P],
             "patch_pack_from_logits": [P, I64, I64, P, P, I64, P, P, P, P, P],
             "patch_gemm_workspace_size": [I64, WP, ctypes.POINTER(SZ)],
             "patch_gemm": [P, I64, WP, P, P, SZ, P, P],
@@ -486,15 +487,20 @@ def patch_gemm_mlp(X: torch.Tensor, gate: PackedWeight, up: PackedWeight, H: tor
     return H
 
 
-def shard_rows(bitmap, n_shards: int) -> list[tuple[int, int]]:
+SHARD_BY = {"bytes": 0, "flops": 1}  # PATCH_SHARD_BY_BYTES / PATCH_SHARD_BY_FLOPS
+
+
+def shard_rows(bitmap, n_shards: int, by: str = "bytes") -> list[tuple[int, int]]:
     """Column-parallel split of a layer into n_shards contiguous tile-row ranges
-    balanced by stored bytes (host computation): [(row_begin, row_end), ...]."""
+    (host computation): [(row_begin, row_end), ...], balanced by stored bytes
+    (by="bytes": decode) or by the tensor cores' work (by="flops": prefill, a
+    dense tile counting twice a sparse one)."""
     import numpy as np
     bm = np.ascontiguousarray(bitmap.cpu().numpy() if isinstance(bitmap, torch.Tensor) else bitmap, dtype=np.uint8)
     Tn, Tk = bm.shape
     out = np.zeros(n_shards + 1, dtype=np.int64)
-    _check(lib().patch_shard_rows(bm.ctypes.data_as(ctypes.c_void_p), Tn, Tk, n_shards,
-                                  out.ctypes.data_as(ctypes.c_void_p)), "patch_shard_rows")
+    _check(lib().patch_shard_rows_by(bm.ctypes.data_as(ctypes.c_void_p), Tn, Tk, n_shards, SHARD_BY[by],
+                                     out.ctypes.data_as(ctypes.c_void_p)), "patch_shard_rows_by")
     return [(int(out[i]), int(out[i + 1])) for i in range(n_shards)]
 
 

@@ -456,27 +456,33 @@ patch_status_t patch_gemm_mlp(const uint16_t* X, int64_t M, const patch_weight* 
   return PATCH_OK;
 }
 
-patch_status_t patch_shard_rows(const uint8_t* bitmap, int64_t Tn, int64_t Tk, int64_t n_shards,
-                                int64_t* row_begin) {
-  if (!bitmap || !row_begin || Tn < 1 || Tk < 1 || n_shards < 1 || n_shards > Tn) return PATCH_ERR_INVALID_ARG;
-  // prefix sums of the stored bytes of the tile rows
-  int64_t total = 0;
-  for (int64_t r = 0; r < Tn; ++r) {
-    int64_t b = 16 * Tk;
-    for (int64_t k = 0; k < Tk; ++k)
-      b += bitmap[r * Tk + k] ? int64_t(PATCH_SPARSE_TILE_BYTES + PATCH_META_TILE_BYTES) : int64_t(PATCH_DENSE_TILE_BYTES);
-    total += b;
+// Weight of tile row r under a shard balance: stored bytes (decode streams
+// them) or the tensor cores' MMA work in units of a sparse tile's (prefill:
+// a dense tile does 2, a sparse tile 1).
+static int64_t row_weight(const uint8_t* bitmap, int64_t r, int64_t Tk, int64_t by) {
+  int64_t w = by == PATCH_SHARD_BY_FLOPS ? 0 : 16 * Tk;
+  for (int64_t k = 0; k < Tk; ++k) {
+    const bool sparse = bitmap[r * Tk + k] != 0;
+    if (by == PATCH_SHARD_BY_FLOPS)
+      w += sparse ? 1 : 2;
+    else
+      w += sparse ? int64_t(PATCH_SPARSE_TILE_BYTES + PATCH_META_TILE_BYTES) : int64_t(PATCH_DENSE_TILE_BYTES);
   }
+  return w;
+}
+
+patch_status_t patch_shard_rows_by(const uint8_t* bitmap, int64_t Tn, int64_t Tk, int64_t n_shards, int64_t by,
+                                   int64_t* row_begin) {
+  if (!bitmap || !row_begin || Tn < 1 || Tk < 1 || n_shards < 1 || n_shards > Tn) return PATCH_ERR_INVALID_ARG;
+  if (by != PATCH_SHARD_BY_BYTES && by != PATCH_SHARD_BY_FLOPS) return PATCH_ERR_INVALID_ARG;
+  int64_t total = 0;
+  for (int64_t r = 0; r < Tn; ++r) total += row_weight(bitmap, r, Tk, by);
   row_begin[0] = 0;
-  int64_t r = 0, before = 0;  // rows [0, r) hold `before` bytes
+  int64_t r = 0, before = 0;  // rows [0, r) weigh `before`
   for (int64_t i = 1; i < n_shards; ++i) {
     // first row whose prefix reaches i / n of the total (compared without rounding)
     while (r < Tn && before * n_shards < i * total) {
-      int64_t b = 16 * Tk;
-      for (int64_t k = 0; k < Tk; ++k)
-        b += bitmap[r * Tk + k] ? int64_t(PATCH_SPARSE_TILE_BYTES + PATCH_META_TILE_BYTES)
-                                : int64_t(PATCH_DENSE_TILE_BYTES);
-      before += b;
+      before += row_weight(bitmap, r, Tk, by);
       ++r;
     }
     // strictly increasing, and leave at least one row for each later shard
@@ -487,6 +493,11 @@ patch_status_t patch_shard_rows(const uint8_t* bitmap, int64_t Tn, int64_t Tk, i
   }
   row_begin[n_shards] = Tn;
   return PATCH_OK;
+}
+
+patch_status_t patch_shard_rows(const uint8_t* bitmap, int64_t Tn, int64_t Tk, int64_t n_shards,
+                                int64_t* row_begin) {
+  return patch_shard_rows_by(bitmap, Tn, Tk, n_shards, PATCH_SHARD_BY_BYTES, row_begin);
 }
 
 patch_status_t patch_mma_probe_m(int m, int sparse, int64_t iters, int32_t* dev_status, void* stream) {
