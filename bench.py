@@ -39,6 +39,7 @@ C, fp64) on a bounded sample of the decode workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import functools
 import json
 import os
 import statistics
@@ -1099,13 +1100,38 @@ def run_block(args, workload, rank, world, dev, pk, status, sparse_ratio=None):
     import torch
     layers = build_layers(workload, args.layers, args.fracs, args.tokens)
     full_layers = layers
-    shard = getattr(args, "shard", False) and world > 1 and workload == "decode"
+    shard = getattr(args, "shard", False) and world > 1 and workload in ("decode", "prefill")
     if shard:
         import tile_sparse_gemm_b200 as tsg
-        layers = shard_layers(full_layers, rank, world, tsg.shard_rows)
+        # decode streams stored bytes, prefill spends tensor-core work: balance each by its own
+        by = "bytes" if workload == "decode" else "flops"
+        split_rows = functools.partial(tsg.shard_rows, by=by)
+        layers = shard_layers(full_layers, rank, world, split_rows)
     packed = pack_layers(layers, dev, status)
     resident = sum(p.stored_bytes for p in packed)
     full = not (args.layers or args.fracs or args.tokens)
+    if shard:  # one column-parallel shard per rank, the step's Y shards all-gathered once per step
+        calls = calls_of(layers)
+        _, _, seg = gather_layout(full_layers, calls, world, split_rows)
+        if workload == "decode":  # this rank's shards of the step's independent GEMMs as one chain launch
+            t = time_calls(args, layers, packed, calls, dev, world, status, chain=True, after=False, gather=seg)
+            out = bytes_block(args, workload, full_layers, calls, t, pk, 1, segments=[(0, len(calls))],
+                              seg_names=["step"], chain=True)
+            out["metric"] = "hybrid GEMM HBM GB/s over stored bytes (decode, sharded)"
+        else:  # this rank's shards as separate patch_gemm calls
+            t = time_calls(args, layers, packed, calls, dev, world, status, gather=seg)
+            out = flops_block(args, workload, full_layers, calls, t, pk, 1, sparse_ratio)[0]
+            out.pop("per_call", None)  # eager steps carry no per-call split
+            out["metric"] = "hybrid GEMM TFLOP/s, dense-equivalent (prefill, sharded)"
+        out["scaling"] = "strong"
+        out["step"] = (f"column-parallel: each of {world} ranks multiplies its tile rows of every layer (balanced by "
+                       f"{'stored bytes' if by == 'bytes' else 'tensor-core work'}), then one NCCL all-gather of the "
+                       "step's Y shards")
+        out["config"] = {"workload": f"LLaMA-2-7B linear layers ({workload}), column-parallel shards",
+                         "parallelism": f"column-parallel x{world}", "shard_balance": by}
+        del packed
+        torch.cuda.synchronize()
+        return out
     if workload in ("decode", "decode_fused"):
         calls = calls_of(layers)
         # the step's 21 GEMMs are independent (every X is an input of the step):
@@ -1281,7 +1307,7 @@ def main():
     ap.add_argument("--fracs", nargs="*", type=float, help="profiling: only these sparse-tile fractions")
     ap.add_argument("--tokens", nargs="*", type=int, help="profiling: only these token counts M")
     ap.add_argument("--shard", action="store_true",
-                    help="decode under torchrun: each rank multiplies a column-parallel shard of every layer, "
+                    help="decode or prefill under torchrun: each rank multiplies a column-parallel shard of every layer, "
                          "then one all-gather of Y per step (strong scaling) instead of independent replicas")
     args = ap.parse_args()
     if args.impl == "ours" and args.warmup < 3:

@@ -195,7 +195,45 @@ def test_run_ours_assembles_every_block_on_fake_timings(monkeypatch, workload):
     json.dumps(out)  # serialisable
 
 
-def bench_small_layers(workload):
+@pytest.mark.parametrize("workload", ["decode", "prefill"])
+def test_run_ours_sharded_blocks_on_fake_timings(monkeypatch, workload):
+    """--shard with two ranks: each rank's block is its column-parallel shard
+    plus one all-gather per step (the timer is faked); the line reports the
+    whole job's throughput as strong scaling, balanced by bytes for decode and
+    by tensor-core work for prefill."""
+    import types
+
+    import torch
+    seen = {}
+
+    class FakePacked:
+        def __init__(self, L):
+            self.stored_bytes = bench.stored_bytes(L["N"], L["K"], int(L["bm"].sum()))
+
+    def fake_time_calls(args, layers, packed, calls, dev, world, status, segments=None, chain=False, after=True,
+                        gather=None, group=False):
+        seen["gather"], seen["N"] = gather, [L["N"] for L in layers]
+        return {"ms": 1.0 * args.steps, "e2e_ms": 2.0 * args.steps, "seg_ms": None, "clocks": {"sm_mhz": 1965.0},
+                "h2d": 1, "d2h": 1, "launches": 2}
+
+    monkeypatch.setattr(bench, "pack_layers", lambda layers, dev, status: [FakePacked(L) for L in layers])
+    monkeypatch.setattr(bench, "time_calls", fake_time_calls)
+    monkeypatch.setattr(bench, "mma_rates", lambda dev: {"sparse_over_dense": 1.5})
+    monkeypatch.setattr(bench, "build_layers", lambda w, *a: bench_small_layers(w, rows=6))
+    monkeypatch.setattr(torch.cuda, "set_device", lambda d: None)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    monkeypatch.setattr(torch.cuda, "empty_cache", lambda: None)
+    import tile_sparse_gemm_b200 as tsg
+    monkeypatch.setattr(tsg, "new_status", lambda dev=None: None)
+    args = types.SimpleNamespace(steps=4, warmup=3, no_graph=False, layers=None, fracs=None, tokens=None,
+                                 shard=True, workload=workload)
+    out = bench.run_ours(args, 0, 2)
+    assert out["scaling"] == "strong" and "sharded" in out["metric"] and out["value"] > 0
+    assert out["config"]["shard_balance"] == ("bytes" if workload == "decode" else "flops")
+    assert seen["gather"] > 0 and all(n < 6 * 128 for n in seen["N"])  # rank 0 holds a part of every layer
+
+
+def bench_small_layers(workload, rows=2):
     """Small stand-ins for each workload's layers (shapes, bitmaps and X only)."""
     rng = np.random.default_rng(0)
 
@@ -206,9 +244,9 @@ def bench_small_layers(workload):
         return dict(name=name, N=N, K=K, bm=bm.reshape(N // 128, K // 128), frac=frac,
                     xs={M: np.zeros((M, K), np.uint16) for M in ms}, **kw)
     if workload in ("decode", "decode_fused"):
-        return [L(n, 256, 256, 0.5, (1, 4, 16)) for n in ("q", "gate")]
+        return [L(n, 128 * rows, 256, 0.5, (1, 4, 16)) for n in ("q", "gate")]
     if workload == "prefill":
-        return [L(n, 256, 256, f, (2048,)) for n in ("q", "down") for f in bench.FRACS]
+        return [L(n, 128 * rows, 256, f, (2048,)) for n in ("q", "down") for f in bench.FRACS]
     if workload == "stack":
         return [L(f"L{i}.{n}", 256, 256, 0.1, (1, 8), proj=n) for i in range(2) for n in ("q", "down")]
     if workload == "llama3_qwen":

@@ -1,6 +1,7 @@
 """Column-parallel sharding of a layer over several GPUs (host logic, CPU):
 the tile-row split balanced by stored bytes or by MMA work, and -- with two gloo ranks --
 that the shards' outputs concatenate to the whole layer's output."""
+import functools
 import os
 import socket
 import sys
@@ -125,9 +126,10 @@ def test_two_ranks_concatenate_to_the_whole_layer():
         assert np.array_equal(out[r], ref)
 
 
-def _bench_rank(rank, world, port, out):
-    """bench.py's sharded decode step on CPU: its shard plan, its gather layout and
-    one all-gather (gloo), with the oracle standing in for each rank's GEMMs."""
+def _bench_rank(rank, world, port, out, by):
+    """bench.py's sharded step on CPU: its shard plan (balanced by `by`), its
+    gather layout and one all-gather (gloo), with the oracle standing in for each
+    rank's GEMMs."""
     import datetime
 
     import torch
@@ -147,8 +149,9 @@ def _bench_rank(rank, world, port, out):
             layers.append(dict(name=f"l{i}", N=N, K=K, w=w, bm=s.tiles_clustered(N, K, 0.5, 18, i),
                                ids=s.patterns_top2(w), xs={M: s.gen_x(M, K, 18, 10 * i + M) for M in (1, 5)}))
         calls = bench.calls_of(layers)
-        mine = bench.shard_layers(layers, rank, world, t.shard_rows)
-        offset, sizes, seg = bench.gather_layout(layers, calls, world, t.shard_rows)
+        split = functools.partial(t.shard_rows, by=by)
+        mine = bench.shard_layers(layers, rank, world, split)
+        offset, sizes, seg = bench.gather_layout(layers, calls, world, split)
         buf = torch.zeros(seg, dtype=torch.float64)
         for j, (li, M) in enumerate(calls):
             L = mine[li]
@@ -166,10 +169,11 @@ def _bench_rank(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_bench_shard_plan_and_gather_reassemble_every_call():
+@pytest.mark.parametrize("by", ["bytes", "flops"])
+def test_bench_shard_plan_and_gather_reassemble_every_call(by):
     world = 2
     out = mp.get_context("spawn").Manager().dict()
-    mp.start_processes(_bench_rank, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+    mp.start_processes(_bench_rank, args=(world, _free_port(), out, by), nprocs=world, start_method="spawn")
     for i, (N, K) in enumerate([(128 * 7, 256), (128 * 3, 384), (128 * 10, 128)]):
         w = si.gen_w(N, K, 18, i)
         bm, ids = si.tiles_clustered(N, K, 0.5, 18, i), si.patterns_top2(w)
