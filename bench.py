@@ -1354,7 +1354,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     out = run_ours(args, rank, world)
     if rank == 0:
-        if not args.no_cpu_baseline and args.workload in ("all", "decode", "decode_fused", "prefill"):
+        # the oracle's host-core baseline: single-GPU runs only
+        if world == 1 and not args.no_cpu_baseline and args.workload in ("all", "decode", "decode_fused", "prefill"):
             out["cpu_baseline"] = cpu_baseline(ref_workload, budget_s=30.0, min_s=10.0)
             if args.workload == "all":
                 out["prefill"]["cpu_baseline"] = cpu_baseline("prefill", budget_s=15.0, min_s=5.0)
