@@ -317,12 +317,12 @@ def _layer(N, K, M, kind, frac, cfg=3, shape_idx=0):
     return x, w, bm, si.patterns_top2(w)
 
 
-def test_gemm_config1_decode():
+def test_gemm_512x512_bernoulli_tiles_m16():
     """512 x 512 weight, Bernoulli(0.5) tiles, M = 16 tokens."""
     x, w, bm, ids = _layer(512, 512, 16, "bernoulli", 0.5, cfg=1)
     ref = oracle.hybrid_gemm(x, w, bm, ids)
     y = gemm_on_gpu(x, pack_on_gpu(w, bm, ids))
-    check_gemm(y, ref, "config 1")
+    check_gemm(y, ref, "512 x 512, Bernoulli(0.5) tiles, M = 16")
 
 
 @pytest.mark.parametrize("path", [tsg.PATH_DECODE, tsg.PATH_DECODE_SIMT])
